@@ -1,0 +1,231 @@
+/*
+ * nvfp4_moe.h - C ABI of libnvfp4moe.so: the NVFP4 W4A4 routed-expert MoE
+ * layer on NVIDIA B200 (sm_100a).
+ *
+ * What the layer computes
+ *   "K-EXAONE-152B-A23B-REAP-80E-NVFP4" model card, section "Quantization
+ *   Setup": routed-expert weights are FP4 E2M1 in groups of 16 with FP8 E4M3
+ *   block scales, quantised round-to-nearest per expert Linear; activations
+ *   are quantised dynamically to FP4 under calibrated global scales; the
+ *   router (mlp.gate) stays BF16.
+ *   "[NetsPresso AQ Deep Dive] How to Quantize the K-EXAONE-236B Model to
+ *   4-Bit (NVFP4)", section "The Standard NVFP4 Serving Spec": NVFP4 scales a
+ *   block by a global scale times a block scale.
+ *   "K-EXAONE-152B-A23B-REAP-80E-BF16" model card, section "Pruning Setup",
+ *   "Routing behavior": renormalised sigmoid routing with an
+ *   e_score_correction_bias and a routed_scaling_factor.
+ *
+ * Conventions for every call
+ *   - Every data pointer is DEVICE memory owned by the caller; the library
+ *     never allocates, frees or keeps a pointer after the call returns.
+ *   - Work is queued on `stream` (a cudaStream_t passed as void*; NULL is the
+ *     legacy default stream) and the call returns without synchronising.
+ *     Argument checks happen on the host before anything is queued; a failed
+ *     check queues nothing.
+ *   - Errors come back as an nvfp4_status; nvfp4_last_error() gives a message
+ *     for the calling host thread.  Nothing is thrown across the ABI.
+ *   - bf16 tensors are row-major with the last index contiguous.
+ *   - Packed codes: two E2M1 codes per byte, the element with the even index
+ *     in the low nibble; the sign is bit 3 of a code.
+ *   - Scale layouts (one E4M3 byte per 16 consecutive elements of a row):
+ *       NVFP4_LAYOUT_CANONICAL: [rows][cols/16] row-major.
+ *       NVFP4_LAYOUT_TILED: the layout the tensor-core MMA reads.  Rows are
+ *       grouped in tiles of 128 and 16-element blocks in groups of 4; each
+ *       (row tile, block group) is a 512-byte atom, atoms ordered row tile
+ *       major, and inside an atom row r (0..127), block b (0..3) sits at byte
+ *       (r % 32) * 16 + (r / 32) * 4 + b.  The buffer holds
+ *       ceil(rows/128) * 128 * cols / 16 bytes; needs cols % 64 == 0.
+ *   - Workspace: calls that take (ws, ws_bytes) need at least the size their
+ *     *_workspace_size() function returns, 256-byte aligned.  Its first word
+ *     is a status word: each call clears it when it starts and a device-side
+ *     wait that gives up sets it; read it with nvfp4_workspace_status().
+ */
+#ifndef NVFP4_MOE_H
+#define NVFP4_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define NVFP4_API __attribute__((visibility("default")))
+#else
+#define NVFP4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum nvfp4_status {
+  NVFP4_OK = 0,
+  NVFP4_ERR_INVALID_ARG = 1,       /* null pointer, bad enum, negative size   */
+  NVFP4_ERR_UNSUPPORTED_SHAPE = 2, /* a size the kernels do not handle        */
+  NVFP4_ERR_CUDA = 3,              /* a CUDA runtime or driver call failed    */
+  NVFP4_ERR_TIMEOUT = 4,           /* a device-side wait gave up              */
+  NVFP4_ERR_WORKSPACE = 5,         /* workspace missing, misaligned or small  */
+  NVFP4_ERR_DEVICE = 6             /* the current device is not an sm_100 GPU */
+} nvfp4_status;
+
+enum { NVFP4_LAYOUT_CANONICAL = 0, NVFP4_LAYOUT_TILED = 1 };
+
+/* Message for the last failed call on this host thread ("" if none). */
+NVFP4_API const char* nvfp4_last_error(void);
+
+/* Version of this interface (incremented on any signature change). */
+NVFP4_API int nvfp4_abi_version(void);
+
+/* Synchronises `stream`, then reads the status word a call left at the start
+ * of `ws`: NVFP4_OK, or NVFP4_ERR_TIMEOUT if a device-side wait gave up (the
+ * outputs of that call are then undefined).  Resets the word to 0. */
+NVFP4_API nvfp4_status nvfp4_workspace_status(void* ws, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Offline RTN weight quantiser ("Quantization Setup": round-to-nearest weight
+ * quantisation at per-expert Linear granularity).
+ *
+ * Quantises n_mats independent bf16 matrices w[n_mats][rows][cols].  For each
+ * matrix: g = amax|w| / (6 * 448) (fp32 division); for each 16-element block
+ * of a row: s = E4M3(amax_block / (6 g)), S = s * g, codes = E2M1(x * (1/S))
+ * with round-to-nearest-even and saturation; a zero block or matrix gives
+ * scale 0 and codes +-0.
+ *   codes        [n_mats][rows][cols/2]
+ *   scales       CANONICAL: [n_mats][rows][cols/16];
+ *                TILED: n_mats * rows rows in the tiled layout (rows % 128 == 0)
+ *   global_scale [n_mats] fp32
+ * Needs cols % 32 == 0 (TILED: cols % 64 == 0, rows % 128 == 0).
+ * Each matrix is read twice (amax pass, then quantise pass) with the second
+ * read scheduled while the matrix is still in L2.
+ * ---------------------------------------------------------------------- */
+NVFP4_API size_t nvfp4_quantize_weights_workspace_size(int n_mats);
+NVFP4_API nvfp4_status nvfp4_quantize_weights(const void* w_bf16, int n_mats, int rows, int cols, int layout,
+                                    uint8_t* codes, uint8_t* scales, float* global_scale, void* ws,
+                                    size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Dynamic activation quantiser ("Quantization Setup": activations dynamically
+ * quantised to FP4 with calibrated global scales).
+ *
+ * x[rows][cols] bf16 under the caller's calibrated global scale (one fp32 in
+ * device memory), same block arithmetic as the weight quantiser.
+ *   codes  [rows][cols/2];  scales CANONICAL [rows][cols/16] or TILED
+ *   (rows beyond `rows` in the last 128-row tile get scale 0).
+ * Needs cols % 32 == 0 (TILED: cols % 64 == 0).
+ * ---------------------------------------------------------------------- */
+NVFP4_API nvfp4_status nvfp4_quantize_act(const void* x_bf16, int rows, int cols, const float* global_scale,
+                                int layout, uint8_t* codes, uint8_t* scales, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Router and permutation ("Pruning Setup", "Routing behavior").
+ *
+ * logits = x W^T + logit_offset (bf16 operands, fp32 accumulation; the
+ * optional per-expert logit_offset is a synthetic load-skew knob, not part of
+ * the method), or the caller's logits_in when that is non-NULL (then x_bf16,
+ * router_weight_bf16 and logit_offset must be NULL).
+ * sigma = 1 / (1 + exp(-logit)) with a fixed fp32 exp (Cody-Waite reduction by
+ * ln 2, degree-7 Taylor polynomial, IEEE operations only, |logit| clamped to
+ * 80); the k experts with the largest sigma + bias are selected (ties to the
+ * lower index) in descending order; w_j = (sigma_j / sum_sel sigma) * rsf
+ * with the sum taken in fp32 in that order.
+ * Permutation: pairs (token t, slot j) ordered by expert, token, slot; each
+ * expert's segment padded to a multiple of 128 rows.
+ *   logits_out     [T][E] fp32 (nullable)
+ *   topk_idx       [T][k] int32;  topk_w [T][k] fp32
+ *   expert_offsets [E+1] int32 (row where each expert's segment starts)
+ *   perm           [moe_route_rows_capacity(T,E,k)] int32: token of each row,
+ *                  -1 on padding rows and beyond expert_offsets[E]
+ *   inv_perm       [T][k] int32: row of each (token, slot)
+ * Needs 1 <= k <= 16, k <= E <= 256, H % 64 == 0.
+ * ---------------------------------------------------------------------- */
+NVFP4_API int moe_route_rows_capacity(int T, int E, int k);
+NVFP4_API size_t moe_route_workspace_size(int T, int E, int k);
+NVFP4_API nvfp4_status moe_route(const void* x_bf16, const void* router_weight_bf16, const float* logits_in,
+                       const float* bias, const float* logit_offset, int T, int H, int E, int k,
+                       float routed_scaling_factor, float* logits_out, int32_t* topk_idx, float* topk_w,
+                       int32_t* expert_offsets, int32_t* perm, int32_t* inv_perm, void* ws, size_t ws_bytes,
+                       void* stream);
+
+/* ------------------------------------------------------------------------
+ * The layer.
+ * ---------------------------------------------------------------------- */
+typedef struct moe_nvfp4_weights {
+  int E, H, I, k;                 /* experts, hidden, expert intermediate, top-k */
+  float routed_scaling_factor;
+  const void* router_weight;      /* bf16 [E][H] (kept BF16)                     */
+  const float* bias;              /* fp32 [E] e_score_correction_bias            */
+  const uint8_t* gate_codes;      /* [E][I][H/2]                                 */
+  const uint8_t* gate_scales;     /* TILED, E*I rows x H cols                    */
+  const float* gate_gscale;       /* [E]                                         */
+  const uint8_t* up_codes;        /* [E][I][H/2]                                 */
+  const uint8_t* up_scales;       /* TILED, E*I rows x H cols                    */
+  const float* up_gscale;         /* [E]                                         */
+  const uint8_t* down_codes;      /* [E][H][I/2]                                 */
+  const uint8_t* down_scales;     /* TILED, E*H rows x I cols                    */
+  const float* down_gscale;       /* [E]                                         */
+} moe_nvfp4_weights;
+
+/* Optional copies of intermediate results (every pointer nullable; device
+ * memory; row-indexed buffers have moe_route_rows_capacity(T,E,k) rows). */
+typedef struct moe_nvfp4_debug {
+  float* logits;                  /* [T][E]                                      */
+  int32_t* topk_idx;              /* [T][k]                                      */
+  float* topk_w;                  /* [T][k]                                      */
+  int32_t* expert_offsets;        /* [E+1]                                       */
+  int32_t* perm;                  /* [rows]                                      */
+  int32_t* inv_perm;              /* [T][k]                                      */
+  uint8_t* a_codes;               /* [rows][H/2] quantised x in permuted order   */
+  uint8_t* a_scales;              /* TILED, rows x H                             */
+  float* h;                       /* [rows][I] silu(gate)*up before requantising */
+  float* h_amax;                  /* max |h| over real rows (fp32, caller zeroes)*/
+  uint8_t* h_codes;               /* [rows][I/2]                                 */
+  uint8_t* h_scales;              /* TILED, rows x I                             */
+  float* y;                       /* [rows][H] weighted down-projection rows     */
+  /* cudaEvent_t handles (nullable, each created by the caller): recorded on
+   * `stream` at the start and after each stage (0 start, 1 routing and
+   * permutation, 2 quantise x, 3 gate/up GEMM, 4 down GEMM, 5 combine), so a
+   * caller can time every stage of a call on the device. */
+  void* stage_events[6];
+} moe_nvfp4_debug;
+
+NVFP4_API size_t moe_nvfp4_workspace_size(int T, int E, int H, int I, int k);
+
+/* out[T][H] bf16 = sum_j w_j * down_e( quant_g2( silu(gate_e(xq)) * up_e(xq) ) )
+ * with xq = x quantised under act_gscale (g1) and the intermediate quantised
+ * under h_gscale (g2), both one fp32 in device memory.  Steps: router GEMM ->
+ * top-k -> permutation -> quantise x into permuted rows -> grouped FP4 GEMM
+ * gate/up with SiLU*up and requantisation fused -> grouped FP4 GEMM down with
+ * g2 * g_down * w_j fused -> combine in slot order (fp32 sum, bf16 out).
+ * Needs H % 256 == 0, I % 128 == 0, 1 <= k <= 16, k <= E <= 256, T >= 1. */
+NVFP4_API nvfp4_status moe_nvfp4_forward(const moe_nvfp4_weights* W, const void* x_bf16, int T,
+                               const float* act_gscale, const float* h_gscale, const float* logit_offset,
+                               void* out_bf16, const moe_nvfp4_debug* dbg, void* ws, size_t ws_bytes,
+                               void* stream);
+
+/* ------------------------------------------------------------------------
+ * The two grouped GEMMs on caller-supplied quantised operands (the same
+ * kernels moe_nvfp4_forward runs).  Rows are grouped by expert_offsets
+ * ([E+1], each segment a multiple of 128 rows, expert_offsets[E] <=
+ * rows_capacity); expert_counts ([E], nullable) gives the rows of each segment
+ * that hold data (rows past it are written as zeros / skipped).
+ * ---------------------------------------------------------------------- */
+NVFP4_API size_t moe_nvfp4_gemm_workspace_size(int rows_capacity);
+
+/* h = silu(g1 g_gate[e] acc_gate) * (g1 g_up[e] acc_up), then quantised under
+ * h_gscale into h_codes [rows][I/2] and TILED h_scales.  h_f32 ([rows][I]) and
+ * h_amax (one fp32, caller zeroes) are optional outputs. */
+NVFP4_API nvfp4_status moe_nvfp4_gate_up(const moe_nvfp4_weights* W, const uint8_t* a_codes, const uint8_t* a_scales,
+                               const int32_t* expert_offsets, const int32_t* expert_counts, int rows_capacity,
+                               const float* act_gscale, const float* h_gscale, uint8_t* h_codes,
+                               uint8_t* h_scales, float* h_f32, float* h_amax, void* ws, size_t ws_bytes,
+                               void* stream);
+
+/* y[r] = g2 g_down[e] row_weight[r] acc_down[r]: y_bf16 [rows][H] and/or
+ * y_f32 [rows][H] (each nullable, not both).  row_weight nullable (= 1). */
+NVFP4_API nvfp4_status moe_nvfp4_down(const moe_nvfp4_weights* W, const uint8_t* h_codes, const uint8_t* h_scales,
+                            const int32_t* expert_offsets, const int32_t* expert_counts, int rows_capacity,
+                            const float* h_gscale, const float* row_weight, void* y_bf16, float* y_f32,
+                            void* ws, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NVFP4_MOE_H */

@@ -1,0 +1,44 @@
+/*
+ * nvfp4_moe_testing.h - test hooks of libnvfp4moe.so.
+ *
+ * These entry points expose the device-side building blocks of the layer so
+ * that tests can compare them element by element with an independent CPU
+ * implementation: the E2M1 and E4M3 conversions used by every quantiser
+ * (element formats of the "K-EXAONE-152B-A23B-REAP-80E-NVFP4" model card,
+ * "Quantization Setup") and the fixed fp32 sigmoid of the router
+ * ("K-EXAONE-152B-A23B-REAP-80E-BF16" model card, "Routing behavior").
+ * Same conventions as nvfp4_moe.h: device pointers, asynchronous on `stream`,
+ * nvfp4_status results.  They are not needed to run the layer.
+ */
+#ifndef NVFP4_MOE_TESTING_H
+#define NVFP4_MOE_TESTING_H
+
+#include "nvfp4_moe.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* For each y[i] (fp32), hw[i] = the E2M1 code the quantisers produce (the
+ * hardware conversion, round to nearest even, saturating) and sw[i] = the
+ * same rounding written as comparisons against the grid midpoints. */
+NVFP4_API nvfp4_status nvfp4_test_e2m1(const float* y, int n, uint8_t* hw, uint8_t* sw, void* stream);
+
+/* Counts, over the fp32 bit patterns [first, first + count) that are not
+ * NaN, how many give different hardware and comparison E2M1 codes; adds the
+ * count to *mismatches (device uint64) and records one offending pattern in
+ * *example (device uint32; left unchanged if none). */
+NVFP4_API nvfp4_status nvfp4_test_e2m1_sweep(uint32_t first, uint64_t count, unsigned long long* mismatches,
+                                             uint32_t* example, void* stream);
+
+/* codes[i] = E4M3 code of s[i] >= 0 (nearest even, saturating at 448) and
+ * value[i] = the value of that code. */
+NVFP4_API nvfp4_status nvfp4_test_e4m3(const float* s, int n, uint8_t* codes, float* value, void* stream);
+
+/* out[i] = the router's fp32 sigmoid of l[i]. */
+NVFP4_API nvfp4_status nvfp4_test_sigmoid(const float* l, int n, float* out, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NVFP4_MOE_TESTING_H */

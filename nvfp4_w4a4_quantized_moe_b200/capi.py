@@ -1,0 +1,381 @@
+"""ctypes binding of libnvfp4moe.so (argument marshalling only).
+
+Every function here has the name of the C entry point it calls (see
+``include/nvfp4_moe.h``) and does nothing but check tensor placement, dtypes
+and shapes, allocate outputs and workspace with torch, pass raw device
+pointers and torch's current CUDA stream, and turn a non-OK status into an
+exception.  All arithmetic of the layer runs in the library's CUDA kernels;
+there is no CPU path.  Importing this module loads the library and fails
+loudly when it has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnvfp4moe.so")
+
+LAYOUT_CANONICAL = 0
+LAYOUT_TILED = 1
+_LAYOUTS = {"canonical": LAYOUT_CANONICAL, "tiled": LAYOUT_TILED}
+
+STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED_SHAPE", 3: "CUDA", 4: "TIMEOUT", 5: "WORKSPACE",
+                6: "DEVICE"}
+
+
+class Nvfp4Error(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m nvfp4_w4a4_quantized_moe_b200.build` "
+                      "(the layer has no other implementation)")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+_vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+
+
+class MoeWeightsStruct(ctypes.Structure):
+    _fields_ = [("E", _i), ("H", _i), ("I", _i), ("k", _i), ("routed_scaling_factor", _f),
+                ("router_weight", _vp), ("bias", _vp),
+                ("gate_codes", _vp), ("gate_scales", _vp), ("gate_gscale", _vp),
+                ("up_codes", _vp), ("up_scales", _vp), ("up_gscale", _vp),
+                ("down_codes", _vp), ("down_scales", _vp), ("down_gscale", _vp)]
+
+
+DEBUG_FIELDS = ("logits", "topk_idx", "topk_w", "expert_offsets", "perm", "inv_perm", "a_codes", "a_scales", "h",
+                "h_amax", "h_codes", "h_scales", "y")
+N_STAGE_EVENTS = 6
+
+
+class MoeDebugStruct(ctypes.Structure):
+    _fields_ = [(n, _vp) for n in DEBUG_FIELDS] + [("stage_events", _vp * N_STAGE_EVENTS)]
+
+
+def _declare(name, restype, *argtypes):
+    fn = getattr(lib, name)
+    fn.restype = restype
+    fn.argtypes = list(argtypes)
+    return fn
+
+
+_declare("nvfp4_last_error", ctypes.c_char_p)
+_declare("nvfp4_abi_version", _i)
+_declare("nvfp4_workspace_status", _i, _vp, _vp)
+_declare("nvfp4_quantize_weights_workspace_size", _sz, _i)
+_declare("nvfp4_quantize_weights", _i, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp)
+_declare("nvfp4_quantize_act", _i, _vp, _i, _i, _vp, _i, _vp, _vp, _vp)
+_declare("moe_route_rows_capacity", _i, _i, _i, _i)
+_declare("moe_route_workspace_size", _sz, _i, _i, _i)
+_declare("moe_route", _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
+         _vp)
+_declare("moe_nvfp4_workspace_size", _sz, _i, _i, _i, _i, _i)
+_declare("moe_nvfp4_forward", _i, ctypes.POINTER(MoeWeightsStruct), _vp, _i, _vp, _vp, _vp, _vp,
+         ctypes.POINTER(MoeDebugStruct), _vp, _sz, _vp)
+_declare("moe_nvfp4_gemm_workspace_size", _sz, _i)
+_declare("moe_nvfp4_gate_up", _i, ctypes.POINTER(MoeWeightsStruct), _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp,
+         _vp, _vp, _vp, _sz, _vp)
+_declare("moe_nvfp4_down", _i, ctypes.POINTER(MoeWeightsStruct), _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp,
+         _vp, _sz, _vp)
+
+_declare("nvfp4_test_e2m1", _i, _vp, _i, _vp, _vp, _vp)
+_declare("nvfp4_test_e2m1_sweep", _i, ctypes.c_uint32, ctypes.c_uint64, _vp, _vp, _vp)
+_declare("nvfp4_test_e4m3", _i, _vp, _i, _vp, _vp, _vp)
+_declare("nvfp4_test_sigmoid", _i, _vp, _i, _vp, _vp)
+
+# Every symbol the public headers declare (checked by the CPU test suite).
+EXPORTS = ("nvfp4_last_error", "nvfp4_abi_version", "nvfp4_workspace_status",
+           "nvfp4_quantize_weights_workspace_size", "nvfp4_quantize_weights", "nvfp4_quantize_act",
+           "moe_route_rows_capacity", "moe_route_workspace_size", "moe_route", "moe_nvfp4_workspace_size",
+           "moe_nvfp4_forward", "moe_nvfp4_gemm_workspace_size", "moe_nvfp4_gate_up", "moe_nvfp4_down",
+           "nvfp4_test_e2m1", "nvfp4_test_e2m1_sweep", "nvfp4_test_e4m3", "nvfp4_test_sigmoid")
+
+
+def _check(status: int):
+    if status != 0:
+        raise Nvfp4Error(status, lib.nvfp4_last_error().decode(errors="replace"))
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _cuda(t, dtype, name):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _workspace(nbytes: int, device) -> torch.Tensor:
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def tiled_scale_bytes(rows: int, cols: int) -> int:
+    return (rows + 127) // 128 * 128 * (cols // 16)
+
+
+def abi_version() -> int:
+    return lib.nvfp4_abi_version()
+
+
+def nvfp4_workspace_status(ws: torch.Tensor):
+    """Raises Nvfp4Error(TIMEOUT) if a device-side wait of the call that used
+    ``ws`` gave up; synchronises the current stream."""
+    _check(lib.nvfp4_workspace_status(_p(ws), _stream()))
+
+
+def moe_route_rows_capacity(T: int, E: int, k: int) -> int:
+    return lib.moe_route_rows_capacity(T, E, k)
+
+
+# ---------------------------------------------------------------------------
+# quantisers
+# ---------------------------------------------------------------------------
+
+def nvfp4_quantize_weights(w: torch.Tensor, layout: str = "tiled", workspace: torch.Tensor | None = None):
+    """w [n_mats, rows, cols] bf16 -> (codes [n, rows, cols/2] u8, scales u8, gscale [n] f32)."""
+    _cuda(w, torch.bfloat16, "w")
+    if w.dim() == 2:
+        w = w.unsqueeze(0)
+    n, rows, cols = w.shape
+    lay = _LAYOUTS[layout]
+    codes = torch.empty((n, rows, cols // 2), dtype=torch.uint8, device=w.device)
+    if lay == LAYOUT_TILED:
+        scales = torch.empty(tiled_scale_bytes(n * rows, cols), dtype=torch.uint8, device=w.device)
+    else:
+        scales = torch.empty((n, rows, cols // 16), dtype=torch.uint8, device=w.device)
+    gscale = torch.empty(n, dtype=torch.float32, device=w.device)
+    need = lib.nvfp4_quantize_weights_workspace_size(n)
+    ws = workspace if workspace is not None else _workspace(need, w.device)
+    _check(lib.nvfp4_quantize_weights(_p(w), n, rows, cols, lay, _p(codes), _p(scales), _p(gscale), _p(ws),
+                                      ws.numel(), _stream()))
+    return codes, scales, gscale
+
+
+def nvfp4_quantize_act(x: torch.Tensor, gscale: torch.Tensor, layout: str = "canonical"):
+    """x [rows, cols] bf16 under gscale (one f32 on the device) -> (codes, scales)."""
+    _cuda(x, torch.bfloat16, "x")
+    _cuda(gscale, torch.float32, "gscale")
+    rows, cols = x.shape
+    lay = _LAYOUTS[layout]
+    codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=x.device)
+    if lay == LAYOUT_TILED:
+        scales = torch.empty(tiled_scale_bytes(rows, cols), dtype=torch.uint8, device=x.device)
+    else:
+        scales = torch.empty((rows, cols // 16), dtype=torch.uint8, device=x.device)
+    _check(lib.nvfp4_quantize_act(_p(x), rows, cols, _p(gscale), lay, _p(codes), _p(scales), _stream()))
+    return codes, scales
+
+
+# ---------------------------------------------------------------------------
+# router
+# ---------------------------------------------------------------------------
+
+def moe_route(x, router_weight, bias, k: int, rsf: float, logit_offset=None, logits_in=None):
+    """Router + permutation.  Pass either (x, router_weight) or logits_in."""
+    _cuda(bias, torch.float32, "bias")
+    E = bias.numel()
+    if logits_in is not None:
+        _cuda(logits_in, torch.float32, "logits_in")
+        T, H = logits_in.shape[0], 64
+        dev = logits_in.device
+    else:
+        _cuda(x, torch.bfloat16, "x")
+        _cuda(router_weight, torch.bfloat16, "router_weight")
+        T, H = x.shape
+        dev = x.device
+        if logit_offset is not None:
+            _cuda(logit_offset, torch.float32, "logit_offset")
+    cap = moe_route_rows_capacity(T, E, k)
+    out = {
+        "logits": torch.empty((T, E), dtype=torch.float32, device=dev),
+        "topk_idx": torch.empty((T, k), dtype=torch.int32, device=dev),
+        "topk_w": torch.empty((T, k), dtype=torch.float32, device=dev),
+        "expert_offsets": torch.empty(E + 1, dtype=torch.int32, device=dev),
+        "perm": torch.empty(cap, dtype=torch.int32, device=dev),
+        "inv_perm": torch.empty((T, k), dtype=torch.int32, device=dev),
+    }
+    ws = _workspace(lib.moe_route_workspace_size(T, E, k), dev)
+    _check(lib.moe_route(_p(x) if logits_in is None else None, _p(router_weight) if logits_in is None else None,
+                         _p(logits_in), _p(bias), _p(logit_offset) if logits_in is None else None, T, H, E, k,
+                         float(rsf), _p(out["logits"]), _p(out["topk_idx"]), _p(out["topk_w"]),
+                         _p(out["expert_offsets"]), _p(out["perm"]), _p(out["inv_perm"]), _p(ws), ws.numel(),
+                         _stream()))
+    out["workspace"] = ws
+    return out
+
+
+# ---------------------------------------------------------------------------
+# the layer
+# ---------------------------------------------------------------------------
+
+@dataclass
+class MoeWeights:
+    """Device tensors of one NVFP4 MoE layer (scales in the tiled layout)."""
+    E: int
+    H: int
+    I: int
+    k: int
+    rsf: float
+    router_weight: torch.Tensor      # bf16 [E, H]
+    bias: torch.Tensor               # f32 [E]
+    gate_codes: torch.Tensor         # u8 [E, I, H/2]
+    gate_scales: torch.Tensor
+    gate_gscale: torch.Tensor        # f32 [E]
+    up_codes: torch.Tensor
+    up_scales: torch.Tensor
+    up_gscale: torch.Tensor
+    down_codes: torch.Tensor         # u8 [E, H, I/2]
+    down_scales: torch.Tensor
+    down_gscale: torch.Tensor
+
+    def struct(self) -> MoeWeightsStruct:
+        return MoeWeightsStruct(self.E, self.H, self.I, self.k, float(self.rsf), _p(self.router_weight),
+                                _p(self.bias), _p(self.gate_codes), _p(self.gate_scales), _p(self.gate_gscale),
+                                _p(self.up_codes), _p(self.up_scales), _p(self.up_gscale), _p(self.down_codes),
+                                _p(self.down_scales), _p(self.down_gscale))
+
+    @classmethod
+    def quantize(cls, gate, up, down, router_weight, bias, k: int, rsf: float) -> "MoeWeights":
+        """RTN-quantise bf16 expert weights (gate/up [E, I, H], down [E, H, I])
+        with the library's weight quantiser, tiled scales."""
+        E, I, H = gate.shape
+        gc, gs, gg = nvfp4_quantize_weights(gate, "tiled")
+        uc, us, ug = nvfp4_quantize_weights(up, "tiled")
+        dc, ds, dg = nvfp4_quantize_weights(down, "tiled")
+        return cls(E, H, I, k, rsf, _cuda(router_weight, torch.bfloat16, "router_weight"),
+                   _cuda(bias, torch.float32, "bias"), gc, gs, gg, uc, us, ug, dc, ds, dg)
+
+
+def moe_nvfp4_workspace_size(T: int, E: int, H: int, I: int, k: int) -> int:
+    return lib.moe_nvfp4_workspace_size(T, E, H, I, k)
+
+
+def moe_nvfp4_forward(W: MoeWeights, x: torch.Tensor, act_gscale: torch.Tensor, h_gscale: torch.Tensor,
+                      logit_offset: torch.Tensor | None = None, debug: bool = False,
+                      out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                      stage_events=None):
+    """out [T, H] bf16; with debug=True also a dict of intermediate results.
+    ``stage_events``: optional list of 6 torch.cuda.Event(enable_timing=True)
+    recorded by the library between the stages of the layer."""
+    _cuda(x, torch.bfloat16, "x")
+    _cuda(act_gscale, torch.float32, "act_gscale")
+    _cuda(h_gscale, torch.float32, "h_gscale")
+    T, H = x.shape
+    dev = x.device
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=dev) if out is None else _cuda(out, torch.bfloat16, "out")
+    if workspace is None:
+        workspace = _workspace(moe_nvfp4_workspace_size(T, W.E, W.H, W.I, W.k), dev)
+    dbg_tensors = None
+    dbg_ptr = None
+    if debug:
+        cap = moe_route_rows_capacity(T, W.E, W.k)
+        z = lambda *s, dt=torch.float32: torch.zeros(s, dtype=dt, device=dev)  # noqa: E731
+        dbg_tensors = {
+            "logits": z(T, W.E), "topk_idx": z(T, W.k, dt=torch.int32), "topk_w": z(T, W.k),
+            "expert_offsets": z(W.E + 1, dt=torch.int32), "perm": z(cap, dt=torch.int32),
+            "inv_perm": z(T, W.k, dt=torch.int32), "a_codes": z(cap, W.H // 2, dt=torch.uint8),
+            "a_scales": z(tiled_scale_bytes(cap, W.H), dt=torch.uint8), "h": z(cap, W.I), "h_amax": z(1),
+            "h_codes": z(cap, W.I // 2, dt=torch.uint8), "h_scales": z(tiled_scale_bytes(cap, W.I), dt=torch.uint8),
+            "y": z(cap, W.H),
+        }
+    if debug or stage_events is not None:
+        dbg = MoeDebugStruct()
+        if debug:
+            for n in DEBUG_FIELDS:
+                setattr(dbg, n, dbg_tensors[n].data_ptr())
+        if stage_events is not None:
+            for i, ev in enumerate(stage_events):
+                dbg.stage_events[i] = ev.cuda_event
+        dbg_ptr = ctypes.pointer(dbg)
+    ws_struct = W.struct()
+    _check(lib.moe_nvfp4_forward(ctypes.byref(ws_struct), _p(x), T, _p(act_gscale), _p(h_gscale), _p(logit_offset),
+                                 _p(out), dbg_ptr, _p(workspace), workspace.numel(), _stream()))
+    if debug:
+        dbg_tensors["workspace"] = workspace
+        return out, dbg_tensors
+    return out
+
+
+def moe_nvfp4_gate_up(W: MoeWeights, a_codes, a_scales, expert_offsets, expert_counts, act_gscale, h_gscale,
+                      want_h: bool = True, want_amax: bool = False):
+    """Grouped gate/up GEMM on caller-supplied quantised rows."""
+    rows = a_codes.shape[0]
+    dev = a_codes.device
+    h_codes = torch.empty((rows, W.I // 2), dtype=torch.uint8, device=dev)
+    h_scales = torch.empty(tiled_scale_bytes(rows, W.I), dtype=torch.uint8, device=dev)
+    h = torch.empty((rows, W.I), dtype=torch.float32, device=dev) if want_h else None
+    amax = torch.zeros(1, dtype=torch.float32, device=dev) if want_amax else None
+    ws = _workspace(lib.moe_nvfp4_gemm_workspace_size(rows), dev)
+    st = W.struct()
+    _check(lib.moe_nvfp4_gate_up(ctypes.byref(st), _p(a_codes), _p(a_scales), _p(expert_offsets), _p(expert_counts),
+                                 rows, _p(act_gscale), _p(h_gscale), _p(h_codes), _p(h_scales), _p(h), _p(amax),
+                                 _p(ws), ws.numel(), _stream()))
+    return {"h_codes": h_codes, "h_scales": h_scales, "h": h, "h_amax": amax, "workspace": ws}
+
+
+def moe_nvfp4_down(W: MoeWeights, h_codes, h_scales, expert_offsets, expert_counts, h_gscale, row_weight=None,
+                   out_dtype=torch.float32):
+    """Grouped down GEMM on caller-supplied quantised rows; y [rows, H]."""
+    rows = h_codes.shape[0]
+    dev = h_codes.device
+    y = torch.zeros((rows, W.H), dtype=out_dtype, device=dev)
+    ws = _workspace(lib.moe_nvfp4_gemm_workspace_size(rows), dev)
+    st = W.struct()
+    yb = y if out_dtype == torch.bfloat16 else None
+    yf = y if out_dtype == torch.float32 else None
+    _check(lib.moe_nvfp4_down(ctypes.byref(st), _p(h_codes), _p(h_scales), _p(expert_offsets), _p(expert_counts),
+                              rows, _p(h_gscale), _p(row_weight), _p(yb), _p(yf), _p(ws), ws.numel(), _stream()))
+    return {"y": y, "workspace": ws}
+
+
+# ---------------------------------------------------------------------------
+# test hooks (include/nvfp4_moe_testing.h)
+# ---------------------------------------------------------------------------
+
+def nvfp4_test_e2m1(y: torch.Tensor):
+    """(hardware codes, comparison codes) of fp32 values, one code per byte."""
+    _cuda(y, torch.float32, "y")
+    hw = torch.empty(y.numel(), dtype=torch.uint8, device=y.device)
+    sw = torch.empty_like(hw)
+    _check(lib.nvfp4_test_e2m1(_p(y), y.numel(), _p(hw), _p(sw), _stream()))
+    return hw, sw
+
+
+def nvfp4_test_e2m1_sweep(first: int, count: int, device="cuda"):
+    """(number of disagreeing non-NaN fp32 patterns in [first, first+count), one example or None)."""
+    mism = torch.zeros(1, dtype=torch.int64, device=device)
+    ex = torch.full((1,), 0xFFFFFFFF, dtype=torch.int64, device=device)
+    ex32 = torch.zeros(1, dtype=torch.int32, device=device)
+    _check(lib.nvfp4_test_e2m1_sweep(first, count, _p(mism), _p(ex32), _stream()))
+    n = int(mism.item())
+    return n, (int(ex32.item()) & 0xFFFFFFFF) if n else None
+
+
+def nvfp4_test_e4m3(s: torch.Tensor):
+    _cuda(s, torch.float32, "s")
+    codes = torch.empty(s.numel(), dtype=torch.uint8, device=s.device)
+    val = torch.empty(s.numel(), dtype=torch.float32, device=s.device)
+    _check(lib.nvfp4_test_e4m3(_p(s), s.numel(), _p(codes), _p(val), _stream()))
+    return codes, val
+
+
+def nvfp4_test_sigmoid(l: torch.Tensor):
+    _cuda(l, torch.float32, "l")
+    out = torch.empty_like(l)
+    _check(lib.nvfp4_test_sigmoid(_p(l), l.numel(), _p(out), _stream()))
+    return out

@@ -1,0 +1,275 @@
+// Device helpers shared by the NVFP4 MoE kernels (sm_100a only).
+//
+// NVFP4 element formats follow the "K-EXAONE-152B-A23B-REAP-80E-NVFP4" model
+// card, section "Quantization Setup": FP4 E2M1 values in groups of 16 with an
+// FP8 E4M3 block scale, under an fp32 per-tensor global scale (the
+// double-scale structure of the NetsPresso AQ article, section "The Standard
+// NVFP4 Serving Spec").
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#define NVDEV __device__ __forceinline__
+
+namespace nvfp4moe {
+
+constexpr int kQBlock = 16;          // elements per E4M3 block scale
+constexpr int kRowTile = 128;        // rows per MMA tile and per scale atom
+constexpr int kAtomBytes = 512;      // 128 rows x 4 scales
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s per wait, then give up
+
+// Device status word values (first word of every workspace).
+enum : uint32_t { kDevOk = 0, kDevTimeout = 1 };
+
+NVDEV uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// ---------------------------------------------------------------------------
+// bf16 <-> fp32
+// ---------------------------------------------------------------------------
+NVDEV float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+NVDEV float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+NVDEV void unpack_bf16x8(const uint4& u, float* v) {
+  v[0] = bf16_lo(u.x); v[1] = bf16_hi(u.x); v[2] = bf16_lo(u.y); v[3] = bf16_hi(u.y);
+  v[4] = bf16_lo(u.z); v[5] = bf16_hi(u.z); v[6] = bf16_lo(u.w); v[7] = bf16_hi(u.w);
+}
+// Round two fp32 values to bf16 (nearest, ties to even); `lo` in the low half.
+NVDEV uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// ---------------------------------------------------------------------------
+// FP4 E2M1 and FP8 E4M3 conversions
+// ---------------------------------------------------------------------------
+// Eight fp32 values -> four bytes of packed E2M1 codes, element 2i in the low
+// nibble of byte i.  Hardware conversion: round to nearest even, saturating
+// to +-6, sign kept.
+NVDEV uint32_t e2m1x8_hw(const float* v) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(r)
+      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+  return r;
+}
+
+// The same rounding written as the seven midpoint decisions of the E2M1 grid
+// {0, .5, 1, 1.5, 2, 3, 4, 6}; a midpoint goes to the even code.  Used only to
+// cross-check the hardware conversion.
+NVDEV uint32_t e2m1_sw(float y) {
+  const float a = fabsf(y);
+  uint32_t m = (a > 0.25f) + (a >= 0.75f) + (a > 1.25f) + (a >= 1.75f) +
+               (a > 2.5f) + (a >= 3.5f) + (a > 5.0f);
+  return m | ((__float_as_uint(y) >> 31) << 3);
+}
+
+// Non-negative fp32 -> E4M3 code (nearest, ties to even, saturating at 448).
+NVDEV uint32_t e4m3_code(float s) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(s));
+  return r & 0xFFu;
+}
+// E4M3 code -> its value (exact).
+NVDEV float e4m3_value(uint32_t code) {
+  uint32_t h2;
+  const uint16_t in = (uint16_t)(code & 0xFFu);
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
+  return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+}
+
+// Quantise one 16-element block under global scale g (d = 6 g), one IEEE
+// rounding per step:  s = E4M3(amax / d);  S = s * g;  inv = 1 / S;
+// q_i = E2M1(x_i * inv).  Zero d or S gives scale code 0 and codes +-0.
+// Returns the scale code; writes 8 bytes of packed codes.
+NVDEV uint32_t quant_block16(const float* v, float g, float d, uint2& codes) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const float s_raw = (d == 0.0f) ? 0.0f : __fdiv_rn(amax, d);
+  const uint32_t s = e4m3_code(s_raw);
+  const float S = __fmul_rn(e4m3_value(s), g);
+  const float inv = (S == 0.0f) ? 0.0f : __frcp_rn(S);
+  float y[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) y[i] = __fmul_rn(v[i], inv);
+  codes.x = e2m1x8_hw(y);
+  codes.y = e2m1x8_hw(y + 8);
+  return s;
+}
+
+// Byte offset of (row, 16-element block kb) in the tiled scale layout that the
+// tensor-core MMA reads: 128-row x 4-block atoms of 512 bytes, atoms ordered
+// (row tile, block group) with nblk4 = K / 64 groups per row tile; inside an
+// atom row r sits at (r % 32) * 16 + (r / 32 % 4) * 4.
+NVDEV size_t tiled_scale_offset(int row, int kb, int nblk4) {
+  const size_t atom = (size_t)(row >> 7) * nblk4 + (kb >> 2);
+  return atom * kAtomBytes + (row & 31) * 16 + ((row >> 5) & 3) * 4 + (kb & 3);
+}
+
+// ---------------------------------------------------------------------------
+// Shared memory, mbarriers, TMA
+// ---------------------------------------------------------------------------
+NVDEV uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+NVDEV void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+NVDEV void fence_barrier_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+NVDEV void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+NVDEV void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+NVDEV void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+NVDEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Wait for the phase with the given parity to complete.  Gives up (returns
+// false) after kWaitLimitNs or when *abort is set by another warp.
+NVDEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+  }
+  return true;
+}
+
+NVDEV void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+          "r"(smem_u32(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+NVDEV void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+NVDEV void prefetch_tmap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// tcgen05: tensor memory, MMA, copies
+// ---------------------------------------------------------------------------
+NVDEV void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols));
+}
+NVDEV void tmem_relinquish() { asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;"); }
+NVDEV void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols));
+}
+NVDEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+NVDEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+// Arrive once on `bar` when every earlier tcgen05 async op of this thread is done.
+NVDEV void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+// D[tmem] (+)= (A * sfA) x (B * sfB)^T, FP4 E2M1 operands from shared memory,
+// UE4M3 scales (one per 16 elements) from tensor memory, fp32 accumulate.
+NVDEV void mma_fp4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t sfa_tmem,
+                   uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::
+          "r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem));
+}
+// D[tmem] (+)= A x B^T, bf16 operands, fp32 accumulate.
+NVDEV void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
+}
+// Copy one 512-byte scale atom (32 rows of 16 bytes) from shared memory into
+// 4 tensor-memory columns, replicated into all four 32-lane sub-partitions.
+NVDEV void tc_cp_scale_atom(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc));
+}
+
+// Shared-memory matrix descriptor, K-major operand with 128-byte swizzle:
+// rows of 128 bytes, groups of 8 rows 1024 bytes apart.
+NVDEV uint64_t sdesc_sw128(uint32_t saddr) {
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1 << 16;                    // leading offset (unused when swizzled)
+  d |= (uint64_t)(1024 >> 4) << 32;          // stride offset: 8 rows x 128 B
+  d |= (uint64_t)1 << 46;                    // descriptor version for sm_100
+  d |= (uint64_t)2 << 61;                    // 128-byte swizzle
+  return d;
+}
+// Descriptor of a scale atom: 32 rows of 16 bytes, contiguous, no swizzle.
+NVDEV uint64_t sdesc_scale_atom(uint32_t saddr) {
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)(128 >> 4) << 16;
+  d |= (uint64_t)(128 >> 4) << 32;           // 8 rows x 16 B
+  d |= (uint64_t)1 << 46;
+  return d;
+}
+// Instruction descriptor: kind::mxf4nvf4, E2M1 x E2M1, UE4M3 scales, K-major
+// operands, M x N tile.
+__host__ __device__ constexpr uint32_t idesc_fp4(int M, int N) {
+  return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+// Instruction descriptor: kind::f16 with bf16 operands and fp32 accumulator.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// 32 consecutive fp32 columns of this warp's 32 TMEM lanes (one lane per thread).
+NVDEV void tmem_ld32(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+NVDEV void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+NVDEV uint32_t elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .b32 r;\n\t.reg .pred p;\n\t"
+      "elect.sync r|p, 0xffffffff;\n\t"
+      "selp.b32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred;
+}
+
+}  // namespace nvfp4moe

@@ -1,0 +1,257 @@
+// The NVFP4 W4A4 routed-expert MoE layer, end to end on one stream:
+//   router logits -> top-k -> permutation -> quantise x into permuted rows ->
+//   grouped FP4 GEMM gate/up (+ SiLU*up, requantise) -> grouped FP4 GEMM down
+//   (+ g2 g_down w) -> combine.
+// Sources: "K-EXAONE-152B-A23B-REAP-80E-NVFP4" model card ("Quantization
+// Setup"), "K-EXAONE-152B-A23B-REAP-80E-BF16" model card ("Pruning Setup",
+// "Routing behavior").
+#include "common.cuh"
+#include "gemm.cuh"
+#include "host.cuh"
+#include "route.cuh"
+
+namespace nvfp4moe {
+
+// Quantises token t's row once under g1 and writes it to each of its k
+// permuted rows: packed codes and tiled scales.  One thread per 16-element
+// block; groups of four lanes assemble a 32-bit scale word.
+__global__ void __launch_bounds__(128) quantize_scatter_kernel(const uint4* __restrict__ x, int T, int H,
+                                                               const float* __restrict__ gscale,
+                                                               const int32_t* __restrict__ inv_perm, int k,
+                                                               uint2* __restrict__ a_codes,
+                                                               uint8_t* __restrict__ a_scales) {
+  __shared__ int32_t rows[16];
+  const int t = blockIdx.x;
+  if (threadIdx.x < k) rows[threadIdx.x] = inv_perm[(size_t)t * k + threadIdx.x];
+  __syncthreads();
+  const float g = *gscale;
+  const float d = __fmul_rn(6.0f, g);
+  const int nblk = H / kQBlock;
+  const int lane = threadIdx.x & 31;
+  for (int kb0 = 0; kb0 < nblk; kb0 += blockDim.x) {
+    const int kb = kb0 + threadIdx.x;
+    const bool valid = kb < nblk;
+    uint2 c = make_uint2(0, 0);
+    uint32_t s = 0;
+    if (valid) {
+      float v[16];
+      const uint4* src = x + ((size_t)t * H + (size_t)kb * kQBlock) / 8;
+      unpack_bf16x8(__ldg(src), v);
+      unpack_bf16x8(__ldg(src + 1), v + 8);
+      s = quant_block16(v, g, d, c);
+    }
+    uint32_t w1 = __shfl_down_sync(0xffffffffu, s, 1);
+    uint32_t w2 = __shfl_down_sync(0xffffffffu, s, 2);
+    uint32_t w3 = __shfl_down_sync(0xffffffffu, s, 3);
+    const uint32_t word = s | (w1 << 8) | (w2 << 16) | (w3 << 24);
+    if (valid) {
+      for (int j = 0; j < k; ++j) {
+        const int row = rows[j];
+        a_codes[(size_t)row * nblk + kb] = c;
+        if ((lane & 3) == 0)
+          *reinterpret_cast<uint32_t*>(a_scales + tiled_scale_offset(row, kb, nblk >> 2)) = word;
+      }
+    }
+  }
+}
+
+// Zeroes the padding rows [offsets[e] + counts[e], offsets[e+1]) of expert e:
+// codes and tiled scales, so that padded rows hold exact zeros.
+__global__ void __launch_bounds__(256) zero_padding_rows_kernel(const int32_t* __restrict__ offsets,
+                                                                const int32_t* __restrict__ counts, int H,
+                                                                uint4* __restrict__ a_codes,
+                                                                uint8_t* __restrict__ a_scales) {
+  const int e = blockIdx.x;
+  const int r0 = offsets[e] + counts[e], r1 = offsets[e + 1];
+  const int vec_per_row = H / 32;             // uint4 of codes per row
+  const int nblk = H / kQBlock;
+  for (int i = threadIdx.x; i < (r1 - r0) * vec_per_row; i += blockDim.x) {
+    const int row = r0 + i / vec_per_row;
+    a_codes[(size_t)row * vec_per_row + i % vec_per_row] = make_uint4(0, 0, 0, 0);
+  }
+  for (int i = threadIdx.x; i < (r1 - r0) * (nblk / 4); i += blockDim.x) {
+    const int row = r0 + i / (nblk / 4), kb = (i % (nblk / 4)) * 4;
+    *reinterpret_cast<uint32_t*>(a_scales + tiled_scale_offset(row, kb, nblk >> 2)) = 0;
+  }
+}
+
+// out[t] = bf16( sum_j y[inv_perm[t, j]] ), fp32 sum in slot order.  The
+// routing weight is already folded into y by the down-projection epilogue.
+__global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ inv_perm,
+                                                      int T, int H, int k, uint4* __restrict__ out) {
+  __shared__ int32_t rows[16];
+  const int t = blockIdx.x;
+  if (threadIdx.x < k) rows[threadIdx.x] = inv_perm[(size_t)t * k + threadIdx.x];
+  __syncthreads();
+  const int vpr = H / 8;
+  for (int c = threadIdx.x; c < vpr; c += blockDim.x) {
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int j = 0; j < k; ++j) {
+      float v[8];
+      unpack_bf16x8(__ldg(y + (size_t)rows[j] * vpr + c), v);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc[q] = __fadd_rn(acc[q], v[q]);
+    }
+    out[(size_t)t * vpr + c] = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                                          pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+  }
+}
+
+struct ForwardScratch {
+  RouteScratch route;
+  float* logits;
+  int32_t* topk_idx;
+  float* topk_w;
+  int32_t* offsets;
+  int32_t* perm;
+  int32_t* inv_perm;
+  uint8_t* a_codes;
+  uint8_t* a_scales;
+  uint8_t* h_codes;
+  uint8_t* h_scales;
+  uint16_t* y;
+};
+
+static ForwardScratch carve_forward(Carver& c, int T, int E, int H, int I, int k) {
+  ForwardScratch f;
+  const int cap = route_rows_capacity(T, E, k);
+  f.route = carve_route_scratch(c, T, E, k);
+  f.logits = c.take<float>((size_t)T * E);
+  f.topk_idx = c.take<int32_t>((size_t)T * k);
+  f.topk_w = c.take<float>((size_t)T * k);
+  f.offsets = c.take<int32_t>((size_t)E + 1);
+  f.perm = c.take<int32_t>((size_t)cap);
+  f.inv_perm = c.take<int32_t>((size_t)T * k);
+  f.a_codes = c.take<uint8_t>((size_t)cap * H / 2);
+  f.a_scales = c.take<uint8_t>((size_t)cap * H / 16);
+  f.h_codes = c.take<uint8_t>((size_t)cap * I / 2);
+  f.h_scales = c.take<uint8_t>((size_t)cap * I / 16);
+  f.y = c.take<uint16_t>((size_t)cap * H);
+  return f;
+}
+
+static nvfp4_status mark(const moe_nvfp4_debug* dbg, int i, cudaStream_t s) {
+  if (!dbg || !dbg->stage_events[i]) return NVFP4_OK;
+  return check_cuda(cudaEventRecord(static_cast<cudaEvent_t>(dbg->stage_events[i]), s), "cudaEventRecord");
+}
+
+static nvfp4_status copy_out(void* dst, const void* src, size_t bytes, cudaStream_t s) {
+  if (!dst || bytes == 0) return NVFP4_OK;
+  return check_cuda(cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, s), "copy debug output");
+}
+
+}  // namespace nvfp4moe
+
+using namespace nvfp4moe;
+
+extern "C" size_t moe_nvfp4_workspace_size(int T, int E, int H, int I, int k) {
+  if (T < 0 || E < 0 || H < 0 || I < 0 || k < 0) return 0;
+  Carver c(nullptr);
+  carve_forward(c, T, E, H, I, k);
+  return c.size();
+}
+
+extern "C" nvfp4_status moe_nvfp4_forward(const moe_nvfp4_weights* W, const void* x_bf16, int T,
+                                          const float* act_gscale, const float* h_gscale, const float* logit_offset,
+                                          void* out_bf16, const moe_nvfp4_debug* dbg, void* ws, size_t ws_bytes,
+                                          void* stream) {
+  NV_CHECK(nvfp4moe_check_weights(W));
+  NV_REQUIRE(x_bf16 && act_gscale && h_gscale && out_bf16, NVFP4_ERR_INVALID_ARG,
+             "moe_nvfp4_forward: x, act_gscale, h_gscale and out are required");
+  NV_REQUIRE(W->router_weight && W->bias && W->gate_codes && W->gate_scales && W->gate_gscale && W->up_codes &&
+                 W->up_scales && W->up_gscale && W->down_codes && W->down_scales && W->down_gscale,
+             NVFP4_ERR_INVALID_ARG, "moe_nvfp4_forward: a weight pointer is NULL");
+  NV_REQUIRE(T >= 1, NVFP4_ERR_INVALID_ARG, "moe_nvfp4_forward: T=%d", T);
+  NV_CHECK(check_route_shape(T, W->H, W->E, W->k));
+  NV_REQUIRE(aligned(x_bf16, 16) && aligned(out_bf16, 16) && aligned(W->router_weight, 16) &&
+                 aligned(W->gate_codes, 16) && aligned(W->up_codes, 16) && aligned(W->down_codes, 16) &&
+                 aligned(W->gate_scales, 16) && aligned(W->up_scales, 16) && aligned(W->down_scales, 16),
+             NVFP4_ERR_INVALID_ARG, "moe_nvfp4_forward: tensors need 16-byte alignment");
+  const int E = W->E, H = W->H, I = W->I, k = W->k;
+  const size_t need = moe_nvfp4_workspace_size(T, E, H, I, k);
+  NV_REQUIRE(ws && ws_bytes >= need && aligned(ws, 256), NVFP4_ERR_WORKSPACE,
+             "moe_nvfp4_forward: needs a 256-byte aligned workspace of %zu bytes", need);
+  int sms = 0;
+  NV_CHECK(device_sm_count(&sms));
+  cudaStream_t s = as_stream(stream);
+  Carver c(ws);
+  ForwardScratch f = carve_forward(c, T, E, H, I, k);
+  const int cap = route_rows_capacity(T, E, k);
+
+  NV_CHECK(check_cuda(cudaMemsetAsync(f.route.status, 0, sizeof(uint32_t), s), "clear status word"));
+  NV_CHECK(mark(dbg, 0, s));
+  // 1-3: router, top-k, permutation
+  RouteArgs ra;
+  ra.x = x_bf16;
+  ra.router_weight = W->router_weight;
+  ra.logit_offset = logit_offset;
+  ra.bias = W->bias;
+  ra.T = T; ra.H = H; ra.E = E; ra.k = k; ra.rsf = W->routed_scaling_factor;
+  ra.logits = f.logits;
+  ra.topk_idx = f.topk_idx; ra.topk_w = f.topk_w; ra.expert_offsets = f.offsets;
+  ra.perm = f.perm; ra.inv_perm = f.inv_perm;
+  NV_CHECK(launch_route(ra, f.route, s));
+  NV_CHECK(mark(dbg, 1, s));
+
+  // 4: quantise x once per token into its k permuted rows; zero the padding
+  quantize_scatter_kernel<<<T, 128, 0, s>>>(static_cast<const uint4*>(x_bf16), T, H, act_gscale, f.inv_perm, k,
+                                            reinterpret_cast<uint2*>(f.a_codes), f.a_scales);
+  NV_CHECK(check_launch("quantize_scatter_kernel"));
+  zero_padding_rows_kernel<<<E, 256, 0, s>>>(f.offsets, f.route.counts, H, reinterpret_cast<uint4*>(f.a_codes),
+                                            f.a_scales);
+  NV_CHECK(check_launch("zero_padding_rows_kernel"));
+  NV_CHECK(mark(dbg, 2, s));
+
+  // 5-6: gate/up GEMM with SiLU*up and requantisation
+  GroupedGemmArgs g1;
+  g1.epi = kEpiGateUp;
+  g1.E = E; g1.H = H; g1.I = I;
+  g1.rows_capacity = cap;
+  g1.a_codes = f.a_codes; g1.a_scales = f.a_scales;
+  g1.b0_codes = W->gate_codes; g1.b0_scales = W->gate_scales; g1.b0_gscale = W->gate_gscale;
+  g1.b1_codes = W->up_codes; g1.b1_scales = W->up_scales; g1.b1_gscale = W->up_gscale;
+  g1.act_gscale = act_gscale;
+  g1.tile_expert = f.route.tile_expert; g1.num_mtiles = f.route.num_mtiles;
+  g1.expert_offsets = f.offsets; g1.expert_counts = f.route.counts;
+  g1.h_gscale = h_gscale; g1.h_codes = f.h_codes; g1.h_scales = f.h_scales;
+  g1.h_f32 = dbg ? dbg->h : nullptr;
+  g1.h_amax = dbg ? dbg->h_amax : nullptr;
+  g1.status = f.route.status;
+  NV_CHECK(launch_grouped_gemm(g1, s));
+  NV_CHECK(mark(dbg, 3, s));
+
+  // 7: down GEMM with g2 * g_down * routing weight
+  GroupedGemmArgs g2;
+  g2.epi = kEpiDown;
+  g2.E = E; g2.H = H; g2.I = I;
+  g2.rows_capacity = cap;
+  g2.a_codes = f.h_codes; g2.a_scales = f.h_scales;
+  g2.b0_codes = W->down_codes; g2.b0_scales = W->down_scales; g2.b0_gscale = W->down_gscale;
+  g2.act_gscale = h_gscale;
+  g2.tile_expert = f.route.tile_expert; g2.num_mtiles = f.route.num_mtiles;
+  g2.expert_offsets = f.offsets; g2.expert_counts = f.route.counts;
+  g2.row_w = f.route.row_w; g2.y_bf16 = f.y; g2.y_f32 = dbg ? dbg->y : nullptr;
+  g2.status = f.route.status;
+  NV_CHECK(launch_grouped_gemm(g2, s));
+  NV_CHECK(mark(dbg, 4, s));
+
+  // 8: combine
+  combine_kernel<<<T, 256, 0, s>>>(reinterpret_cast<const uint4*>(f.y), f.inv_perm, T, H, k,
+                                   static_cast<uint4*>(out_bf16));
+  NV_CHECK(check_launch("combine_kernel"));
+  NV_CHECK(mark(dbg, 5, s));
+
+  if (dbg) {
+    NV_CHECK(copy_out(dbg->logits, f.logits, sizeof(float) * (size_t)T * E, s));
+    NV_CHECK(copy_out(dbg->topk_idx, f.topk_idx, sizeof(int32_t) * (size_t)T * k, s));
+    NV_CHECK(copy_out(dbg->topk_w, f.topk_w, sizeof(float) * (size_t)T * k, s));
+    NV_CHECK(copy_out(dbg->expert_offsets, f.offsets, sizeof(int32_t) * (size_t)(E + 1), s));
+    NV_CHECK(copy_out(dbg->perm, f.perm, sizeof(int32_t) * (size_t)cap, s));
+    NV_CHECK(copy_out(dbg->inv_perm, f.inv_perm, sizeof(int32_t) * (size_t)T * k, s));
+    NV_CHECK(copy_out(dbg->a_codes, f.a_codes, (size_t)cap * H / 2, s));
+    NV_CHECK(copy_out(dbg->a_scales, f.a_scales, (size_t)cap * H / 16, s));
+    NV_CHECK(copy_out(dbg->h_codes, f.h_codes, (size_t)cap * I / 2, s));
+    NV_CHECK(copy_out(dbg->h_scales, f.h_scales, (size_t)cap * I / 16, s));
+  }
+  return NVFP4_OK;
+}

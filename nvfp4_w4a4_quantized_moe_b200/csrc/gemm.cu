@@ -1,0 +1,540 @@
+// Grouped block-scaled FP4 GEMMs of the routed experts on the 5th-generation
+// tensor cores (tcgen05, sm_100a).
+//
+// The expert GEMMs of an NVFP4 W4A4 MoE layer ("K-EXAONE-152B-A23B-REAP-80E-
+// NVFP4" model card, "Quantization Setup": E2M1 weights and activations with
+// one E4M3 scale per 16 elements, per-expert Linear granularity; the global
+// times block scale structure of the NetsPresso AQ article, "The Standard
+// NVFP4 Serving Spec").  The block scales are applied inside the MMA
+// (kind::mxf4nvf4, scale_vec::4X); the per-tensor global scales in the
+// epilogue.
+//
+// Tile: 128 permuted rows x 256 weight rows x 256 K elements per stage.
+//   gate/up: the 256 weight rows are 128 gate rows and the same 128 up rows,
+//            so one tile yields 128 columns of h = silu(gate) * up, which the
+//            epilogue re-quantises to NVFP4 (16-column blocks stay in-thread).
+//   down:    256 output columns, scaled by g2 * g_down[e] * w(row).
+// Warp roles (320 threads): warp 0 issues TMA loads, warp 1 owns tensor memory
+// and issues MMAs, warps 2..9 drain the accumulator (warp w reads TMEM lanes
+// 32*(w%4).., columns split in two halves).  The grid is persistent: one CTA
+// per SM walks the (m-tile, n-tile) list, whose length is read on the device.
+// Every wait is bounded in time; a wait that gives up sets the workspace
+// status word and the CTA winds down after its outstanding copies land.
+#include "common.cuh"
+#include "gemm.cuh"
+#include "host.cuh"
+
+namespace nvfp4moe {
+
+constexpr int kBM = 128, kBN = 256;
+constexpr int kBK = 256;                         // K elements per stage
+constexpr int kBKBytes = kBK / 2;                // 128 bytes of packed FP4 per row
+constexpr int kStages = 4;
+constexpr int kABytes = kBM * kBKBytes;          // 16 KiB
+constexpr int kBBytes = kBN * kBKBytes;          // 32 KiB
+constexpr int kSfaBytes = kBM * kBK / kQBlock;   // 2 KiB (4 scale atoms)
+constexpr int kSfbBytes = kBN * kBK / kQBlock;   // 4 KiB (8 scale atoms)
+constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
+constexpr int kSmemBytes = kStages * kStageBytes + 1024;
+constexpr int kThreads = 320;
+constexpr int kEpiWarps = 8;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kAccCol = 0;                  // 256 fp32 accumulator columns
+constexpr uint32_t kSfaCol = 256;                // 4 MMA k-steps x 4 columns
+constexpr uint32_t kSfbCol = 272;                // 4 MMA k-steps x 8 columns
+
+struct GemmParams {
+  const uint8_t* a_sf;
+  const uint8_t* b0_sf;
+  const uint8_t* b1_sf;
+  int K;                // reduction length (elements)
+  int E;                // experts (tile_expert entries are clamped to [0, E))
+  int Nw;               // weight rows per expert in B0 / B1
+  int n_tiles;          // n-tiles per m-tile
+  const int32_t* tile_expert;
+  const int32_t* num_mtiles;
+  const int32_t* expert_offsets;
+  const int32_t* expert_counts;
+  const float* g_act;
+  const float* g_b0;
+  const float* g_b1;
+  const float* g_h;
+  uint8_t* h_codes;
+  uint8_t* h_sf;
+  float* h_f32;
+  float* h_amax;
+  int I;
+  const float* row_w;
+  uint16_t* y_bf16;
+  float* y_f32;
+  int H;
+  uint32_t* status;
+};
+
+NVDEV void give_up(uint32_t* status, volatile int* abort_flag) {
+  *abort_flag = 1;
+  if (status) atomicExch(status, kDevTimeout);
+}
+
+NVDEV float silu(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
+
+template <int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+                            const __grid_constant__ CUtensorMap tmB1, const GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t full_bar[kStages];
+  __shared__ __align__(8) uint64_t empty_bar[kStages];
+  __shared__ __align__(8) uint64_t acc_full_bar;
+  __shared__ __align__(8) uint64_t acc_empty_bar;
+  __shared__ __align__(8) uint64_t drain_bar;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int abort_s;
+  volatile int* abort_flag = &abort_s;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    mbar_init(&acc_full_bar, 1);
+    mbar_init(&acc_empty_bar, kEpiWarps);
+    mbar_init(&drain_bar, 1);
+    abort_s = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB0);
+    if (EPI == kEpiGateUp) prefetch_tmap(&tmB1);
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_s, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_s;
+
+  const int num_tiles = (*p.num_mtiles) * p.n_tiles;
+  const int KT = (p.K + kBK - 1) / kBK;
+  const int nblk4 = p.K / 64;                    // scale atoms per 128-row tile
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t filled = 0, fill_parity = 0;     // per stage: ever filled / parity of last fill
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
+        const int mt = t / p.n_tiles, nt = t % p.n_tiles;
+        const int e = min(max(p.tile_expert[mt], 0), p.E - 1);
+        for (int kt = 0; kt < KT; ++kt) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) {
+            give_up(p.status, abort_flag);
+            ok = false;
+            break;
+          }
+          uint8_t* sA = smem + stage * kStageBytes;
+          uint8_t* sB = sA + kABytes;
+          uint8_t* sSFA = sB + kBBytes;
+          uint8_t* sSFB = sSFA + kSfaBytes;
+          const int katoms = min(4, (p.K - kt * kBK) / 64);
+          const uint32_t sf_bytes = (uint32_t)katoms * kAtomBytes;
+          mbar_arrive_expect_tx(&full_bar[stage], kABytes + kBBytes + 3 * sf_bytes);
+          tma_load_2d(sA, &tmA, kt * kBKBytes, mt * kBM, &full_bar[stage]);
+          bulk_load(sSFA, p.a_sf + ((size_t)mt * nblk4 + kt * 4) * kAtomBytes, sf_bytes, &full_bar[stage]);
+          if (EPI == kEpiGateUp) {
+            const int brow = e * p.Nw + nt * 128;
+            tma_load_2d(sB, &tmB0, kt * kBKBytes, brow, &full_bar[stage]);
+            tma_load_2d(sB + kBBytes / 2, &tmB1, kt * kBKBytes, brow, &full_bar[stage]);
+            const size_t off = ((size_t)(brow / kRowTile) * nblk4 + kt * 4) * kAtomBytes;
+            bulk_load(sSFB, p.b0_sf + off, sf_bytes, &full_bar[stage]);
+            bulk_load(sSFB + kSfbBytes / 2, p.b1_sf + off, sf_bytes, &full_bar[stage]);
+          } else {
+            const int brow = e * p.Nw + nt * kBN;
+            tma_load_2d(sB, &tmB0, kt * kBKBytes, brow, &full_bar[stage]);
+            const size_t off0 = ((size_t)(brow / kRowTile) * nblk4 + kt * 4) * kAtomBytes;
+            const size_t off1 = ((size_t)(brow / kRowTile + 1) * nblk4 + kt * 4) * kAtomBytes;
+            bulk_load(sSFB, p.b0_sf + off0, sf_bytes, &full_bar[stage]);
+            bulk_load(sSFB + kSfbBytes / 2, p.b0_sf + off1, sf_bytes, &full_bar[stage]);
+          }
+          filled |= 1u << stage;
+          fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        // let every copy already issued land before the CTA's shared memory goes away
+        volatile int never = 0;
+        for (int s = 0; s < kStages; ++s)
+          if ((filled >> s) & 1u) mbar_wait(&full_bar[s], (fill_parity >> s) & 1u, &never);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_fp4(kBM, kBN);
+      int stage = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
+        if (!mbar_wait(&acc_empty_bar, acc_phase ^ 1u, abort_flag)) {
+          give_up(p.status, abort_flag);
+          break;
+        }
+        tc_fence_after();
+        for (int kt = 0; kt < KT; ++kt) {
+          if (!mbar_wait(&full_bar[stage], phase, abort_flag)) {
+            give_up(p.status, abort_flag);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sA = smem_u32(smem + stage * kStageBytes);
+          const uint32_t sB = sA + kABytes, sSFA = sB + kBBytes, sSFB = sSFA + kSfaBytes;
+          const int katoms = min(4, (p.K - kt * kBK) / 64);
+          for (int j = 0; j < katoms; ++j) {
+            tc_cp_scale_atom(tmem + kSfaCol + 4 * j, sdesc_scale_atom(sSFA + kAtomBytes * j));
+            tc_cp_scale_atom(tmem + kSfbCol + 8 * j, sdesc_scale_atom(sSFB + kAtomBytes * j));
+            tc_cp_scale_atom(tmem + kSfbCol + 8 * j + 4, sdesc_scale_atom(sSFB + kSfbBytes / 2 + kAtomBytes * j));
+          }
+          const uint64_t adesc = sdesc_sw128(sA), bdesc = sdesc_sw128(sB);
+          for (int j = 0; j < katoms; ++j) {
+            // +32 bytes (64 FP4 values) along K inside the 128-byte swizzle atom
+            mma_fp4(tmem + kAccCol, adesc + 2 * j, bdesc + 2 * j, idesc, tmem + kSfaCol + 4 * j,
+                    tmem + kSfbCol + 8 * j, (kt | j) != 0);
+          }
+          tc_commit(&empty_bar[stage]);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(&acc_full_bar);
+        acc_phase ^= 1u;
+      }
+      // every MMA issued by this thread completes before tensor memory is freed
+      tc_commit(&drain_bar);
+      volatile int never = 0;
+      mbar_wait(&drain_bar, 0, &never);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quad = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int row_in_tile = quad * 32 + lane;
+    const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16);
+    const float g_act = *p.g_act;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+      const int mt = t / p.n_tiles, nt = t % p.n_tiles;
+      const int e = min(max(p.tile_expert[mt], 0), p.E - 1);
+      const int grow = mt * kBM + row_in_tile;
+      const bool real = p.expert_counts ? (grow - p.expert_offsets[e] < p.expert_counts[e]) : true;
+      if (!mbar_wait(&acc_full_bar, acc_phase, abort_flag)) {
+        give_up(p.status, abort_flag);
+        break;
+      }
+      tc_fence_after();
+      if (EPI == kEpiGateUp) {
+        const float sg = __fmul_rn(g_act, p.g_b0[e]);
+        const float su = __fmul_rn(g_act, p.g_b1[e]);
+        float h[64];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t rg[32], ru[32];
+          tmem_ld32(tbase + kAccCol + half * 64 + 32 * c, rg);
+          tmem_ld32(tbase + kAccCol + 128 + half * 64 + 32 * c, ru);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float gate = __fmul_rn(__uint_as_float(rg[i]), sg);
+            const float up = __fmul_rn(__uint_as_float(ru[i]), su);
+            h[32 * c + i] = __fmul_rn(silu(gate), up);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty_bar);
+        const int hcol0 = nt * 128 + half * 64;
+        uint4 cw0 = make_uint4(0, 0, 0, 0), cw1 = make_uint4(0, 0, 0, 0);
+        uint32_t sw = 0;
+        if (real) {
+          const float g2 = *p.g_h;
+          const float d2 = __fmul_rn(6.0f, g2);
+          uint2 c0, c1, c2, c3;
+          const uint32_t s0 = quant_block16(h, g2, d2, c0);
+          const uint32_t s1 = quant_block16(h + 16, g2, d2, c1);
+          const uint32_t s2 = quant_block16(h + 32, g2, d2, c2);
+          const uint32_t s3 = quant_block16(h + 48, g2, d2, c3);
+          cw0 = make_uint4(c0.x, c0.y, c1.x, c1.y);
+          cw1 = make_uint4(c2.x, c2.y, c3.x, c3.y);
+          sw = s0 | (s1 << 8) | (s2 << 16) | (s3 << 24);
+          if (p.h_f32) {
+            float4* dst = reinterpret_cast<float4*>(p.h_f32 + (size_t)grow * p.I + hcol0);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) dst[i] = make_float4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
+          }
+          if (p.h_amax) {
+            float m = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 64; ++i) m = fmaxf(m, fabsf(h[i]));
+            atomicMax(reinterpret_cast<unsigned int*>(p.h_amax), __float_as_uint(m));
+          }
+        }
+        uint4* cdst = reinterpret_cast<uint4*>(p.h_codes + (size_t)grow * (p.I / 2) + hcol0 / 2);
+        cdst[0] = cw0;
+        cdst[1] = cw1;
+        *reinterpret_cast<uint32_t*>(p.h_sf + tiled_scale_offset(grow, hcol0 / kQBlock, p.I / 64)) = sw;
+      } else {
+        const float scale = __fmul_rn(__fmul_rn(g_act, p.g_b0[e]), p.row_w ? p.row_w[grow] : 1.0f);
+        const int col0 = nt * kBN + half * 128;
+        uint32_t packed[64];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tbase + kAccCol + half * 128 + 32 * c, r);
+          tmem_ld_wait();
+          float v[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(__uint_as_float(r[i]), scale);
+          if (p.y_f32 && real) {
+            float4* dst = reinterpret_cast<float4*>(p.y_f32 + (size_t)grow * p.H + col0 + 32 * c);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+          }
+#pragma unroll
+          for (int i = 0; i < 16; ++i) packed[16 * c + i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty_bar);
+        if (p.y_bf16 && real) {
+          uint4* dst = reinterpret_cast<uint4*>(p.y_bf16 + (size_t)grow * p.H + col0);
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+        }
+      }
+      acc_phase ^= 1u;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// Opts a kernel into the large dynamic shared memory once per device.
+static nvfp4_status set_smem_attr(const void* fn, int which) {
+  static bool done[2][64] = {};
+  int dev = 0;
+  NV_CHECK(check_cuda(cudaGetDevice(&dev), "cudaGetDevice"));
+  if (dev < 0 || dev >= 64) dev = 63;
+  if (!done[which][dev]) {
+    NV_CHECK(check_cuda(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes),
+                        "cudaFuncSetAttribute"));
+    done[which][dev] = true;
+  }
+  return NVFP4_OK;
+}
+
+nvfp4_status launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t s) {
+  int sms = 0;
+  NV_CHECK(device_sm_count(&sms));
+  const bool gu = a.epi == kEpiGateUp;
+  const int K = gu ? a.H : a.I;
+  const int Nw = gu ? a.I : a.H;
+  CUtensorMap tmA, tmB0, tmB1;
+  NV_CHECK(make_tmap_2d(&tmA, a.a_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, (uint64_t)K / 2, (uint64_t)a.rows_capacity,
+                        (uint64_t)K / 2, kBKBytes, kBM));
+  NV_CHECK(make_tmap_2d(&tmB0, a.b0_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, (uint64_t)K / 2, (uint64_t)a.E * Nw,
+                        (uint64_t)K / 2, kBKBytes, gu ? 128 : kBN));
+  if (gu) {
+    NV_CHECK(make_tmap_2d(&tmB1, a.b1_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, (uint64_t)K / 2, (uint64_t)a.E * Nw,
+                          (uint64_t)K / 2, kBKBytes, 128));
+  } else {
+    tmB1 = tmB0;
+  }
+  GemmParams p;
+  p.a_sf = a.a_scales;
+  p.b0_sf = a.b0_scales;
+  p.b1_sf = a.b1_scales;
+  p.K = K;
+  p.E = a.E;
+  p.Nw = Nw;
+  p.n_tiles = gu ? a.I / 128 : a.H / kBN;
+  p.tile_expert = a.tile_expert;
+  p.num_mtiles = a.num_mtiles;
+  p.expert_offsets = a.expert_offsets;
+  p.expert_counts = a.expert_counts;
+  p.g_act = a.act_gscale;
+  p.g_b0 = a.b0_gscale;
+  p.g_b1 = a.b1_gscale;
+  p.g_h = a.h_gscale;
+  p.h_codes = a.h_codes;
+  p.h_sf = a.h_scales;
+  p.h_f32 = a.h_f32;
+  p.h_amax = a.h_amax;
+  p.I = a.I;
+  p.row_w = a.row_w;
+  p.y_bf16 = static_cast<uint16_t*>(a.y_bf16);
+  p.y_f32 = a.y_f32;
+  p.H = a.H;
+  p.status = a.status;
+  const int max_tiles = a.rows_capacity / kBM * p.n_tiles;
+  const int grid = std::max(1, std::min(sms, max_tiles));
+  if (gu) {
+    NV_CHECK(set_smem_attr((const void*)grouped_fp4_gemm_kernel<kEpiGateUp>, 0));
+    grouped_fp4_gemm_kernel<kEpiGateUp><<<grid, kThreads, kSmemBytes, s>>>(tmA, tmB0, tmB1, p);
+  } else {
+    NV_CHECK(set_smem_attr((const void*)grouped_fp4_gemm_kernel<kEpiDown>, 1));
+    grouped_fp4_gemm_kernel<kEpiDown><<<grid, kThreads, kSmemBytes, s>>>(tmA, tmB0, tmB1, p);
+  }
+  return check_launch("grouped_fp4_gemm_kernel");
+}
+
+// Builds the m-tile -> expert map from caller-supplied segment offsets,
+// clamped so that every tile stays inside the row capacity.
+__global__ void tiles_from_offsets_kernel(const int32_t* __restrict__ offsets, int E, int cap_tiles,
+                                          int32_t* __restrict__ tile_expert, int32_t* __restrict__ num_mtiles) {
+  for (int m = threadIdx.x; m < cap_tiles; m += blockDim.x) tile_expert[m] = 0;
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const int lo = min(max(offsets[e] / kRowTile, 0), cap_tiles);
+    const int hi = min(max(offsets[e + 1] / kRowTile, lo), cap_tiles);
+    for (int m = lo; m < hi; ++m) tile_expert[m] = e;
+  }
+  if (threadIdx.x == 0) *num_mtiles = min(max(offsets[E] / kRowTile, 0), cap_tiles);
+}
+
+struct GemmScratch {
+  uint32_t* status;
+  int32_t* tile_expert;
+  int32_t* num_mtiles;
+};
+
+static GemmScratch carve_gemm_scratch(Carver& c, int rows_capacity) {
+  GemmScratch g;
+  g.status = c.take<uint32_t>(64);
+  g.tile_expert = c.take<int32_t>((size_t)rows_capacity / kRowTile + 1);
+  g.num_mtiles = c.take<int32_t>(1);
+  return g;
+}
+
+static nvfp4_status check_weights(const moe_nvfp4_weights* W) {
+  NV_REQUIRE(W != nullptr, NVFP4_ERR_INVALID_ARG, "weights struct is NULL");
+  NV_REQUIRE(W->E >= 1 && W->E <= 256 && W->k >= 1 && W->k <= 16 && W->k <= W->E, NVFP4_ERR_UNSUPPORTED_SHAPE,
+             "needs 1 <= k <= 16 and k <= E <= 256 (E=%d k=%d)", W->E, W->k);
+  NV_REQUIRE(W->H > 0 && W->H % 256 == 0, NVFP4_ERR_UNSUPPORTED_SHAPE, "H=%d must be a positive multiple of 256",
+             W->H);
+  NV_REQUIRE(W->I > 0 && W->I % 128 == 0, NVFP4_ERR_UNSUPPORTED_SHAPE, "I=%d must be a positive multiple of 128",
+             W->I);
+  return NVFP4_OK;
+}
+
+}  // namespace nvfp4moe
+
+using namespace nvfp4moe;
+
+nvfp4_status nvfp4moe_check_weights(const moe_nvfp4_weights* W) { return check_weights(W); }
+
+extern "C" size_t moe_nvfp4_gemm_workspace_size(int rows_capacity) {
+  if (rows_capacity < 0) return 0;
+  Carver c(nullptr);
+  carve_gemm_scratch(c, rows_capacity);
+  return c.size();
+}
+
+static nvfp4_status step_common(const moe_nvfp4_weights* W, const int32_t* expert_offsets, int rows_capacity,
+                                void* ws, size_t ws_bytes, const char* name) {
+  NV_CHECK(check_weights(W));
+  NV_REQUIRE(expert_offsets != nullptr, NVFP4_ERR_INVALID_ARG, "%s: expert_offsets is NULL", name);
+  NV_REQUIRE(rows_capacity >= 0 && rows_capacity % 128 == 0, NVFP4_ERR_UNSUPPORTED_SHAPE,
+             "%s: rows_capacity=%d must be a non-negative multiple of 128", name, rows_capacity);
+  const size_t need = moe_nvfp4_gemm_workspace_size(rows_capacity);
+  NV_REQUIRE(ws && ws_bytes >= need && aligned(ws, 256), NVFP4_ERR_WORKSPACE,
+             "%s: needs a 256-byte aligned workspace of %zu bytes", name, need);
+  return NVFP4_OK;
+}
+
+extern "C" nvfp4_status moe_nvfp4_gate_up(const moe_nvfp4_weights* W, const uint8_t* a_codes,
+                                          const uint8_t* a_scales, const int32_t* expert_offsets,
+                                          const int32_t* expert_counts, int rows_capacity, const float* act_gscale,
+                                          const float* h_gscale, uint8_t* h_codes, uint8_t* h_scales, float* h_f32,
+                                          float* h_amax, void* ws, size_t ws_bytes, void* stream) {
+  NV_CHECK(step_common(W, expert_offsets, rows_capacity, ws, ws_bytes, "moe_nvfp4_gate_up"));
+  NV_REQUIRE(a_codes && a_scales && act_gscale && h_gscale && h_codes && h_scales && W->gate_codes &&
+                 W->gate_scales && W->gate_gscale && W->up_codes && W->up_scales && W->up_gscale,
+             NVFP4_ERR_INVALID_ARG, "moe_nvfp4_gate_up: a required pointer is NULL");
+  NV_REQUIRE(aligned(a_codes, 16) && aligned(h_codes, 16) && aligned(a_scales, 16) && aligned(h_scales, 16) &&
+                 aligned(W->gate_codes, 16) && aligned(W->up_codes, 16) && aligned(W->gate_scales, 16) &&
+                 aligned(W->up_scales, 16) && (!h_f32 || aligned(h_f32, 16)),
+             NVFP4_ERR_INVALID_ARG, "moe_nvfp4_gate_up: operands need 16-byte alignment");
+  if (rows_capacity == 0) return NVFP4_OK;
+  cudaStream_t s = as_stream(stream);
+  Carver c(ws);
+  GemmScratch g = carve_gemm_scratch(c, rows_capacity);
+  NV_CHECK(check_cuda(cudaMemsetAsync(g.status, 0, sizeof(uint32_t), s), "clear status word"));
+  tiles_from_offsets_kernel<<<1, 256, 0, s>>>(expert_offsets, W->E, rows_capacity / kRowTile, g.tile_expert,
+                                              g.num_mtiles);
+  NV_CHECK(check_launch("tiles_from_offsets_kernel"));
+  GroupedGemmArgs a;
+  a.epi = kEpiGateUp;
+  a.E = W->E; a.H = W->H; a.I = W->I;
+  a.rows_capacity = rows_capacity;
+  a.a_codes = a_codes; a.a_scales = a_scales;
+  a.b0_codes = W->gate_codes; a.b0_scales = W->gate_scales; a.b0_gscale = W->gate_gscale;
+  a.b1_codes = W->up_codes; a.b1_scales = W->up_scales; a.b1_gscale = W->up_gscale;
+  a.act_gscale = act_gscale;
+  a.tile_expert = g.tile_expert; a.num_mtiles = g.num_mtiles;
+  a.expert_offsets = expert_offsets; a.expert_counts = expert_counts;
+  a.h_gscale = h_gscale; a.h_codes = h_codes; a.h_scales = h_scales; a.h_f32 = h_f32; a.h_amax = h_amax;
+  a.status = g.status;
+  return launch_grouped_gemm(a, s);
+}
+
+extern "C" nvfp4_status moe_nvfp4_down(const moe_nvfp4_weights* W, const uint8_t* h_codes, const uint8_t* h_scales,
+                                       const int32_t* expert_offsets, const int32_t* expert_counts, int rows_capacity,
+                                       const float* h_gscale, const float* row_weight, void* y_bf16, float* y_f32,
+                                       void* ws, size_t ws_bytes, void* stream) {
+  NV_CHECK(step_common(W, expert_offsets, rows_capacity, ws, ws_bytes, "moe_nvfp4_down"));
+  NV_REQUIRE(h_codes && h_scales && h_gscale && W->down_codes && W->down_scales && W->down_gscale,
+             NVFP4_ERR_INVALID_ARG, "moe_nvfp4_down: a required pointer is NULL");
+  NV_REQUIRE((y_bf16 != nullptr) != (y_f32 != nullptr), NVFP4_ERR_INVALID_ARG,
+             "moe_nvfp4_down: pass exactly one of y_bf16 and y_f32");
+  NV_REQUIRE(aligned(h_codes, 16) && aligned(h_scales, 16) && aligned(W->down_codes, 16) &&
+                 aligned(W->down_scales, 16) && (!y_bf16 || aligned(y_bf16, 16)) && (!y_f32 || aligned(y_f32, 16)),
+             NVFP4_ERR_INVALID_ARG, "moe_nvfp4_down: operands need 16-byte alignment");
+  if (rows_capacity == 0) return NVFP4_OK;
+  cudaStream_t s = as_stream(stream);
+  Carver c(ws);
+  GemmScratch g = carve_gemm_scratch(c, rows_capacity);
+  NV_CHECK(check_cuda(cudaMemsetAsync(g.status, 0, sizeof(uint32_t), s), "clear status word"));
+  tiles_from_offsets_kernel<<<1, 256, 0, s>>>(expert_offsets, W->E, rows_capacity / kRowTile, g.tile_expert,
+                                              g.num_mtiles);
+  NV_CHECK(check_launch("tiles_from_offsets_kernel"));
+  GroupedGemmArgs a;
+  a.epi = kEpiDown;
+  a.E = W->E; a.H = W->H; a.I = W->I;
+  a.rows_capacity = rows_capacity;
+  a.a_codes = h_codes; a.a_scales = h_scales;
+  a.b0_codes = W->down_codes; a.b0_scales = W->down_scales; a.b0_gscale = W->down_gscale;
+  a.act_gscale = h_gscale;
+  a.tile_expert = g.tile_expert; a.num_mtiles = g.num_mtiles;
+  a.expert_offsets = expert_offsets; a.expert_counts = expert_counts;
+  a.row_w = row_weight; a.y_bf16 = y_bf16; a.y_f32 = y_f32;
+  a.status = g.status;
+  return launch_grouped_gemm(a, s);
+}

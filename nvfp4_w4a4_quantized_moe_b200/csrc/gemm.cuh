@@ -1,0 +1,51 @@
+// Internal interface of the grouped NVFP4 GEMM (used by the layer).
+#pragma once
+
+#include "host.cuh"
+
+namespace nvfp4moe {
+
+enum GemmEpilogue { kEpiGateUp = 0, kEpiDown = 1 };
+
+// One grouped GEMM over the permuted rows: row tile m (128 rows) belongs to
+// expert tile_expert[m]; m-tiles beyond *num_mtiles are not computed.
+struct GroupedGemmArgs {
+  int epi = kEpiGateUp;
+  int E = 0, H = 0, I = 0;
+  int rows_capacity = 0;
+  // A operand: packed codes [rows][K/2], tiled scales
+  const uint8_t* a_codes = nullptr;
+  const uint8_t* a_scales = nullptr;
+  // B operands (gate and up for kEpiGateUp; down for kEpiDown)
+  const uint8_t* b0_codes = nullptr;
+  const uint8_t* b0_scales = nullptr;
+  const float* b0_gscale = nullptr;
+  const uint8_t* b1_codes = nullptr;
+  const uint8_t* b1_scales = nullptr;
+  const float* b1_gscale = nullptr;
+  const float* act_gscale = nullptr;        // g1 (gate/up) or g2 (down)
+  // row grouping
+  const int32_t* tile_expert = nullptr;
+  const int32_t* num_mtiles = nullptr;
+  const int32_t* expert_offsets = nullptr;
+  const int32_t* expert_counts = nullptr;   // nullable: every row of a segment is data
+  // gate/up outputs
+  const float* h_gscale = nullptr;          // g2
+  uint8_t* h_codes = nullptr;
+  uint8_t* h_scales = nullptr;
+  float* h_f32 = nullptr;
+  float* h_amax = nullptr;
+  // down outputs
+  const float* row_w = nullptr;
+  void* y_bf16 = nullptr;
+  float* y_f32 = nullptr;
+  uint32_t* status = nullptr;
+};
+
+nvfp4_status launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t s);
+
+}  // namespace nvfp4moe
+
+// Host-side shape checks of a weights struct.
+nvfp4_status nvfp4moe_check_weights(const moe_nvfp4_weights* W);
+

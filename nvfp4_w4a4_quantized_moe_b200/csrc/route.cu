@@ -1,0 +1,345 @@
+// Router and permutation ("K-EXAONE-152B-A23B-REAP-80E-BF16" model card,
+// section "Pruning Setup", "Routing behavior": renormalised sigmoid routing,
+// sigmoid-and-bias selection, routed_scaling_factor; the router stays BF16 per
+// the NVFP4 model card's "Quantization Setup").
+#include "common.cuh"
+#include "host.cuh"
+#include "route.cuh"
+#include "route_math.cuh"
+
+namespace nvfp4moe {
+
+// ---------------------------------------------------------------------------
+// Router logits, CUDA cores: a 64-token x 64-expert tile per block, each
+// thread a 4 x 4 register tile, bf16 operands staged through shared memory as
+// fp32, fp32 accumulation in k order.
+// ---------------------------------------------------------------------------
+constexpr int kLT = 64, kLE = 64, kLK = 32;
+
+__global__ void __launch_bounds__(256) router_logits_kernel(const uint16_t* __restrict__ x,
+                                                            const uint16_t* __restrict__ wg, const float* offset,
+                                                            int T, int H, int E, float* __restrict__ logits) {
+  __shared__ float xs[kLT][kLK + 1];
+  __shared__ float ws[kLE][kLK + 1];
+  const int t0 = blockIdx.x * kLT, e0 = blockIdx.y * kLE;
+  const int tid = threadIdx.x;
+  const int tt = (tid >> 4) * 4, ee = tid & 15;
+  float acc[4][4] = {};
+  // loader: 256 threads x 8 bf16 = a 64 x 32 tile
+  const int lr = tid >> 2, lc = (tid & 3) * 8;
+  for (int k0 = 0; k0 < H; k0 += kLK) {
+    {
+      const int t = t0 + lr;
+      uint4 u = make_uint4(0, 0, 0, 0);
+      if (t < T) u = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * H + k0 + lc));
+      float v[8];
+      unpack_bf16x8(u, v);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) xs[lr][lc + q] = v[q];
+      const int e = e0 + lr;
+      u = make_uint4(0, 0, 0, 0);
+      if (e < E) u = __ldg(reinterpret_cast<const uint4*>(wg + (size_t)e * H + k0 + lc));
+      unpack_bf16x8(u, v);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) ws[lr][lc + q] = v[q];
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int k = 0; k < kLK; ++k) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = xs[tt + i][k];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) b[j] = ws[ee + 16 * j][k];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int t = t0 + tt + i;
+    if (t >= T) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e = e0 + ee + 16 * j;
+      if (e < E) logits[(size_t)t * E + e] = offset ? __fadd_rn(acc[i][j], offset[e]) : acc[i][j];
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Top-k: one warp per token.  Lane l holds experts l, l+32, ...; each of the k
+// rounds is a warp-wide argmax of sigma + bias (ties to the lower expert).
+// ---------------------------------------------------------------------------
+constexpr int kMaxE = 256, kMaxK = 16;
+
+__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
+                                                   int T, int E, int k, float rsf, int32_t* __restrict__ topk_idx,
+                                                   float* __restrict__ topk_w) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;
+  float sig[kMaxE / 32], c[kMaxE / 32];
+  const int per = (E + 31) >> 5;
+#pragma unroll
+  for (int i = 0; i < kMaxE / 32; ++i) {
+    const int e = lane + 32 * i;
+    if (i < per && e < E) {
+      sig[i] = sigmoid_fixed(logits[(size_t)t * E + e]);
+      c[i] = __fadd_rn(sig[i], bias[e]);
+    } else {
+      sig[i] = 0.0f;
+      c[i] = -INFINITY;
+    }
+  }
+  uint32_t taken = 0;
+  float sum = 0.0f, my_sig = 0.0f;
+  int my_idx = 0;
+  for (int j = 0; j < k; ++j) {
+    float bc = -INFINITY;
+    int be = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < kMaxE / 32; ++i) {
+      const int e = lane + 32 * i;
+      if (i < per && e < E && !((taken >> i) & 1u) && (c[i] > bc || (c[i] == bc && e < be))) {
+        bc = c[i];
+        be = e;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float oc = __shfl_xor_sync(0xffffffffu, bc, o);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+      if (oc > bc || (oc == bc && oe < be)) {
+        bc = oc;
+        be = oe;
+      }
+    }
+    // the owner lane marks the winner and broadcasts its sigma
+    float s_own = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kMaxE / 32; ++i)
+      if (lane + 32 * i == be) {
+        s_own = sig[i];
+        taken |= 1u << i;
+      }
+    const float s_sel = __shfl_sync(0xffffffffu, s_own, be & 31);
+    sum = __fadd_rn(sum, s_sel);
+    if (lane == j) {
+      my_sig = s_sel;
+      my_idx = be;
+    }
+  }
+  if (lane < k) {
+    topk_idx[(size_t)t * k + lane] = my_idx;
+    topk_w[(size_t)t * k + lane] = __fmul_rn(__fdiv_rn(my_sig, sum), rsf);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Permutation.  Tokens are cut into chunks of 256; inside a chunk a bitmap per
+// expert marks the tokens that chose it, so the rank of (token, expert) among
+// the chunk's tokens is a popcount.  A single-block scan turns per-chunk
+// counts into row bases.  Everything is integer and order-independent.
+// ---------------------------------------------------------------------------
+constexpr int kChunk = 256;
+
+NVDEV void build_bitmap(uint32_t (*bm)[kChunk / 32], const int32_t* topk_idx, int T, int E, int k, int t) {
+  for (int i = threadIdx.x; i < E * (kChunk / 32); i += blockDim.x) bm[i / (kChunk / 32)][i % (kChunk / 32)] = 0;
+  __syncthreads();
+  if (t < T)
+    for (int j = 0; j < k; ++j) atomicOr(&bm[topk_idx[(size_t)t * k + j]][threadIdx.x >> 5], 1u << (threadIdx.x & 31));
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kChunk) perm_count_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
+                                                            int32_t* __restrict__ chunk_counts) {
+  __shared__ uint32_t bm[kMaxE][kChunk / 32];
+  build_bitmap(bm, topk_idx, T, E, k, blockIdx.x * kChunk + threadIdx.x);
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int n = 0;
+#pragma unroll
+    for (int w = 0; w < kChunk / 32; ++w) n += __popc(bm[e][w]);
+    chunk_counts[(size_t)blockIdx.x * E + e] = n;
+  }
+}
+
+// One block of 256 threads (E <= 256): per-expert totals, 128-row padding,
+// exclusive scan into expert_offsets, per-chunk row bases (in place) and the
+// m-tile -> expert map.
+__global__ void __launch_bounds__(256) perm_scan_kernel(int32_t* __restrict__ chunk_counts, int nchunks, int E,
+                                                        int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                                                        int32_t* __restrict__ tile_expert,
+                                                        int32_t* __restrict__ num_mtiles) {
+  __shared__ int32_t sp[256];
+  const int e = threadIdx.x;
+  int total = 0;
+  if (e < E)
+    for (int c = 0; c < nchunks; ++c) total += chunk_counts[(size_t)c * E + e];
+  const int padded = (total + kRowTile - 1) / kRowTile * kRowTile;
+  sp[e] = (e < E) ? padded : 0;
+  __syncthreads();
+  // inclusive scan (Hillis-Steele) over 256 entries
+  for (int o = 1; o < 256; o <<= 1) {
+    const int v = (e >= o) ? sp[e - o] : 0;
+    __syncthreads();
+    sp[e] += v;
+    __syncthreads();
+  }
+  const int start = sp[e] - ((e < E) ? padded : 0);
+  if (e < E) {
+    offsets[e] = start;
+    counts[e] = total;
+    int run = start;
+    for (int c = 0; c < nchunks; ++c) {
+      const int n = chunk_counts[(size_t)c * E + e];
+      chunk_counts[(size_t)c * E + e] = run;
+      run += n;
+    }
+    for (int m = start / kRowTile; m < (start + padded) / kRowTile; ++m) tile_expert[m] = e;
+  }
+  if (e == E - 1) {
+    offsets[E] = start + padded;
+    *num_mtiles = (start + padded) / kRowTile;
+  }
+}
+
+__global__ void __launch_bounds__(kChunk) perm_scatter_kernel(const int32_t* __restrict__ topk_idx,
+                                                              const float* __restrict__ topk_w, int T, int E, int k,
+                                                              const int32_t* __restrict__ chunk_base,
+                                                              int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm,
+                                                              float* __restrict__ row_w) {
+  __shared__ uint32_t bm[kMaxE][kChunk / 32];
+  const int t = blockIdx.x * kChunk + threadIdx.x;
+  build_bitmap(bm, topk_idx, T, E, k, t);
+  if (t >= T) return;
+  const int wi = threadIdx.x >> 5;
+  const uint32_t below = (1u << (threadIdx.x & 31)) - 1u;
+  for (int j = 0; j < k; ++j) {
+    const int e = topk_idx[(size_t)t * k + j];
+    int rank = __popc(bm[e][wi] & below);
+    for (int w = 0; w < wi; ++w) rank += __popc(bm[e][w]);
+    const int row = chunk_base[(size_t)blockIdx.x * E + e] + rank;
+    perm[row] = t;
+    inv_perm[(size_t)t * k + j] = row;
+    if (row_w) row_w[row] = topk_w[(size_t)t * k + j];
+  }
+}
+
+RouteScratch carve_route_scratch(Carver& c, int T, int E, int k) {
+  RouteScratch r;
+  const int nchunks = (T + kChunk - 1) / kChunk;
+  const int cap = route_rows_capacity(T, E, k);
+  r.status = c.take<uint32_t>(64);
+  r.chunk_counts = c.take<int32_t>((size_t)nchunks * E);
+  r.counts = c.take<int32_t>((size_t)E);
+  r.tile_expert = c.take<int32_t>((size_t)cap / kRowTile + 1);
+  r.num_mtiles = c.take<int32_t>(1);
+  r.row_w = c.take<float>((size_t)cap);
+  return r;
+}
+
+int route_rows_capacity(int T, int E, int k) {
+  const long long rows = (long long)T * k + (long long)E * (kRowTile - 1);
+  return (int)((rows + kRowTile - 1) / kRowTile * kRowTile);
+}
+
+nvfp4_status launch_route(const RouteArgs& a, const RouteScratch& r, cudaStream_t s) {
+  const int cap = route_rows_capacity(a.T, a.E, a.k);
+  const int nchunks = (a.T + kChunk - 1) / kChunk;
+  if (a.x) {
+    dim3 grid((a.T + kLT - 1) / kLT, (a.E + kLE - 1) / kLE);
+    router_logits_kernel<<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(a.x),
+                                              static_cast<const uint16_t*>(a.router_weight), a.logit_offset, a.T, a.H,
+                                              a.E, a.logits);
+    NV_CHECK(check_launch("router_logits_kernel"));
+  }
+  NV_CHECK(check_cuda(cudaMemsetAsync(a.perm, 0xFF, sizeof(int32_t) * (size_t)cap, s), "memset perm"));
+  NV_CHECK(check_cuda(cudaMemsetAsync(r.row_w, 0, sizeof(float) * (size_t)cap, s), "memset row_w"));
+  topk_kernel<<<(a.T + 7) / 8, 256, 0, s>>>(a.logits, a.bias, a.T, a.E, a.k, a.rsf, a.topk_idx, a.topk_w);
+  NV_CHECK(check_launch("topk_kernel"));
+  perm_count_kernel<<<nchunks, kChunk, 0, s>>>(a.topk_idx, a.T, a.E, a.k, r.chunk_counts);
+  NV_CHECK(check_launch("perm_count_kernel"));
+  perm_scan_kernel<<<1, 256, 0, s>>>(r.chunk_counts, nchunks, a.E, r.counts, a.expert_offsets, r.tile_expert,
+                                     r.num_mtiles);
+  NV_CHECK(check_launch("perm_scan_kernel"));
+  perm_scatter_kernel<<<nchunks, kChunk, 0, s>>>(a.topk_idx, a.topk_w, a.T, a.E, a.k, r.chunk_counts, a.perm,
+                                                 a.inv_perm, r.row_w);
+  return check_launch("perm_scatter_kernel");
+}
+
+nvfp4_status check_route_shape(int T, int H, int E, int k) {
+  NV_REQUIRE(T >= 1 && E >= 1 && k >= 1, NVFP4_ERR_INVALID_ARG, "route: T=%d E=%d k=%d", T, E, k);
+  NV_REQUIRE(k <= kMaxK && k <= E && E <= kMaxE, NVFP4_ERR_UNSUPPORTED_SHAPE,
+             "route: needs 1 <= k <= 16 and k <= E <= 256 (k=%d E=%d)", k, E);
+  NV_REQUIRE(H % 64 == 0 && H > 0, NVFP4_ERR_UNSUPPORTED_SHAPE, "route: H=%d must be a positive multiple of 64", H);
+  NV_REQUIRE((long long)T * k + (long long)E * 128 < (1ll << 30), NVFP4_ERR_UNSUPPORTED_SHAPE,
+             "route: T*k=%lld too large", (long long)T * k);
+  return NVFP4_OK;
+}
+
+}  // namespace nvfp4moe
+
+using namespace nvfp4moe;
+
+extern "C" int moe_route_rows_capacity(int T, int E, int k) {
+  if (T < 0 || E < 0 || k < 0) return 0;
+  return route_rows_capacity(T, E, k);
+}
+
+extern "C" size_t moe_route_workspace_size(int T, int E, int k) {
+  if (T < 0 || E < 0 || k < 0) return 0;
+  Carver c(nullptr);
+  carve_route_scratch(c, T, E, k);
+  c.take<float>((size_t)T * E);     // logits when the caller does not keep them
+  return c.size();
+}
+
+extern "C" nvfp4_status moe_route(const void* x_bf16, const void* router_weight_bf16, const float* logits_in,
+                                  const float* bias, const float* logit_offset, int T, int H, int E, int k,
+                                  float routed_scaling_factor, float* logits_out, int32_t* topk_idx, float* topk_w,
+                                  int32_t* expert_offsets, int32_t* perm, int32_t* inv_perm, void* ws,
+                                  size_t ws_bytes, void* stream) {
+  NV_REQUIRE(bias && topk_idx && topk_w && expert_offsets && perm && inv_perm, NVFP4_ERR_INVALID_ARG,
+             "moe_route: a required pointer is NULL");
+  if (logits_in) {
+    NV_REQUIRE(!x_bf16 && !router_weight_bf16 && !logit_offset, NVFP4_ERR_INVALID_ARG,
+               "moe_route: with logits_in, x, router weight and logit_offset must be NULL");
+    NV_CHECK(check_route_shape(T, 64, E, k));
+  } else {
+    NV_REQUIRE(x_bf16 && router_weight_bf16, NVFP4_ERR_INVALID_ARG, "moe_route: x and router weight are required");
+    NV_REQUIRE(aligned(x_bf16, 16) && aligned(router_weight_bf16, 16), NVFP4_ERR_INVALID_ARG,
+               "moe_route: x and router weight need 16-byte alignment");
+    NV_CHECK(check_route_shape(T, H, E, k));
+  }
+  const size_t need = moe_route_workspace_size(T, E, k);
+  NV_REQUIRE(ws && ws_bytes >= need && aligned(ws, 256), NVFP4_ERR_WORKSPACE,
+             "moe_route: needs a 256-byte aligned workspace of %zu bytes", need);
+  int sms = 0;
+  NV_CHECK(device_sm_count(&sms));
+  cudaStream_t s = as_stream(stream);
+  Carver c(ws);
+  RouteScratch r = carve_route_scratch(c, T, E, k);
+  float* own_logits = c.take<float>((size_t)T * E);
+  NV_CHECK(check_cuda(cudaMemsetAsync(r.status, 0, sizeof(uint32_t), s), "clear status word"));
+  RouteArgs a;
+  a.x = logits_in ? nullptr : x_bf16;
+  a.router_weight = router_weight_bf16;
+  a.logit_offset = logit_offset;
+  a.bias = bias;
+  a.T = T; a.H = H; a.E = E; a.k = k; a.rsf = routed_scaling_factor;
+  a.topk_idx = topk_idx; a.topk_w = topk_w; a.expert_offsets = expert_offsets; a.perm = perm; a.inv_perm = inv_perm;
+  if (logits_in) {
+    a.logits = const_cast<float*>(logits_in);
+  } else {
+    a.logits = logits_out ? logits_out : own_logits;
+  }
+  NV_CHECK(launch_route(a, r, s));
+  if (logits_in && logits_out)
+    NV_CHECK(check_cuda(cudaMemcpyAsync(logits_out, logits_in, sizeof(float) * (size_t)T * E,
+                                        cudaMemcpyDeviceToDevice, s), "copy logits"));
+  return NVFP4_OK;
+}

@@ -1,0 +1,37 @@
+// Internal interface of the router / permutation kernels (used by the layer).
+#pragma once
+
+#include "host.cuh"
+
+namespace nvfp4moe {
+
+struct RouteArgs {
+  const void* x = nullptr;              // bf16 [T][H]; NULL when logits are given
+  const void* router_weight = nullptr;  // bf16 [E][H]
+  const float* logit_offset = nullptr;  // [E] or NULL
+  const float* bias = nullptr;          // [E]
+  int T = 0, H = 0, E = 0, k = 0;
+  float rsf = 1.0f;
+  float* logits = nullptr;              // [T][E]: written when x is given, read always
+  int32_t* topk_idx = nullptr;
+  float* topk_w = nullptr;
+  int32_t* expert_offsets = nullptr;    // [E+1]
+  int32_t* perm = nullptr;              // [capacity]
+  int32_t* inv_perm = nullptr;          // [T][k]
+};
+
+struct RouteScratch {
+  uint32_t* status = nullptr;           // device status word (start of the workspace)
+  int32_t* chunk_counts = nullptr;      // [chunks][E], then per-chunk row bases
+  int32_t* counts = nullptr;            // [E] rows routed to each expert
+  int32_t* tile_expert = nullptr;       // [capacity / 128] expert of each m-tile
+  int32_t* num_mtiles = nullptr;        // [1]
+  float* row_w = nullptr;               // [capacity] routing weight of each row (0 on padding)
+};
+
+int route_rows_capacity(int T, int E, int k);
+RouteScratch carve_route_scratch(Carver& c, int T, int E, int k);
+nvfp4_status check_route_shape(int T, int H, int E, int k);
+nvfp4_status launch_route(const RouteArgs& a, const RouteScratch& r, cudaStream_t s);
+
+}  // namespace nvfp4moe

@@ -1,0 +1,55 @@
+"""The C ABI library builds for sm_100a, loads, exports what the headers
+declare and rejects bad arguments on the host (CPU only, no kernel launch)."""
+import ctypes
+import subprocess
+
+import pytest
+
+from _util import ROOT, capi, header_functions
+
+
+def test_library_exports_every_declared_function():
+    c = capi()
+    declared = header_functions()
+    assert len(declared) >= 18
+    out = subprocess.run(["nm", "-D", "--defined-only", c.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+    missing = [n for n in declared if n not in exported]
+    assert not missing, missing
+    assert set(c.EXPORTS) == set(declared)
+    for n in declared:
+        assert hasattr(c.lib, n)
+
+
+def test_abi_version_and_sizes():
+    c = capi()
+    assert c.abi_version() == 1
+    assert c.moe_route_rows_capacity(8192, 80, 8) == 75776
+    assert c.moe_route_rows_capacity(16, 80, 8) % 128 == 0
+    assert c.lib.moe_nvfp4_workspace_size(16, 80, 6144, 2048, 8) > 0
+    assert c.lib.nvfp4_quantize_weights_workspace_size(240) >= 256
+
+
+def test_host_side_argument_checks():
+    c = capi()
+    lib = c.lib
+    # NULL pointers: rejected before any CUDA call
+    assert lib.nvfp4_quantize_act(None, 4, 64, None, 0, None, None, None) == 1
+    assert b"NULL" in lib.nvfp4_last_error()
+    fake = ctypes.c_void_p(0x1000)
+    # unsupported shapes and layouts
+    assert lib.nvfp4_quantize_act(fake, 4, 48, fake, 0, fake, fake, None) == 2
+    assert lib.nvfp4_quantize_act(fake, 4, 64, fake, 7, fake, fake, None) == 1
+    assert lib.nvfp4_quantize_weights(fake, 1, 100, 64, 1, fake, fake, fake, fake, 1 << 20, None) == 2
+    # workspace too small
+    assert lib.nvfp4_quantize_weights(fake, 1, 128, 64, 1, fake, fake, fake, fake, 8, None) == 5
+    # routing shapes
+    assert lib.moe_route(fake, fake, None, fake, None, 4, 64, 8, 9, 1.0, None, fake, fake, fake, fake, fake, fake,
+                         1 << 20, None) == 2
+    assert lib.moe_route(fake, fake, None, fake, None, 4, 64, 300, 8, 1.0, None, fake, fake, fake, fake, fake, fake,
+                         1 << 20, None) == 2
+    # layer shapes: H must be a multiple of 256
+    W = c.MoeWeightsStruct(8, 192, 128, 2, 2.5, *([fake] * 11))
+    assert lib.moe_nvfp4_forward(ctypes.byref(W), fake, 4, fake, fake, None, fake, None, fake, 1 << 30, None) == 2
+    W = c.MoeWeightsStruct(8, 256, 128, 2, 2.5, *([fake] * 11))
+    assert lib.moe_nvfp4_forward(ctypes.byref(W), fake, 4, fake, fake, None, fake, None, fake, 16, None) == 5

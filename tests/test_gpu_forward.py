@@ -1,0 +1,109 @@
+"""The whole layer (moe_nvfp4_forward) against the oracle.
+
+Routing is computed on both sides from the same bf16 inputs; the logits
+differ in fp32 summation order only, so a token whose k-th and (k+1)-th
+biased scores are closer than that error may legitimately route differently.
+Those tokens are excluded from the value comparisons (and must be rare)."""
+import numpy as np
+import pytest
+import torch
+
+from _util import capi, host, rel_l2, require_cuda, tiled_rows
+from nvfp4_w4a4_quantized_moe_b200 import workloads
+from oracle import moe, nvfp4
+
+pytestmark = pytest.mark.gpu
+F32 = np.float32
+
+CASES = {
+    "tiny": workloads.CONFIGS["tiny"],
+    "mid_skewed": workloads.LayerConfig("mid", T=300, H=1024, I=512, E=16, k=4, x_outlier_p=0.001,
+                                        logit_offset_std=0.5),
+    "ragged_small": workloads.LayerConfig("rs", T=3, H=512, I=256, E=6, k=3),
+}
+
+
+def _setup(cfg):
+    c = capi()
+    x = workloads.hidden_states(cfg, device="cpu")
+    wg, bias, off = workloads.router_params(cfg, device="cpu")
+    gate, up, down = workloads.stacked_expert_weights(cfg, device="cpu")
+    W = c.MoeWeights.quantize(gate.cuda(), up.cuda(), down.cuda(), wg.cuda(), bias.cuda(), cfg.k, cfg.rsf)
+    q = {e: tuple(nvfp4.quantize_weight(t[e].float().numpy()) for t in (gate, up, down)) for e in range(cfg.E)}
+    return c, x, wg, bias, off, W, q
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_forward_matches_oracle(name):
+    require_cuda()
+    cfg = CASES[name]
+    c, x, wg, bias, off, W, q = _setup(cfg)
+    xf, wf, bf = x.float().numpy(), wg.float().numpy(), bias.numpy()
+    offn = None if off is None else off.numpy()
+    g1 = F32(F32(np.abs(xf).max()) / F32(2688))
+    # calibrate g2 on the oracle's own h (max over every routed pair)
+    cal = moe.moe_layer(xf, wf, bf, cfg.k, cfg.rsf, lambda e: q[e], g1, F32(1.0), logit_offset=offn)
+    g2 = F32(F32(max(np.abs(h).max() for h in cal["h"].values())) / F32(2688))
+    ref = moe.moe_layer(xf, wf, bf, cfg.k, cfg.rsf, lambda e: q[e], g1, g2, logit_offset=offn)
+
+    out, dbg = c.moe_nvfp4_forward(W, x.cuda(), torch.tensor([g1]).cuda(), torch.tensor([g2]).cuda(),
+                                   logit_offset=None if off is None else off.cuda(), debug=True)
+    c.nvfp4_workspace_status(dbg["workspace"])
+
+    # routing: same sets wherever the oracle's selection margin is safe
+    gidx, gw = host(dbg["topk_idx"]), host(dbg["topk_w"])
+    L = ref["logits"].astype(np.float64)
+    sig = moe.sigmoid_f32(ref["logits"]).astype(np.float64)
+    cb = np.sort(sig + bf[None, :], axis=1)[:, ::-1]
+    mag = np.abs(xf.astype(np.float64)) @ np.abs(wf.astype(np.float64)).T
+    safe = (cb[:, cfg.k - 1] - cb[:, cfg.k]) > 0.5 * (1e-5 * mag.max(axis=1) + 1e-6) + 1e-6
+    same = np.all(gidx == ref["topk_idx"], axis=1)
+    assert np.all(same[safe])
+    assert same.mean() >= 0.97
+    assert np.all(np.abs(host(dbg["logits"]) - L) <= 1e-5 * mag + 1e-6)
+    np.testing.assert_allclose(gw[same], ref["topk_w"][same], rtol=2e-5)
+
+    # permutation consistent with the GPU's own selection
+    off_g, perm_g, inv_g = host(dbg["expert_offsets"]), host(dbg["perm"]), host(dbg["inv_perm"])
+    ro, rp, ri = moe.permute(ref["topk_idx"], cfg.E)
+    if np.all(same):
+        np.testing.assert_array_equal(off_g, ro)
+        np.testing.assert_array_equal(perm_g[: rp.size], rp)
+        np.testing.assert_array_equal(inv_g, ri)
+
+    # quantised x in permuted rows: bit-exact
+    ac = host(dbg["a_codes"])
+    asc = host(dbg["a_scales"])
+    for t in range(cfg.T):
+        for j in range(cfg.k):
+            r = inv_g[t, j]
+            np.testing.assert_array_equal(ac[r], ref["a_codes"][t])
+            np.testing.assert_array_equal(tiled_rows(asc, [r], cfg.H)[0], ref["a_scales"][t])
+
+    # h before requantisation, requantised codes, weighted y, and the output
+    h_g, hc_g, y_g = host(dbg["h"]), host(dbg["h_codes"]), host(dbg["y"])
+    hs, hr, flips, total = [], [], 0, 0
+    for t in np.nonzero(same)[0]:
+        for j in range(cfg.k):
+            r = inv_g[t, j]
+            hs.append(h_g[r])
+            hr.append(ref["h"][(t, j)])
+            rc, _ = nvfp4.quantize(ref["h"][(t, j)][None, :], g2)
+            flips += int(np.count_nonzero(nvfp4.unpack_codes(hc_g[r:r + 1]) != nvfp4.unpack_codes(rc)))
+            total += cfg.I
+    assert rel_l2(np.array(hs), np.array(hr)) <= 1e-3
+    assert flips <= 0.001 * total, f"{flips}/{total} requantised codes differ"
+    err = rel_l2(host(out)[same], ref["out"][same])
+    assert err <= 1e-2, err
+
+
+def test_forward_status_word_is_clear_and_repeatable():
+    require_cuda()
+    cfg = CASES["tiny"]
+    c, x, wg, bias, off, W, q = _setup(cfg)
+    g = torch.tensor([0.01]).cuda()
+    ws = torch.empty(c.moe_nvfp4_workspace_size(cfg.T, cfg.E, cfg.H, cfg.I, cfg.k), dtype=torch.uint8, device="cuda")
+    o1 = c.moe_nvfp4_forward(W, x.cuda(), g, g, workspace=ws).clone()
+    o2 = c.moe_nvfp4_forward(W, x.cuda(), g, g, workspace=ws)
+    c.nvfp4_workspace_status(ws)
+    assert torch.equal(o1, o2)        # deterministic: no atomics in the value path
