@@ -36,7 +36,7 @@ from nvfp4_w4a4_quantized_moe_b200 import workloads  # noqa: E402
 METRIC = "MoE-layer tokens/s and TFLOPS (% NVFP4 peak); quantiser GB/s (% HBM) at 1 B200"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP4_OVER_BF16 = 4.0            # nominal dense ratio (9 vs 2.25 PFLOP/s)
-KERNELS_PER_STEP = 10          # router, top-k, 3 permutation, quantise, pad, 2 GEMMs, combine
+KERNELS_PER_STEP = 9           # router GEMM, top-k, 3 permutation, quantise, 2 GEMMs, combine
 NVFP4_BYTES_PER_ELEM = 0.5 + 1.0 / 16
 
 
@@ -46,7 +46,7 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["decode", "prefill", "outlier", "tiny"], default="decode")
+    ap.add_argument("--workload", choices=["decode", "prefill", "outlier", "tiny", "prefill16"], default="decode")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -289,6 +289,10 @@ def run_ours(args, cfg):
         torch.cuda.synchronize()
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(c.N_STAGE_EVENTS)] for _ in range(args.steps)]
+    for row in evs:                 # torch creates the CUDA events lazily, on first record
+        for ev in row:
+            ev.record(stream)
+    torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     dist.barrier()
     torch.cuda.synchronize()

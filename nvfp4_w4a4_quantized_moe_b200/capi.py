@@ -270,8 +270,9 @@ def moe_nvfp4_forward(W: MoeWeights, x: torch.Tensor, act_gscale: torch.Tensor, 
                       out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
                       stage_events=None):
     """out [T, H] bf16; with debug=True also a dict of intermediate results.
-    ``stage_events``: optional list of 6 torch.cuda.Event(enable_timing=True)
-    recorded by the library between the stages of the layer."""
+    ``stage_events``: optional list of 6 torch.cuda.Event(enable_timing=True),
+    each already recorded once (torch creates the CUDA event lazily), which
+    the library records again between the stages of the layer."""
     _cuda(x, torch.bfloat16, "x")
     _cuda(act_gscale, torch.float32, "act_gscale")
     _cuda(h_gscale, torch.float32, "h_gscale")
@@ -300,6 +301,8 @@ def moe_nvfp4_forward(W: MoeWeights, x: torch.Tensor, act_gscale: torch.Tensor, 
                 setattr(dbg, n, dbg_tensors[n].data_ptr())
         if stage_events is not None:
             for i, ev in enumerate(stage_events):
+                if not ev.cuda_event:
+                    raise ValueError("stage_events must have been recorded once (so that the CUDA event exists)")
                 dbg.stage_events[i] = ev.cuda_event
         dbg_ptr = ctypes.pointer(dbg)
     ws_struct = W.struct()

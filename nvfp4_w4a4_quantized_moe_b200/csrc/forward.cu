@@ -55,26 +55,6 @@ __global__ void __launch_bounds__(128) quantize_scatter_kernel(const uint4* __re
   }
 }
 
-// Zeroes the padding rows [offsets[e] + counts[e], offsets[e+1]) of expert e:
-// codes and tiled scales, so that padded rows hold exact zeros.
-__global__ void __launch_bounds__(256) zero_padding_rows_kernel(const int32_t* __restrict__ offsets,
-                                                                const int32_t* __restrict__ counts, int H,
-                                                                uint4* __restrict__ a_codes,
-                                                                uint8_t* __restrict__ a_scales) {
-  const int e = blockIdx.x;
-  const int r0 = offsets[e] + counts[e], r1 = offsets[e + 1];
-  const int vec_per_row = H / 32;             // uint4 of codes per row
-  const int nblk = H / kQBlock;
-  for (int i = threadIdx.x; i < (r1 - r0) * vec_per_row; i += blockDim.x) {
-    const int row = r0 + i / vec_per_row;
-    a_codes[(size_t)row * vec_per_row + i % vec_per_row] = make_uint4(0, 0, 0, 0);
-  }
-  for (int i = threadIdx.x; i < (r1 - r0) * (nblk / 4); i += blockDim.x) {
-    const int row = r0 + i / (nblk / 4), kb = (i % (nblk / 4)) * 4;
-    *reinterpret_cast<uint32_t*>(a_scales + tiled_scale_offset(row, kb, nblk >> 2)) = 0;
-  }
-}
-
 // out[t] = bf16( sum_j y[inv_perm[t, j]] ), fp32 sum in slot order.  The
 // routing weight is already folded into y by the down-projection epilogue.
 __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ inv_perm,
@@ -193,13 +173,12 @@ extern "C" nvfp4_status moe_nvfp4_forward(const moe_nvfp4_weights* W, const void
   NV_CHECK(launch_route(ra, f.route, s));
   NV_CHECK(mark(dbg, 1, s));
 
-  // 4: quantise x once per token into its k permuted rows; zero the padding
+  // 4: quantise x once per token into its k permuted rows.  Padding rows are
+  // left as they are: an MMA row only feeds the same output row, and the
+  // epilogues skip padding rows.
   quantize_scatter_kernel<<<T, 128, 0, s>>>(static_cast<const uint4*>(x_bf16), T, H, act_gscale, f.inv_perm, k,
                                             reinterpret_cast<uint2*>(f.a_codes), f.a_scales);
   NV_CHECK(check_launch("quantize_scatter_kernel"));
-  zero_padding_rows_kernel<<<E, 256, 0, s>>>(f.offsets, f.route.counts, H, reinterpret_cast<uint4*>(f.a_codes),
-                                            f.a_scales);
-  NV_CHECK(check_launch("zero_padding_rows_kernel"));
   NV_CHECK(mark(dbg, 2, s));
 
   // 5-6: gate/up GEMM with SiLU*up and requantisation

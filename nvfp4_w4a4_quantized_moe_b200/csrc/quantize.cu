@@ -84,16 +84,20 @@ __global__ void zero_tiled_scale_rows(uint8_t* scales, int rows, int padded_rows
 }
 
 // ---------------------------------------------------------------------------
-// Weights: a persistent kernel walking a queue of 8192-element chunks.  The
+// Weights: a persistent kernel walking a queue of 32768-element items.  The
 // queue interleaves the amax pass of matrix m+1 with the quantise pass of
-// matrix m, so the second read of a matrix finds it in L2.  A quantise chunk
-// waits (bounded) until every amax chunk of its matrix has finished; those
-// chunks were taken from the queue earlier by running blocks, so the wait
-// always ends.
+// matrix m, so the second read of a matrix finds it in L2 (the first read
+// asks L2 to keep the lines, the second lets them go).  A quantise item waits
+// (bounded) until every amax item of its matrix has finished; those items
+// were taken from the queue earlier by running blocks, so the wait always
+// ends.  Each thread owns 4 x 32 consecutive elements of an item and issues
+// all of its loads before it waits or computes.
 // ---------------------------------------------------------------------------
 constexpr int kWThreads = 256;
 constexpr int kWPerThread = 32;                       // two 16-element blocks
-constexpr int kWChunk = kWThreads * kWPerThread;      // 8192 elements
+constexpr int kWSub = 4;                              // sub-chunks per item
+constexpr int kWSubElems = kWThreads * kWPerThread;   // 8192
+constexpr int kWItem = kWSub * kWSubElems;            // 32768 elements
 
 struct WeightQuantState {
   uint32_t status;          // device status word (first word of the workspace)
@@ -108,6 +112,24 @@ NVDEV uint32_t ld_acquire_u32(const uint32_t* p) {
   return v;
 }
 
+NVDEV uint64_t l2_policy_evict_last() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+NVDEV uint64_t l2_policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+NVDEV uint4 ld_hint(const uint4* p, uint64_t pol) {
+  uint4 v;
+  asm volatile("ld.global.nc.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p), "l"(pol));
+  return v;
+}
+
 __global__ void __launch_bounds__(kWThreads) quantize_weights_kernel(
     const uint4* __restrict__ w, int n_mats, int rows, int cols, int layout, uint2* __restrict__ codes,
     uint8_t* __restrict__ scales, float* __restrict__ gscale, WeightQuantState* st, uint32_t* amax_bits,
@@ -116,10 +138,11 @@ __global__ void __launch_bounds__(kWThreads) quantize_weights_kernel(
   __shared__ uint32_t s_red[kWThreads / 32];
   __shared__ int s_fail;
   const long long per_mat = (long long)rows * cols;
-  const uint32_t chunks = (uint32_t)((per_mat + kWChunk - 1) / kWChunk);
+  const uint32_t chunks = (uint32_t)((per_mat + kWItem - 1) / kWItem);
   const uint32_t total_items = 2u * chunks * (uint32_t)n_mats;
   const int nblk = cols / kQBlock;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint64_t keep = l2_policy_evict_last(), drop = l2_policy_evict_first();
 
   for (;;) {
     if (threadIdx.x == 0) {
@@ -142,21 +165,30 @@ __global__ void __launch_bounds__(kWThreads) quantize_weights_kernel(
         is_amax = false; mat = n_mats - 1; chunk = r;
       }
     }
-    const long long e0 = (long long)chunk * kWChunk + (long long)threadIdx.x * kWPerThread;
-    const bool valid = e0 < per_mat;
-    const uint4* src = w + ((long long)mat * per_mat + e0) / 8;
-    float v[32];
-    if (valid) {
+    // element offsets of this thread's four 32-element runs
+    long long e0[kWSub];
+    bool valid[kWSub];
+    uint4 raw[kWSub][4];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) unpack_bf16x8(__ldg(src + q), v + 8 * q);
-    } else {
+    for (int q = 0; q < kWSub; ++q) {
+      e0[q] = (long long)chunk * kWItem + (long long)q * kWSubElems + (long long)threadIdx.x * kWPerThread;
+      valid[q] = e0[q] < per_mat;
+      const uint4* src = w + ((long long)mat * per_mat + e0[q]) / 8;
 #pragma unroll
-      for (int q = 0; q < 32; ++q) v[q] = 0.0f;
+      for (int i = 0; i < 4; ++i)
+        raw[q][i] = valid[q] ? ld_hint(src + i, is_amax ? keep : drop) : make_uint4(0, 0, 0, 0);
     }
     if (is_amax) {
       float m = 0.0f;
 #pragma unroll
-      for (int q = 0; q < 32; ++q) m = fmaxf(m, fabsf(v[q]));
+      for (int q = 0; q < kWSub; ++q)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          float v[8];
+          unpack_bf16x8(raw[q][i], v);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(v[j]));
+        }
       uint32_t mb = __float_as_uint(m);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, o));
@@ -188,19 +220,24 @@ __global__ void __launch_bounds__(kWThreads) quantize_weights_kernel(
       const float g = __fdiv_rn(amax, 2688.0f);
       const float d = __fmul_rn(6.0f, g);
       if (chunk == 0 && threadIdx.x == 0) gscale[mat] = g;
-      uint32_t s[2] = {0, 0};
-      int row = 0, kb = 0;
-      if (valid) {
-        row = (int)(e0 / cols);
-        kb = (int)((e0 % cols) / kQBlock);
-        uint2 c0, c1;
-        s[0] = quant_block16(v, g, d, c0);
-        s[1] = quant_block16(v + 16, g, d, c1);
-        uint4 cc = make_uint4(c0.x, c0.y, c1.x, c1.y);
-        *reinterpret_cast<uint4*>(codes + ((long long)mat * per_mat + e0) / 16) = cc;
+#pragma unroll
+      for (int q = 0; q < kWSub; ++q) {
+        uint32_t s[2] = {0, 0};
+        int row = 0, kb = 0;
+        if (valid[q]) {
+          float v[32];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) unpack_bf16x8(raw[q][i], v + 8 * i);
+          row = (int)(e0[q] / cols);
+          kb = (int)((e0[q] % cols) / kQBlock);
+          uint2 c0, c1;
+          s[0] = quant_block16(v, g, d, c0);
+          s[1] = quant_block16(v + 16, g, d, c1);
+          *reinterpret_cast<uint4*>(codes + ((long long)mat * per_mat + e0[q]) / 16) =
+              make_uint4(c0.x, c0.y, c1.x, c1.y);
+        }
+        store_scales<2>(scales, layout, mat * rows + row, kb, nblk, s, valid[q]);
       }
-      store_scales<2>(scales, layout, mat * rows + row, kb, nblk,
-                      s, valid);
     }
     __syncthreads();
   }
@@ -264,7 +301,7 @@ extern "C" nvfp4_status nvfp4_quantize_weights(const void* w_bf16, int n_mats, i
   NV_REQUIRE(layout == NVFP4_LAYOUT_CANONICAL || (cols % 64 == 0 && rows % 128 == 0), NVFP4_ERR_UNSUPPORTED_SHAPE,
              "nvfp4_quantize_weights: the tiled layout needs rows %% 128 == 0 and cols %% 64 == 0 (got %d x %d)", rows,
              cols);
-  NV_REQUIRE((long long)rows * cols / 8192 < (1ll << 30) / 2 && (long long)n_mats * 2 * ((long long)rows * cols / 8192 + 1) < (1ll << 32),
+  NV_REQUIRE((long long)n_mats * 2 * ((long long)rows * cols / 32768 + 1) < (1ll << 32),
              NVFP4_ERR_UNSUPPORTED_SHAPE, "nvfp4_quantize_weights: too many elements");
   const size_t need = nvfp4_quantize_weights_workspace_size(n_mats);
   NV_REQUIRE(ws != nullptr && ws_bytes >= need && aligned(ws, 256), NVFP4_ERR_WORKSPACE,

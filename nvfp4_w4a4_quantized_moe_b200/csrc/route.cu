@@ -10,63 +10,169 @@
 namespace nvfp4moe {
 
 // ---------------------------------------------------------------------------
-// Router logits, CUDA cores: a 64-token x 64-expert tile per block, each
-// thread a 4 x 4 register tile, bf16 operands staged through shared memory as
-// fp32, fp32 accumulation in k order.
+// Router logits on the tensor cores: a bf16 x bf16 -> fp32 tcgen05 GEMM.
+// One CTA computes a 128-token tile against all E experts (N = E rounded up
+// to 16) over one slice of H; the slices' partial sums land in
+// partial[split][T][E] and the top-k kernel adds them in split order, so the
+// result does not depend on scheduling.  Warp 0 issues TMA loads (64 bf16 =
+// 128 bytes of K per stage, 128-byte swizzle), warp 1 issues the MMAs from
+// one thread, warps 2..5 read the accumulator out of tensor memory.
 // ---------------------------------------------------------------------------
-constexpr int kLT = 64, kLE = 64, kLK = 32;
+constexpr int kRBM = 128;
+constexpr int kRBK = 64;                      // bf16 elements of K per stage
+constexpr int kRStages = 4;
+constexpr int kRThreads = 192;
+constexpr int kRAbytes = kRBM * kRBK * 2;     // 16 KiB
 
-__global__ void __launch_bounds__(256) router_logits_kernel(const uint16_t* __restrict__ x,
-                                                            const uint16_t* __restrict__ wg, const float* offset,
-                                                            int T, int H, int E, float* __restrict__ logits) {
-  __shared__ float xs[kLT][kLK + 1];
-  __shared__ float ws[kLE][kLK + 1];
-  const int t0 = blockIdx.x * kLT, e0 = blockIdx.y * kLE;
-  const int tid = threadIdx.x;
-  const int tt = (tid >> 4) * 4, ee = tid & 15;
-  float acc[4][4] = {};
-  // loader: 256 threads x 8 bf16 = a 64 x 32 tile
-  const int lr = tid >> 2, lc = (tid & 3) * 8;
-  for (int k0 = 0; k0 < H; k0 += kLK) {
-    {
-      const int t = t0 + lr;
-      uint4 u = make_uint4(0, 0, 0, 0);
-      if (t < T) u = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * H + k0 + lc));
-      float v[8];
-      unpack_bf16x8(u, v);
-#pragma unroll
-      for (int q = 0; q < 8; ++q) xs[lr][lc + q] = v[q];
-      const int e = e0 + lr;
-      u = make_uint4(0, 0, 0, 0);
-      if (e < E) u = __ldg(reinterpret_cast<const uint4*>(wg + (size_t)e * H + k0 + lc));
-      unpack_bf16x8(u, v);
-#pragma unroll
-      for (int q = 0; q < 8; ++q) ws[lr][lc + q] = v[q];
+struct RouterGemmParams {
+  int T, E, H, n_mma, kt_per_split, splits;
+  float* partial;
+  uint32_t* status;
+};
+
+static inline int router_n_mma(int E) { return (E + 15) / 16 * 16; }
+static inline int router_stage_bytes(int E) { return kRAbytes + (router_n_mma(E) * 128 + 1023) / 1024 * 1024; }
+static inline int router_smem_bytes(int E) { return kRStages * router_stage_bytes(E) + 1024; }
+
+// Split count: enough CTAs to cover the SMs of a B200 (148) with at least
+// four K stages each.  A function of the shape only, so results are the same
+// on every device.
+int router_splits(int T, int H) {
+  const int mt = (T + kRBM - 1) / kRBM;
+  const int kt = H / kRBK;
+  int sp = (148 + mt - 1) / mt;
+  sp = std::min(sp, std::max(1, kt / 4));
+  return std::max(1, sp);
+}
+
+__global__ void __launch_bounds__(kRThreads, 1)
+    router_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                       const RouterGemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t full_bar[kRStages];
+  __shared__ __align__(8) uint64_t empty_bar[kRStages];
+  __shared__ __align__(8) uint64_t acc_bar;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int abort_s;
+  volatile int* abort_flag = &abort_s;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int stage_bytes = kRAbytes + (p.n_mma * 128 + 1023) / 1024 * 1024;
+  const uint32_t tcols = p.n_mma <= 32 ? 32 : p.n_mma <= 64 ? 64 : p.n_mma <= 128 ? 128 : 256;
+  const int mt = blockIdx.x;
+  const int KT = p.H / kRBK;
+  const int kt0 = blockIdx.y * p.kt_per_split;
+  const int kt1 = min(kt0 + p.kt_per_split, KT);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kRStages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
     }
-    __syncthreads();
-#pragma unroll 8
-    for (int k = 0; k < kLK; ++k) {
-      float a[4], b[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) a[i] = xs[tt + i][k];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) b[j] = ws[ee + 16 * j][k];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
-    }
-    __syncthreads();
+    mbar_init(&acc_bar, 1);
+    abort_s = 0;
+    fence_barrier_init();
   }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int t = t0 + tt + i;
-    if (t >= T) continue;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int e = e0 + ee + 16 * j;
-      if (e < E) logits[(size_t)t * E + e] = offset ? __fadd_rn(acc[i][j], offset[e]) : acc[i][j];
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmX);
+    prefetch_tmap(&tmW);
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_s, tcols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_s;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, filled = 0, fill_parity = 0;
+      bool ok = true;
+      for (int kt = kt0; kt < kt1; ++kt) {
+        if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) {
+          *abort_flag = 1;
+          atomicExch(p.status, kDevTimeout);
+          ok = false;
+          break;
+        }
+        uint8_t* sA = smem + stage * stage_bytes;
+        mbar_arrive_expect_tx(&full_bar[stage], kRAbytes + p.n_mma * 128);
+        tma_load_2d(sA, &tmX, kt * kRBK, mt * kRBM, &full_bar[stage]);
+        tma_load_2d(sA + kRAbytes, &tmW, kt * kRBK, 0, &full_bar[stage]);
+        filled |= 1u << stage;
+        fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
+        if (++stage == kRStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) {
+        volatile int never = 0;
+        for (int s = 0; s < kRStages; ++s)
+          if ((filled >> s) & 1u) mbar_wait(&full_bar[s], (fill_parity >> s) & 1u, &never);
+      }
     }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16(kRBM, p.n_mma);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int kt = kt0; kt < kt1; ++kt) {
+        if (!mbar_wait(&full_bar[stage], phase, abort_flag)) {
+          *abort_flag = 1;
+          atomicExch(p.status, kDevTimeout);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sA = smem_u32(smem + stage * stage_bytes);
+        const uint64_t adesc = sdesc_sw128(sA), bdesc = sdesc_sw128(sA + kRAbytes);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)      // 16 bf16 = 32 bytes of K per MMA
+          mma_bf16(tmem, adesc + 2 * j, bdesc + 2 * j, idesc, (kt > kt0 || j > 0) ? 1u : 0u);
+        tc_commit(&empty_bar[stage]);
+        if (++stage == kRStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      tc_commit(&acc_bar);
+      if (!ok) {
+        volatile int never = 0;
+        mbar_wait(&acc_bar, 0, &never);
+      }
+    }
+  } else {
+    const int quad = warp & 3;
+    const int row = mt * kRBM + quad * 32 + lane;
+    if (mbar_wait(&acc_bar, 0, abort_flag)) {
+      tc_fence_after();
+      const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16);
+      float* dst = p.partial + ((size_t)blockIdx.y * p.T + row) * p.E;
+      for (int c = 0; c < p.n_mma; c += 32) {
+        uint32_t r[32];
+        tmem_ld32(tbase + c, r);
+        tmem_ld_wait();
+        if (row < p.T) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (c + i < p.E) dst[c + i] = __uint_as_float(r[i]);
+        }
+      }
+    } else {
+      *abort_flag = 1;
+      atomicExch(p.status, kDevTimeout);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, tcols);
   }
 }
 
@@ -76,9 +182,13 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const uint16_t* __re
 // ---------------------------------------------------------------------------
 constexpr int kMaxE = 256, kMaxK = 16;
 
-__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
-                                                   int T, int E, int k, float rsf, int32_t* __restrict__ topk_idx,
-                                                   float* __restrict__ topk_w) {
+// With splits > 0 the logits are the split-ordered sum of the router GEMM's
+// partial sums (plus the optional offset) and are written to `logits`; with
+// splits == 0 `src` already holds the logits.
+__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ src, int splits,
+                                                   const float* __restrict__ offset, float* __restrict__ logits,
+                                                   const float* __restrict__ bias, int T, int E, int k, float rsf,
+                                                   int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;
@@ -88,7 +198,16 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
   for (int i = 0; i < kMaxE / 32; ++i) {
     const int e = lane + 32 * i;
     if (i < per && e < E) {
-      sig[i] = sigmoid_fixed(logits[(size_t)t * E + e]);
+      float l;
+      if (splits > 0) {
+        l = src[(size_t)t * E + e];
+        for (int q = 1; q < splits; ++q) l = __fadd_rn(l, src[((size_t)q * T + t) * E + e]);
+        if (offset) l = __fadd_rn(l, offset[e]);
+        logits[(size_t)t * E + e] = l;
+      } else {
+        l = src[(size_t)t * E + e];
+      }
+      sig[i] = sigmoid_fixed(l);
       c[i] = __fadd_rn(sig[i], bias[e]);
     } else {
       sig[i] = 0.0f;
@@ -239,6 +358,8 @@ RouteScratch carve_route_scratch(Carver& c, int T, int E, int k) {
   r.tile_expert = c.take<int32_t>((size_t)cap / kRowTile + 1);
   r.num_mtiles = c.take<int32_t>(1);
   r.row_w = c.take<float>((size_t)cap);
+  // router_splits() never exceeds ceil(148 / m-tiles), whatever H is
+  r.partial = c.take<float>((size_t)((148 + (T + kRBM - 1) / kRBM - 1) / ((T + kRBM - 1) / kRBM)) * T * E);
   return r;
 }
 
@@ -250,16 +371,32 @@ int route_rows_capacity(int T, int E, int k) {
 nvfp4_status launch_route(const RouteArgs& a, const RouteScratch& r, cudaStream_t s) {
   const int cap = route_rows_capacity(a.T, a.E, a.k);
   const int nchunks = (a.T + kChunk - 1) / kChunk;
+  int splits = 0;
   if (a.x) {
-    dim3 grid((a.T + kLT - 1) / kLT, (a.E + kLE - 1) / kLE);
-    router_logits_kernel<<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(a.x),
-                                              static_cast<const uint16_t*>(a.router_weight), a.logit_offset, a.T, a.H,
-                                              a.E, a.logits);
-    NV_CHECK(check_launch("router_logits_kernel"));
+    splits = router_splits(a.T, a.H);
+    const int n_mma = router_n_mma(a.E);
+    CUtensorMap tmX, tmW;
+    NV_CHECK(make_tmap_2d(&tmX, a.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)a.H, (uint64_t)a.T,
+                          (uint64_t)a.H * 2, kRBK, kRBM));
+    NV_CHECK(make_tmap_2d(&tmW, a.router_weight, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)a.H, (uint64_t)a.E,
+                          (uint64_t)a.H * 2, kRBK, (uint32_t)n_mma));
+    RouterGemmParams p;
+    p.T = a.T; p.E = a.E; p.H = a.H; p.n_mma = n_mma;
+    p.kt_per_split = (a.H / kRBK + splits - 1) / splits;
+    p.splits = splits;
+    p.partial = r.partial;
+    p.status = r.status;
+    const int smem = router_smem_bytes(a.E);
+    NV_CHECK(check_cuda(cudaFuncSetAttribute(router_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
+                        "cudaFuncSetAttribute"));
+    dim3 grid((a.T + kRBM - 1) / kRBM, splits);
+    router_gemm_kernel<<<grid, kRThreads, smem, s>>>(tmX, tmW, p);
+    NV_CHECK(check_launch("router_gemm_kernel"));
   }
   NV_CHECK(check_cuda(cudaMemsetAsync(a.perm, 0xFF, sizeof(int32_t) * (size_t)cap, s), "memset perm"));
   NV_CHECK(check_cuda(cudaMemsetAsync(r.row_w, 0, sizeof(float) * (size_t)cap, s), "memset row_w"));
-  topk_kernel<<<(a.T + 7) / 8, 256, 0, s>>>(a.logits, a.bias, a.T, a.E, a.k, a.rsf, a.topk_idx, a.topk_w);
+  topk_kernel<<<(a.T + 7) / 8, 256, 0, s>>>(splits ? r.partial : a.logits, splits, a.logit_offset, a.logits, a.bias,
+                                            a.T, a.E, a.k, a.rsf, a.topk_idx, a.topk_w);
   NV_CHECK(check_launch("topk_kernel"));
   perm_count_kernel<<<nchunks, kChunk, 0, s>>>(a.topk_idx, a.T, a.E, a.k, r.chunk_counts);
   NV_CHECK(check_launch("perm_count_kernel"));

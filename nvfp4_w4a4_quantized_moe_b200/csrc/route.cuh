@@ -27,6 +27,7 @@ struct RouteScratch {
   int32_t* tile_expert = nullptr;       // [capacity / 128] expert of each m-tile
   int32_t* num_mtiles = nullptr;        // [1]
   float* row_w = nullptr;               // [capacity] routing weight of each row (0 on padding)
+  float* partial = nullptr;             // [splits][T][E] router GEMM partial sums
 };
 
 int route_rows_capacity(int T, int E, int k);

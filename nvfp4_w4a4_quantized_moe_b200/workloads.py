@@ -62,6 +62,9 @@ CONFIGS = {
     # 128 experts with 1% weight outliers, 4096 tokens
     "outlier": LayerConfig("outlier", T=4096, H=6144, I=2048, E=128, k=8,
                            w_outlier_p=0.01, gen_device="cuda"),
+    # a prefill-shaped layer small enough for profiler captures (16 experts)
+    "prefill16": LayerConfig("prefill16", T=2048, H=6144, I=2048, E=16, k=8,
+                             x_outlier_p=0.001, logit_offset_std=0.5, gen_device="cuda"),
     # offline weight quantiser over one 80-expert layer (weights only)
     "quantiser": LayerConfig("quantiser", T=0, H=6144, I=2048, E=80, k=8,
                              gen_device="cuda"),
