@@ -49,6 +49,8 @@ def parse_args():
     ap.add_argument("--workload", choices=["decode", "prefill", "outlier", "tiny", "prefill16"], default="decode")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--mma-peak", action="store_true",
+                    help="measure the FP4 tensor-core rate with no memory traffic and exit")
     return ap.parse_args()
 
 
@@ -422,8 +424,27 @@ def run_ours(args, cfg):
     return 0
 
 
+def run_mma_peak():
+    """FP4 MMA rate per SM clock with operands resident in shared memory."""
+    from nvfp4_w4a4_quantized_moe_b200 import capi as c
+    res = {}
+    for n in (256, 128):
+        for cp in (False, True):
+            c.nvfp4_test_mma_peak(200, n, cp)                      # warm-up
+            fpc, cyc = c.nvfp4_test_mma_peak(20000, n, cp)
+            res[f"n{n}{'_with_scale_copies' if cp else ''}"] = {
+                "flop_per_sm_clock": float(fpc.median()), "cycles_median": float(cyc.median())}
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    best = max(v["flop_per_sm_clock"] for v in res.values())
+    print(json.dumps({"mma_peak": res, "sms": sms,
+                      "pflops_at_1965mhz": best * sms * 1.965e9 / 1e15}), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
+    if args.mma_peak:
+        return run_mma_peak()
     cfg = workloads.CONFIGS[args.workload]
     if args.impl == "reference":
         return run_reference(args, cfg)

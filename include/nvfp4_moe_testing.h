@@ -35,6 +35,15 @@ NVFP4_API nvfp4_status nvfp4_test_e2m1_sweep(uint32_t first, uint64_t count, uns
  * value[i] = the value of that code. */
 NVFP4_API nvfp4_status nvfp4_test_e4m3(const float* s, int n, uint8_t* codes, float* value, void* stream);
 
+/* FP4 tensor-core rate without memory traffic: `ctas` CTAs (at most one per
+ * SM) each issue `iters` x 4 block-scaled 128 x n x 64 MMAs (n = 128 or 256)
+ * from fixed shared-memory operands, with (with_cp != 0) or without the 12
+ * scale-factor copies of a 256-wide K stage before every 4 MMAs.
+ * cycles[c] (device uint64) = SM clock cycles CTA c spent; *status (device
+ * uint32) is set non-zero if the final wait gave up. */
+NVFP4_API nvfp4_status nvfp4_test_mma_peak(int iters, int n, int with_cp, int ctas, unsigned long long* cycles,
+                                           uint32_t* status, void* stream);
+
 /* out[i] = the router's fp32 sigmoid of l[i]. */
 NVFP4_API nvfp4_status nvfp4_test_sigmoid(const float* l, int n, float* out, void* stream);
 

@@ -88,13 +88,15 @@ _declare("nvfp4_test_e2m1", _i, _vp, _i, _vp, _vp, _vp)
 _declare("nvfp4_test_e2m1_sweep", _i, ctypes.c_uint32, ctypes.c_uint64, _vp, _vp, _vp)
 _declare("nvfp4_test_e4m3", _i, _vp, _i, _vp, _vp, _vp)
 _declare("nvfp4_test_sigmoid", _i, _vp, _i, _vp, _vp)
+_declare("nvfp4_test_mma_peak", _i, _i, _i, _i, _i, _vp, _vp, _vp)
 
 # Every symbol the public headers declare (checked by the CPU test suite).
 EXPORTS = ("nvfp4_last_error", "nvfp4_abi_version", "nvfp4_workspace_status",
            "nvfp4_quantize_weights_workspace_size", "nvfp4_quantize_weights", "nvfp4_quantize_act",
            "moe_route_rows_capacity", "moe_route_workspace_size", "moe_route", "moe_nvfp4_workspace_size",
            "moe_nvfp4_forward", "moe_nvfp4_gemm_workspace_size", "moe_nvfp4_gate_up", "moe_nvfp4_down",
-           "nvfp4_test_e2m1", "nvfp4_test_e2m1_sweep", "nvfp4_test_e4m3", "nvfp4_test_sigmoid")
+           "nvfp4_test_e2m1", "nvfp4_test_e2m1_sweep", "nvfp4_test_e4m3", "nvfp4_test_sigmoid",
+           "nvfp4_test_mma_peak")
 
 
 def _check(status: int):
@@ -382,3 +384,17 @@ def nvfp4_test_sigmoid(l: torch.Tensor):
     out = torch.empty_like(l)
     _check(lib.nvfp4_test_sigmoid(_p(l), l.numel(), _p(out), _stream()))
     return out
+
+
+def nvfp4_test_mma_peak(iters: int, n: int = 256, with_cp: bool = False, ctas: int | None = None):
+    """(FLOP per SM clock per CTA, cycles per CTA) of back-to-back FP4 MMAs."""
+    ctas = ctas or torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    cycles = torch.zeros(ctas, dtype=torch.int64, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    _check(lib.nvfp4_test_mma_peak(iters, n, int(with_cp), ctas, _p(cycles), _p(status), _stream()))
+    torch.cuda.synchronize()
+    if int(status.item()) != 0:
+        raise Nvfp4Error(4, "mma peak kernel: the completion wait gave up")
+    cyc = cycles.cpu().double()
+    flops = iters * 4 * 2.0 * 128 * n * 64
+    return flops / cyc, cyc

@@ -66,9 +66,80 @@ __global__ void test_sigmoid_kernel(const float* l, int n, float* out) {
   if (i < n) out[i] = sigmoid_fixed(l[i]);
 }
 
+// FP4 tensor-core rate without memory traffic: one thread per CTA issues
+// `iters` groups of four 128 x N x 64 block-scaled MMAs on fixed shared-memory
+// operands (zeros), optionally preceded by the 12 scale-factor copies a
+// 256-wide K stage needs, then waits for completion.  Cycles are the CTA's
+// clock64 span.
+__global__ void __launch_bounds__(128, 1) mma_peak_kernel(int iters, int n, int with_cp,
+                                                          unsigned long long* cycles, uint32_t* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ uint32_t tmem_s;
+  __shared__ int abort_s;
+  const int warp = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < (16384 + 32768 + 6144) / 16; i += blockDim.x)
+    reinterpret_cast<uint4*>(smem)[i] = make_uint4(0, 0, 0, 0);
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_s = 0;
+    fence_barrier_init();
+  }
+  fence_proxy_async();
+  if (warp == 0) {
+    tmem_alloc(&tmem_s, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_s;
+  if (threadIdx.x == 32) {
+    const uint32_t sA = smem_u32(smem), sB = sA + 16384, sSF = sB + 32768;
+    const uint64_t adesc = sdesc_sw128(sA), bdesc = sdesc_sw128(sB);
+    const uint32_t idesc = idesc_fp4(128, n);
+    const unsigned long long t0 = clock64();
+    for (int it = 0; it < iters; ++it) {
+      if (with_cp) {
+        for (int j = 0; j < 4; ++j) {
+          tc_cp_scale_atom(tmem + 256 + 4 * j, sdesc_scale_atom(sSF + 512 * j));
+          tc_cp_scale_atom(tmem + 272 + 8 * j, sdesc_scale_atom(sSF + 2048 + 512 * j));
+          tc_cp_scale_atom(tmem + 276 + 8 * j, sdesc_scale_atom(sSF + 4096 + 512 * j));
+        }
+      }
+      for (int j = 0; j < 4; ++j)
+        mma_fp4(tmem, adesc + 2 * j, bdesc + 2 * j, idesc, tmem + 256 + 4 * j, tmem + 272 + 8 * j, (it | j) != 0);
+    }
+    tc_commit(&bar);
+    if (!mbar_wait(&bar, 0, &abort_s)) atomicExch(status, kDevTimeout);
+    const unsigned long long t1 = clock64();
+    cycles[blockIdx.x] = t1 - t0;
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 }  // namespace nvfp4moe
 
 using namespace nvfp4moe;
+
+extern "C" nvfp4_status nvfp4_test_mma_peak(int iters, int n, int with_cp, int ctas, unsigned long long* cycles,
+                                            uint32_t* status, void* stream) {
+  NV_REQUIRE(cycles && status && iters > 0 && ctas > 0 && (n == 128 || n == 256), NVFP4_ERR_INVALID_ARG,
+             "nvfp4_test_mma_peak: bad arguments");
+  int sms = 0;
+  NV_CHECK(device_sm_count(&sms));
+  const int smem = 16384 + 32768 + 6144 + 1024;
+  NV_CHECK(check_cuda(cudaFuncSetAttribute(mma_peak_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
+                      "cudaFuncSetAttribute"));
+  mma_peak_kernel<<<ctas, 128, smem, as_stream(stream)>>>(iters, n, with_cp, cycles, status);
+  return check_launch("mma_peak_kernel");
+}
 
 extern "C" nvfp4_status nvfp4_test_e2m1(const float* y, int n, uint8_t* hw, uint8_t* sw, void* stream) {
   NV_REQUIRE(y && hw && sw && n >= 0, NVFP4_ERR_INVALID_ARG, "nvfp4_test_e2m1: bad arguments");
