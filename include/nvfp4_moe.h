@@ -101,6 +101,28 @@ NVFP4_API nvfp4_status nvfp4_quantize_weights(const void* w_bf16, int n_mats, in
                                     uint8_t* codes, uint8_t* scales, float* global_scale, void* ws,
                                     size_t ws_bytes, void* stream);
 
+/* Same quantiser, for callers that cannot allocate device memory.  The pages
+ * have no counterpart to this entry point; it exists for hosts whose device
+ * memory is owned by another allocator (a serving engine's arena, a plugin
+ * host's fixed pool) so that they cannot provide the workspace above, or that
+ * run where device allocation calls are not allowed.  It takes no workspace
+ * and allocates nothing: its scratch is a 8448-byte array inside the library,
+ * which every GPU that loads the library keeps until the process exits.
+ *   - At most 1024 matrices per call; more returns
+ *     NVFP4_ERR_UNSUPPORTED_SHAPE (split the call or use the workspace form).
+ *   - The first call on a device looks up the array's device address (once,
+ *     with that device current); make that first call before any stream
+ *     capture on the device.
+ *   - Every call shares the one array and clears it when it starts, so calls
+ *     whose work overlaps on the GPU (different streams, or different host
+ *     threads on one device) race; serialise them on one stream.
+ *   - A device-side wait that gives up leaves no status word to read: the
+ *     outputs are then undefined, as with the workspace form.
+ * Arguments, layouts and results are those of nvfp4_quantize_weights. */
+NVFP4_API nvfp4_status nvfp4_quantize_weights_noalloc(const void* w_bf16, int n_mats, int rows, int cols,
+                                                      int layout, uint8_t* codes, uint8_t* scales,
+                                                      float* global_scale, void* stream);
+
 /* ------------------------------------------------------------------------
  * Dynamic activation quantiser ("Quantization Setup": activations dynamically
  * quantised to FP4 with calibrated global scales).

@@ -70,6 +70,7 @@ _declare("nvfp4_abi_version", _i)
 _declare("nvfp4_workspace_status", _i, _vp, _vp)
 _declare("nvfp4_quantize_weights_workspace_size", _sz, _i)
 _declare("nvfp4_quantize_weights", _i, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp)
+_declare("nvfp4_quantize_weights_noalloc", _i, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp)
 _declare("nvfp4_quantize_act", _i, _vp, _i, _i, _vp, _i, _vp, _vp, _vp)
 _declare("moe_route_rows_capacity", _i, _i, _i, _i)
 _declare("moe_route_workspace_size", _sz, _i, _i, _i)
@@ -92,7 +93,8 @@ _declare("nvfp4_test_mma_peak", _i, _i, _i, _i, _i, _vp, _vp, _vp)
 
 # Every symbol the public headers declare (checked by the CPU test suite).
 EXPORTS = ("nvfp4_last_error", "nvfp4_abi_version", "nvfp4_workspace_status",
-           "nvfp4_quantize_weights_workspace_size", "nvfp4_quantize_weights", "nvfp4_quantize_act",
+           "nvfp4_quantize_weights_workspace_size", "nvfp4_quantize_weights", "nvfp4_quantize_weights_noalloc",
+           "nvfp4_quantize_act",
            "moe_route_rows_capacity", "moe_route_workspace_size", "moe_route", "moe_nvfp4_workspace_size",
            "moe_nvfp4_forward", "moe_nvfp4_gemm_workspace_size", "moe_nvfp4_gate_up", "moe_nvfp4_down",
            "nvfp4_test_e2m1", "nvfp4_test_e2m1_sweep", "nvfp4_test_e4m3", "nvfp4_test_sigmoid",
@@ -165,6 +167,27 @@ def nvfp4_quantize_weights(w: torch.Tensor, layout: str = "tiled", workspace: to
     ws = workspace if workspace is not None else _workspace(need, w.device)
     _check(lib.nvfp4_quantize_weights(_p(w), n, rows, cols, lay, _p(codes), _p(scales), _p(gscale), _p(ws),
                                       ws.numel(), _stream()))
+    return codes, scales, gscale
+
+
+def nvfp4_quantize_weights_noalloc(w: torch.Tensor, layout: str = "tiled", out=None):
+    """The weight quantiser without a workspace (its scratch is built into the
+    library).  ``out`` = (codes, scales, gscale) to write into; allocated here
+    with torch when None (the library itself allocates nothing)."""
+    _cuda(w, torch.bfloat16, "w")
+    if w.dim() == 2:
+        w = w.unsqueeze(0)
+    n, rows, cols = w.shape
+    lay = _LAYOUTS[layout]
+    if out is None:
+        codes = torch.empty((n, rows, cols // 2), dtype=torch.uint8, device=w.device)
+        scales = (torch.empty(tiled_scale_bytes(n * rows, cols), dtype=torch.uint8, device=w.device)
+                  if lay == LAYOUT_TILED else torch.empty((n, rows, cols // 16), dtype=torch.uint8, device=w.device))
+        gscale = torch.empty(n, dtype=torch.float32, device=w.device)
+    else:
+        codes, scales, gscale = out
+    _check(lib.nvfp4_quantize_weights_noalloc(_p(w), n, rows, cols, lay, _p(codes), _p(scales), _p(gscale),
+                                              _stream()))
     return codes, scales, gscale
 
 

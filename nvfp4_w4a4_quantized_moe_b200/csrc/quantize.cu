@@ -2,6 +2,8 @@
 // weight quantiser ("K-EXAONE-152B-A23B-REAP-80E-NVFP4" model card, section
 // "Quantization Setup").  Both are HBM-bound streams: 128-bit loads of bf16,
 // 64-bit stores of packed codes, one scale byte per 16 elements.
+#include <mutex>
+
 #include "common.cuh"
 #include "host.cuh"
 
@@ -317,6 +319,90 @@ extern "C" nvfp4_status nvfp4_quantize_weights(const void* w_bf16, int n_mats, i
   uint32_t* amax = c.take<uint32_t>((size_t)n_mats);
   uint32_t* done = c.take<uint32_t>((size_t)n_mats);
   NV_CHECK(check_cuda(cudaMemsetAsync(ws, 0, need, s), "cudaMemsetAsync(workspace)"));
+  int per_sm = 0;
+  NV_CHECK(check_cuda(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quantize_weights_kernel, kWThreads, 0),
+                      "occupancy"));
+  per_sm = per_sm < 1 ? 1 : per_sm;
+  quantize_weights_kernel<<<sms * per_sm, kWThreads, 0, s>>>(static_cast<const uint4*>(w_bf16), n_mats, rows, cols,
+                                                             layout, reinterpret_cast<uint2*>(codes), scales,
+                                                             global_scale, st, amax, done);
+  return check_launch("quantize_weights_kernel");
+}
+
+namespace nvfp4moe {
+
+// ---------------------------------------------------------------------------
+// Weight quantiser for callers that cannot allocate device memory.
+//
+// Some hosts of this library cannot hand it a workspace: the process's device
+// memory belongs to another allocator (a serving engine's arena, a plugin
+// host's fixed pool) that the caller has no way to draw an extra buffer from,
+// or the caller runs where device allocation calls are not permitted.  This
+// entry point needs no workspace: the quantiser's scratch (work-queue head,
+// status word, per-matrix amax and completion counters) lives in the array
+// below, which every GPU that loads the library holds until the process
+// exits.
+// ---------------------------------------------------------------------------
+constexpr int kStaticMaxMats = 1024;
+constexpr size_t kStaticScratchBytes = 256 + 2 * 4 * kStaticMaxMats;   // state, amax[], done[]
+
+static __device__ __align__(256) uint8_t g_weight_quant_scratch[kStaticScratchBytes];
+
+// Device address of the scratch array, looked up once per device (the host
+// symbol is only a stand-in and must never be passed to a kernel).
+static nvfp4_status static_scratch_address(uint8_t** out) {
+  static std::mutex mu;
+  static uint8_t* addr[64] = {};
+  int dev = 0;
+  NV_CHECK(check_cuda(cudaGetDevice(&dev), "cudaGetDevice"));
+  NV_REQUIRE(dev >= 0 && dev < 64, NVFP4_ERR_DEVICE, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    NV_CHECK(check_cuda(cudaGetSymbolAddress(&p, g_weight_quant_scratch), "cudaGetSymbolAddress"));
+    addr[dev] = static_cast<uint8_t*>(p);
+  }
+  *out = addr[dev];
+  return NVFP4_OK;
+}
+
+}  // namespace nvfp4moe
+
+extern "C" nvfp4_status nvfp4_quantize_weights_noalloc(const void* w_bf16, int n_mats, int rows, int cols,
+                                                       int layout, uint8_t* codes, uint8_t* scales,
+                                                       float* global_scale, void* stream) {
+  using namespace nvfp4moe;
+  NV_REQUIRE(w_bf16 && codes && scales && global_scale, NVFP4_ERR_INVALID_ARG,
+             "nvfp4_quantize_weights_noalloc: a pointer argument is NULL");
+  NV_REQUIRE(n_mats >= 0 && rows >= 0 && cols > 0, NVFP4_ERR_INVALID_ARG,
+             "nvfp4_quantize_weights_noalloc: n_mats=%d rows=%d cols=%d", n_mats, rows, cols);
+  NV_REQUIRE(n_mats <= kStaticMaxMats, NVFP4_ERR_UNSUPPORTED_SHAPE,
+             "nvfp4_quantize_weights_noalloc: n_mats=%d exceeds the built-in scratch limit of %d matrices per call "
+             "(use nvfp4_quantize_weights with a workspace, or split the call)",
+             n_mats, kStaticMaxMats);
+  NV_REQUIRE(layout == NVFP4_LAYOUT_CANONICAL || layout == NVFP4_LAYOUT_TILED, NVFP4_ERR_INVALID_ARG,
+             "nvfp4_quantize_weights_noalloc: unknown layout %d", layout);
+  NV_REQUIRE(cols % 32 == 0, NVFP4_ERR_UNSUPPORTED_SHAPE,
+             "nvfp4_quantize_weights_noalloc: cols=%d must be a multiple of 32", cols);
+  NV_REQUIRE(layout == NVFP4_LAYOUT_CANONICAL || (cols % 64 == 0 && rows % 128 == 0), NVFP4_ERR_UNSUPPORTED_SHAPE,
+             "nvfp4_quantize_weights_noalloc: the tiled layout needs rows %% 128 == 0 and cols %% 64 == 0");
+  NV_REQUIRE((long long)n_mats * 2 * ((long long)rows * cols / 32768 + 1) < (1ll << 32),
+             NVFP4_ERR_UNSUPPORTED_SHAPE, "nvfp4_quantize_weights_noalloc: too many elements");
+  NV_REQUIRE(aligned(w_bf16, 16) && aligned(codes, 16) && aligned(scales, 4), NVFP4_ERR_INVALID_ARG,
+             "nvfp4_quantize_weights_noalloc: w and codes need 16-byte alignment, scales 4-byte");
+  if (n_mats == 0 || rows == 0) return NVFP4_OK;
+  int sms = 0;
+  NV_CHECK(device_sm_count(&sms));
+  uint8_t* scratch = nullptr;
+  NV_CHECK(static_scratch_address(&scratch));
+  cudaStream_t s = as_stream(stream);
+  // the array keeps the previous call's contents: clear the queue head, the
+  // status word and the per-matrix amax and counters this call uses
+  Carver c(scratch);
+  WeightQuantState* st = c.take<WeightQuantState>(1);
+  uint32_t* amax = c.take<uint32_t>((size_t)n_mats);
+  uint32_t* done = c.take<uint32_t>((size_t)n_mats);
+  NV_CHECK(check_cuda(cudaMemsetAsync(scratch, 0, c.size(), s), "cudaMemsetAsync(static scratch)"));
   int per_sm = 0;
   NV_CHECK(check_cuda(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quantize_weights_kernel, kWThreads, 0),
                       "occupancy"));
