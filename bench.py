@@ -429,10 +429,14 @@ def run_mma_peak():
     from nvfp4_w4a4_quantized_moe_b200 import capi as c
     res = {}
     for n in (256, 128):
-        for cp in (False, True):
+        for cp in (0, 1, 5, 6, 9, 10, 11, 12):
             c.nvfp4_test_mma_peak(200, n, cp)                      # warm-up
             fpc, cyc = c.nvfp4_test_mma_peak(20000, n, cp)
-            res[f"n{n}{'_with_scale_copies' if cp else ''}"] = {
+            res[f"n{n}" + ("", "_scale_copies_one_buffer", "_scale_copies_4_buffers",
+                           "_scale_copies_one_stage_ahead", "_scale_copies_6_wide", "_stage_handshake",
+                           "_stage_handshake_scale_copies", "_stage_handshake_spin",
+                           "_stage_handshake_spin_scale_copies", "_8_stages", "_8_stages_scale_copies",
+                           "_8_half_stages", "_8_half_stages_scale_copies")[cp]] = {
                 "flop_per_sm_clock": float(fpc.median()), "cycles_median": float(cyc.median())}
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     best = max(v["flop_per_sm_clock"] for v in res.values())

@@ -37,8 +37,10 @@ NVFP4_API nvfp4_status nvfp4_test_e4m3(const float* s, int n, uint8_t* codes, fl
 
 /* FP4 tensor-core rate without memory traffic: `ctas` CTAs (at most one per
  * SM) each issue `iters` x 4 block-scaled 128 x n x 64 MMAs (n = 128 or 256)
- * from fixed shared-memory operands, with (with_cp != 0) or without the 12
- * scale-factor copies of a 256-wide K stage before every 4 MMAs.
+ * from fixed shared-memory operands, without (with_cp == 0) or with the 12
+ * scale-factor copies of a 256-wide K stage before every 4 MMAs, into one set
+ * of tensor-memory columns (with_cp == 1) or rotating over four sets
+ * (with_cp == 2).
  * cycles[c] (device uint64) = SM clock cycles CTA c spent; *status (device
  * uint32) is set non-zero if the final wait gave up. */
 NVFP4_API nvfp4_status nvfp4_test_mma_peak(int iters, int n, int with_cp, int ctas, unsigned long long* cycles,

@@ -409,7 +409,7 @@ def nvfp4_test_sigmoid(l: torch.Tensor):
     return out
 
 
-def nvfp4_test_mma_peak(iters: int, n: int = 256, with_cp: bool = False, ctas: int | None = None):
+def nvfp4_test_mma_peak(iters: int, n: int = 256, with_cp: int = 0, ctas: int | None = None):
     """(FLOP per SM clock per CTA, cycles per CTA) of back-to-back FP4 MMAs."""
     ctas = ctas or torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
     cycles = torch.zeros(ctas, dtype=torch.int64, device="cuda")

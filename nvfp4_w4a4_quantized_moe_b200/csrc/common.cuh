@@ -146,16 +146,56 @@ NVDEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Non-blocking probe of a phase (never suspends the thread).
+NVDEV bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Like mbar_wait, but spinning on test_wait: the latency-critical single
+// threads (TMA producer, MMA issuer) see a completed phase at once.
+NVDEV bool mbar_wait_spin(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  if (mbar_test_wait(bar, parity)) return true;
+  uint64_t t0 = 0;
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_test_wait(bar, parity)) return true;
+    if ((i & 1023u) == 0) {
+      if (*abort) return false;
+      const uint64_t now = globaltimer_ns();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > kWaitLimitNs) {
+        return false;
+      }
+    }
+  }
+}
+
 // Wait for the phase with the given parity to complete.  Gives up (returns
-// false) after kWaitLimitNs or when *abort is set by another warp.
+// false) after kWaitLimitNs or when *abort is set by another warp.  The
+// abort flag and the clock are looked at only every 256 polls, so a phase
+// that completes is seen without the cost of a timer read.
 NVDEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (*abort) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+  uint64_t t0 = 0;
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 255u) == 0) {
+      if (*abort) return false;
+      const uint64_t now = globaltimer_ns();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > kWaitLimitNs) {
+        return false;
+      }
+    }
   }
-  return true;
 }
 
 NVDEV void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
@@ -218,6 +258,22 @@ NVDEV void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t 
 // 4 tensor-memory columns, replicated into all four 32-lane sub-partitions.
 NVDEV void tc_cp_scale_atom(uint32_t taddr, uint64_t sdesc) {
   asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc));
+}
+
+// Copy 128 rows x 32 bytes from shared memory into 8 tensor-memory columns of
+// all 128 lanes (no replication).
+NVDEV void tc_cp_128x256b(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc));
+}
+// Descriptor of a no-swizzle K-major source with 8-row x 16-byte core
+// matrices: `lbo` bytes between the two 16-byte halves of a 32-byte row
+// group, `sbo` bytes between groups of 8 rows.
+NVDEV uint64_t sdesc_interleave(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  return d;
 }
 
 // Shared-memory matrix descriptor, K-major operand with 128-byte swizzle:

@@ -40,8 +40,11 @@ constexpr int kThreads = 320;
 constexpr int kEpiWarps = 8;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCol = 0;                  // 256 fp32 accumulator columns
-constexpr uint32_t kSfaCol = 256;                // 4 MMA k-steps x 4 columns
-constexpr uint32_t kSfbCol = 272;                // 4 MMA k-steps x 8 columns
+// Scale factors of one stage: 4 MMA k-steps x (4 SFA + 8 SFB) columns.  The
+// copies and MMAs of one thread run in issue order, so every stage reuses the
+// same 48 columns.
+constexpr uint32_t kSfCol = 256;
+constexpr uint32_t kSfaOff = 0, kSfbOff = 16;
 
 struct GemmParams {
   const uint8_t* a_sf;
@@ -130,39 +133,38 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       uint32_t filled = 0, fill_parity = 0;     // per stage: ever filled / parity of last fill
       bool ok = true;
+      uint8_t* const st0 = smem;
+      const size_t tile_sf_bytes = (size_t)nblk4 * kAtomBytes;     // one 128-row tile's scales
       for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
         const int mt = t / p.n_tiles, nt = t % p.n_tiles;
         const int e = min(max(p.tile_expert[mt], 0), p.E - 1);
+        const int arow = mt * kBM;
+        const int brow = e * p.Nw + nt * (EPI == kEpiGateUp ? 128 : kBN);
+        const uint8_t* asf = p.a_sf + (size_t)mt * tile_sf_bytes;
+        const uint8_t* bsf0 = p.b0_sf + (size_t)(brow / kRowTile) * tile_sf_bytes;
+        const uint8_t* bsf1 = (EPI == kEpiGateUp ? p.b1_sf + (size_t)(brow / kRowTile) * tile_sf_bytes
+                                                 : bsf0 + tile_sf_bytes);
         for (int kt = 0; kt < KT; ++kt) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) {
             give_up(p.status, abort_flag);
             ok = false;
             break;
           }
-          uint8_t* sA = smem + stage * kStageBytes;
+          uint8_t* sA = st0 + stage * kStageBytes;
           uint8_t* sB = sA + kABytes;
           uint8_t* sSFA = sB + kBBytes;
           uint8_t* sSFB = sSFA + kSfaBytes;
           const int katoms = min(4, (p.K - kt * kBK) / 64);
           const uint32_t sf_bytes = (uint32_t)katoms * kAtomBytes;
+          const int x = kt * kBKBytes;
+          const size_t sf_off = (size_t)kt * 4 * kAtomBytes;
           mbar_arrive_expect_tx(&full_bar[stage], kABytes + kBBytes + 3 * sf_bytes);
-          tma_load_2d(sA, &tmA, kt * kBKBytes, mt * kBM, &full_bar[stage]);
-          bulk_load(sSFA, p.a_sf + ((size_t)mt * nblk4 + kt * 4) * kAtomBytes, sf_bytes, &full_bar[stage]);
-          if (EPI == kEpiGateUp) {
-            const int brow = e * p.Nw + nt * 128;
-            tma_load_2d(sB, &tmB0, kt * kBKBytes, brow, &full_bar[stage]);
-            tma_load_2d(sB + kBBytes / 2, &tmB1, kt * kBKBytes, brow, &full_bar[stage]);
-            const size_t off = ((size_t)(brow / kRowTile) * nblk4 + kt * 4) * kAtomBytes;
-            bulk_load(sSFB, p.b0_sf + off, sf_bytes, &full_bar[stage]);
-            bulk_load(sSFB + kSfbBytes / 2, p.b1_sf + off, sf_bytes, &full_bar[stage]);
-          } else {
-            const int brow = e * p.Nw + nt * kBN;
-            tma_load_2d(sB, &tmB0, kt * kBKBytes, brow, &full_bar[stage]);
-            const size_t off0 = ((size_t)(brow / kRowTile) * nblk4 + kt * 4) * kAtomBytes;
-            const size_t off1 = ((size_t)(brow / kRowTile + 1) * nblk4 + kt * 4) * kAtomBytes;
-            bulk_load(sSFB, p.b0_sf + off0, sf_bytes, &full_bar[stage]);
-            bulk_load(sSFB + kSfbBytes / 2, p.b0_sf + off1, sf_bytes, &full_bar[stage]);
-          }
+          tma_load_2d(sA, &tmA, x, arow, &full_bar[stage]);
+          tma_load_2d(sB, &tmB0, x, brow, &full_bar[stage]);
+          if (EPI == kEpiGateUp) tma_load_2d(sB + kBBytes / 2, &tmB1, x, brow, &full_bar[stage]);
+          bulk_load(sSFA, asf + sf_off, sf_bytes, &full_bar[stage]);
+          bulk_load(sSFB, bsf0 + sf_off, sf_bytes, &full_bar[stage]);
+          bulk_load(sSFB + kSfbBytes / 2, bsf1 + sf_off, sf_bytes, &full_bar[stage]);
           filled |= 1u << stage;
           fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == kStages) {
@@ -180,8 +182,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // One thread issues everything; its own instruction latency bounds the
+    // MMA rate, so all shared-memory descriptors are built once here and a
+    // stage only adds constant offsets to their start-address fields.
     if (lane == 0) {
       const uint32_t idesc = idesc_fp4(kBM, kBN);
+      const uint32_t s0 = smem_u32(smem);
+      const uint64_t a0 = sdesc_sw128(s0), b0 = sdesc_sw128(s0 + kABytes);
+      const uint64_t sfa0 = sdesc_scale_atom(s0 + kABytes + kBBytes);
+      const uint64_t sfb0 = sdesc_scale_atom(s0 + kABytes + kBBytes + kSfaBytes);
+      constexpr uint64_t kStageStep = kStageBytes >> 4;        // start address is in 16-byte units
+      constexpr uint64_t kAtomStep = kAtomBytes >> 4;
+      constexpr uint64_t kSfbHalfStep = (kSfbBytes / 2) >> 4;
+      const uint32_t sfa_t = tmem + kSfCol + kSfaOff, sfb_t = tmem + kSfCol + kSfbOff;
+      const uint32_t acc_t = tmem + kAccCol;
       int stage = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
@@ -191,26 +205,40 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
+        uint32_t accumulate = 0;
         for (int kt = 0; kt < KT; ++kt) {
+          // TMA wrote this stage through the async proxy that the MMAs read
+          // through; the completed barrier phase is all the ordering needed
           if (!mbar_wait(&full_bar[stage], phase, abort_flag)) {
             give_up(p.status, abort_flag);
             ok = false;
             break;
           }
-          tc_fence_after();
-          const uint32_t sA = smem_u32(smem + stage * kStageBytes);
-          const uint32_t sB = sA + kABytes, sSFA = sB + kBBytes, sSFB = sSFA + kSfaBytes;
+          const uint64_t d = (uint64_t)stage * kStageStep;
           const int katoms = min(4, (p.K - kt * kBK) / 64);
-          for (int j = 0; j < katoms; ++j) {
-            tc_cp_scale_atom(tmem + kSfaCol + 4 * j, sdesc_scale_atom(sSFA + kAtomBytes * j));
-            tc_cp_scale_atom(tmem + kSfbCol + 8 * j, sdesc_scale_atom(sSFB + kAtomBytes * j));
-            tc_cp_scale_atom(tmem + kSfbCol + 8 * j + 4, sdesc_scale_atom(sSFB + kSfbBytes / 2 + kAtomBytes * j));
-          }
-          const uint64_t adesc = sdesc_sw128(sA), bdesc = sdesc_sw128(sB);
-          for (int j = 0; j < katoms; ++j) {
-            // +32 bytes (64 FP4 values) along K inside the 128-byte swizzle atom
-            mma_fp4(tmem + kAccCol, adesc + 2 * j, bdesc + 2 * j, idesc, tmem + kSfaCol + 4 * j,
-                    tmem + kSfbCol + 8 * j, (kt | j) != 0);
+          if (katoms == 4) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              tc_cp_scale_atom(sfa_t + 4 * j, sfa0 + d + j * kAtomStep);
+              tc_cp_scale_atom(sfb_t + 8 * j, sfb0 + d + j * kAtomStep);
+              tc_cp_scale_atom(sfb_t + 8 * j + 4, sfb0 + d + kSfbHalfStep + j * kAtomStep);
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              // +32 bytes (64 FP4 values) along K inside the 128-byte swizzle atom
+              mma_fp4(acc_t, a0 + d + 2 * j, b0 + d + 2 * j, idesc, sfa_t + 4 * j, sfb_t + 8 * j, accumulate);
+              accumulate = 1;
+            }
+          } else {
+            for (int j = 0; j < katoms; ++j) {
+              tc_cp_scale_atom(sfa_t + 4 * j, sfa0 + d + j * kAtomStep);
+              tc_cp_scale_atom(sfb_t + 8 * j, sfb0 + d + j * kAtomStep);
+              tc_cp_scale_atom(sfb_t + 8 * j + 4, sfb0 + d + kSfbHalfStep + j * kAtomStep);
+            }
+            for (int j = 0; j < katoms; ++j) {
+              mma_fp4(acc_t, a0 + d + 2 * j, b0 + d + 2 * j, idesc, sfa_t + 4 * j, sfb_t + 8 * j, accumulate);
+              accumulate = 1;
+            }
           }
           tc_commit(&empty_bar[stage]);
           if (++stage == kStages) {

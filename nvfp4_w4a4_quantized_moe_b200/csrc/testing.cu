@@ -76,6 +76,8 @@ __global__ void __launch_bounds__(128, 1) mma_peak_kernel(int iters, int n, int 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   __shared__ __align__(8) uint64_t bar;
+  __shared__ __align__(8) uint64_t full_bar[8];
+  __shared__ __align__(8) uint64_t empty_bar[8];
   __shared__ uint32_t tmem_s;
   __shared__ int abort_s;
   const int warp = threadIdx.x >> 5;
@@ -83,6 +85,10 @@ __global__ void __launch_bounds__(128, 1) mma_peak_kernel(int iters, int n, int 
     reinterpret_cast<uint4*>(smem)[i] = make_uint4(0, 0, 0, 0);
   if (threadIdx.x == 0) {
     mbar_init(&bar, 1);
+    for (int i = 0; i < 8; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&empty_bar[i], 1);
+    }
     abort_s = 0;
     fence_barrier_init();
   }
@@ -100,21 +106,69 @@ __global__ void __launch_bounds__(128, 1) mma_peak_kernel(int iters, int n, int 
     const uint64_t adesc = sdesc_sw128(sA), bdesc = sdesc_sw128(sB);
     const uint32_t idesc = idesc_fp4(128, n);
     const unsigned long long t0 = clock64();
-    for (int it = 0; it < iters; ++it) {
-      if (with_cp) {
-        for (int j = 0; j < 4; ++j) {
-          tc_cp_scale_atom(tmem + 256 + 4 * j, sdesc_scale_atom(sSF + 512 * j));
-          tc_cp_scale_atom(tmem + 272 + 8 * j, sdesc_scale_atom(sSF + 2048 + 512 * j));
-          tc_cp_scale_atom(tmem + 276 + 8 * j, sdesc_scale_atom(sSF + 4096 + 512 * j));
-        }
+    auto copies = [&](uint32_t sf) {
+      for (int j = 0; j < 4; ++j) {
+        tc_cp_scale_atom(sf + 4 * j, sdesc_scale_atom(sSF + 512 * j));
+        tc_cp_scale_atom(sf + 16 + 8 * j, sdesc_scale_atom(sSF + 2048 + 512 * j));
+        tc_cp_scale_atom(sf + 20 + 8 * j, sdesc_scale_atom(sSF + 4096 + 512 * j));
       }
+    };
+    auto wide_copies = [&](uint32_t sf) {      // 6 copies of 128 lanes x 8 columns
+      for (int j = 0; j < 2; ++j) tc_cp_128x256b(sf + 8 * j, sdesc_interleave(sSF + 2048 * j, 128, 256));
+      for (int j = 0; j < 4; ++j) tc_cp_128x256b(sf + 16 + 8 * j, sdesc_interleave(sSF + 512 * j, 128, 256));
+    };
+    if (with_cp == 3) copies(tmem + 256);
+    if (with_cp >= 5) {
+      // the GEMM's stage handshake: wait "full" (arrived by a second warp once
+      // it has seen the "empty" commit of `stages` stages back), MMAs, commit
+      // "empty".  Modes 9-12: 8 stages; 11-12: stages of 2 MMAs (K = 128).
+      const int stages = with_cp >= 9 ? 8 : 4;
+      const int per = with_cp >= 11 ? 2 : 4;
+      const bool cps = with_cp == 6 || with_cp == 8 || with_cp == 10 || with_cp == 12;
+      uint32_t phase = 0;
+      for (int it = 0; it < iters * (4 / per); ++it) {
+        const int st = it & (stages - 1);
+        if (!(with_cp == 7 || with_cp == 8 ? mbar_wait_spin(&full_bar[st], phase, &abort_s) : mbar_wait(&full_bar[st], phase, &abort_s))) { atomicExch(status, kDevTimeout); break; }
+        tc_fence_after();
+        const uint32_t sf = tmem + 256 + (uint32_t)(st & 3) * 48;
+        if (cps) {
+          for (int j = 0; j < per; ++j) {
+            tc_cp_scale_atom(sf + 4 * j, sdesc_scale_atom(sSF + 512 * j));
+            tc_cp_scale_atom(sf + 16 + 8 * j, sdesc_scale_atom(sSF + 2048 + 512 * j));
+            tc_cp_scale_atom(sf + 20 + 8 * j, sdesc_scale_atom(sSF + 4096 + 512 * j));
+          }
+        }
+        for (int j = 0; j < per; ++j)
+          mma_fp4(tmem, adesc + 2 * j, bdesc + 2 * j, idesc, sf + 4 * j, sf + 16 + 8 * j, (it | j) != 0);
+        tc_commit(&empty_bar[st]);
+        if (st == stages - 1) phase ^= 1u;
+      }
+    }
+    for (int it = 0; with_cp < 5 && it < iters; ++it) {
+      // with_cp: 1 one buffer; 2 four rotating buffers; 3 rotating buffers,
+      // copies issued one iteration ahead; 4 six 128x256b copies
+      const uint32_t sf = tmem + 256 + (with_cp >= 2 ? (uint32_t)(it & 3) * 48 : 0u);
+      if (with_cp == 1 || with_cp == 2) copies(sf);
+      if (with_cp == 3) copies(tmem + 256 + (uint32_t)((it + 1) & 3) * 48);
+      if (with_cp == 4) wide_copies(sf);
       for (int j = 0; j < 4; ++j)
-        mma_fp4(tmem, adesc + 2 * j, bdesc + 2 * j, idesc, tmem + 256 + 4 * j, tmem + 272 + 8 * j, (it | j) != 0);
+        mma_fp4(tmem, adesc + 2 * j, bdesc + 2 * j, idesc, sf + 4 * j, sf + 16 + 8 * j, (it | j) != 0);
     }
     tc_commit(&bar);
     if (!mbar_wait(&bar, 0, &abort_s)) atomicExch(status, kDevTimeout);
     const unsigned long long t1 = clock64();
     cycles[blockIdx.x] = t1 - t0;
+  } else if (threadIdx.x == 64 && with_cp >= 5) {
+    // the producer side of the handshake, with no loads
+    const int stages = with_cp >= 9 ? 8 : 4;
+    const int per = with_cp >= 11 ? 2 : 4;
+    uint32_t phase = 0;
+    for (int it = 0; it < iters * (4 / per); ++it) {
+      const int st = it & (stages - 1);
+      if (!(with_cp == 7 || with_cp == 8 ? mbar_wait_spin(&empty_bar[st], phase ^ 1u, &abort_s) : mbar_wait(&empty_bar[st], phase ^ 1u, &abort_s))) { atomicExch(status, kDevTimeout); break; }
+      mbar_arrive(&full_bar[st]);
+      if (st == stages - 1) phase ^= 1u;
+    }
   }
   tc_fence_before();
   __syncthreads();
