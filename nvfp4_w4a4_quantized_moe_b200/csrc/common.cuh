@@ -211,6 +211,10 @@ NVDEV void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) 
                "l"(src), "r"(bytes), "r"(smem_u32(bar))
                : "memory");
 }
+// Bring a byte range into L2 ahead of its loads (no shared memory involved).
+NVDEV void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 NVDEV void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }

@@ -206,14 +206,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         uint32_t accumulate = 0;
+        bool ready = false;                     // this stage already seen complete
         for (int kt = 0; kt < KT; ++kt) {
           // TMA wrote this stage through the async proxy that the MMAs read
           // through; the completed barrier phase is all the ordering needed
-          if (!mbar_wait(&full_bar[stage], phase, abort_flag)) {
+          if (!ready && !mbar_wait(&full_bar[stage], phase, abort_flag)) {
             give_up(p.status, abort_flag);
             ok = false;
             break;
           }
+          // look at the next stage now; the answer is used only after this
+          // stage's copies and MMAs have been issued
+          const int nstage = stage + 1 == kStages ? 0 : stage + 1;
+          const uint32_t nphase = stage + 1 == kStages ? phase ^ 1u : phase;
+          ready = (kt + 1 < KT) && mbar_test_wait(&full_bar[nstage], nphase);
           const uint64_t d = (uint64_t)stage * kStageStep;
           const int katoms = min(4, (p.K - kt * kBK) / 64);
           if (katoms == 4) {
@@ -276,20 +282,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (EPI == kEpiGateUp) {
         const float sg = __fmul_rn(g_act, p.g_b0[e]);
         const float su = __fmul_rn(g_act, p.g_b1[e]);
-        float h[64];
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t rg[32], ru[32];
-          tmem_ld32(tbase + kAccCol + half * 64 + 32 * c, rg);
-          tmem_ld32(tbase + kAccCol + 128 + half * 64 + 32 * c, ru);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float gate = __fmul_rn(__uint_as_float(rg[i]), sg);
-            const float up = __fmul_rn(__uint_as_float(ru[i]), su);
-            h[32 * c + i] = __fmul_rn(silu(gate), up);
-          }
-        }
+        // drain this thread's 64 gate and 64 up columns, then hand the
+        // accumulator back before any arithmetic
+        uint32_t rg[64], ru[64];
+        tmem_ld32(tbase + kAccCol + half * 64, rg);
+        tmem_ld32(tbase + kAccCol + half * 64 + 32, rg + 32);
+        tmem_ld32(tbase + kAccCol + 128 + half * 64, ru);
+        tmem_ld32(tbase + kAccCol + 128 + half * 64 + 32, ru + 32);
+        tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty_bar);
@@ -297,6 +297,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint4 cw0 = make_uint4(0, 0, 0, 0), cw1 = make_uint4(0, 0, 0, 0);
         uint32_t sw = 0;
         if (real) {
+          float h[64];
+#pragma unroll
+          for (int i = 0; i < 64; ++i) {
+            const float gate = __fmul_rn(__uint_as_float(rg[i]), sg);
+            const float up = __fmul_rn(__uint_as_float(ru[i]), su);
+            h[i] = __fmul_rn(silu(gate), up);
+          }
           const float g2 = *p.g_h;
           const float d2 = __fmul_rn(6.0f, g2);
           uint2 c0, c1, c2, c3;
@@ -326,31 +333,36 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         const float scale = __fmul_rn(__fmul_rn(g_act, p.g_b0[e]), p.row_w ? p.row_w[grow] : 1.0f);
         const int col0 = nt * kBN + half * 128;
-        uint32_t packed[64];
+        // drain this thread's 128 columns, then hand the accumulator back
+        uint32_t r[128];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tbase + kAccCol + half * 128 + 32 * c, r);
-          tmem_ld_wait();
-          float v[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(__uint_as_float(r[i]), scale);
-          if (p.y_f32 && real) {
-            float4* dst = reinterpret_cast<float4*>(p.y_f32 + (size_t)grow * p.H + col0 + 32 * c);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-          }
-#pragma unroll
-          for (int i = 0; i < 16; ++i) packed[16 * c + i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
-        }
+        for (int c = 0; c < 4; ++c) tmem_ld32(tbase + kAccCol + half * 128 + 32 * c, r + 32 * c);
+        tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty_bar);
-        if (p.y_bf16 && real) {
-          uint4* dst = reinterpret_cast<uint4*>(p.y_bf16 + (size_t)grow * p.H + col0);
+        if (real) {
+          if (p.y_f32) {
+            float4* dst = reinterpret_cast<float4*>(p.y_f32 + (size_t)grow * p.H + col0);
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+            for (int i = 0; i < 32; ++i)
+              dst[i] = make_float4(__fmul_rn(__uint_as_float(r[4 * i]), scale),
+                                   __fmul_rn(__uint_as_float(r[4 * i + 1]), scale),
+                                   __fmul_rn(__uint_as_float(r[4 * i + 2]), scale),
+                                   __fmul_rn(__uint_as_float(r[4 * i + 3]), scale));
+          }
+          if (p.y_bf16) {
+            uint4* dst = reinterpret_cast<uint4*>(p.y_bf16 + (size_t)grow * p.H + col0);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              uint32_t w[4];
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                w[q] = pack_bf16x2(__fmul_rn(__uint_as_float(r[8 * i + 2 * q]), scale),
+                                   __fmul_rn(__uint_as_float(r[8 * i + 2 * q + 1]), scale));
+              dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+          }
         }
       }
       acc_phase ^= 1u;

@@ -86,25 +86,26 @@ __global__ void zero_tiled_scale_rows(uint8_t* scales, int rows, int padded_rows
 }
 
 // ---------------------------------------------------------------------------
-// Weights: a persistent kernel walking a queue of 32768-element items.  The
-// queue interleaves the amax pass of matrix m+1 with the quantise pass of
-// matrix m, so the second read of a matrix finds it in L2 (the first read
-// asks L2 to keep the lines, the second lets them go).  A quantise item waits
-// (bounded) until every amax item of its matrix has finished; those items
-// were taken from the queue earlier by running blocks, so the wait always
-// ends.  Each thread owns 4 x 32 consecutive elements of an item and issues
-// all of its loads before it waits or computes.
+// Weights: one cooperative launch (every CTA resident).  Each CTA owns an
+// even share of every matrix and splits its warps in two groups that run side
+// by side:
+//   * amax warps stream matrix after matrix, publish one atomic max and one
+//     completion count per matrix, and stay at most two matrices ahead of
+//     their own CTA's quantise warps (so the matrices in flight fit in L2);
+//   * quantise warps take matrix m once every CTA has published its amax
+//     (a bounded wait), re-read their share (from L2: the amax pass asked L2
+//     to keep the lines, this pass lets them go) and write codes and scales.
+// Waits only ever point at earlier matrices, so with all CTAs resident they
+// always end.
 // ---------------------------------------------------------------------------
-constexpr int kWThreads = 256;
-constexpr int kWPerThread = 32;                       // two 16-element blocks
-constexpr int kWSub = 4;                              // sub-chunks per item
-constexpr int kWSubElems = kWThreads * kWPerThread;   // 8192
-constexpr int kWItem = kWSub * kWSubElems;            // 32768 elements
+constexpr int kWAmax = 256;                     // amax threads per CTA (the DRAM stream)
+constexpr int kWQuant = 256;                    // quantise threads per CTA (re-read from L2)
+constexpr int kWThreads = kWAmax + kWQuant;
+constexpr int kWAhead = 2;                      // amax may lead quantise by this many matrices
 
 struct WeightQuantState {
   uint32_t status;          // device status word (first word of the workspace)
-  uint32_t next_item;       // queue head
-  uint32_t pad[62];
+  uint32_t pad[63];
   // followed by amax_bits[n_mats], done[n_mats]
 };
 
@@ -113,7 +114,6 @@ NVDEV uint32_t ld_acquire_u32(const uint32_t* p) {
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
-
 NVDEV uint64_t l2_policy_evict_last() {
   uint64_t pol;
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
@@ -131,118 +131,164 @@ NVDEV uint4 ld_hint(const uint4* p, uint64_t pol) {
                : "l"(p), "l"(pol));
   return v;
 }
+template <int N>
+NVDEV void group_sync(int id) { asm volatile("bar.sync %0, %1;" ::"r"(id), "n"(N) : "memory"); }
 
 __global__ void __launch_bounds__(kWThreads) quantize_weights_kernel(
     const uint4* __restrict__ w, int n_mats, int rows, int cols, int layout, uint2* __restrict__ codes,
     uint8_t* __restrict__ scales, float* __restrict__ gscale, WeightQuantState* st, uint32_t* amax_bits,
     uint32_t* done) {
-  __shared__ uint32_t s_item;
-  __shared__ uint32_t s_red[kWThreads / 32];
-  __shared__ int s_fail;
+  __shared__ uint32_t s_red[kWAmax / 32];
+  __shared__ int s_ok_amax, s_ok_quant;
+  __shared__ volatile int quantised;            // matrices this CTA's quantise warps have finished
+  __shared__ volatile int failed;
   const long long per_mat = (long long)rows * cols;
-  const uint32_t chunks = (uint32_t)((per_mat + kWItem - 1) / kWItem);
-  const uint32_t total_items = 2u * chunks * (uint32_t)n_mats;
+  const long long blocks = per_mat / kQBlock;                  // 16-element blocks per matrix
   const int nblk = cols / kQBlock;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const uint64_t keep = l2_policy_evict_last(), drop = l2_policy_evict_first();
+  const int lane = threadIdx.x & 31;
+  const int gt = threadIdx.x < kWAmax ? threadIdx.x : threadIdx.x - kWAmax;   // index within its group
+  // this CTA's share of every matrix, in whole groups of 4 blocks
+  const long long share = ((blocks + gridDim.x - 1) / gridDim.x + 3) / 4 * 4;
+  const long long b_begin = min(blocks, share * blockIdx.x), b_end = min(blocks, b_begin + share);
+  if (threadIdx.x == 0) {
+    quantised = 0;
+    failed = 0;
+  }
+  __syncthreads();
 
-  for (;;) {
-    if (threadIdx.x == 0) {
-      s_item = atomicAdd(&st->next_item, 1u);
-      s_fail = 0;
-    }
-    __syncthreads();
-    const uint32_t item = s_item;
-    if (item >= total_items) break;
-    // decode the queue position: step 0 = amax(0); step s = amax(s), quant(s-1)
-    bool is_amax;
-    uint32_t mat, chunk;
-    if (item < chunks) {
-      is_amax = true; mat = 0; chunk = item;
-    } else {
-      const uint32_t j = item - chunks, step = 1 + j / (2 * chunks), r = j % (2 * chunks);
-      if (step < (uint32_t)n_mats) {
-        is_amax = r < chunks; mat = is_amax ? step : step - 1; chunk = is_amax ? r : r - chunks;
-      } else {
-        is_amax = false; mat = n_mats - 1; chunk = r;
+  if (threadIdx.x < kWAmax) {
+    // ------------------------------------------------------------ amax warps
+    const uint64_t keep = l2_policy_evict_last();
+    for (int mat = 0; mat < n_mats; ++mat) {
+      if (gt == 0) {
+        const uint64_t t0 = globaltimer_ns();
+        while (quantised < mat - kWAhead && !failed) {
+          if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            failed = 1;
+            atomicExch(&st->status, kDevTimeout);
+          }
+        }
+        s_ok_amax = !failed;
       }
-    }
-    // element offsets of this thread's four 32-element runs
-    long long e0[kWSub];
-    bool valid[kWSub];
-    uint4 raw[kWSub][4];
-#pragma unroll
-    for (int q = 0; q < kWSub; ++q) {
-      e0[q] = (long long)chunk * kWItem + (long long)q * kWSubElems + (long long)threadIdx.x * kWPerThread;
-      valid[q] = e0[q] < per_mat;
-      const uint4* src = w + ((long long)mat * per_mat + e0[q]) / 8;
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        raw[q][i] = valid[q] ? ld_hint(src + i, is_amax ? keep : drop) : make_uint4(0, 0, 0, 0);
-    }
-    if (is_amax) {
+      group_sync<kWAmax>(1);
+      if (!s_ok_amax) break;
+      const uint4* src = w + (long long)mat * per_mat / 8;
+      const long long v1 = b_end * 2;                          // uint4 range (8 bf16 each)
       float m = 0.0f;
+      long long i = b_begin * 2 + gt;
+      for (; i + 7 * kWAmax < v1; i += 8 * kWAmax) {
+        uint4 u[8];
 #pragma unroll
-      for (int q = 0; q < kWSub; ++q)
+        for (int q = 0; q < 8; ++q) u[q] = ld_hint(src + i + q * kWAmax, keep);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int q = 0; q < 8; ++q) {
           float v[8];
-          unpack_bf16x8(raw[q][i], v);
+          unpack_bf16x8(u[q], v);
 #pragma unroll
           for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(v[j]));
         }
+      }
+      for (; i < v1; i += kWAmax) {
+        float v[8];
+        unpack_bf16x8(ld_hint(src + i, keep), v);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(v[j]));
+      }
       uint32_t mb = __float_as_uint(m);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, o));
-      if (lane == 0) s_red[warp] = mb;
-      __syncthreads();
-      if (threadIdx.x == 0) {
+      if (lane == 0) s_red[gt >> 5] = mb;
+      group_sync<kWAmax>(1);
+      if (gt == 0) {
         uint32_t bm = 0;
-        for (int q = 0; q < kWThreads / 32; ++q) bm = max(bm, s_red[q]);
-        atomicMax(amax_bits + mat, bm);     // non-negative floats order like their bits
+        for (int q = 0; q < kWAmax / 32; ++q) bm = max(bm, s_red[q]);
+        atomicMax(amax_bits + mat, bm);         // non-negative floats order like their bits
         __threadfence();
         atomicAdd(done + mat, 1u);
       }
-    } else {
-      if (threadIdx.x == 0) {
-        if (ld_acquire_u32(done + mat) < chunks) {
+    }
+  } else {
+    // ------------------------------------------------------------ quantise warps
+    const uint64_t drop = l2_policy_evict_first();
+    for (int mat = 0; mat < n_mats; ++mat) {
+      if (gt == 0) {
+        int ok = 1;
+        if (ld_acquire_u32(done + mat) < gridDim.x) {
           const uint64_t t0 = globaltimer_ns();
-          while (ld_acquire_u32(done + mat) < chunks) {
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+          while (ld_acquire_u32(done + mat) < gridDim.x) {
+            if (failed || globaltimer_ns() - t0 > kWaitLimitNs) {
+              ok = 0;
+              failed = 1;
               atomicExch(&st->status, kDevTimeout);
-              s_fail = 1;
               break;
             }
           }
         }
+        s_ok_quant = ok;
       }
-      __syncthreads();
-      if (s_fail) break;
+      group_sync<kWQuant>(2);
+      if (!s_ok_quant) break;
       const float amax = __uint_as_float(ld_acquire_u32(amax_bits + mat));
       const float g = __fdiv_rn(amax, 2688.0f);
       const float d = __fmul_rn(6.0f, g);
-      if (chunk == 0 && threadIdx.x == 0) gscale[mat] = g;
+      if (blockIdx.x == 0 && gt == 0) gscale[mat] = g;
+      const uint4* src = w + (long long)mat * per_mat / 8;
+      // every lane of a warp runs the same number of iterations (shuffles
+      // below); each iteration has two blocks per thread in flight
+      const long long n_iter = (b_end - b_begin + 2 * kWQuant - 1) / (2 * kWQuant);
+      for (long long it = 0; it < n_iter; ++it) {
+        uint4 u[2][2];
+        bool valid[2];
+        long long b[2];
 #pragma unroll
-      for (int q = 0; q < kWSub; ++q) {
-        uint32_t s[2] = {0, 0};
-        int row = 0, kb = 0;
-        if (valid[q]) {
-          float v[32];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) unpack_bf16x8(raw[q][i], v + 8 * i);
-          row = (int)(e0[q] / cols);
-          kb = (int)((e0[q] % cols) / kQBlock);
-          uint2 c0, c1;
-          s[0] = quant_block16(v, g, d, c0);
-          s[1] = quant_block16(v + 16, g, d, c1);
-          *reinterpret_cast<uint4*>(codes + ((long long)mat * per_mat + e0[q]) / 16) =
-              make_uint4(c0.x, c0.y, c1.x, c1.y);
+        for (int q = 0; q < 2; ++q) {
+          b[q] = b_begin + (2 * it + q) * kWQuant + gt;
+          valid[q] = b[q] < b_end;
+          if (valid[q]) {
+            u[q][0] = ld_hint(src + 2 * b[q], drop);
+            u[q][1] = ld_hint(src + 2 * b[q] + 1, drop);
+          }
         }
-        store_scales<2>(scales, layout, mat * rows + row, kb, nblk, s, valid[q]);
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          uint32_t sc = 0;
+          int row = 0, kb = 0;
+          if (valid[q]) {
+            float v[16];
+            unpack_bf16x8(u[q][0], v);
+            unpack_bf16x8(u[q][1], v + 8);
+            uint2 c;
+            sc = quant_block16(v, g, d, c);
+            codes[(long long)mat * blocks + b[q]] = c;
+            row = (int)(b[q] / nblk);
+            kb = (int)(b[q] % nblk);
+          }
+          store_scales<1>(scales, layout, mat * rows + row, kb, nblk, &sc, valid[q]);
+        }
       }
+      group_sync<kWQuant>(2);
+      if (gt == 0) quantised = mat + 1;
     }
-    __syncthreads();
   }
+  __syncthreads();
+}
+
+// Cooperative launch: the phases need every CTA resident at once.
+static nvfp4_status launch_weight_quantiser(const void* w_bf16, int n_mats, int rows, int cols, int layout,
+                                           uint8_t* codes, uint8_t* scales, float* global_scale,
+                                           WeightQuantState* st, uint32_t* amax, uint32_t* done, int sms,
+                                           cudaStream_t s) {
+  int per_sm = 0;
+  NV_CHECK(check_cuda(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quantize_weights_kernel, kWThreads, 0),
+                      "occupancy"));
+  per_sm = std::max(1, std::min(per_sm, 2));
+  const uint4* w = static_cast<const uint4*>(w_bf16);
+  uint2* c = reinterpret_cast<uint2*>(codes);
+  void* args[] = {(void*)&w, (void*)&n_mats, (void*)&rows, (void*)&cols, (void*)&layout, (void*)&c,
+                  (void*)&scales, (void*)&global_scale, (void*)&st, (void*)&amax, (void*)&done};
+  return check_cuda(cudaLaunchCooperativeKernel((const void*)quantize_weights_kernel, dim3(sms * per_sm),
+                                                dim3(kWThreads), args, 0, s),
+                    "cudaLaunchCooperativeKernel(quantize_weights_kernel)");
 }
 
 }  // namespace nvfp4moe
@@ -303,7 +349,7 @@ extern "C" nvfp4_status nvfp4_quantize_weights(const void* w_bf16, int n_mats, i
   NV_REQUIRE(layout == NVFP4_LAYOUT_CANONICAL || (cols % 64 == 0 && rows % 128 == 0), NVFP4_ERR_UNSUPPORTED_SHAPE,
              "nvfp4_quantize_weights: the tiled layout needs rows %% 128 == 0 and cols %% 64 == 0 (got %d x %d)", rows,
              cols);
-  NV_REQUIRE((long long)n_mats * 2 * ((long long)rows * cols / 32768 + 1) < (1ll << 32),
+  NV_REQUIRE((long long)rows * cols < (1ll << 40) && n_mats < (1 << 24),
              NVFP4_ERR_UNSUPPORTED_SHAPE, "nvfp4_quantize_weights: too many elements");
   const size_t need = nvfp4_quantize_weights_workspace_size(n_mats);
   NV_REQUIRE(ws != nullptr && ws_bytes >= need && aligned(ws, 256), NVFP4_ERR_WORKSPACE,
@@ -319,14 +365,8 @@ extern "C" nvfp4_status nvfp4_quantize_weights(const void* w_bf16, int n_mats, i
   uint32_t* amax = c.take<uint32_t>((size_t)n_mats);
   uint32_t* done = c.take<uint32_t>((size_t)n_mats);
   NV_CHECK(check_cuda(cudaMemsetAsync(ws, 0, need, s), "cudaMemsetAsync(workspace)"));
-  int per_sm = 0;
-  NV_CHECK(check_cuda(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quantize_weights_kernel, kWThreads, 0),
-                      "occupancy"));
-  per_sm = per_sm < 1 ? 1 : per_sm;
-  quantize_weights_kernel<<<sms * per_sm, kWThreads, 0, s>>>(static_cast<const uint4*>(w_bf16), n_mats, rows, cols,
-                                                             layout, reinterpret_cast<uint2*>(codes), scales,
-                                                             global_scale, st, amax, done);
-  return check_launch("quantize_weights_kernel");
+  return launch_weight_quantiser(w_bf16, n_mats, rows, cols, layout, codes, scales, global_scale, st, amax, done,
+                                 sms, s);
 }
 
 namespace nvfp4moe {
@@ -386,7 +426,7 @@ extern "C" nvfp4_status nvfp4_quantize_weights_noalloc(const void* w_bf16, int n
              "nvfp4_quantize_weights_noalloc: cols=%d must be a multiple of 32", cols);
   NV_REQUIRE(layout == NVFP4_LAYOUT_CANONICAL || (cols % 64 == 0 && rows % 128 == 0), NVFP4_ERR_UNSUPPORTED_SHAPE,
              "nvfp4_quantize_weights_noalloc: the tiled layout needs rows %% 128 == 0 and cols %% 64 == 0");
-  NV_REQUIRE((long long)n_mats * 2 * ((long long)rows * cols / 32768 + 1) < (1ll << 32),
+  NV_REQUIRE((long long)rows * cols < (1ll << 40) && n_mats < (1 << 24),
              NVFP4_ERR_UNSUPPORTED_SHAPE, "nvfp4_quantize_weights_noalloc: too many elements");
   NV_REQUIRE(aligned(w_bf16, 16) && aligned(codes, 16) && aligned(scales, 4), NVFP4_ERR_INVALID_ARG,
              "nvfp4_quantize_weights_noalloc: w and codes need 16-byte alignment, scales 4-byte");
@@ -403,12 +443,6 @@ extern "C" nvfp4_status nvfp4_quantize_weights_noalloc(const void* w_bf16, int n
   uint32_t* amax = c.take<uint32_t>((size_t)n_mats);
   uint32_t* done = c.take<uint32_t>((size_t)n_mats);
   NV_CHECK(check_cuda(cudaMemsetAsync(scratch, 0, c.size(), s), "cudaMemsetAsync(static scratch)"));
-  int per_sm = 0;
-  NV_CHECK(check_cuda(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quantize_weights_kernel, kWThreads, 0),
-                      "occupancy"));
-  per_sm = per_sm < 1 ? 1 : per_sm;
-  quantize_weights_kernel<<<sms * per_sm, kWThreads, 0, s>>>(static_cast<const uint4*>(w_bf16), n_mats, rows, cols,
-                                                             layout, reinterpret_cast<uint2*>(codes), scales,
-                                                             global_scale, st, amax, done);
-  return check_launch("quantize_weights_kernel");
+  return launch_weight_quantiser(w_bf16, n_mats, rows, cols, layout, codes, scales, global_scale, st, amax, done,
+                                 sms, s);
 }
