@@ -57,8 +57,12 @@ def test_forward_matches_oracle(name):
     cb = np.sort(sig + bf[None, :], axis=1)[:, ::-1]
     mag = np.abs(xf.astype(np.float64)) @ np.abs(wf.astype(np.float64)).T
     safe = (cb[:, cfg.k - 1] - cb[:, cfg.k]) > 0.5 * (1e-5 * mag.max(axis=1) + 1e-6) + 1e-6
+    # sets must agree where the margin is safe; the order inside a set can
+    # differ only between nearly tied scores, so values are compared on
+    # tokens whose ordered selection agrees
+    same_set = np.all(np.sort(gidx, axis=1) == np.sort(ref["topk_idx"], axis=1), axis=1)
+    assert np.all(same_set[safe])
     same = np.all(gidx == ref["topk_idx"], axis=1)
-    assert np.all(same[safe])
     assert same.mean() >= 0.97
     assert np.all(np.abs(host(dbg["logits"]) - L) <= 1e-5 * mag + 1e-6)
     np.testing.assert_allclose(gw[same], ref["topk_w"][same], rtol=2e-5)
