@@ -9,6 +9,7 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <stdint.h>
 
@@ -89,21 +90,72 @@ NVDEV float e4m3_value(uint32_t code) {
   return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
 }
 
-// Quantise one 16-element block under global scale g (d = 6 g), one IEEE
-// rounding per step:  s = E4M3(amax / d);  S = s * g;  inv = 1 / S;
-// q_i = E2M1(x_i * inv).  Zero d or S gives scale code 0 and codes +-0.
-// Returns the scale code; writes 8 bytes of packed codes.
+// Two independent IEEE fp32 multiplies (round to nearest) in one instruction.
+NVDEV uint64_t mul_f32x2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+NVDEV uint64_t pack_f32x2(float lo, float hi) {
+  return (uint64_t)__float_as_uint(lo) | ((uint64_t)__float_as_uint(hi) << 32);
+}
+NVDEV float lo_f32(uint64_t p) { return __uint_as_float((uint32_t)p); }
+NVDEV float hi_f32(uint64_t p) { return __uint_as_float((uint32_t)(p >> 32)); }
+
+// The block scale of R2: s = E4M3(amax / d), S = s * g, inv = 1 / S (zero d
+// or S gives s = 0 and inv = 0).
+NVDEV uint32_t block_scale(float amax, float g, float d, float& inv) {
+  const float s_raw = (d == 0.0f) ? 0.0f : __fdiv_rn(amax, d);
+  const uint32_t s = e4m3_code(s_raw);
+  const float S = __fmul_rn(e4m3_value(s), g);
+  inv = (S == 0.0f) ? 0.0f : __frcp_rn(S);
+  return s;
+}
+
+// Quantise one 16-element block of fp32 values under global scale g
+// (d = 6 g), one IEEE rounding per step:  s = E4M3(amax / d);  S = s * g;
+// inv = 1 / S;  q_i = E2M1(x_i * inv).  Returns the scale code; writes 8
+// bytes of packed codes.
 NVDEV uint32_t quant_block16(const float* v, float g, float d, uint2& codes) {
   float amax = 0.0f;
 #pragma unroll
   for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
-  const float s_raw = (d == 0.0f) ? 0.0f : __fdiv_rn(amax, d);
-  const uint32_t s = e4m3_code(s_raw);
-  const float S = __fmul_rn(e4m3_value(s), g);
-  const float inv = (S == 0.0f) ? 0.0f : __frcp_rn(S);
+  float inv;
+  const uint32_t s = block_scale(amax, g, d, inv);
+  const uint64_t inv2 = pack_f32x2(inv, inv);
   float y[16];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) y[i] = __fmul_rn(v[i], inv);
+  for (int i = 0; i < 16; i += 2) {
+    const uint64_t r = mul_f32x2(pack_f32x2(v[i], v[i + 1]), inv2);
+    y[i] = lo_f32(r);
+    y[i + 1] = hi_f32(r);
+  }
+  codes.x = e2m1x8_hw(y);
+  codes.y = e2m1x8_hw(y + 8);
+  return s;
+}
+
+// max |x| of eight packed bf16 pairs (exact: a bf16 maximum), as fp32.
+NVDEV float amax16_bf16(const uint32_t* w) {
+  __nv_bfloat162 m = __habs2(*reinterpret_cast<const __nv_bfloat162*>(&w[0]));
+#pragma unroll
+  for (int i = 1; i < 8; ++i) m = __hmax2(m, __habs2(*reinterpret_cast<const __nv_bfloat162*>(&w[i])));
+  return fmaxf(__low2float(m), __high2float(m));
+}
+
+// The same quantisation of a block given as 16 packed bf16 values (32 bytes).
+NVDEV uint32_t quant_block16_bf16(const uint4& u0, const uint4& u1, float g, float d, uint2& codes) {
+  const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+  float inv;
+  const uint32_t s = block_scale(amax16_bf16(w), g, d, inv);
+  const uint64_t inv2 = pack_f32x2(inv, inv);
+  float y[16];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint64_t r = mul_f32x2(((uint64_t)(w[i] & 0xFFFF0000u) << 32) | (uint64_t)(w[i] << 16), inv2);
+    y[2 * i] = lo_f32(r);
+    y[2 * i + 1] = hi_f32(r);
+  }
   codes.x = e2m1x8_hw(y);
   codes.y = e2m1x8_hw(y + 8);
   return s;

@@ -34,11 +34,8 @@ __global__ void __launch_bounds__(128) quantize_scatter_kernel(const uint4* __re
     uint2 c = make_uint2(0, 0);
     uint32_t s = 0;
     if (valid) {
-      float v[16];
       const uint4* src = x + ((size_t)t * H + (size_t)kb * kQBlock) / 8;
-      unpack_bf16x8(__ldg(src), v);
-      unpack_bf16x8(__ldg(src + 1), v + 8);
-      s = quant_block16(v, g, d, c);
+      s = quant_block16_bf16(__ldg(src), __ldg(src + 1), g, d, c);
     }
     uint32_t w1 = __shfl_down_sync(0xffffffffu, s, 1);
     uint32_t w2 = __shfl_down_sync(0xffffffffu, s, 2);

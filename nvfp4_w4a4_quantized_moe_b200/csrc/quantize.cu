@@ -63,12 +63,9 @@ __global__ void __launch_bounds__(256) quantize_act_kernel(const uint4* __restri
     if (valid) {
       row = (int)(i / nblk);
       kb = (int)(i % nblk);
-      float v[16];
       const uint4 u0 = __ldg(x + i * 2), u1 = __ldg(x + i * 2 + 1);
-      unpack_bf16x8(u0, v);
-      unpack_bf16x8(u1, v + 8);
       uint2 c;
-      s = quant_block16(v, g, d, c);
+      s = quant_block16_bf16(u0, u1, g, d, c);
       codes[i] = c;
     }
     store_scales<1>(scales, layout, row, kb, nblk, &s, valid);
@@ -101,7 +98,7 @@ __global__ void zero_tiled_scale_rows(uint8_t* scales, int rows, int padded_rows
 constexpr int kWAmax = 256;                     // amax threads per CTA (the DRAM stream)
 constexpr int kWQuant = 256;                    // quantise threads per CTA (re-read from L2)
 constexpr int kWThreads = kWAmax + kWQuant;
-constexpr int kWAhead = 2;                      // amax may lead quantise by this many matrices
+constexpr int kWAhead = 1;                      // amax may lead quantise by this many matrices
 
 struct WeightQuantState {
   uint32_t status;          // device status word (first word of the workspace)
@@ -174,26 +171,23 @@ __global__ void __launch_bounds__(kWThreads) quantize_weights_kernel(
       if (!s_ok_amax) break;
       const uint4* src = w + (long long)mat * per_mat / 8;
       const long long v1 = b_end * 2;                          // uint4 range (8 bf16 each)
-      float m = 0.0f;
+      // running max of |x| on packed bf16 pairs (exact)
+      __nv_bfloat162 m2 = __floats2bfloat162_rn(0.0f, 0.0f);
+      auto absmax4 = [&](const uint4& u) {
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) m2 = __hmax2(m2, __habs2(*reinterpret_cast<const __nv_bfloat162*>(&w[j])));
+      };
       long long i = b_begin * 2 + gt;
       for (; i + 7 * kWAmax < v1; i += 8 * kWAmax) {
         uint4 u[8];
 #pragma unroll
         for (int q = 0; q < 8; ++q) u[q] = ld_hint(src + i + q * kWAmax, keep);
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          float v[8];
-          unpack_bf16x8(u[q], v);
-#pragma unroll
-          for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(v[j]));
-        }
+        for (int q = 0; q < 8; ++q) absmax4(u[q]);
       }
-      for (; i < v1; i += kWAmax) {
-        float v[8];
-        unpack_bf16x8(ld_hint(src + i, keep), v);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(v[j]));
-      }
+      for (; i < v1; i += kWAmax) absmax4(ld_hint(src + i, keep));
+      const float m = fmaxf(__low2float(m2), __high2float(m2));
       uint32_t mb = __float_as_uint(m);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, o));
@@ -233,6 +227,7 @@ __global__ void __launch_bounds__(kWThreads) quantize_weights_kernel(
       const float d = __fmul_rn(6.0f, g);
       if (blockIdx.x == 0 && gt == 0) gscale[mat] = g;
       const uint4* src = w + (long long)mat * per_mat / 8;
+      const float inv_nblk = 1.0f / (float)nblk;
       // every lane of a warp runs the same number of iterations (shuffles
       // below); each iteration has two blocks per thread in flight
       const long long n_iter = (b_end - b_begin + 2 * kWQuant - 1) / (2 * kWQuant);
@@ -254,14 +249,18 @@ __global__ void __launch_bounds__(kWThreads) quantize_weights_kernel(
           uint32_t sc = 0;
           int row = 0, kb = 0;
           if (valid[q]) {
-            float v[16];
-            unpack_bf16x8(u[q][0], v);
-            unpack_bf16x8(u[q][1], v + 8);
             uint2 c;
-            sc = quant_block16(v, g, d, c);
+            sc = quant_block16_bf16(u[q][0], u[q][1], g, d, c);
             codes[(long long)mat * blocks + b[q]] = c;
-            row = (int)(b[q] / nblk);
-            kb = (int)(b[q] % nblk);
+            // b < 2^24 (checked on the host): a float quotient off by at most
+            // one, then an exact integer correction
+            const uint32_t bb = (uint32_t)b[q];
+            uint32_t qt = (uint32_t)__fmul_rz((float)bb, inv_nblk);
+            int32_t rem = (int32_t)(bb - qt * (uint32_t)nblk);
+            if (rem < 0) { --qt; rem += nblk; }
+            if (rem >= nblk) { ++qt; rem -= nblk; }
+            row = (int)qt;
+            kb = rem;
           }
           store_scales<1>(scales, layout, mat * rows + row, kb, nblk, &sc, valid[q]);
         }
@@ -349,7 +348,7 @@ extern "C" nvfp4_status nvfp4_quantize_weights(const void* w_bf16, int n_mats, i
   NV_REQUIRE(layout == NVFP4_LAYOUT_CANONICAL || (cols % 64 == 0 && rows % 128 == 0), NVFP4_ERR_UNSUPPORTED_SHAPE,
              "nvfp4_quantize_weights: the tiled layout needs rows %% 128 == 0 and cols %% 64 == 0 (got %d x %d)", rows,
              cols);
-  NV_REQUIRE((long long)rows * cols < (1ll << 40) && n_mats < (1 << 24),
+  NV_REQUIRE((long long)rows * cols / 16 < (1ll << 24) && n_mats < (1 << 24),
              NVFP4_ERR_UNSUPPORTED_SHAPE, "nvfp4_quantize_weights: too many elements");
   const size_t need = nvfp4_quantize_weights_workspace_size(n_mats);
   NV_REQUIRE(ws != nullptr && ws_bytes >= need && aligned(ws, 256), NVFP4_ERR_WORKSPACE,
@@ -426,7 +425,7 @@ extern "C" nvfp4_status nvfp4_quantize_weights_noalloc(const void* w_bf16, int n
              "nvfp4_quantize_weights_noalloc: cols=%d must be a multiple of 32", cols);
   NV_REQUIRE(layout == NVFP4_LAYOUT_CANONICAL || (cols % 64 == 0 && rows % 128 == 0), NVFP4_ERR_UNSUPPORTED_SHAPE,
              "nvfp4_quantize_weights_noalloc: the tiled layout needs rows %% 128 == 0 and cols %% 64 == 0");
-  NV_REQUIRE((long long)rows * cols < (1ll << 40) && n_mats < (1 << 24),
+  NV_REQUIRE((long long)rows * cols / 16 < (1ll << 24) && n_mats < (1 << 24),
              NVFP4_ERR_UNSUPPORTED_SHAPE, "nvfp4_quantize_weights_noalloc: too many elements");
   NV_REQUIRE(aligned(w_bf16, 16) && aligned(codes, 16) && aligned(scales, 4), NVFP4_ERR_INVALID_ARG,
              "nvfp4_quantize_weights_noalloc: w and codes need 16-byte alignment, scales 4-byte");
