@@ -155,15 +155,25 @@ class ClockSampler:
 # traffic of the dominant kernel, from the committed ncu summary
 # ---------------------------------------------------------------------------
 
+GEMM_SOURCES = ("gemm.cu", "gemm.cuh", "common.cuh")
+
+
+def gemm_source_sha() -> str:
+    """Hash of the sources the GEMM kernel is compiled from."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in GEMM_SOURCES:
+        h.update(open(os.path.join(ROOT, "nvfp4_w4a4_quantized_moe_b200", "csrc", name), "rb").read())
+    return h.hexdigest()[:16]
+
+
 def recorded_traffic(kernel: str, workload: str):
     """dram bytes per launch recorded by ncu for this kernel and workload, or
     None when no record exists or the kernel source changed since."""
-    import hashlib
     path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     if not os.path.exists(path):
         return None
-    src = os.path.join(ROOT, "nvfp4_w4a4_quantized_moe_b200", "csrc", "gemm.cu")
-    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    sha = gemm_source_sha()
     for line in open(path):
         f = dict(kv.split("=", 1) for kv in line.split() if "=" in kv)
         if f.get("kernel") == kernel and f.get("workload") == workload and f.get("source_sha") == sha:
@@ -181,12 +191,17 @@ def _oracle_quantize_expert(args):
 
 
 class OracleSample:
-    """The oracle's layer on a bounded sample: the first token of the batch.
-    The sampled token's experts are quantised by the oracle beforehand
-    (untimed, in a spawn pool); the timed part is the oracle's forward."""
+    """The oracle's layer on a bounded sample of the batch: its first token.
+
+    One step is one (token, expert) pair of that token, cycling through its k
+    experts: the token's routing and x quantisation, then that expert's
+    gate/up, SiLU(gate)*up, requantisation, down and weighted contribution, in
+    the order the oracle's layer takes them.  k steps make one token, so the
+    rate in tokens/s is pairs/s / k.  The token's experts are quantised by the
+    oracle beforehand (untimed, in a spawn pool)."""
 
     def __init__(self, cfg, seed, x, wg, bias, off):
-        from oracle import moe
+        from oracle import moe, nvfp4
         self.cfg = cfg
         self.x = x[:1].float().cpu().numpy()
         self.wg = wg.float().cpu().numpy()
@@ -207,11 +222,30 @@ class OracleSample:
         cal = moe.moe_layer(self.x, self.wg, self.bias, cfg.k, cfg.rsf, lambda e: self.q[e], self.g1,
                             np.float32(1.0), logit_offset=self.off)
         self.g2 = np.float32(np.float32(max(np.abs(h).max() for h in cal["h"].values())) / np.float32(2688))
+        self.slot = 0
+        self.out = np.zeros(self.x.shape, np.float64)
+        self._nvfp4 = nvfp4
 
     def step(self):
+        """One (token, expert) pair; returns the token's partial output."""
         from oracle import moe
-        return moe.moe_layer(self.x, self.wg, self.bias, self.cfg.k, self.cfg.rsf, lambda e: self.q[e], self.g1,
-                             self.g2, logit_offset=self.off)["out"]
+        nvfp4 = self._nvfp4
+        j = self.slot
+        self.slot = (j + 1) % self.cfg.k
+        logits = moe.router_logits(self.x, self.wg, self.off)
+        idx, w = moe.route(logits, self.bias, self.cfg.k, self.cfg.rsf)
+        a_codes, a_scales = nvfp4.quantize(self.x, self.g1)
+        gate, up, down = self.q[int(idx[0, j])]
+        _, _, h = moe.expert_gate_up(a_codes, a_scales, self.g1, gate, up)
+        hc, hs = nvfp4.quantize(h, self.g2)
+        y = moe.expert_down(hc, hs, self.g2, down)
+        if j == 0:
+            self.out[:] = 0.0
+        self.out[0] += float(w[0, j]) * y[0]
+        return self.out
+
+    def tokens_per_step(self):
+        return 1.0 / self.cfg.k
 
     @staticmethod
     def threads():
@@ -223,8 +257,10 @@ class OracleSample:
 
 
 def sample_desc(cfg):
-    return (f"1 token of the {cfg.name} batch (routing, x quantisation, its {cfg.k} experts' gate/up/down on "
-            f"dequantised NVFP4 operands in fp64, combine); its experts quantised by the oracle beforehand, untimed")
+    return (f"token 0 of the {cfg.name} batch, one (token, expert) pair per step cycling through its {cfg.k} "
+            f"experts (routing, x quantisation, the expert's gate/up, SiLU*up, requantisation and down on "
+            f"dequantised NVFP4 operands in fp64, weighted add); tokens/s = pairs/s / {cfg.k}; the token's "
+            f"experts quantised by the oracle beforehand, untimed")
 
 
 def run_reference(args, cfg):
@@ -239,11 +275,11 @@ def run_reference(args, cfg):
     for _ in range(args.steps):
         smp.step()
     dt = (time.perf_counter() - t0) / args.steps
-    v = 1.0 / dt
+    v = smp.tokens_per_step() / dt
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": cfg.name, "tokens_per_step": 1, "T": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E,
+            "config": {"workload": cfg.name, "tokens_per_step": 1.0 / cfg.k, "T": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E,
                        "k": cfg.k},
             "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": OracleSample.threads(), "kind": "oracle",
                              "sample": sample_desc(cfg)},
@@ -394,12 +430,12 @@ def run_ours(args, cfg):
         smp.step()
         t = time.perf_counter()
         n = 0
-        while n < 1 or time.perf_counter() - t < 10.0:
+        while n < cfg.k or time.perf_counter() - t < 10.0:
             smp.step()
             n += 1
         dt = (time.perf_counter() - t) / n
-        cpu = {"value": 1.0 / dt, "unit": "tokens/s", "cores": OracleSample.threads(), "kind": "oracle",
-               "sample": sample_desc(cfg) + f"; {n} repetitions"}
+        cpu = {"value": smp.tokens_per_step() / dt, "unit": "tokens/s", "cores": OracleSample.threads(), "kind": "oracle",
+               "sample": sample_desc(cfg) + f"; {n} pairs timed"}
 
     tokens = cfg.T * dist.world
     line = {
@@ -436,20 +472,24 @@ def weak_scaling_value(tokens_per_rank: int, world: int, max_ms_per_step: float)
     return tokens_per_rank * world / (max_ms_per_step * 1e-3)
 
 
+MMA_PEAK_MODES = {
+    0: "", 1: "_scale_copies_one_buffer", 5: "_stage_handshake", 6: "_stage_handshake_scale_copies",
+    9: "_8_stages", 10: "_8_stages_scale_copies", 13: "_scale_copies_commit", 14: "_commit",
+    15: "_scale_copies_fence", 16: "_scale_copies_commit_every_2nd", 17: "_split_issue",
+    18: "_split_issue_handshake", 19: "_warp_predicated_scale_copies", 20: "_warp_predicated",
+    21: "_warp_branch_scale_copies",
+}
+
+
 def run_mma_peak():
     """FP4 MMA rate per SM clock with operands resident in shared memory."""
     from nvfp4_w4a4_quantized_moe_b200 import capi as c
     res = {}
     for n in (256, 128):
-        for cp in (0, 1, 5, 6, 9, 10, 11, 12):
-            c.nvfp4_test_mma_peak(200, n, cp)                      # warm-up
-            fpc, cyc = c.nvfp4_test_mma_peak(20000, n, cp)
-            res[f"n{n}" + ("", "_scale_copies_one_buffer", "_scale_copies_4_buffers",
-                           "_scale_copies_one_stage_ahead", "_scale_copies_6_wide", "_stage_handshake",
-                           "_stage_handshake_scale_copies", "_stage_handshake_spin",
-                           "_stage_handshake_spin_scale_copies", "_8_stages", "_8_stages_scale_copies",
-                           "_8_half_stages", "_8_half_stages_scale_copies")[cp]] = {
-                "flop_per_sm_clock": float(fpc.median()), "cycles_median": float(cyc.median())}
+        for mode, name in MMA_PEAK_MODES.items():
+            c.nvfp4_test_mma_peak(200, n, mode)                    # warm-up
+            fpc, cyc = c.nvfp4_test_mma_peak(20000, n, mode)
+            res[f"n{n}{name}"] = {"flop_per_sm_clock": float(fpc.median()), "cycles_median": float(cyc.median())}
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     best = max(v["flop_per_sm_clock"] for v in res.values())
     print(json.dumps({"mma_peak": res, "sms": sms,

@@ -37,12 +37,24 @@ NVFP4_API nvfp4_status nvfp4_test_e4m3(const float* s, int n, uint8_t* codes, fl
 
 /* FP4 tensor-core rate without memory traffic: `ctas` CTAs (at most one per
  * SM) each issue `iters` x 4 block-scaled 128 x n x 64 MMAs (n = 128 or 256)
- * from fixed shared-memory operands, without (with_cp == 0) or with the 12
- * scale-factor copies of a 256-wide K stage before every 4 MMAs, into one set
- * of tensor-memory columns (with_cp == 1) or rotating over four sets
- * (with_cp == 2).
+ * from fixed shared-memory operands.  with_cp selects what else one issuing
+ * thread does per 4 MMAs (one 256-wide K stage):
+ *   0 nothing; 1 the stage's 12 scale-factor copies into one set of tensor
+ *   memory columns; 2 the same rotating over four sets; 3 copies issued one
+ *   stage ahead; 4 six 128-lane x 256-bit copies instead of twelve;
+ *   5/6 (without/with copies) a full/empty mbarrier handshake with a second
+ *   thread over 4 stages, 9/10 over 8 stages, 7/8 with spinning waits,
+ *   11/12 over 8 stages of 2 MMAs; 13 copies and a tcgen05.commit (no wait);
+ *   14 a commit only; 15 copies and a tcgen05 after-thread-sync fence;
+ *   16 copies and a commit every second stage; 17 split issue: this thread
+ *   issues only the MMAs and a second thread the copies, into two
+ *   alternating column sets, with mbarrier handshakes; 18 the same plus a
+ *   full/empty handshake with a third thread; 19-21 the whole warp runs
+ *   the loop and one elected lane issues: 19 copies and MMAs as predicated
+ *   instructions, 20 MMAs only, 21 copies and MMAs in a branch.
  * cycles[c] (device uint64) = SM clock cycles CTA c spent; *status (device
- * uint32) is set non-zero if the final wait gave up. */
+ * uint32) is set non-zero if a wait gave up.  INVALID_ARG for with_cp outside
+ * [0, 21]. */
 NVFP4_API nvfp4_status nvfp4_test_mma_peak(int iters, int n, int with_cp, int ctas, unsigned long long* cycles,
                                            uint32_t* status, void* stream);
 

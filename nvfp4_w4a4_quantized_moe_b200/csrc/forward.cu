@@ -20,6 +20,7 @@ __global__ void __launch_bounds__(128) quantize_scatter_kernel(const uint4* __re
                                                                const int32_t* __restrict__ inv_perm, int k,
                                                                uint2* __restrict__ a_codes,
                                                                uint8_t* __restrict__ a_scales) {
+  // block (t, by): token t, 16-element blocks [128 by, 128 by + 128) of its row
   __shared__ int32_t rows[16];
   const int t = blockIdx.x;
   if (threadIdx.x < k) rows[threadIdx.x] = inv_perm[(size_t)t * k + threadIdx.x];
@@ -28,46 +29,58 @@ __global__ void __launch_bounds__(128) quantize_scatter_kernel(const uint4* __re
   const float d = __fmul_rn(6.0f, g);
   const int nblk = H / kQBlock;
   const int lane = threadIdx.x & 31;
-  for (int kb0 = 0; kb0 < nblk; kb0 += blockDim.x) {
-    const int kb = kb0 + threadIdx.x;
-    const bool valid = kb < nblk;
-    uint2 c = make_uint2(0, 0);
-    uint32_t s = 0;
-    if (valid) {
-      const uint4* src = x + ((size_t)t * H + (size_t)kb * kQBlock) / 8;
-      s = quant_block16_bf16(__ldg(src), __ldg(src + 1), g, d, c);
-    }
-    uint32_t w1 = __shfl_down_sync(0xffffffffu, s, 1);
-    uint32_t w2 = __shfl_down_sync(0xffffffffu, s, 2);
-    uint32_t w3 = __shfl_down_sync(0xffffffffu, s, 3);
-    const uint32_t word = s | (w1 << 8) | (w2 << 16) | (w3 << 24);
-    if (valid) {
-      for (int j = 0; j < k; ++j) {
-        const int row = rows[j];
-        a_codes[(size_t)row * nblk + kb] = c;
-        if ((lane & 3) == 0)
-          *reinterpret_cast<uint32_t*>(a_scales + tiled_scale_offset(row, kb, nblk >> 2)) = word;
-      }
+  const int kb = blockIdx.y * blockDim.x + threadIdx.x;
+  const bool valid = kb < nblk;
+  uint2 c = make_uint2(0, 0);
+  uint32_t s = 0;
+  if (valid) {
+    const uint4* src = x + ((size_t)t * H + (size_t)kb * kQBlock) / 8;
+    s = quant_block16_bf16(__ldg(src), __ldg(src + 1), g, d, c);
+  }
+  const uint32_t w1 = __shfl_down_sync(0xffffffffu, s, 1);
+  const uint32_t w2 = __shfl_down_sync(0xffffffffu, s, 2);
+  const uint32_t w3 = __shfl_down_sync(0xffffffffu, s, 3);
+  const uint32_t word = s | (w1 << 8) | (w2 << 16) | (w3 << 24);
+  if (valid) {
+    for (int j = 0; j < k; ++j) {
+      const int row = rows[j];
+      a_codes[(size_t)row * nblk + kb] = c;
+      if ((lane & 3) == 0)
+        *reinterpret_cast<uint32_t*>(a_scales + tiled_scale_offset(row, kb, nblk >> 2)) = word;
     }
   }
 }
 
 // out[t] = bf16( sum_j y[inv_perm[t, j]] ), fp32 sum in slot order.  The
 // routing weight is already folded into y by the down-projection epilogue.
-__global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ inv_perm,
-                                                      int T, int H, int k, uint4* __restrict__ out) {
+// Block (t, by) covers token t's 8-column groups by*blockDim.x + i*gridDim.y*
+// blockDim.x (+ threadIdx.x): a small batch spreads a row over several
+// blocks, a large one keeps whole rows in one block for long contiguous
+// reads.  A thread issues all k row loads of a column group before adding.
+constexpr int kCombineThreads = 256;
+
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(const uint4* __restrict__ y,
+                                                                  const int32_t* __restrict__ inv_perm, int T, int H,
+                                                                  int k, uint4* __restrict__ out) {
   __shared__ int32_t rows[16];
   const int t = blockIdx.x;
   if (threadIdx.x < k) rows[threadIdx.x] = inv_perm[(size_t)t * k + threadIdx.x];
   __syncthreads();
   const int vpr = H / 8;
-  for (int c = threadIdx.x; c < vpr; c += blockDim.x) {
-    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    for (int j = 0; j < k; ++j) {
-      float v[8];
-      unpack_bf16x8(__ldg(y + (size_t)rows[j] * vpr + c), v);
+  for (int c = blockIdx.y * blockDim.x + threadIdx.x; c < vpr; c += gridDim.y * blockDim.x) {
+    uint4 v[16];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) acc[q] = __fadd_rn(acc[q], v[q]);
+    for (int j = 0; j < 16; ++j)
+      if (j < k) v[j] = __ldg(y + (size_t)rows[j] * vpr + c);
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      if (j < k) {
+        float f[8];
+        unpack_bf16x8(v[j], f);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[q] = __fadd_rn(acc[q], f[q]);
+      }
     }
     out[(size_t)t * vpr + c] = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
                                           pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
@@ -173,7 +186,7 @@ extern "C" nvfp4_status moe_nvfp4_forward(const moe_nvfp4_weights* W, const void
   // 4: quantise x once per token into its k permuted rows.  Padding rows are
   // left as they are: an MMA row only feeds the same output row, and the
   // epilogues skip padding rows.
-  quantize_scatter_kernel<<<T, 128, 0, s>>>(static_cast<const uint4*>(x_bf16), T, H, act_gscale, f.inv_perm, k,
+  quantize_scatter_kernel<<<dim3(T, (H / kQBlock + 127) / 128), 128, 0, s>>>(static_cast<const uint4*>(x_bf16), T, H, act_gscale, f.inv_perm, k,
                                             reinterpret_cast<uint2*>(f.a_codes), f.a_scales);
   NV_CHECK(check_launch("quantize_scatter_kernel"));
   NV_CHECK(mark(dbg, 2, s));
@@ -212,7 +225,9 @@ extern "C" nvfp4_status moe_nvfp4_forward(const moe_nvfp4_weights* W, const void
   NV_CHECK(mark(dbg, 4, s));
 
   // 8: combine
-  combine_kernel<<<T, 256, 0, s>>>(reinterpret_cast<const uint4*>(f.y), f.inv_perm, T, H, k,
+  // below about two waves of whole-row blocks, split rows across blocks
+  const int row_blocks = T >= 2 * sms ? 1 : (H / 8 + kCombineThreads - 1) / kCombineThreads;
+  combine_kernel<<<dim3(T, row_blocks), kCombineThreads, 0, s>>>(reinterpret_cast<const uint4*>(f.y), f.inv_perm, T, H, k,
                                    static_cast<uint4*>(out_bf16));
   NV_CHECK(check_launch("combine_kernel"));
   NV_CHECK(mark(dbg, 5, s));

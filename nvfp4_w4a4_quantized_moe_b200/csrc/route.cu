@@ -182,31 +182,43 @@ __global__ void __launch_bounds__(kRThreads, 1)
 // ---------------------------------------------------------------------------
 constexpr int kMaxE = 256, kMaxK = 16;
 
-// With splits > 0 the logits are the split-ordered sum of the router GEMM's
-// partial sums (plus the optional offset) and are written to `logits`; with
+// Logit of (token t, expert e).  With splits > 0 it is the split-ordered sum
+// of the router GEMM's partial sums (plus the optional offset), loaded eight
+// splits at a time so the loads overlap, and is written to `logits`; with
 // splits == 0 `src` already holds the logits.
-__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ src, int splits,
-                                                   const float* __restrict__ offset, float* __restrict__ logits,
-                                                   const float* __restrict__ bias, int T, int E, int k, float rsf,
-                                                   int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
-  const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (t >= T) return;
+NVDEV float token_logit(const float* __restrict__ src, int splits, const float* __restrict__ offset,
+                        float* __restrict__ logits, int T, int E, int t, int e) {
+  const float* p = src + (size_t)t * E + e;
+  if (splits == 0) return *p;
+  const size_t stride = (size_t)T * E;
+  float l = p[0];
+  int q = 1;
+  for (; q + 8 <= splits; q += 8) {
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = p[(size_t)(q + u) * stride];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) l = __fadd_rn(l, v[u]);
+  }
+  for (; q < splits; ++q) l = __fadd_rn(l, p[(size_t)q * stride]);
+  if (offset) l = __fadd_rn(l, offset[e]);
+  logits[(size_t)t * E + e] = l;
+  return l;
+}
+
+// Top-k of token t by one warp.  Lane l holds experts l, l+32, ...; each of
+// the k rounds is a warp-wide argmax of sigma + bias (ties to the lower
+// expert).  Lane j < k returns slot j's expert and weight.
+NVDEV void topk_token(const float* __restrict__ src, int splits, const float* __restrict__ offset,
+                      float* __restrict__ logits, const float* __restrict__ bias, int T, int E, int k, float rsf,
+                      int t, int lane, int& out_idx, float& out_w) {
   float sig[kMaxE / 32], c[kMaxE / 32];
   const int per = (E + 31) >> 5;
 #pragma unroll
   for (int i = 0; i < kMaxE / 32; ++i) {
     const int e = lane + 32 * i;
     if (i < per && e < E) {
-      float l;
-      if (splits > 0) {
-        l = src[(size_t)t * E + e];
-        for (int q = 1; q < splits; ++q) l = __fadd_rn(l, src[((size_t)q * T + t) * E + e]);
-        if (offset) l = __fadd_rn(l, offset[e]);
-        logits[(size_t)t * E + e] = l;
-      } else {
-        l = src[(size_t)t * E + e];
-      }
+      const float l = token_logit(src, splits, offset, logits, T, E, t, e);
       sig[i] = sigmoid_fixed(l);
       c[i] = __fadd_rn(sig[i], bias[e]);
     } else {
@@ -252,9 +264,23 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ src
       my_idx = be;
     }
   }
+  out_idx = my_idx;
+  out_w = __fmul_rn(__fdiv_rn(my_sig, sum), rsf);
+}
+
+__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ src, int splits,
+                                                   const float* __restrict__ offset, float* __restrict__ logits,
+                                                   const float* __restrict__ bias, int T, int E, int k, float rsf,
+                                                   int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;
+  int idx;
+  float w;
+  topk_token(src, splits, offset, logits, bias, T, E, k, rsf, t, lane, idx, w);
   if (lane < k) {
-    topk_idx[(size_t)t * k + lane] = my_idx;
-    topk_w[(size_t)t * k + lane] = __fmul_rn(__fdiv_rn(my_sig, sum), rsf);
+    topk_idx[(size_t)t * k + lane] = idx;
+    topk_w[(size_t)t * k + lane] = w;
   }
 }
 
@@ -348,6 +374,81 @@ __global__ void __launch_bounds__(kChunk) perm_scatter_kernel(const int32_t* __r
   }
 }
 
+// ---------------------------------------------------------------------------
+// Routing of a small batch (T <= 256) in one block: top-k, per-expert counts,
+// the padded scan, and the scatter, with the padding fill of perm and row_w
+// that the large-batch path leaves to memsets.  The arithmetic is the same
+// (topk_token) and so is every integer result.
+// ---------------------------------------------------------------------------
+constexpr int kSmallT = 256;
+constexpr int kSmallThreads = 1024;
+
+__global__ void __launch_bounds__(kSmallThreads, 1)
+    route_small_kernel(const float* __restrict__ src, int splits, const float* __restrict__ offset,
+                       float* __restrict__ logits, const float* __restrict__ bias, int T, int E, int k, float rsf,
+                       int cap, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
+                       int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                       int32_t* __restrict__ tile_expert, int32_t* __restrict__ num_mtiles,
+                       int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm, float* __restrict__ row_w) {
+  __shared__ uint32_t bm[kMaxE][kSmallT / 32];
+  __shared__ int32_t sp[256];
+  __shared__ int32_t base[kMaxE];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int i = tid; i < E * (kSmallT / 32); i += blockDim.x) bm[i / (kSmallT / 32)][i % (kSmallT / 32)] = 0;
+  for (int i = tid; i < cap; i += blockDim.x) {
+    perm[i] = -1;
+    row_w[i] = 0.0f;
+  }
+  __syncthreads();
+  for (int t = warp; t < T; t += blockDim.x >> 5) {
+    int idx;
+    float w;
+    topk_token(src, splits, offset, logits, bias, T, E, k, rsf, t, lane, idx, w);
+    if (lane < k) {
+      topk_idx[(size_t)t * k + lane] = idx;
+      topk_w[(size_t)t * k + lane] = w;
+      atomicOr(&bm[idx][t >> 5], 1u << (t & 31));
+    }
+  }
+  __syncthreads();
+  // per-expert totals, 128-row padding, exclusive scan (threads 0..255)
+  int total = 0, padded = 0;
+  if (tid < E)
+    for (int w = 0; w < kSmallT / 32; ++w) total += __popc(bm[tid][w]);
+  padded = (total + kRowTile - 1) / kRowTile * kRowTile;
+  if (tid < 256) sp[tid] = tid < E ? padded : 0;
+  __syncthreads();
+  for (int o = 1; o < 256; o <<= 1) {
+    const int v = (tid < 256 && tid >= o) ? sp[tid - o] : 0;
+    __syncthreads();
+    if (tid < 256) sp[tid] += v;
+    __syncthreads();
+  }
+  if (tid < E) {
+    const int start = sp[tid] - padded;
+    base[tid] = start;
+    offsets[tid] = start;
+    counts[tid] = total;
+    for (int m = start / kRowTile; m < (start + padded) / kRowTile; ++m) tile_expert[m] = tid;
+    if (tid == E - 1) {
+      offsets[E] = start + padded;
+      *num_mtiles = (start + padded) / kRowTile;
+    }
+  }
+  __syncthreads();
+  // stable scatter: rank of token t among the tokens of expert e
+  for (int i = tid; i < T * k; i += blockDim.x) {
+    const int t = i / k;
+    const int e = topk_idx[i];
+    int rank = __popc(bm[e][t >> 5] & ((1u << (t & 31)) - 1u));
+    for (int w = 0; w < (t >> 5); ++w) rank += __popc(bm[e][w]);
+    const int row = base[e] + rank;
+    perm[row] = t;
+    inv_perm[i] = row;
+    row_w[row] = topk_w[i];
+  }
+}
+
 RouteScratch carve_route_scratch(Carver& c, int T, int E, int k) {
   RouteScratch r;
   const int nchunks = (T + kChunk - 1) / kChunk;
@@ -392,6 +493,13 @@ nvfp4_status launch_route(const RouteArgs& a, const RouteScratch& r, cudaStream_
     dim3 grid((a.T + kRBM - 1) / kRBM, splits);
     router_gemm_kernel<<<grid, kRThreads, smem, s>>>(tmX, tmW, p);
     NV_CHECK(check_launch("router_gemm_kernel"));
+  }
+  if (a.T <= kSmallT) {
+    route_small_kernel<<<1, kSmallThreads, 0, s>>>(splits ? r.partial : a.logits, splits, a.logit_offset, a.logits,
+                                                   a.bias, a.T, a.E, a.k, a.rsf, cap, a.topk_idx, a.topk_w, r.counts,
+                                                   a.expert_offsets, r.tile_expert, r.num_mtiles, a.perm,
+                                                   a.inv_perm, r.row_w);
+    return check_launch("route_small_kernel");
   }
   NV_CHECK(check_cuda(cudaMemsetAsync(a.perm, 0xFF, sizeof(int32_t) * (size_t)cap, s), "memset perm"));
   NV_CHECK(check_cuda(cudaMemsetAsync(r.row_w, 0, sizeof(float) * (size_t)cap, s), "memset row_w"));

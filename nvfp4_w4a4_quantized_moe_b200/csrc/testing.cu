@@ -66,6 +66,26 @@ __global__ void test_sigmoid_kernel(const float* l, int n, float* out) {
   if (i < n) out[i] = sigmoid_fixed(l[i]);
 }
 
+// Issue helpers for a whole warp: every lane executes the instruction, only
+// the lane whose `leader` is non-zero issues it.
+NVDEV void mma_fp4_pred(uint32_t leader, uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                        uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.ne.b32 q, %7, 0;\n\t"
+      "@q tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::
+          "r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem), "r"(leader));
+}
+NVDEV void tc_cp_scale_atom_pred(uint32_t leader, uint32_t taddr, uint64_t sdesc) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\t"
+      "setp.ne.b32 q, %2, 0;\n\t"
+      "@q tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;\n\t}" ::"r"(taddr),
+      "l"(sdesc), "r"(leader));
+}
+
 // FP4 tensor-core rate without memory traffic: one thread per CTA issues
 // `iters` groups of four 128 x N x 64 block-scaled MMAs on fixed shared-memory
 // operands (zeros), optionally preceded by the 12 scale-factor copies a
@@ -78,6 +98,8 @@ __global__ void __launch_bounds__(128, 1) mma_peak_kernel(int iters, int n, int 
   __shared__ __align__(8) uint64_t bar;
   __shared__ __align__(8) uint64_t full_bar[8];
   __shared__ __align__(8) uint64_t empty_bar[8];
+  __shared__ __align__(8) uint64_t sf_bar[2];
+  __shared__ __align__(8) uint64_t cp_drain;
   __shared__ uint32_t tmem_s;
   __shared__ int abort_s;
   const int warp = threadIdx.x >> 5;
@@ -89,6 +111,9 @@ __global__ void __launch_bounds__(128, 1) mma_peak_kernel(int iters, int n, int 
       mbar_init(&full_bar[i], 1);
       mbar_init(&empty_bar[i], 1);
     }
+    mbar_init(&sf_bar[0], 1);
+    mbar_init(&sf_bar[1], 1);
+    mbar_init(&cp_drain, 1);
     abort_s = 0;
     fence_barrier_init();
   }
@@ -101,7 +126,59 @@ __global__ void __launch_bounds__(128, 1) mma_peak_kernel(int iters, int n, int 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_s;
-  if (threadIdx.x == 32) {
+  if (warp == 1 && with_cp >= 19) {
+    // the whole warp runs the loop; one elected lane issues (19: copies and
+    // MMAs predicated; 20: MMAs only, predicated; 21: copies and MMAs inside
+    // a branch taken by the elected lane)
+    const uint32_t leader = elect_one();
+    const uint32_t sA = smem_u32(smem), sB = sA + 16384, sSF = sB + 32768;
+    const uint64_t adesc = sdesc_sw128(sA), bdesc = sdesc_sw128(sB);
+    const uint64_t sf0 = sdesc_scale_atom(sSF);
+    constexpr uint64_t kAtom = 512 >> 4;
+    const uint32_t idesc = idesc_fp4(128, n);
+    const uint32_t sfa = tmem + 256, sfb = tmem + 256 + 16;
+    const unsigned long long t0 = clock64();
+    if (with_cp == 19) {
+      for (int it = 0; it < iters; ++it) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          tc_cp_scale_atom_pred(leader, sfa + 4 * j, sf0 + j * kAtom);
+          tc_cp_scale_atom_pred(leader, sfb + 8 * j, sf0 + (4 + j) * kAtom);
+          tc_cp_scale_atom_pred(leader, sfb + 8 * j + 4, sf0 + (8 + j) * kAtom);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          mma_fp4_pred(leader, tmem, adesc + 2 * j, bdesc + 2 * j, idesc, sfa + 4 * j, sfb + 8 * j, (it | j) != 0);
+      }
+    } else if (with_cp == 20) {
+      for (int it = 0; it < iters; ++it) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          mma_fp4_pred(leader, tmem, adesc + 2 * j, bdesc + 2 * j, idesc, sfa + 4 * j, sfb + 8 * j, (it | j) != 0);
+      }
+    } else {
+      for (int it = 0; it < iters; ++it) {
+        if (leader) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            tc_cp_scale_atom(sfa + 4 * j, sf0 + j * kAtom);
+            tc_cp_scale_atom(sfb + 8 * j, sf0 + (4 + j) * kAtom);
+            tc_cp_scale_atom(sfb + 8 * j + 4, sf0 + (8 + j) * kAtom);
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            mma_fp4(tmem, adesc + 2 * j, bdesc + 2 * j, idesc, sfa + 4 * j, sfb + 8 * j, (it | j) != 0);
+        }
+        __syncwarp();
+      }
+    }
+    if (leader) {
+      tc_commit(&bar);
+      if (!mbar_wait(&bar, 0, &abort_s)) atomicExch(status, kDevTimeout);
+      cycles[blockIdx.x] = clock64() - t0;
+    }
+    __syncwarp();
+  } else if (threadIdx.x == 32) {
     const uint32_t sA = smem_u32(smem), sB = sA + 16384, sSF = sB + 32768;
     const uint64_t adesc = sdesc_sw128(sA), bdesc = sdesc_sw128(sB);
     const uint32_t idesc = idesc_fp4(128, n);
@@ -118,7 +195,29 @@ __global__ void __launch_bounds__(128, 1) mma_peak_kernel(int iters, int n, int 
       for (int j = 0; j < 4; ++j) tc_cp_128x256b(sf + 16 + 8 * j, sdesc_interleave(sSF + 512 * j, 128, 256));
     };
     if (with_cp == 3) copies(tmem + 256);
-    if (with_cp >= 5) {
+    if (with_cp == 17 || with_cp == 18) {
+      // split issue: this thread issues only MMAs; a second thread issues the
+      // scale-factor copies into two alternating column sets and signals
+      // each set with a commit.  Mode 18 also waits for a producer's "full".
+      for (int it = 0; it < iters; ++it) {
+        const int st = it & 3, b = it & 1;
+        if (with_cp == 18 && !mbar_wait(&full_bar[st], (uint32_t)(it >> 2) & 1u, &abort_s)) {
+          atomicExch(status, kDevTimeout);
+          break;
+        }
+        if (!mbar_wait(&sf_bar[b], (uint32_t)(it >> 1) & 1u, &abort_s)) {
+          atomicExch(status, kDevTimeout);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sf = tmem + 256 + (uint32_t)b * 48;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          mma_fp4(tmem, adesc + 2 * j, bdesc + 2 * j, idesc, sf + 4 * j, sf + 16 + 8 * j, (it | j) != 0);
+        tc_commit(&empty_bar[st]);
+      }
+    }
+    if (with_cp >= 5 && with_cp <= 12) {
       // the GEMM's stage handshake: wait "full" (arrived by a second warp once
       // it has seen the "empty" commit of `stages` stages back), MMAs, commit
       // "empty".  Modes 9-12: 8 stages; 11-12: stages of 2 MMAs (K = 128).
@@ -144,24 +243,55 @@ __global__ void __launch_bounds__(128, 1) mma_peak_kernel(int iters, int n, int 
         if (st == stages - 1) phase ^= 1u;
       }
     }
-    for (int it = 0; with_cp < 5 && it < iters; ++it) {
+    for (int it = 0; (with_cp < 5 || (with_cp >= 13 && with_cp <= 16)) && it < iters; ++it) {
       // with_cp: 1 one buffer; 2 four rotating buffers; 3 rotating buffers,
-      // copies issued one iteration ahead; 4 six 128x256b copies
-      const uint32_t sf = tmem + 256 + (with_cp >= 2 ? (uint32_t)(it & 3) * 48 : 0u);
-      if (with_cp == 1 || with_cp == 2) copies(sf);
+      // copies issued one iteration ahead; 4 six 128x256b copies.
+      // 13-16 add one stage's bookkeeping without any wait: 13 copies and a
+      // commit per iteration; 14 a commit only; 15 copies and a
+      // fence::after_thread_sync; 16 copies and a commit every 2nd iteration.
+      const uint32_t sf = tmem + 256 + (with_cp >= 2 && with_cp <= 4 ? (uint32_t)(it & 3) * 48 : 0u);
+      if (with_cp == 1 || with_cp == 2 || with_cp == 13 || with_cp == 15 || with_cp == 16) copies(sf);
       if (with_cp == 3) copies(tmem + 256 + (uint32_t)((it + 1) & 3) * 48);
       if (with_cp == 4) wide_copies(sf);
+      if (with_cp == 15) tc_fence_after();
       for (int j = 0; j < 4; ++j)
         mma_fp4(tmem, adesc + 2 * j, bdesc + 2 * j, idesc, sf + 4 * j, sf + 16 + 8 * j, (it | j) != 0);
+      if (with_cp == 13 || with_cp == 14 || (with_cp == 16 && (it & 1))) tc_commit(&empty_bar[it & 3]);
     }
     tc_commit(&bar);
     if (!mbar_wait(&bar, 0, &abort_s)) atomicExch(status, kDevTimeout);
     const unsigned long long t1 = clock64();
     cycles[blockIdx.x] = t1 - t0;
-  } else if (threadIdx.x == 64 && with_cp >= 5) {
+  } else if (threadIdx.x == 96 && (with_cp == 17 || with_cp == 18)) {
+    // the scale-factor copier of the split-issue modes
+    const uint32_t sSF = smem_u32(smem) + 16384 + 32768;
+    for (int it = 0; it < iters; ++it) {
+      const int b = it & 1;
+      if (it >= 2) {
+        const int prev = it - 2;
+        if (!mbar_wait(&empty_bar[prev & 3], (uint32_t)(prev >> 2) & 1u, &abort_s)) {
+          atomicExch(status, kDevTimeout);
+          break;
+        }
+      }
+      tc_fence_after();
+      const uint32_t sf = tmem + 256 + (uint32_t)b * 48;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        tc_cp_scale_atom(sf + 4 * j, sdesc_scale_atom(sSF + 512 * j));
+        tc_cp_scale_atom(sf + 16 + 8 * j, sdesc_scale_atom(sSF + 2048 + 512 * j));
+        tc_cp_scale_atom(sf + 20 + 8 * j, sdesc_scale_atom(sSF + 4096 + 512 * j));
+      }
+      tc_commit(&sf_bar[b]);
+    }
+    // the copies complete before tensor memory is freed
+    tc_commit(&cp_drain);
+    volatile int never = 0;
+    if (!mbar_wait(&cp_drain, 0, &never)) atomicExch(status, kDevTimeout);
+  } else if (threadIdx.x == 64 && ((with_cp >= 5 && with_cp <= 12) || with_cp == 18)) {
     // the producer side of the handshake, with no loads
-    const int stages = with_cp >= 9 ? 8 : 4;
-    const int per = with_cp >= 11 ? 2 : 4;
+    const int stages = with_cp >= 9 && with_cp <= 12 ? 8 : 4;
+    const int per = with_cp >= 11 && with_cp <= 12 ? 2 : 4;
     uint32_t phase = 0;
     for (int it = 0; it < iters * (4 / per); ++it) {
       const int st = it & (stages - 1);
@@ -184,7 +314,8 @@ using namespace nvfp4moe;
 
 extern "C" nvfp4_status nvfp4_test_mma_peak(int iters, int n, int with_cp, int ctas, unsigned long long* cycles,
                                             uint32_t* status, void* stream) {
-  NV_REQUIRE(cycles && status && iters > 0 && ctas > 0 && (n == 128 || n == 256), NVFP4_ERR_INVALID_ARG,
+  NV_REQUIRE(cycles && status && iters > 0 && ctas > 0 && (n == 128 || n == 256) && with_cp >= 0 && with_cp <= 21,
+             NVFP4_ERR_INVALID_ARG,
              "nvfp4_test_mma_peak: bad arguments");
   int sms = 0;
   NV_CHECK(device_sm_count(&sms));
