@@ -128,28 +128,31 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      uint32_t filled = 0, fill_parity = 0;     // per stage: ever filled / parity of last fill
-      bool ok = true;
-      uint8_t* const st0 = smem;
-      const size_t tile_sf_bytes = (size_t)nblk4 * kAtomBytes;     // one 128-row tile's scales
-      for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
-        const int mt = t / p.n_tiles, nt = t % p.n_tiles;
-        const int e = min(max(p.tile_expert[mt], 0), p.E - 1);
-        const int arow = mt * kBM;
-        const int brow = e * p.Nw + nt * (EPI == kEpiGateUp ? 128 : kBN);
-        const uint8_t* asf = p.a_sf + (size_t)mt * tile_sf_bytes;
-        const uint8_t* bsf0 = p.b0_sf + (size_t)(brow / kRowTile) * tile_sf_bytes;
-        const uint8_t* bsf1 = (EPI == kEpiGateUp ? p.b1_sf + (size_t)(brow / kRowTile) * tile_sf_bytes
-                                                 : bsf0 + tile_sf_bytes);
-        for (int kt = 0; kt < KT; ++kt) {
-          if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) {
-            give_up(p.status, abort_flag);
-            ok = false;
-            break;
-          }
+    // The whole warp runs the loop (waits and bookkeeping stay warp-uniform);
+    // one elected lane issues the copies.
+    const uint32_t leader = elect_one();
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t filled = 0, fill_parity = 0;       // per stage: ever filled / parity of last fill
+    bool ok = true;
+    uint8_t* const st0 = smem;
+    const size_t tile_sf_bytes = (size_t)nblk4 * kAtomBytes;       // one 128-row tile's scales
+    for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
+      const int mt = t / p.n_tiles, nt = t % p.n_tiles;
+      const int e = min(max(p.tile_expert[mt], 0), p.E - 1);
+      const int arow = mt * kBM;
+      const int brow = e * p.Nw + nt * (EPI == kEpiGateUp ? 128 : kBN);
+      const uint8_t* asf = p.a_sf + (size_t)mt * tile_sf_bytes;
+      const uint8_t* bsf0 = p.b0_sf + (size_t)(brow / kRowTile) * tile_sf_bytes;
+      const uint8_t* bsf1 = (EPI == kEpiGateUp ? p.b1_sf + (size_t)(brow / kRowTile) * tile_sf_bytes
+                                               : bsf0 + tile_sf_bytes);
+      for (int kt = 0; kt < KT; ++kt) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag));
+        if (!ok) {
+          if (leader) give_up(p.status, abort_flag);
+          break;
+        }
+        if (leader) {
           uint8_t* sA = st0 + stage * kStageBytes;
           uint8_t* sB = sA + kABytes;
           uint8_t* sSFA = sB + kBBytes;
@@ -165,63 +168,62 @@ __global__ void __launch_bounds__(kThreads, 1)
           bulk_load(sSFA, asf + sf_off, sf_bytes, &full_bar[stage]);
           bulk_load(sSFB, bsf0 + sf_off, sf_bytes, &full_bar[stage]);
           bulk_load(sSFB + kSfbBytes / 2, bsf1 + sf_off, sf_bytes, &full_bar[stage]);
-          filled |= 1u << stage;
-          fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
-          if (++stage == kStages) {
-            stage = 0;
-            phase ^= 1u;
-          }
         }
-      }
-      if (!ok) {
-        // let every copy already issued land before the CTA's shared memory goes away
-        volatile int never = 0;
-        for (int s = 0; s < kStages; ++s)
-          if ((filled >> s) & 1u) mbar_wait(&full_bar[s], (fill_parity >> s) & 1u, &never);
+        __syncwarp();
+        filled |= 1u << stage;
+        fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
       }
     }
+    if (!ok && leader) {
+      // let every copy already issued land before the CTA's shared memory goes away
+      volatile int never = 0;
+      for (int s = 0; s < kStages; ++s)
+        if ((filled >> s) & 1u) mbar_wait(&full_bar[s], (fill_parity >> s) & 1u, &never);
+    }
+    __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // One thread issues everything; its own instruction latency bounds the
-    // MMA rate, so all shared-memory descriptors are built once here and a
-    // stage only adds constant offsets to their start-address fields.
-    if (lane == 0) {
-      const uint32_t idesc = idesc_fp4(kBM, kBN);
-      const uint32_t s0 = smem_u32(smem);
-      const uint64_t a0 = sdesc_sw128(s0), b0 = sdesc_sw128(s0 + kABytes);
-      const uint64_t sfa0 = sdesc_scale_atom(s0 + kABytes + kBBytes);
-      const uint64_t sfb0 = sdesc_scale_atom(s0 + kABytes + kBBytes + kSfaBytes);
-      constexpr uint64_t kStageStep = kStageBytes >> 4;        // start address is in 16-byte units
-      constexpr uint64_t kAtomStep = kAtomBytes >> 4;
-      constexpr uint64_t kSfbHalfStep = (kSfbBytes / 2) >> 4;
-      const uint32_t sfa_t = tmem + kSfCol + kSfaOff, sfb_t = tmem + kSfCol + kSfbOff;
-      const uint32_t acc_t = tmem + kAccCol;
-      int stage = 0;
-      uint32_t phase = 0, acc_phase = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
-        if (!mbar_wait(&acc_empty_bar, acc_phase ^ 1u, abort_flag)) {
-          give_up(p.status, abort_flag);
+    // The whole warp runs the loop and one elected lane issues the tcgen05
+    // instructions: a loop run by a single divergent lane issues them too
+    // slowly to keep the tensor pipe busy.  Shared-memory descriptors are
+    // built once; a stage only adds constant offsets to their address fields.
+    const uint32_t leader = elect_one();
+    const uint32_t idesc = idesc_fp4(kBM, kBN);
+    const uint32_t s0 = smem_u32(smem);
+    const uint64_t a0 = sdesc_sw128(s0), b0 = sdesc_sw128(s0 + kABytes);
+    const uint64_t sfa0 = sdesc_scale_atom(s0 + kABytes + kBBytes);
+    const uint64_t sfb0 = sdesc_scale_atom(s0 + kABytes + kBBytes + kSfaBytes);
+    constexpr uint64_t kStageStep = kStageBytes >> 4;          // start address is in 16-byte units
+    constexpr uint64_t kAtomStep = kAtomBytes >> 4;
+    constexpr uint64_t kSfbHalfStep = (kSfbBytes / 2) >> 4;
+    const uint32_t sfa_t = tmem + kSfCol + kSfaOff, sfb_t = tmem + kSfCol + kSfbOff;
+    const uint32_t acc_t = tmem + kAccCol;
+    int stage = 0;
+    uint32_t phase = 0, acc_phase = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&acc_empty_bar, acc_phase ^ 1u, abort_flag));
+      if (!ok) {
+        if (leader) give_up(p.status, abort_flag);
+        break;
+      }
+      tc_fence_after();
+      uint32_t accumulate = 0;
+      for (int kt = 0; kt < KT; ++kt) {
+        // TMA wrote this stage through the async proxy that the MMAs read
+        // through; the completed barrier phase is all the ordering needed
+        ok = __all_sync(0xffffffffu, mbar_wait(&full_bar[stage], phase, abort_flag));
+        if (!ok) {
+          if (leader) give_up(p.status, abort_flag);
           break;
         }
-        tc_fence_after();
-        uint32_t accumulate = 0;
-        bool ready = false;                     // this stage already seen complete
-        for (int kt = 0; kt < KT; ++kt) {
-          // TMA wrote this stage through the async proxy that the MMAs read
-          // through; the completed barrier phase is all the ordering needed
-          if (!ready && !mbar_wait(&full_bar[stage], phase, abort_flag)) {
-            give_up(p.status, abort_flag);
-            ok = false;
-            break;
-          }
-          // look at the next stage now; the answer is used only after this
-          // stage's copies and MMAs have been issued
-          const int nstage = stage + 1 == kStages ? 0 : stage + 1;
-          const uint32_t nphase = stage + 1 == kStages ? phase ^ 1u : phase;
-          ready = (kt + 1 < KT) && mbar_test_wait(&full_bar[nstage], nphase);
-          const uint64_t d = (uint64_t)stage * kStageStep;
-          const int katoms = min(4, (p.K - kt * kBK) / 64);
+        const uint64_t d = (uint64_t)stage * kStageStep;
+        const int katoms = min(4, (p.K - kt * kBK) / 64);
+        if (leader) {
           if (katoms == 4) {
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -232,8 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               // +32 bytes (64 FP4 values) along K inside the 128-byte swizzle atom
-              mma_fp4(acc_t, a0 + d + 2 * j, b0 + d + 2 * j, idesc, sfa_t + 4 * j, sfb_t + 8 * j, accumulate);
-              accumulate = 1;
+              mma_fp4(acc_t, a0 + d + 2 * j, b0 + d + 2 * j, idesc, sfa_t + 4 * j, sfb_t + 8 * j, accumulate | j);
             }
           } else {
             for (int j = 0; j < katoms; ++j) {
@@ -241,26 +242,30 @@ __global__ void __launch_bounds__(kThreads, 1)
               tc_cp_scale_atom(sfb_t + 8 * j, sfb0 + d + j * kAtomStep);
               tc_cp_scale_atom(sfb_t + 8 * j + 4, sfb0 + d + kSfbHalfStep + j * kAtomStep);
             }
-            for (int j = 0; j < katoms; ++j) {
-              mma_fp4(acc_t, a0 + d + 2 * j, b0 + d + 2 * j, idesc, sfa_t + 4 * j, sfb_t + 8 * j, accumulate);
-              accumulate = 1;
-            }
+            for (int j = 0; j < katoms; ++j)
+              mma_fp4(acc_t, a0 + d + 2 * j, b0 + d + 2 * j, idesc, sfa_t + 4 * j, sfb_t + 8 * j, accumulate | j);
           }
           tc_commit(&empty_bar[stage]);
-          if (++stage == kStages) {
-            stage = 0;
-            phase ^= 1u;
-          }
         }
-        if (!ok) break;
-        tc_commit(&acc_full_bar);
-        acc_phase ^= 1u;
+        __syncwarp();
+        accumulate = 1;
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
       }
-      // every MMA issued by this thread completes before tensor memory is freed
+      if (!ok) break;
+      if (leader) tc_commit(&acc_full_bar);
+      __syncwarp();
+      acc_phase ^= 1u;
+    }
+    // every MMA issued by the elected lane completes before tensor memory is freed
+    if (leader) {
       tc_commit(&drain_bar);
       volatile int never = 0;
       mbar_wait(&drain_bar, 0, &never);
     }
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
     const int quad = warp & 3;
