@@ -20,6 +20,8 @@
 // per SM walks the (m-tile, n-tile) list, whose length is read on the device.
 // Every wait is bounded in time; a wait that gives up sets the workspace
 // status word and the CTA winds down after its outstanding copies land.
+#include <mutex>
+
 #include "common.cuh"
 #include "gemm.cuh"
 #include "host.cuh"
@@ -29,15 +31,22 @@ namespace nvfp4moe {
 constexpr int kBM = 128, kBN = 256;
 constexpr int kBK = 256;                         // K elements per stage
 constexpr int kBKBytes = kBK / 2;                // 128 bytes of packed FP4 per row
-constexpr int kStages = 4;
 constexpr int kABytes = kBM * kBKBytes;          // 16 KiB
 constexpr int kBBytes = kBN * kBKBytes;          // 32 KiB
 constexpr int kSfaBytes = kBM * kBK / kQBlock;   // 2 KiB (4 scale atoms)
 constexpr int kSfbBytes = kBN * kBK / kQBlock;   // 4 KiB (8 scale atoms)
 constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
-constexpr int kSmemBytes = kStages * kStageBytes + 1024;
 constexpr int kThreads = 320;
 constexpr int kEpiWarps = 8;
+// Pipeline stages: the gate/up GEMM keeps four; the down GEMM gives one up
+// for the shared-memory buffer its epilogue stages y through, 32 rows x 64
+// bf16 columns (4 KiB) per warp at a time.
+template <int EPI> constexpr int stages_of() { return EPI == kEpiDown ? 3 : 4; }
+constexpr int kYPassCols = 64;
+constexpr int kYStageBytes = 32 * kYPassCols * 2;
+template <int EPI> constexpr int smem_bytes_of() {
+  return stages_of<EPI>() * kStageBytes + 1024 + (EPI == kEpiDown ? kEpiWarps * kYStageBytes : 0);
+}
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCol = 0;                  // 256 fp32 accumulator columns
 // Scale factors of one stage: 4 MMA k-steps x (4 SFA + 8 SFB) columns.  The
@@ -87,6 +96,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const __grid_constant__ CUtensorMap tmB1, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  constexpr int kStages = stages_of<EPI>();
   __shared__ __align__(8) uint64_t full_bar[kStages];
   __shared__ __align__(8) uint64_t empty_bar[kStages];
   __shared__ __align__(8) uint64_t acc_full_bar;
@@ -346,27 +356,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty_bar);
-        if (real) {
-          if (p.y_f32) {
-            float4* dst = reinterpret_cast<float4*>(p.y_f32 + (size_t)grow * p.H + col0);
+        if (real && p.y_f32) {
+          float4* dst = reinterpret_cast<float4*>(p.y_f32 + (size_t)grow * p.H + col0);
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-              dst[i] = make_float4(__fmul_rn(__uint_as_float(r[4 * i]), scale),
-                                   __fmul_rn(__uint_as_float(r[4 * i + 1]), scale),
-                                   __fmul_rn(__uint_as_float(r[4 * i + 2]), scale),
-                                   __fmul_rn(__uint_as_float(r[4 * i + 3]), scale));
-          }
-          if (p.y_bf16) {
-            uint4* dst = reinterpret_cast<uint4*>(p.y_bf16 + (size_t)grow * p.H + col0);
+          for (int i = 0; i < 32; ++i)
+            dst[i] = make_float4(__fmul_rn(__uint_as_float(r[4 * i]), scale),
+                                 __fmul_rn(__uint_as_float(r[4 * i + 1]), scale),
+                                 __fmul_rn(__uint_as_float(r[4 * i + 2]), scale),
+                                 __fmul_rn(__uint_as_float(r[4 * i + 3]), scale));
+        }
+        // scaled and packed to bf16 pairs right away, which frees r
+        uint32_t yw[64];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              uint32_t w[4];
+        for (int i = 0; i < 64; ++i)
+          yw[i] = pack_bf16x2(__fmul_rn(__uint_as_float(r[2 * i]), scale), __fmul_rn(__uint_as_float(r[2 * i + 1]), scale));
+        const uint32_t real_mask = __ballot_sync(0xffffffffu, real);
+        if (p.y_bf16 && real_mask != 0) {
+          // Each lane holds one row.  Stores straight from registers would
+          // hit 32 rows per instruction, so the warp stages 64 columns of its
+          // 32 rows in shared memory (16-byte chunks XOR-swizzled by row) and
+          // writes them back four whole 128-byte row segments per instruction.
+          uint4* ybuf = reinterpret_cast<uint4*>(smem + kStages * kStageBytes + (warp - 2) * kYStageBytes);
+          const int row0 = mt * kBM + quad * 32;
 #pragma unroll
-              for (int q = 0; q < 4; ++q)
-                w[q] = pack_bf16x2(__fmul_rn(__uint_as_float(r[8 * i + 2 * q]), scale),
-                                   __fmul_rn(__uint_as_float(r[8 * i + 2 * q + 1]), scale));
-              dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+          for (int pass = 0; pass < 2; ++pass) {
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+              ybuf[lane * 8 + (ch ^ (lane & 7))] = make_uint4(yw[pass * 32 + ch * 4], yw[pass * 32 + ch * 4 + 1],
+                                                              yw[pass * 32 + ch * 4 + 2], yw[pass * 32 + ch * 4 + 3]);
             }
+            __syncwarp();
+#pragma unroll
+            for (int it = 0; it < 8; ++it) {
+              const int rr = it * 4 + (lane >> 3), ch = lane & 7;
+              const uint4 v = ybuf[rr * 8 + (ch ^ (rr & 7))];
+              if ((real_mask >> rr) & 1u)
+                *reinterpret_cast<uint4*>(p.y_bf16 + (size_t)(row0 + rr) * p.H + col0 + pass * kYPassCols + ch * 8) = v;
+            }
+            __syncwarp();
           }
         }
       }
@@ -382,13 +409,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Opts a kernel into the large dynamic shared memory once per device.
-static nvfp4_status set_smem_attr(const void* fn, int which) {
+static nvfp4_status set_smem_attr(const void* fn, int which, int smem) {
+  static std::mutex mu;
   static bool done[2][64] = {};
   int dev = 0;
   NV_CHECK(check_cuda(cudaGetDevice(&dev), "cudaGetDevice"));
   if (dev < 0 || dev >= 64) dev = 63;
+  std::lock_guard<std::mutex> lock(mu);
   if (!done[which][dev]) {
-    NV_CHECK(check_cuda(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes),
+    NV_CHECK(check_cuda(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
                         "cudaFuncSetAttribute"));
     done[which][dev] = true;
   }
@@ -441,11 +470,11 @@ nvfp4_status launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t s) {
   const int max_tiles = a.rows_capacity / kBM * p.n_tiles;
   const int grid = std::max(1, std::min(sms, max_tiles));
   if (gu) {
-    NV_CHECK(set_smem_attr((const void*)grouped_fp4_gemm_kernel<kEpiGateUp>, 0));
-    grouped_fp4_gemm_kernel<kEpiGateUp><<<grid, kThreads, kSmemBytes, s>>>(tmA, tmB0, tmB1, p);
+    NV_CHECK(set_smem_attr((const void*)grouped_fp4_gemm_kernel<kEpiGateUp>, 0, smem_bytes_of<kEpiGateUp>()));
+    grouped_fp4_gemm_kernel<kEpiGateUp><<<grid, kThreads, smem_bytes_of<kEpiGateUp>(), s>>>(tmA, tmB0, tmB1, p);
   } else {
-    NV_CHECK(set_smem_attr((const void*)grouped_fp4_gemm_kernel<kEpiDown>, 1));
-    grouped_fp4_gemm_kernel<kEpiDown><<<grid, kThreads, kSmemBytes, s>>>(tmA, tmB0, tmB1, p);
+    NV_CHECK(set_smem_attr((const void*)grouped_fp4_gemm_kernel<kEpiDown>, 1, smem_bytes_of<kEpiDown>()));
+    grouped_fp4_gemm_kernel<kEpiDown><<<grid, kThreads, smem_bytes_of<kEpiDown>(), s>>>(tmA, tmB0, tmB1, p);
   }
   return check_launch("grouped_fp4_gemm_kernel");
 }
