@@ -41,10 +41,10 @@ constexpr int kEpiWarps = 8;
 // Pipeline stages: the gate/up GEMM keeps four; the down GEMM gives one up
 // for the shared-memory buffer its epilogue stages y through, 32 rows x 64
 // bf16 columns (4 KiB) per warp at a time.
-template <int EPI> constexpr int stages_of() { return EPI == kEpiDown ? 3 : 4; }
+template <int EPI> __host__ __device__ constexpr int stages_of() { return EPI == kEpiDown ? 3 : 4; }
 constexpr int kYPassCols = 64;
 constexpr int kYStageBytes = 32 * kYPassCols * 2;
-template <int EPI> constexpr int smem_bytes_of() {
+template <int EPI> __host__ __device__ constexpr int smem_bytes_of() {
   return stages_of<EPI>() * kStageBytes + 1024 + (EPI == kEpiDown ? kEpiWarps * kYStageBytes : 0);
 }
 constexpr uint32_t kTmemCols = 512;

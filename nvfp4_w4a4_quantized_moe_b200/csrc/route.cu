@@ -183,22 +183,32 @@ __global__ void __launch_bounds__(kRThreads, 1)
 constexpr int kMaxE = 256, kMaxK = 16;
 
 // Logit of (token t, expert e).  With splits > 0 it is the split-ordered sum
-// of the router GEMM's partial sums (plus the optional offset), loaded eight
-// splits at a time so the loads overlap, and is written to `logits`; with
-// splits == 0 `src` already holds the logits.
+// of the router GEMM's partial sums (plus the optional offset), with up to
+// sixteen loads in flight, and is written to `logits`; with splits == 0 `src`
+// already holds the logits, and with splits < 0 it holds logits that this
+// kernel wrote itself.
 NVDEV float token_logit(const float* __restrict__ src, int splits, const float* __restrict__ offset,
                         float* __restrict__ logits, int T, int E, int t, int e) {
   const float* p = src + (size_t)t * E + e;
   if (splits == 0) return *p;
+  if (splits < 0) return __ldcg(p);      // written earlier by this kernel: read through L2
   const size_t stride = (size_t)T * E;
   float l = p[0];
   int q = 1;
-  for (; q + 8 <= splits; q += 8) {
+  for (; q + 16 <= splits; q += 16) {
+    float v[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) v[u] = p[(size_t)(q + u) * stride];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) l = __fadd_rn(l, v[u]);
+  }
+  if (q + 8 <= splits) {
     float v[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u) v[u] = p[(size_t)(q + u) * stride];
 #pragma unroll
     for (int u = 0; u < 8; ++u) l = __fadd_rn(l, v[u]);
+    q += 8;
   }
   for (; q < splits; ++q) l = __fadd_rn(l, p[(size_t)q * stride]);
   if (offset) l = __fadd_rn(l, offset[e]);
@@ -218,7 +228,7 @@ NVDEV void topk_token(const float* __restrict__ src, int splits, const float* __
   for (int i = 0; i < kMaxE / 32; ++i) {
     const int e = lane + 32 * i;
     if (i < per && e < E) {
-      const float l = token_logit(src, splits, offset, logits, T, E, t, e);
+      const float l = token_logit(src, splits, offset, logits, T, E, t, e);   // splits < 0: no write
       sig[i] = sigmoid_fixed(l);
       c[i] = __fadd_rn(sig[i], bias[e]);
     } else {
@@ -398,6 +408,13 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
   for (int i = tid; i < cap; i += blockDim.x) {
     perm[i] = -1;
     row_w[i] = 0.0f;
+  }
+  // all logits first, one (token, expert) per thread, so that every thread's
+  // partial-sum loads are in flight at once
+  if (splits > 0) {
+    for (int i = tid; i < T * E; i += blockDim.x) token_logit(src, splits, offset, logits, T, E, i / E, i % E);
+    src = logits;
+    splits = -1;
   }
   __syncthreads();
   for (int t = warp; t < T; t += blockDim.x >> 5) {
