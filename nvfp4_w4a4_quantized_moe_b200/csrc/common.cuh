@@ -374,6 +374,13 @@ NVDEV void tmem_ld32(uint32_t taddr, uint32_t* r) {
 }
 NVDEV void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// Programmatic dependent launch.  griddep_wait() blocks until the previous
+// kernel in the stream has finished and its memory is visible (a no-op for a
+// kernel launched without the attribute); griddep_launch() lets the next
+// kernel's blocks be scheduled before this one finishes.
+NVDEV void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+NVDEV void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 NVDEV uint32_t elect_one() {
   uint32_t pred = 0;
   asm volatile(

@@ -22,6 +22,8 @@ __global__ void __launch_bounds__(128) quantize_scatter_kernel(const uint4* __re
                                                                uint8_t* __restrict__ a_scales) {
   // block (t, by): token t, 16-element blocks [128 by, 128 by + 128) of its row
   __shared__ int32_t rows[16];
+  griddep_wait();
+  griddep_launch();
   const int t = blockIdx.x;
   if (threadIdx.x < k) rows[threadIdx.x] = inv_perm[(size_t)t * k + threadIdx.x];
   __syncthreads();
@@ -63,6 +65,7 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const uint4* _
                                                                   const int32_t* __restrict__ inv_perm, int T, int H,
                                                                   int k, uint4* __restrict__ out) {
   __shared__ int32_t rows[16];
+  griddep_wait();
   const int t = blockIdx.x;
   if (threadIdx.x < k) rows[threadIdx.x] = inv_perm[(size_t)t * k + threadIdx.x];
   __syncthreads();
@@ -186,9 +189,9 @@ extern "C" nvfp4_status moe_nvfp4_forward(const moe_nvfp4_weights* W, const void
   // 4: quantise x once per token into its k permuted rows.  Padding rows are
   // left as they are: an MMA row only feeds the same output row, and the
   // epilogues skip padding rows.
-  quantize_scatter_kernel<<<dim3(T, (H / kQBlock + 127) / 128), 128, 0, s>>>(static_cast<const uint4*>(x_bf16), T, H, act_gscale, f.inv_perm, k,
-                                            reinterpret_cast<uint2*>(f.a_codes), f.a_scales);
-  NV_CHECK(check_launch("quantize_scatter_kernel"));
+  NV_CHECK(launch_dependent("quantize_scatter_kernel", quantize_scatter_kernel, dim3(T, (H / kQBlock + 127) / 128),
+                            dim3(128), 0, s, static_cast<const uint4*>(x_bf16), T, H, act_gscale,
+                            (const int32_t*)f.inv_perm, k, reinterpret_cast<uint2*>(f.a_codes), f.a_scales));
   NV_CHECK(mark(dbg, 2, s));
 
   // 5-6: gate/up GEMM with SiLU*up and requantisation
@@ -227,9 +230,9 @@ extern "C" nvfp4_status moe_nvfp4_forward(const moe_nvfp4_weights* W, const void
   // 8: combine
   // below about two waves of whole-row blocks, split rows across blocks
   const int row_blocks = T >= 2 * sms ? 1 : (H / 8 + kCombineThreads - 1) / kCombineThreads;
-  combine_kernel<<<dim3(T, row_blocks), kCombineThreads, 0, s>>>(reinterpret_cast<const uint4*>(f.y), f.inv_perm, T, H, k,
-                                   static_cast<uint4*>(out_bf16));
-  NV_CHECK(check_launch("combine_kernel"));
+  NV_CHECK(launch_dependent("combine_kernel", combine_kernel, dim3(T, row_blocks), dim3(kCombineThreads), 0, s,
+                            reinterpret_cast<const uint4*>(f.y), (const int32_t*)f.inv_perm, T, H, k,
+                            static_cast<uint4*>(out_bf16)));
   NV_CHECK(mark(dbg, 5, s));
 
   if (dbg) {

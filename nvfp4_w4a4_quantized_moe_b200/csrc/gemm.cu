@@ -131,6 +131,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_s;
+  // everything above overlaps the previous kernel; its outputs are read below
+  griddep_wait();
+  griddep_launch();
 
   const int num_tiles = (*p.num_mtiles) * p.n_tiles;
   const int KT = (p.K + kBK - 1) / kBK;
@@ -471,12 +474,12 @@ nvfp4_status launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t s) {
   const int grid = std::max(1, std::min(sms, max_tiles));
   if (gu) {
     NV_CHECK(set_smem_attr((const void*)grouped_fp4_gemm_kernel<kEpiGateUp>, 0, smem_bytes_of<kEpiGateUp>()));
-    grouped_fp4_gemm_kernel<kEpiGateUp><<<grid, kThreads, smem_bytes_of<kEpiGateUp>(), s>>>(tmA, tmB0, tmB1, p);
-  } else {
-    NV_CHECK(set_smem_attr((const void*)grouped_fp4_gemm_kernel<kEpiDown>, 1, smem_bytes_of<kEpiDown>()));
-    grouped_fp4_gemm_kernel<kEpiDown><<<grid, kThreads, smem_bytes_of<kEpiDown>(), s>>>(tmA, tmB0, tmB1, p);
+    return launch_dependent("grouped_fp4_gemm_kernel<gate_up>", grouped_fp4_gemm_kernel<kEpiGateUp>, dim3(grid),
+                            dim3(kThreads), smem_bytes_of<kEpiGateUp>(), s, tmA, tmB0, tmB1, p);
   }
-  return check_launch("grouped_fp4_gemm_kernel");
+  NV_CHECK(set_smem_attr((const void*)grouped_fp4_gemm_kernel<kEpiDown>, 1, smem_bytes_of<kEpiDown>()));
+  return launch_dependent("grouped_fp4_gemm_kernel<down>", grouped_fp4_gemm_kernel<kEpiDown>, dim3(grid),
+                          dim3(kThreads), smem_bytes_of<kEpiDown>(), s, tmA, tmB0, tmB1, p);
 }
 
 // Builds the m-tile -> expert map from caller-supplied segment offsets,

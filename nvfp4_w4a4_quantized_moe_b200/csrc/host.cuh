@@ -8,6 +8,8 @@
 #include <stdint.h>
 #include <stdio.h>
 
+#include <utility>
+
 #include "../../include/nvfp4_moe.h"
 
 namespace nvfp4moe {
@@ -42,6 +44,27 @@ struct Carver {
 };
 
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Launches `kernel` as a programmatic dependent of the stream's previous
+// kernel: its blocks may start once every block of that kernel has signalled
+// (griddepcontrol.launch_dependents), and the kernel itself waits for the
+// previous one to finish (griddepcontrol.wait) before it touches memory that
+// kernel wrote.  Every kernel launched this way calls griddep_wait() first.
+template <typename... Params, typename... Args>
+nvfp4_status launch_dependent(const char* what, void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return check_cuda(cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...), what);
+}
 
 }  // namespace nvfp4moe
 

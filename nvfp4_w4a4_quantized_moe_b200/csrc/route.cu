@@ -85,6 +85,8 @@ __global__ void __launch_bounds__(kRThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_s;
+  griddep_wait();
+  griddep_launch();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -404,11 +406,15 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
   __shared__ int32_t sp[256];
   __shared__ int32_t base[kMaxE];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // the router GEMM before this kernel writes none of these, so the fill
+  // overlaps it
   for (int i = tid; i < E * (kSmallT / 32); i += blockDim.x) bm[i / (kSmallT / 32)][i % (kSmallT / 32)] = 0;
   for (int i = tid; i < cap; i += blockDim.x) {
     perm[i] = -1;
     row_w[i] = 0.0f;
   }
+  griddep_wait();
+  griddep_launch();
   // all logits first, one (token, expert) per thread, so that every thread's
   // partial-sum loads are in flight at once
   if (splits > 0) {
@@ -512,11 +518,10 @@ nvfp4_status launch_route(const RouteArgs& a, const RouteScratch& r, cudaStream_
     NV_CHECK(check_launch("router_gemm_kernel"));
   }
   if (a.T <= kSmallT) {
-    route_small_kernel<<<1, kSmallThreads, 0, s>>>(splits ? r.partial : a.logits, splits, a.logit_offset, a.logits,
-                                                   a.bias, a.T, a.E, a.k, a.rsf, cap, a.topk_idx, a.topk_w, r.counts,
-                                                   a.expert_offsets, r.tile_expert, r.num_mtiles, a.perm,
-                                                   a.inv_perm, r.row_w);
-    return check_launch("route_small_kernel");
+    return launch_dependent("route_small_kernel", route_small_kernel, dim3(1), dim3(kSmallThreads), 0, s,
+                            (const float*)(splits ? r.partial : a.logits), splits, a.logit_offset, a.logits, a.bias,
+                            a.T, a.E, a.k, a.rsf, cap, a.topk_idx, a.topk_w, r.counts, a.expert_offsets,
+                            r.tile_expert, r.num_mtiles, a.perm, a.inv_perm, r.row_w);
   }
   NV_CHECK(check_cuda(cudaMemsetAsync(a.perm, 0xFF, sizeof(int32_t) * (size_t)cap, s), "memset perm"));
   NV_CHECK(check_cuda(cudaMemsetAsync(r.row_w, 0, sizeof(float) * (size_t)cap, s), "memset row_w"));
