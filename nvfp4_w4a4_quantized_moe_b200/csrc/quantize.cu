@@ -83,22 +83,47 @@ __global__ void zero_tiled_scale_rows(uint8_t* scales, int rows, int padded_rows
 }
 
 // ---------------------------------------------------------------------------
-// Weights: one cooperative launch (every CTA resident).  Each CTA owns an
-// even share of every matrix and splits its warps in two groups that run side
-// by side:
-//   * amax warps stream matrix after matrix, publish one atomic max and one
-//     completion count per matrix, and stay at most two matrices ahead of
-//     their own CTA's quantise warps (so the matrices in flight fit in L2);
-//   * quantise warps take matrix m once every CTA has published its amax
-//     (a bounded wait), re-read their share (from L2: the amax pass asked L2
-//     to keep the lines, this pass lets them go) and write codes and scales.
-// Waits only ever point at earlier matrices, so with all CTAs resident they
+// Weights: one cooperative launch (every CTA resident, one per SM).  Each CTA
+// owns an even share of every matrix and runs two streams over it side by
+// side.  Each stream is a ring of 16 KiB shared-memory chunks that its own
+// producer warp fills with bulk asynchronous copies (the copy engine holds the
+// bytes in flight, not registers), and eight consumer warps drain:
+//   * the amax stream reads matrix after matrix from HBM (L2 evict_last); its
+//     consumers keep a running max and, at the end of each matrix, publish
+//     one atomic max and one completion count.  Its producer stays at most
+//     one matrix ahead of this CTA's quantise consumers, so the matrices in
+//     flight stay in L2;
+//   * the quantise stream's producer waits (bounded) until every CTA has
+//     published matrix m's amax, then re-reads this CTA's share from L2
+//     (evict_first); its consumers write codes and tiled scales.
+// Waits only ever point at earlier work, so with all CTAs resident they
 // always end.
 // ---------------------------------------------------------------------------
-constexpr int kWAmax = 256;                     // amax threads per CTA (the DRAM stream)
-constexpr int kWQuant = 256;                    // quantise threads per CTA (re-read from L2)
-constexpr int kWThreads = kWAmax + kWQuant;
-constexpr int kWAhead = 1;                      // amax may lead quantise by this many matrices
+// Quantising a block costs far more instructions than taking its max, so the
+// quantise stream gets four times the amax stream's consumer warps.  One
+// 1024-thread CTA per SM: with two CTAs per SM the later one fell behind by
+// a fifth, and every matrix waits for the slowest CTA.
+constexpr int kWChunkBlocks = 768;                       // 16-element blocks per chunk
+constexpr int kWChunkBytes = kWChunkBlocks * 32;         // 24 KiB of bf16
+constexpr int kWSlotsA = 4;                              // ring depth of the amax stream (HBM)
+constexpr int kWSlotsQ = 3;                              // ring depth of the quantise stream (L2)
+constexpr int kWAmaxConsumers = 192;                     // 8 x 16 bytes of each chunk per thread
+constexpr int kWQuantConsumers = 768;                    // one block of each chunk per thread
+constexpr int kWThreads = 64 + kWAmaxConsumers + kWQuantConsumers;   // + one producer warp per stream
+// The amax stream may start matrix m once this CTA's quantise consumers are
+// no more than kWLagEighths eighths of a matrix behind it: (8 m - kWLag) / 8
+// matrices' worth of chunks done.  The matrices in flight must stay in L2,
+// and the amax stream should not stall at the end of every quantise pass.
+constexpr int kWLagEighths = 14;
+constexpr int kWDynSmem = (kWSlotsA + kWSlotsQ) * kWChunkBytes + 128;
+// warp roles
+constexpr int kWAmaxProducer = 0;                        // warp 0
+constexpr int kWQuantProducer = 1;                       // warp 1
+constexpr int kWAmaxWarp0 = 2;                           // warps 2..7
+constexpr int kWQuantWarp0 = 2 + kWAmaxConsumers / 32;   // warps 8..31
+static_assert(kWChunkBlocks % kWQuantConsumers == 0 && (2 * kWChunkBlocks) % kWAmaxConsumers == 0,
+              "chunks split evenly over the consumers");
+static_assert(kWChunkBlocks % 4 == 0, "a chunk holds whole 4-block scale words");
 
 struct WeightQuantState {
   uint32_t status;          // device status word (first word of the workspace)
@@ -121,152 +146,299 @@ NVDEV uint64_t l2_policy_evict_first() {
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
   return pol;
 }
-NVDEV uint4 ld_hint(const uint4* p, uint64_t pol) {
-  uint4 v;
-  asm volatile("ld.global.nc.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p), "l"(pol));
-  return v;
+// cp.async.bulk global -> shared with an L2 cache policy.
+NVDEV void bulk_load_hint(void* dst, const void* src, uint32_t bytes, uint64_t* bar, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::
+          "r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
+      : "memory");
 }
 template <int N>
 NVDEV void group_sync(int id) { asm volatile("bar.sync %0, %1;" ::"r"(id), "n"(N) : "memory"); }
+// Named-barrier AND over the N threads of a group: every thread gets the same
+// answer, so a group leaves its loops together.
+template <int N>
+NVDEV bool group_all(int id, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(id), "n"(N)
+      : "memory");
+  return r != 0;
+}
 
-__global__ void __launch_bounds__(kWThreads) quantize_weights_kernel(
+// The producer side of one stream: fills ring slots in order with this CTA's
+// share of matrices [0, n_mats).  `ready(mat)` is a bounded wait for the
+// stream's precondition on matrix mat (it returns false on give-up).  Before
+// returning it waits for every copy it issued, so none lands after the CTA
+// exits.
+template <int SLOTS, class Ready>
+NVDEV void weight_stream_producer(const uint8_t* w, long long mat_bytes, long long byte_begin, long long byte_end,
+                                  int n_mats, uint8_t* ring, uint64_t* full, uint64_t* empty, uint64_t pol,
+                                  volatile int* abort_flag, uint32_t* status, Ready ready) {
+  int slot = 0;
+  uint32_t phase = 0;
+  uint32_t filled = 0, fill_parity = 0;
+  bool ok = true;
+  for (int mat = 0; ok && mat < n_mats; ++mat) {
+    if (!ready(mat)) {
+      ok = false;
+      break;
+    }
+    for (long long off = byte_begin; off < byte_end; off += kWChunkBytes) {
+      if (!mbar_wait(&empty[slot], phase ^ 1u, abort_flag)) {
+        ok = false;
+        break;
+      }
+      const uint32_t bytes = (uint32_t)min((long long)kWChunkBytes, byte_end - off);
+      mbar_arrive_expect_tx(&full[slot], bytes);
+      bulk_load_hint(ring + slot * kWChunkBytes, w + mat * mat_bytes + off, bytes, &full[slot], pol);
+      filled |= 1u << slot;
+      fill_parity = (fill_parity & ~(1u << slot)) | (phase << slot);
+      if (++slot == SLOTS) {
+        slot = 0;
+        phase ^= 1u;
+      }
+    }
+  }
+  if (!ok) {
+    *abort_flag = 1;
+    atomicExch(status, kDevTimeout);
+  }
+  volatile int never = 0;
+  for (int s = 0; s < SLOTS; ++s)
+    if ((filled >> s) & 1u) mbar_wait(&full[s], (fill_parity >> s) & 1u, &never);
+}
+
+__global__ void __launch_bounds__(kWThreads, 1) quantize_weights_kernel(
     const uint4* __restrict__ w, int n_mats, int rows, int cols, int layout, uint2* __restrict__ codes,
     uint8_t* __restrict__ scales, float* __restrict__ gscale, WeightQuantState* st, uint32_t* amax_bits,
     uint32_t* done) {
-  __shared__ uint32_t s_red[kWAmax / 32];
-  __shared__ int s_ok_amax, s_ok_quant;
-  __shared__ volatile int quantised;            // matrices this CTA's quantise warps have finished
-  __shared__ volatile int failed;
+  extern __shared__ uint8_t wq_smem_raw[];
+  uint8_t* ring_a = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(wq_smem_raw) + 127) & ~uintptr_t(127));
+  uint8_t* ring_q = ring_a + kWSlotsA * kWChunkBytes;
+  __shared__ __align__(8) uint64_t full_a[kWSlotsA], empty_a[kWSlotsA], full_q[kWSlotsQ], empty_q[kWSlotsQ];
+  __shared__ uint32_t s_red[kWAmaxConsumers / 32];
+  __shared__ float s_amax[4];                   // amax of matrix m at [m % 4], set by the quantise producer
+  __shared__ float s_inv[2][256];               // matrix m's 1 / (E4M3(s) g) for every scale code s, at [m % 2]
+  __shared__ volatile int quantised;            // matrices this CTA's quantise consumers have finished
+  __shared__ unsigned int q_chunk_warps;        // (chunk, warp) pairs the quantise consumers have finished
+  __shared__ int abort_s;
+  volatile int* abort_flag = &abort_s;
   const long long per_mat = (long long)rows * cols;
   const long long blocks = per_mat / kQBlock;                  // 16-element blocks per matrix
   const int nblk = cols / kQBlock;
-  const int lane = threadIdx.x & 31;
-  const int gt = threadIdx.x < kWAmax ? threadIdx.x : threadIdx.x - kWAmax;   // index within its group
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // this CTA's share of every matrix, in whole groups of 4 blocks
   const long long share = ((blocks + gridDim.x - 1) / gridDim.x + 3) / 4 * 4;
   const long long b_begin = min(blocks, share * blockIdx.x), b_end = min(blocks, b_begin + share);
+  const int n_chunks = (int)((b_end - b_begin + kWChunkBlocks - 1) / kWChunkBlocks);
   if (threadIdx.x == 0) {
+    for (int i = 0; i < kWSlotsA; ++i) {
+      mbar_init(&full_a[i], 1);
+      mbar_init(&empty_a[i], kWAmaxConsumers / 32);
+    }
+    for (int i = 0; i < kWSlotsQ; ++i) {
+      mbar_init(&full_q[i], 1);
+      mbar_init(&empty_q[i], kWQuantConsumers / 32);
+    }
     quantised = 0;
-    failed = 0;
+    q_chunk_warps = 0;
+    abort_s = 0;
+    fence_barrier_init();
   }
   __syncthreads();
+  const uint8_t* wb = reinterpret_cast<const uint8_t*>(w);
 
-  if (threadIdx.x < kWAmax) {
-    // ------------------------------------------------------------ amax warps
-    const uint64_t keep = l2_policy_evict_last();
-    for (int mat = 0; mat < n_mats; ++mat) {
-      if (gt == 0) {
+  if (warp == kWAmaxProducer) {
+    // ------------------------------------------------------------ amax producer
+    if (lane == 0) {
+      auto gate = [&](int mat) {
+        const long long need_eighths = 8ll * mat - kWLagEighths;
+        if (need_eighths <= 0) return true;
+        const long long need = (need_eighths * n_chunks + 7) / 8 * (kWQuantConsumers / 32);
         const uint64_t t0 = globaltimer_ns();
-        while (quantised < mat - kWAhead && !failed) {
-          if (globaltimer_ns() - t0 > kWaitLimitNs) {
-            failed = 1;
-            atomicExch(&st->status, kDevTimeout);
-          }
+        while ((long long)*reinterpret_cast<volatile unsigned int*>(&q_chunk_warps) < need) {
+          if (*abort_flag || globaltimer_ns() - t0 > kWaitLimitNs) return false;
         }
-        s_ok_amax = !failed;
-      }
-      group_sync<kWAmax>(1);
-      if (!s_ok_amax) break;
-      const uint4* src = w + (long long)mat * per_mat / 8;
-      const long long v1 = b_end * 2;                          // uint4 range (8 bf16 each)
+        return true;
+      };
+      weight_stream_producer<kWSlotsA>(wb, per_mat * 2, b_begin * 32, b_end * 32, n_mats, ring_a, full_a, empty_a,
+                             l2_policy_evict_last(), abort_flag, &st->status, gate);
+    }
+  } else if (warp == kWQuantProducer) {
+    // ------------------------------------------------------------ quantise producer
+    if (lane == 0) {
+      auto amax_ready = [&](int mat) {
+        const uint64_t t0 = globaltimer_ns();
+        while (ld_acquire_u32(done + mat) < gridDim.x) {
+          if (*abort_flag || globaltimer_ns() - t0 > kWaitLimitNs) return false;
+        }
+        // published before the matrix's first chunk is announced, so the
+        // consumers see it once that chunk's barrier completes
+        s_amax[mat & 3] = __uint_as_float(ld_acquire_u32(amax_bits + mat));
+        return true;
+      };
+      weight_stream_producer<kWSlotsQ>(wb, per_mat * 2, b_begin * 32, b_end * 32, n_mats, ring_q, full_q, empty_q,
+                             l2_policy_evict_first(), abort_flag, &st->status, amax_ready);
+    }
+  } else if (warp < kWQuantWarp0) {
+    // ------------------------------------------------------------ amax consumers
+    const int gt = threadIdx.x - kWAmaxWarp0 * 32;
+    int slot = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int mat = 0; mat < n_mats; ++mat) {
       // running max of |x| on packed bf16 pairs (exact)
       __nv_bfloat162 m2 = __floats2bfloat162_rn(0.0f, 0.0f);
-      auto absmax4 = [&](const uint4& u) {
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+      for (int c = 0; ok && c < n_chunks; ++c) {
+        if (!mbar_wait(&full_a[slot], phase, abort_flag)) {
+          ok = false;
+          break;
+        }
+        const long long c0 = b_begin + (long long)c * kWChunkBlocks;
+        const int nvec = (int)min((long long)kWChunkBlocks, b_end - c0) * 2;     // uint4 in this chunk
+        const uint4* src = reinterpret_cast<const uint4*>(ring_a + slot * kWChunkBytes);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) m2 = __hmax2(m2, __habs2(*reinterpret_cast<const __nv_bfloat162*>(&w[j])));
-      };
-      long long i = b_begin * 2 + gt;
-      for (; i + 7 * kWAmax < v1; i += 8 * kWAmax) {
-        uint4 u[8];
+        for (int i = 0; i < 2 * kWChunkBlocks / kWAmaxConsumers; ++i) {
+          const int v = gt + i * kWAmaxConsumers;
+          if (v < nvec) {
+            const uint4 u = src[v];
+            const uint32_t ws[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-        for (int q = 0; q < 8; ++q) u[q] = ld_hint(src + i + q * kWAmax, keep);
-#pragma unroll
-        for (int q = 0; q < 8; ++q) absmax4(u[q]);
+            for (int j = 0; j < 4; ++j)
+              m2 = __hmax2(m2, __habs2(*reinterpret_cast<const __nv_bfloat162*>(&ws[j])));
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty_a[slot]);
+        if (++slot == kWSlotsA) {
+          slot = 0;
+          phase ^= 1u;
+        }
       }
-      for (; i < v1; i += kWAmax) absmax4(ld_hint(src + i, keep));
       const float m = fmaxf(__low2float(m2), __high2float(m2));
       uint32_t mb = __float_as_uint(m);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, o));
       if (lane == 0) s_red[gt >> 5] = mb;
-      group_sync<kWAmax>(1);
+      ok = group_all<kWAmaxConsumers>(1, ok && !*abort_flag);
       if (gt == 0) {
         uint32_t bm = 0;
-        for (int q = 0; q < kWAmax / 32; ++q) bm = max(bm, s_red[q]);
+        for (int q = 0; q < kWAmaxConsumers / 32; ++q) bm = max(bm, s_red[q]);
         atomicMax(amax_bits + mat, bm);         // non-negative floats order like their bits
         __threadfence();
         atomicAdd(done + mat, 1u);
       }
+      group_sync<kWAmaxConsumers>(1);
+      if (!ok) {
+        // publish the remaining matrices so that no other CTA waits on them
+        if (gt == 0)
+          for (int mm = mat + 1; mm < n_mats; ++mm) atomicAdd(done + mm, 1u);
+        *abort_flag = 1;
+        atomicExch(&st->status, kDevTimeout);
+        break;
+      }
     }
   } else {
-    // ------------------------------------------------------------ quantise warps
-    const uint64_t drop = l2_policy_evict_first();
-    for (int mat = 0; mat < n_mats; ++mat) {
-      if (gt == 0) {
-        int ok = 1;
-        if (ld_acquire_u32(done + mat) < gridDim.x) {
-          const uint64_t t0 = globaltimer_ns();
-          while (ld_acquire_u32(done + mat) < gridDim.x) {
-            if (failed || globaltimer_ns() - t0 > kWaitLimitNs) {
-              ok = 0;
-              failed = 1;
-              atomicExch(&st->status, kDevTimeout);
-              break;
+    // ------------------------------------------------------------ quantise consumers
+    const int gt = threadIdx.x - kWQuantWarp0 * 32;
+    int slot = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    const float inv_nblk = 1.0f / (float)nblk;
+    for (int mat = 0; ok && mat < n_mats; ++mat) {
+      float g = 0.0f, d = 0.0f;
+      float* inv_tab = s_inv[mat & 1];
+      for (int c = 0; c < n_chunks; ++c) {
+        const bool landed = mbar_wait(&full_q[slot], phase, abort_flag);
+        if (c == 0) {
+          // the matrix's global scale and, for each of the 256 scale codes,
+          // the reciprocal its blocks multiply by: 1 / (E4M3(s) g), 0 for 0.
+          // Every warp takes part in the barrier, landed or not.
+          if (landed) {
+            g = __fdiv_rn(s_amax[mat & 3], 2688.0f);
+            d = __fmul_rn(6.0f, g);
+            if (gt < 256) {
+              const float S = __fmul_rn(e4m3_value((uint32_t)gt), g);
+              inv_tab[gt] = (S == 0.0f) ? 0.0f : __frcp_rn(S);
             }
           }
-        }
-        s_ok_quant = ok;
-      }
-      group_sync<kWQuant>(2);
-      if (!s_ok_quant) break;
-      const float amax = __uint_as_float(ld_acquire_u32(amax_bits + mat));
-      const float g = __fdiv_rn(amax, 2688.0f);
-      const float d = __fmul_rn(6.0f, g);
-      if (blockIdx.x == 0 && gt == 0) gscale[mat] = g;
-      const uint4* src = w + (long long)mat * per_mat / 8;
-      const float inv_nblk = 1.0f / (float)nblk;
-      // every lane of a warp runs the same number of iterations (shuffles
-      // below); each iteration has two blocks per thread in flight
-      const long long n_iter = (b_end - b_begin + 2 * kWQuant - 1) / (2 * kWQuant);
-      for (long long it = 0; it < n_iter; ++it) {
-        uint4 u[2][2];
-        bool valid[2];
-        long long b[2];
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          b[q] = b_begin + (2 * it + q) * kWQuant + gt;
-          valid[q] = b[q] < b_end;
-          if (valid[q]) {
-            u[q][0] = ld_hint(src + 2 * b[q], drop);
-            u[q][1] = ld_hint(src + 2 * b[q] + 1, drop);
+          if (!group_all<kWQuantConsumers>(2, landed)) {
+            ok = false;
+            break;
           }
+        } else if (!landed) {
+          ok = false;
+          break;
         }
+        const long long c0 = b_begin + (long long)c * kWChunkBlocks;
+        const int nb = (int)min((long long)kWChunkBlocks, b_end - c0);
+        const uint4* src = reinterpret_cast<const uint4*>(ring_q + slot * kWChunkBytes);
+        const int j = gt;                             // this thread's block within the chunk
+        const bool valid = j < nb;
+        uint32_t sc = 0;
+        int row = 0, kb = 0;
+        if (valid) {
+          const uint4 u0 = src[2 * j], u1 = src[2 * j + 1];
+          const uint32_t w8[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+          const float amax = amax16_bf16(w8);
+          const float s_raw = (d == 0.0f) ? 0.0f : __fdiv_rn(amax, d);
+          sc = e4m3_code(s_raw);
+          const float inv = inv_tab[sc];
+          const uint64_t inv2 = pack_f32x2(inv, inv);
+          float y[16];
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          uint32_t sc = 0;
-          int row = 0, kb = 0;
-          if (valid[q]) {
-            uint2 c;
-            sc = quant_block16_bf16(u[q][0], u[q][1], g, d, c);
-            codes[(long long)mat * blocks + b[q]] = c;
-            // b < 2^24 (checked on the host): a float quotient off by at most
-            // one, then an exact integer correction
-            const uint32_t bb = (uint32_t)b[q];
-            uint32_t qt = (uint32_t)__fmul_rz((float)bb, inv_nblk);
-            int32_t rem = (int32_t)(bb - qt * (uint32_t)nblk);
-            if (rem < 0) { --qt; rem += nblk; }
-            if (rem >= nblk) { ++qt; rem -= nblk; }
-            row = (int)qt;
-            kb = rem;
+          for (int i = 0; i < 8; ++i) {
+            const uint64_t r = mul_f32x2(((uint64_t)(w8[i] & 0xFFFF0000u) << 32) | (uint64_t)(w8[i] << 16), inv2);
+            y[2 * i] = lo_f32(r);
+            y[2 * i + 1] = hi_f32(r);
           }
-          store_scales<1>(scales, layout, mat * rows + row, kb, nblk, &sc, valid[q]);
+          const long long b = c0 + j;
+          codes[(long long)mat * blocks + b] = make_uint2(e2m1x8_hw(y), e2m1x8_hw(y + 8));
+          // b < 2^24 (checked on the host): a float quotient off by at most
+          // one, then an exact integer correction
+          const uint32_t bb = (uint32_t)b;
+          uint32_t qt = (uint32_t)__fmul_rz((float)bb, inv_nblk);
+          int32_t rem = (int32_t)(bb - qt * (uint32_t)nblk);
+          if (rem < 0) { --qt; rem += nblk; }
+          if (rem >= nblk) { ++qt; rem -= nblk; }
+          row = (int)qt;
+          kb = rem;
+        }
+        store_scales<1>(scales, layout, mat * rows + row, kb, nblk, &sc, valid);
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&empty_q[slot]);
+          atomicAdd(&q_chunk_warps, 1u);
+        }
+        if (++slot == kWSlotsQ) {
+          slot = 0;
+          phase ^= 1u;
         }
       }
-      group_sync<kWQuant>(2);
-      if (gt == 0) quantised = mat + 1;
+      if (ok && n_chunks == 0) {
+        // an empty share still waits for the matrix so that its gscale is written
+        const uint64_t t0 = globaltimer_ns();
+        while (ld_acquire_u32(done + mat) < gridDim.x)
+          if (*abort_flag || globaltimer_ns() - t0 > kWaitLimitNs) {
+            ok = false;
+            break;
+          }
+        if (ok) g = __fdiv_rn(__uint_as_float(ld_acquire_u32(amax_bits + mat)), 2688.0f);
+      }
+      if (blockIdx.x == 0 && gt == 0 && ok) gscale[mat] = g;
+      ok = group_all<kWQuantConsumers>(2, ok);
+      if (gt == 0 && ok) quantised = mat + 1;
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      atomicExch(&st->status, kDevTimeout);
     }
   }
   __syncthreads();
@@ -277,16 +449,31 @@ static nvfp4_status launch_weight_quantiser(const void* w_bf16, int n_mats, int 
                                            uint8_t* codes, uint8_t* scales, float* global_scale,
                                            WeightQuantState* st, uint32_t* amax, uint32_t* done, int sms,
                                            cudaStream_t s) {
+  {
+    static std::mutex mu;
+    static bool attr_set[64] = {};
+    int dev = 0;
+    NV_CHECK(check_cuda(cudaGetDevice(&dev), "cudaGetDevice"));
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+      NV_CHECK(check_cuda(cudaFuncSetAttribute(quantize_weights_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               kWDynSmem),
+                          "cudaFuncSetAttribute"));
+      if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    }
+  }
   int per_sm = 0;
-  NV_CHECK(check_cuda(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quantize_weights_kernel, kWThreads, 0),
-                      "occupancy"));
-  per_sm = std::max(1, std::min(per_sm, 2));
+  NV_CHECK(check_cuda(
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quantize_weights_kernel, kWThreads, kWDynSmem),
+      "occupancy"));
+  NV_REQUIRE(per_sm >= 1, NVFP4_ERR_CUDA, "quantize_weights_kernel cannot be resident");
+  per_sm = 1;
   const uint4* w = static_cast<const uint4*>(w_bf16);
   uint2* c = reinterpret_cast<uint2*>(codes);
   void* args[] = {(void*)&w, (void*)&n_mats, (void*)&rows, (void*)&cols, (void*)&layout, (void*)&c,
                   (void*)&scales, (void*)&global_scale, (void*)&st, (void*)&amax, (void*)&done};
   return check_cuda(cudaLaunchCooperativeKernel((const void*)quantize_weights_kernel, dim3(sms * per_sm),
-                                                dim3(kWThreads), args, 0, s),
+                                                dim3(kWThreads), args, kWDynSmem, s),
                     "cudaLaunchCooperativeKernel(quantize_weights_kernel)");
 }
 
