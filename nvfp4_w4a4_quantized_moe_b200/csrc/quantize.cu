@@ -351,9 +351,14 @@ __global__ void __launch_bounds__(kWThreads, 1) quantize_weights_kernel(
     int slot = 0;
     uint32_t phase = 0;
     bool ok = true;
-    const float inv_nblk = 1.0f / (float)nblk;
+    // (row, block column) of this thread's block in chunk 0; each further
+    // chunk moves it kWChunkBlocks blocks on
+    const long long bt0 = b_begin + gt;
+    const int row_t0 = (int)(bt0 / nblk), kb_t0 = (int)(bt0 % nblk);
+    const int step_rows = kWChunkBlocks / nblk, step_kb = kWChunkBlocks % nblk;
     for (int mat = 0; ok && mat < n_mats; ++mat) {
       float g = 0.0f, d = 0.0f;
+      int row = row_t0, kb = kb_t0;
       float* inv_tab = s_inv[mat & 1];
       for (int c = 0; c < n_chunks; ++c) {
         const bool landed = mbar_wait(&full_q[slot], phase, abort_flag);
@@ -381,15 +386,12 @@ __global__ void __launch_bounds__(kWThreads, 1) quantize_weights_kernel(
         const int nb = (int)min((long long)kWChunkBlocks, b_end - c0);
         const uint4* src = reinterpret_cast<const uint4*>(ring_q + slot * kWChunkBytes);
         const int j = gt;                             // this thread's block within the chunk
-        const bool valid = j < nb;
-        uint32_t sc = 0;
-        int row = 0, kb = 0;
-        if (valid) {
+        if (j < nb) {
           const uint4 u0 = src[2 * j], u1 = src[2 * j + 1];
           const uint32_t w8[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
           const float amax = amax16_bf16(w8);
           const float s_raw = (d == 0.0f) ? 0.0f : __fdiv_rn(amax, d);
-          sc = e4m3_code(s_raw);
+          const uint32_t sc = e4m3_code(s_raw);
           const float inv = inv_tab[sc];
           const uint64_t inv2 = pack_f32x2(inv, inv);
           float y[16];
@@ -399,19 +401,17 @@ __global__ void __launch_bounds__(kWThreads, 1) quantize_weights_kernel(
             y[2 * i] = lo_f32(r);
             y[2 * i + 1] = hi_f32(r);
           }
-          const long long b = c0 + j;
-          codes[(long long)mat * blocks + b] = make_uint2(e2m1x8_hw(y), e2m1x8_hw(y + 8));
-          // b < 2^24 (checked on the host): a float quotient off by at most
-          // one, then an exact integer correction
-          const uint32_t bb = (uint32_t)b;
-          uint32_t qt = (uint32_t)__fmul_rz((float)bb, inv_nblk);
-          int32_t rem = (int32_t)(bb - qt * (uint32_t)nblk);
-          if (rem < 0) { --qt; rem += nblk; }
-          if (rem >= nblk) { ++qt; rem -= nblk; }
-          row = (int)qt;
-          kb = rem;
+          codes[(long long)mat * blocks + c0 + j] = make_uint2(e2m1x8_hw(y), e2m1x8_hw(y + 8));
+          const int srow = mat * rows + row;
+          scales[layout == NVFP4_LAYOUT_CANONICAL ? (size_t)srow * nblk + kb
+                                                  : tiled_scale_offset(srow, kb, nblk >> 2)] = (uint8_t)sc;
         }
-        store_scales<1>(scales, layout, mat * rows + row, kb, nblk, &sc, valid);
+        row += step_rows;
+        kb += step_kb;
+        if (kb >= nblk) {
+          kb -= nblk;
+          ++row;
+        }
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(&empty_q[slot]);
