@@ -414,6 +414,9 @@ def run_ours(args, cfg):
     torch.cuda.synchronize()
     q_ms = dist.max(q0.elapsed_time(q1)) / qsteps
     q_gbs = qbytes / (q_ms * 1e-3) / 1e9
+
+    # block-scale distortion statistics of the layer's quantised experts
+    diag = block_stats_report(c, cfg, (gate, up, down), W, stream, dist, peaks)
     c.nvfp4_workspace_status(qws)
 
     # roofline of the dominant kernel
@@ -468,6 +471,7 @@ def run_ours(args, cfg):
                  "frac_of_fp4_peak": (gu_flops + dn_flops) / (gemm_ms * 1e-3) / 1e12 / fp4_peak},
         "stages_ms": stage_ms,
         "roofline": roof,
+        "diagnostics": diag,
         "quantiser": {"workload": f"quantiser: {cfg.E} x (gate, up {cfg.I}x{cfg.H}; down {cfg.H}x{cfg.I}) bf16",
                       "ms": q_ms, "gbs": q_gbs, "bytes": qbytes, "bound": "hbm", "peak": peaks["hbm_gbs"],
                       "frac": q_gbs / peaks["hbm_gbs"]},
@@ -481,6 +485,52 @@ def run_ours(args, cfg):
         print(json.dumps(line), flush=True)
     dist.close()
     return 0
+
+
+def block_stats_report(c, cfg, bf16_weights, W, stream, dist, peaks):
+    """Block-scale distortion statistics of the quantised experts (gate, up and
+    down of every expert): outlier share (|w| > 0.1), relative RMS error over
+    all weights, over the neighbours of outliers and over clean blocks, and
+    the share of subnormal-scale blocks and clamped elements; plus the time
+    and bandwidth of the statistics kernel (2.5625 bytes read per element)."""
+    enc = ((W.gate_codes, W.gate_scales, W.gate_gscale), (W.up_codes, W.up_scales, W.up_gscale),
+           (W.down_codes, W.down_scales, W.down_gscale))
+    bufs = [torch.empty((w.shape[0], len(c.BLOCK_STATS_FIELDS)), dtype=torch.int64, device=w.device)
+            for w in bf16_weights]
+
+    def run():
+        for w, (cd, sc, g), b in zip(bf16_weights, enc, bufs):
+            c.nvfp4_block_stats_compute(w, cd, sc, g, "tiled", 0.1, stats=b)
+
+    run()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(5):
+        run()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = dist.max(e0.elapsed_time(e1)) / 5
+    tot = dict.fromkeys(c.BLOCK_STATS_FIELDS, 0)
+    for b in bufs:
+        for d in c.block_stats_to_dicts(b):
+            for k, v in d.items():
+                tot[k] += v
+    rel = lambda sse, sq: (sse / sq) ** 0.5 if sq > 0 else 0.0   # noqa: E731
+    nbytes = tot["elements"] * 2.5625
+    return {
+        "tensors": f"{cfg.E} x (gate, up, down)", "outlier_threshold": 0.1,
+        "outlier_share": tot["outliers"] / tot["elements"],
+        "outlier_block_share": tot["outlier_blocks"] / tot["blocks"],
+        "rel_rms_error": rel(tot["sse"], tot["sum_sq"]),
+        "rel_rms_error_neighbours": rel(tot["sse_neighbours"], tot["sum_sq_neighbours"]),
+        "rel_rms_error_clean": rel(tot["sse_clean"], tot["sum_sq_clean"]),
+        "subnormal_scale_block_share": tot["subnormal_scale_blocks"] / tot["blocks"],
+        "zero_scale_block_share": tot["zero_scale_blocks"] / tot["blocks"],
+        "saturated_share": tot["saturated_elements"] / tot["elements"],
+        "kernel": {"ms": ms, "gbs": nbytes / (ms * 1e-3) / 1e9, "bytes": nbytes, "bound": "hbm",
+                   "frac": nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+    }
 
 
 def weak_scaling_value(tokens_per_rank: int, world: int, max_ms_per_step: float) -> float:

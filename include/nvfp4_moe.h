@@ -247,6 +247,44 @@ NVFP4_API nvfp4_status moe_nvfp4_down(const moe_nvfp4_weights* W, const uint8_t*
                             const float* h_gscale, const float* row_weight, void* y_bf16, float* y_f32,
                             void* ws, size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------------------------------
+ * Block-scale distortion statistics (NetsPresso AQ article, section "Why
+ * 4-Bit Quantization of MoE Models Is Hard: Outliers in the Final Two
+ * Layers": the share of weights with |w| > 0.1, and the way concentrated
+ * outliers distort the NVFP4 block scale and the precision of the other
+ * weights of their block).
+ *
+ * For each of n_mats matrices w[m] ([rows][cols] bf16) and its NVFP4 encoding
+ * (codes [n_mats][rows][cols/2], scales in `layout` as the weight quantiser
+ * writes them, global_scale[n_mats]), stats[m] receives:
+ *   elements, outliers            elements; elements with |w| > threshold
+ *   blocks, outlier_blocks        16-element blocks; blocks holding an outlier
+ *   zero_scale_blocks             blocks with scale code 0
+ *   subnormal_scale_blocks        blocks with an E4M3 subnormal scale (codes 1..7)
+ *   saturated_elements            |fl32(w * fl32(1/S))| > 6, S = fl32(E4M3(s) g):
+ *                                 elements the E2M1 conversion clamps
+ *   neighbours, clean             non-outlier elements of outlier blocks;
+ *                                 elements of blocks without outliers
+ *   sum_sq, sse                   sum of w^2 and of (w - dq)^2, where
+ *                                 dq = fl32(fl32(E2M1(q) E4M3(s)) g)
+ *   *_neighbours, *_clean         the same two sums over those subsets
+ * Counts are exact.  The sums are taken in fp32 within a block and in fp64
+ * across blocks, which keeps them within about 1e-6 relative.  `stats`
+ * is device memory of n_mats entries; the call overwrites it.  Needs
+ * cols % 16 == 0 (TILED: cols % 64 == 0, rows % 128 == 0), w 16-byte and
+ * codes and stats 8-byte aligned.  Reads 2.5625 bytes per element.
+ * ---------------------------------------------------------------------- */
+typedef struct {
+  uint64_t elements, outliers, blocks, outlier_blocks, zero_scale_blocks, subnormal_scale_blocks,
+      saturated_elements, neighbours, clean;
+  double sum_sq, sse, sum_sq_neighbours, sse_neighbours, sum_sq_clean, sse_clean;
+} nvfp4_block_stats;
+
+NVFP4_API nvfp4_status nvfp4_block_stats_compute(const void* w_bf16, const uint8_t* codes, const uint8_t* scales,
+                                                 const float* global_scale, int n_mats, int rows, int cols,
+                                                 int layout, float outlier_threshold, nvfp4_block_stats* stats,
+                                                 void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -85,6 +85,7 @@ _declare("moe_nvfp4_gate_up", _i, ctypes.POINTER(MoeWeightsStruct), _vp, _vp, _v
 _declare("moe_nvfp4_down", _i, ctypes.POINTER(MoeWeightsStruct), _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp,
          _vp, _sz, _vp)
 
+_declare("nvfp4_block_stats_compute", _i, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _vp)
 _declare("nvfp4_test_e2m1", _i, _vp, _i, _vp, _vp, _vp)
 _declare("nvfp4_test_e2m1_sweep", _i, ctypes.c_uint32, ctypes.c_uint64, _vp, _vp, _vp)
 _declare("nvfp4_test_e4m3", _i, _vp, _i, _vp, _vp, _vp)
@@ -97,6 +98,7 @@ EXPORTS = ("nvfp4_last_error", "nvfp4_abi_version", "nvfp4_workspace_status",
            "nvfp4_quantize_act",
            "moe_route_rows_capacity", "moe_route_workspace_size", "moe_route", "moe_nvfp4_workspace_size",
            "moe_nvfp4_forward", "moe_nvfp4_gemm_workspace_size", "moe_nvfp4_gate_up", "moe_nvfp4_down",
+           "nvfp4_block_stats_compute",
            "nvfp4_test_e2m1", "nvfp4_test_e2m1_sweep", "nvfp4_test_e4m3", "nvfp4_test_sigmoid",
            "nvfp4_test_mma_peak")
 
@@ -204,6 +206,36 @@ def nvfp4_quantize_act(x: torch.Tensor, gscale: torch.Tensor, layout: str = "can
         scales = torch.empty((rows, cols // 16), dtype=torch.uint8, device=x.device)
     _check(lib.nvfp4_quantize_act(_p(x), rows, cols, _p(gscale), lay, _p(codes), _p(scales), _stream()))
     return codes, scales
+
+
+#: Fields of nvfp4_block_stats, in declaration order (9 uint64 counts, 6 fp64 sums).
+BLOCK_STATS_FIELDS = ("elements", "outliers", "blocks", "outlier_blocks", "zero_scale_blocks",
+                      "subnormal_scale_blocks", "saturated_elements", "neighbours", "clean", "sum_sq", "sse",
+                      "sum_sq_neighbours", "sse_neighbours", "sum_sq_clean", "sse_clean")
+
+
+def nvfp4_block_stats_compute(w: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, gscale: torch.Tensor,
+                              layout: str = "tiled", threshold: float = 0.1, stats: torch.Tensor | None = None):
+    """Block-scale distortion statistics of n_mats NVFP4 tensors.  Returns the
+    device buffer ([n_mats, 15] int64 words: 9 counts, then 6 fp64 sums bit-cast);
+    ``block_stats_to_dicts`` turns it into one dict per matrix."""
+    _cuda(w, torch.bfloat16, "w")
+    if w.dim() == 2:
+        w = w.unsqueeze(0)
+    n, rows, cols = w.shape
+    _cuda(gscale, torch.float32, "gscale")
+    if stats is None:
+        stats = torch.empty((n, len(BLOCK_STATS_FIELDS)), dtype=torch.int64, device=w.device)
+    _check(lib.nvfp4_block_stats_compute(_p(w), _p(codes), _p(scales), _p(gscale), n, rows, cols,
+                                         _LAYOUTS[layout], float(threshold), _p(stats), _stream()))
+    return stats
+
+
+def block_stats_to_dicts(stats: torch.Tensor) -> list[dict]:
+    h = stats.cpu()
+    counts = h[:, :9].tolist()
+    sums = h[:, 9:].contiguous().view(torch.float64).tolist()
+    return [dict(zip(BLOCK_STATS_FIELDS, c + s)) for c, s in zip(counts, sums)]
 
 
 # ---------------------------------------------------------------------------
