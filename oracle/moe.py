@@ -28,6 +28,13 @@ R12 the routing weight scales each expert's down-projection output; the
     combine sums the k weighted rows of a token in slot order.
 R13 each expert's rows are padded to a multiple of 128; padded rows hold no
     token (perm = -1) and never reach the output.
+R16 activation global scales, beyond R8 (the extension "per-expert
+    activation global scales plus an on-device dynamic amax mode"): g1 and g2
+    may instead be one fp32 per expert, the rows of expert e quantised under
+    g1[e] and g2[e]; in the dynamic modes g1 is derived from the batch itself
+    with the weight rule R1, g1 = fl32(amax / 2688), over the whole batch x
+    ("dynamic") or over the tokens routed to each expert ("dynamic_expert";
+    an expert without tokens gets 0).  h keeps a caller-supplied g2.
 """
 from __future__ import annotations
 
@@ -174,23 +181,62 @@ def expert_down(h_codes, h_scales, g2, down) -> np.ndarray:
     return acc * (float(g2) * float(down[2]))
 
 
+def activation_scales(x, g1, num_experts, topk_idx_all=None):
+    """The x global scale(s) of R8/R16: a scalar or [E] array as given, or
+    derived from the batch ``x`` ([T, H], all tokens) for "dynamic" (one
+    scalar) and "dynamic_expert" (one per expert over the tokens that
+    ``topk_idx_all`` [T, k] routes to it)."""
+    if isinstance(g1, str):
+        x = np.abs(np.asarray(x, F32))
+        if g1 == "dynamic":
+            return F32(F32(x.max() if x.size else 0) / nvfp4.GLOBAL_DIVISOR)
+        if g1 == "dynamic_expert":
+            tmax = x.max(axis=1) if x.size else np.zeros(x.shape[0], F32)
+            g = np.zeros(num_experts, F32)
+            for e in range(num_experts):
+                t = np.nonzero(np.any(topk_idx_all == e, axis=1))[0]
+                g[e] = F32(F32(tmax[t].max()) / nvfp4.GLOBAL_DIVISOR) if t.size else F32(0)
+            return g
+        raise ValueError(f"unknown activation scale mode {g1!r}")
+    return np.asarray(g1, F32) if np.ndim(g1) else F32(g1)
+
+
+def _scale_of(g, e):
+    """The global scale of expert e: g itself when per tensor, g[e] when per expert."""
+    return F32(g[e]) if np.ndim(g) else F32(g)
+
+
 def moe_layer(x, router_weight, bias, k, rsf, experts, g1, g2,
-              logit_offset=None, tokens=None, logits=None):
+              logit_offset=None, tokens=None, logits=None, topk_idx_all=None):
     """The NVFP4 W4A4 routed-expert layer for the tokens ``tokens`` (all if None).
 
     ``experts(e)`` returns ((gate codes, scales, g), (up ...), (down ...)) for
-    expert e, canonical layouts.  Activations are quantised once per token
-    under g1; h under g2.  Returns a dict with ``out`` (bf16 values as fp32,
-    [len(tokens), H]), the routing and each token's per-slot h and y.
+    expert e, canonical layouts.  ``g1`` is the x global scale: a scalar (R8),
+    an [E] array, or "dynamic" / "dynamic_expert" (R16); ``g2`` (for h) is a
+    scalar or an [E] array.  The rows of expert e are quantised under its
+    scales.  Returns a dict with ``out`` (bf16 values as fp32, [len(tokens),
+    H]), the routing, each token's per-slot h and y, and the scales used.
 
-    Because routing is per token, evaluating a subset of tokens is exact."""
+    Because routing is per token, evaluating a subset of tokens is exact; the
+    dynamic modes take their amax over the whole batch ``x``, and
+    "dynamic_expert" needs the routing of every token (``topk_idx_all``,
+    computed here when not given)."""
     x = np.asarray(x, F32)
     T, H = x.shape
     tok = np.arange(T) if tokens is None else np.asarray(tokens)
     if logits is None:
         logits = router_logits(x[tok], router_weight, logit_offset)
     topk_idx, topk_w = route(logits, bias, k, rsf)
-    a_codes, a_scales = nvfp4.quantize(x[tok], g1)
+    E = len(bias)
+    if isinstance(g1, str) and g1 == "dynamic_expert" and topk_idx_all is None:
+        topk_idx_all = route(router_logits(x, router_weight, logit_offset), bias, k, rsf)[0]
+    g1 = activation_scales(x, g1, E, topk_idx_all)
+    g2 = np.asarray(g2, F32) if np.ndim(g2) else F32(g2)
+    per_expert_x = np.ndim(g1) > 0
+    if not per_expert_x:
+        a_codes, a_scales = nvfp4.quantize(x[tok], g1)
+    else:
+        a_codes = a_scales = None
     cache = {}
     out = np.zeros((len(tok), H), np.float64)
     h_all, y_all = {}, {}
@@ -200,16 +246,21 @@ def moe_layer(x, router_weight, bias, k, rsf, experts, g1, g2,
         if e not in cache:
             cache[e] = experts(int(e))
         gate, up, down = cache[e]
-        _, _, h = expert_gate_up(a_codes[ti], a_scales[ti], g1, gate, up)
-        hc, hs = nvfp4.quantize(h, g2)
-        y = expert_down(hc, hs, g2, down)
+        g1e, g2e = _scale_of(g1, e), _scale_of(g2, e)
+        if per_expert_x:
+            ac, asc = nvfp4.quantize(x[tok[ti]], g1e)
+        else:
+            ac, asc = a_codes[ti], a_scales[ti]
+        _, _, h = expert_gate_up(ac, asc, g1e, gate, up)
+        hc, hs = nvfp4.quantize(h, g2e)
+        y = expert_down(hc, hs, g2e, down)
         for r in range(len(ti)):
             out[ti[r]] += float(topk_w[ti[r], sj[r]]) * y[r]
             h_all[(int(tok[ti[r]]), int(sj[r]))] = h[r]
             y_all[(int(tok[ti[r]]), int(sj[r]))] = y[r]
     return {"out": nvfp4.bf16_round(out), "out_f64": out, "topk_idx": topk_idx,
             "topk_w": topk_w, "logits": logits, "h": h_all, "y": y_all,
-            "a_codes": a_codes, "a_scales": a_scales}
+            "a_codes": a_codes, "a_scales": a_scales, "g1": g1, "g2": g2}
 
 
 def dense_moe_layer(x, router_weight, bias, k, rsf, experts_bf16,

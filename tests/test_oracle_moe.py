@@ -186,3 +186,69 @@ def test_layer_token_subset_is_exact():
     full = moe.moe_layer(x, wg, bias, cfg.k, cfg.rsf, lambda e: q[e], g1, g2)
     sub = moe.moe_layer(x, wg, bias, cfg.k, cfg.rsf, lambda e: q[e], g1, g2, tokens=[3, 17, 30])
     np.testing.assert_array_equal(sub["out"], full["out"][[3, 17, 30]])
+
+
+# --- activation global scales per expert and from the batch (reading R16) ---
+
+def _zero_except(q, keep):
+    """Expert weights with every expert but ``keep`` replaced by zeros."""
+    def ex(e):
+        if e == keep:
+            return q[e]
+        return tuple((np.zeros_like(c), np.zeros_like(s), g) for c, s, g in q[e])
+    return ex
+
+
+def test_per_expert_scales_equal_to_one_value_reproduce_the_tensor_mode():
+    cfg, x, wg, bias, bf, q = _tiny_layer()
+    g1, g2 = F32(0.0023), F32(0.0004)
+    ref = moe.moe_layer(x, wg, bias, cfg.k, cfg.rsf, lambda e: q[e], g1, g2)
+    got = moe.moe_layer(x, wg, bias, cfg.k, cfg.rsf, lambda e: q[e], np.full(cfg.E, g1, F32),
+                        np.full(cfg.E, g2, F32))
+    np.testing.assert_array_equal(got["out_f64"], ref["out_f64"])
+
+
+def test_per_expert_scales_sum_of_single_expert_layers():
+    """The per-expert layer equals the sum over experts of the per-tensor layer
+    run with that expert's (g1, g2) and every other expert zeroed: a second
+    route through the per-tensor code for each expert's share."""
+    cfg, x, wg, bias, bf, q = _tiny_layer()
+    rng = np.random.default_rng(5)
+    g1 = (F32(0.002) * (1 + rng.random(cfg.E))).astype(F32)
+    g2 = (F32(0.0003) * (1 + rng.random(cfg.E))).astype(F32)
+    got = moe.moe_layer(x, wg, bias, cfg.k, cfg.rsf, lambda e: q[e], g1, g2)
+    acc = np.zeros_like(got["out_f64"])
+    for e in range(cfg.E):
+        acc += moe.moe_layer(x, wg, bias, cfg.k, cfg.rsf, _zero_except(q, e), g1[e], g2[e])["out_f64"]
+    np.testing.assert_allclose(got["out_f64"], acc, rtol=1e-12, atol=1e-15)
+
+
+def test_dynamic_scale_is_invariant_to_power_of_two_rescaling():
+    """With g1 taken from the batch, x and 2^j x quantise to the same codes
+    and block scales: the global scale moves by exactly 2^j."""
+    cfg, x, wg, bias, bf, q = _tiny_layer()
+    a = moe.moe_layer(x, wg, bias, cfg.k, cfg.rsf, lambda e: q[e], "dynamic", F32(0.0004))
+    b = moe.moe_layer((x * F32(8.0)).astype(F32), wg, bias, cfg.k, cfg.rsf, lambda e: q[e], "dynamic", F32(0.0004),
+                      logits=a["logits"])
+    assert b["g1"] == a["g1"] * 8
+    np.testing.assert_array_equal(a["a_codes"], b["a_codes"])
+    np.testing.assert_array_equal(a["a_scales"], b["a_scales"])
+    # the batch amax block lands on the top of the E4M3 range
+    assert a["a_scales"].max() == 0x7E
+
+
+def test_dynamic_expert_scales_bound_the_dynamic_scale():
+    cfg, x, wg, bias, bf, q = _tiny_layer()
+    res = moe.moe_layer(x, wg, bias, cfg.k, cfg.rsf, lambda e: q[e], "dynamic_expert", np.full(cfg.E, F32(4e-4)))
+    g_all = moe.activation_scales(x, "dynamic", cfg.E)
+    g = res["g1"]
+    assert g.shape == (cfg.E,) and np.all(g <= g_all)
+    t_max = int(np.argmax(np.abs(x).max(axis=1)))
+    for e in res["topk_idx"][t_max]:
+        assert g[e] == g_all                       # experts of the batch-max token
+    idle = np.setdiff1d(np.arange(cfg.E), res["topk_idx"])
+    assert np.all(g[idle] == 0)
+    # a token subset gives the same rows as the whole batch
+    sub = moe.moe_layer(x, wg, bias, cfg.k, cfg.rsf, lambda e: q[e], "dynamic_expert", np.full(cfg.E, F32(4e-4)),
+                        tokens=[1, 9])
+    np.testing.assert_array_equal(sub["out"], res["out"][[1, 9]])
