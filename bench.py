@@ -372,6 +372,27 @@ def run_ours(args, cfg):
     stage_ms = {n: dist.max(float(np.mean([evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps)])))
                 for j, n in enumerate(stage_names)}
 
+    # the activation global-scale modes beyond the calibrated per-tensor one
+    # (same workload, K steps each, nothing between the kernels)
+    mode_ms = {}
+    for mode in ("expert", "dynamic", "dynamic_expert"):
+        n = cfg.E if mode in ("expert", "dynamic_expert") else 1
+        a = g1.repeat(n).contiguous() if mode == "expert" else torch.zeros(n, device=dev)
+        h = g2.repeat(n).contiguous()
+        run = lambda: c.moe_nvfp4_forward(W, x, a, h, logit_offset=off, out=out, workspace=ws,  # noqa: E731
+                                          act_scale_mode=mode)
+        for _ in range(3):
+            run()
+        torch.cuda.synchronize()
+        m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        m0.record(stream)
+        for _ in range(args.steps):
+            run()
+        m1.record(stream)
+        torch.cuda.synchronize()
+        mode_ms[mode] = dist.max(m0.elapsed_time(m1)) / args.steps
+    c.nvfp4_workspace_status(ws)
+
     # end to end: pinned host x in, host out back, through the same call
     x_h = x.cpu().pin_memory()
     out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
@@ -470,6 +491,7 @@ def run_ours(args, cfg):
         "gemm": {"ms": gemm_ms, "tflops": (gu_flops + dn_flops) / (gemm_ms * 1e-3) / 1e12,
                  "frac_of_fp4_peak": (gu_flops + dn_flops) / (gemm_ms * 1e-3) / 1e12 / fp4_peak},
         "stages_ms": stage_ms,
+        "act_scale_modes_ms_per_step": dict({"tensor": ms_step}, **mode_ms),
         "roofline": roof,
         "diagnostics": diag,
         "quantiser": {"workload": f"quantiser: {cfg.E} x (gate, up {cfg.I}x{cfg.H}; down {cfg.H}x{cfg.I}) bf16",

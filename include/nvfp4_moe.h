@@ -197,7 +197,8 @@ typedef struct moe_nvfp4_debug {
   uint8_t* a_codes;               /* [rows][H/2] quantised x in permuted order   */
   uint8_t* a_scales;              /* TILED, rows x H                             */
   float* h;                       /* [rows][I] silu(gate)*up before requantising */
-  float* h_amax;                  /* max |h| over real rows (fp32, caller zeroes)*/
+  float* h_amax;                  /* max |h| over real rows (fp32, caller zeroes);
+                                     [E], one per expert, in the per-expert modes */
   uint8_t* h_codes;               /* [rows][I/2]                                 */
   uint8_t* h_scales;              /* TILED, rows x I                             */
   float* y;                       /* [rows][H] weighted down-projection rows     */
@@ -221,6 +222,35 @@ NVFP4_API nvfp4_status moe_nvfp4_forward(const moe_nvfp4_weights* W, const void*
                                const float* act_gscale, const float* h_gscale, const float* logit_offset,
                                void* out_bf16, const moe_nvfp4_debug* dbg, void* ws, size_t ws_bytes,
                                void* stream);
+
+/* Activation global-scale modes of moe_nvfp4_forward_scaled.  The pages fix
+ * one calibrated fp32 global scale per activation tensor ("Quantization
+ * Setup"); the other modes are an extension: one scale per expert, and g1
+ * derived on the device from the batch with the weight rule
+ * g1 = fl32(amax|x| / 2688), taken over the whole batch or over the tokens
+ * routed to each expert (0 for an expert without tokens).
+ *   mode                          act_gscale              h_gscale
+ *   NVFP4_ACT_SCALE_TENSOR         [1] read                [1]
+ *   NVFP4_ACT_SCALE_EXPERT         [E] read                [E]
+ *   NVFP4_ACT_SCALE_DYNAMIC        [1] written (batch g1)  [1]
+ *   NVFP4_ACT_SCALE_DYNAMIC_EXPERT [E] written (per expert) [E]
+ * With one g1 per expert, each of a token's k permuted rows is quantised under
+ * its own expert's g1, and expert e's h rows under h_gscale[e]. */
+enum {
+  NVFP4_ACT_SCALE_TENSOR = 0,
+  NVFP4_ACT_SCALE_EXPERT = 1,
+  NVFP4_ACT_SCALE_DYNAMIC = 2,
+  NVFP4_ACT_SCALE_DYNAMIC_EXPERT = 3
+};
+
+/* moe_nvfp4_forward with a choice of activation global-scale mode (above);
+ * moe_nvfp4_forward is this call with NVFP4_ACT_SCALE_TENSOR.  Same workspace,
+ * layouts and errors; an unknown mode returns NVFP4_ERR_INVALID_ARG. */
+NVFP4_API nvfp4_status moe_nvfp4_forward_scaled(const moe_nvfp4_weights* W, const void* x_bf16, int T,
+                                                int act_scale_mode, float* act_gscale, const float* h_gscale,
+                                                const float* logit_offset, void* out_bf16,
+                                                const moe_nvfp4_debug* dbg, void* ws, size_t ws_bytes,
+                                                void* stream);
 
 /* ------------------------------------------------------------------------
  * The two grouped GEMMs on caller-supplied quantised operands (the same

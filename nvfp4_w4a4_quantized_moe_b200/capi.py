@@ -79,6 +79,8 @@ _declare("moe_route", _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _vp,
 _declare("moe_nvfp4_workspace_size", _sz, _i, _i, _i, _i, _i)
 _declare("moe_nvfp4_forward", _i, ctypes.POINTER(MoeWeightsStruct), _vp, _i, _vp, _vp, _vp, _vp,
          ctypes.POINTER(MoeDebugStruct), _vp, _sz, _vp)
+_declare("moe_nvfp4_forward_scaled", _i, ctypes.POINTER(MoeWeightsStruct), _vp, _i, _i, _vp, _vp, _vp, _vp,
+         ctypes.POINTER(MoeDebugStruct), _vp, _sz, _vp)
 _declare("moe_nvfp4_gemm_workspace_size", _sz, _i)
 _declare("moe_nvfp4_gate_up", _i, ctypes.POINTER(MoeWeightsStruct), _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp,
          _vp, _vp, _vp, _sz, _vp)
@@ -97,7 +99,8 @@ EXPORTS = ("nvfp4_last_error", "nvfp4_abi_version", "nvfp4_workspace_status",
            "nvfp4_quantize_weights_workspace_size", "nvfp4_quantize_weights", "nvfp4_quantize_weights_noalloc",
            "nvfp4_quantize_act",
            "moe_route_rows_capacity", "moe_route_workspace_size", "moe_route", "moe_nvfp4_workspace_size",
-           "moe_nvfp4_forward", "moe_nvfp4_gemm_workspace_size", "moe_nvfp4_gate_up", "moe_nvfp4_down",
+           "moe_nvfp4_forward", "moe_nvfp4_forward_scaled", "moe_nvfp4_gemm_workspace_size", "moe_nvfp4_gate_up",
+           "moe_nvfp4_down",
            "nvfp4_block_stats_compute",
            "nvfp4_test_e2m1", "nvfp4_test_e2m1_sweep", "nvfp4_test_e4m3", "nvfp4_test_sigmoid",
            "nvfp4_test_mma_peak")
@@ -322,17 +325,28 @@ def moe_nvfp4_workspace_size(T: int, E: int, H: int, I: int, k: int) -> int:
     return lib.moe_nvfp4_workspace_size(T, E, H, I, k)
 
 
+#: Activation global-scale modes of moe_nvfp4_forward_scaled (NVFP4_ACT_SCALE_*).
+ACT_SCALE_MODES = {"tensor": 0, "expert": 1, "dynamic": 2, "dynamic_expert": 3}
+
+
 def moe_nvfp4_forward(W: MoeWeights, x: torch.Tensor, act_gscale: torch.Tensor, h_gscale: torch.Tensor,
                       logit_offset: torch.Tensor | None = None, debug: bool = False,
                       out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
-                      stage_events=None):
+                      stage_events=None, act_scale_mode: str = "tensor"):
     """out [T, H] bf16; with debug=True also a dict of intermediate results.
+    ``act_scale_mode`` is one of ACT_SCALE_MODES: in "tensor" act_gscale and
+    h_gscale hold one fp32 each, in "expert" E each; in "dynamic" and
+    "dynamic_expert" the library writes g1 into act_gscale ([1] or [E]).
     ``stage_events``: optional list of 6 torch.cuda.Event(enable_timing=True),
     each already recorded once (torch creates the CUDA event lazily), which
     the library records again between the stages of the layer."""
+    mode = ACT_SCALE_MODES[act_scale_mode]
     _cuda(x, torch.bfloat16, "x")
     _cuda(act_gscale, torch.float32, "act_gscale")
     _cuda(h_gscale, torch.float32, "h_gscale")
+    n_scales = W.E if mode & 1 else 1
+    if act_gscale.numel() != n_scales or h_gscale.numel() != n_scales:
+        raise ValueError(f"act_scale_mode {act_scale_mode!r} needs {n_scales} value(s) in act_gscale and h_gscale")
     T, H = x.shape
     dev = x.device
     out = torch.empty((T, H), dtype=torch.bfloat16, device=dev) if out is None else _cuda(out, torch.bfloat16, "out")
@@ -347,7 +361,7 @@ def moe_nvfp4_forward(W: MoeWeights, x: torch.Tensor, act_gscale: torch.Tensor, 
             "logits": z(T, W.E), "topk_idx": z(T, W.k, dt=torch.int32), "topk_w": z(T, W.k),
             "expert_offsets": z(W.E + 1, dt=torch.int32), "perm": z(cap, dt=torch.int32),
             "inv_perm": z(T, W.k, dt=torch.int32), "a_codes": z(cap, W.H // 2, dt=torch.uint8),
-            "a_scales": z(tiled_scale_bytes(cap, W.H), dt=torch.uint8), "h": z(cap, W.I), "h_amax": z(1),
+            "a_scales": z(tiled_scale_bytes(cap, W.H), dt=torch.uint8), "h": z(cap, W.I), "h_amax": z(n_scales),
             "h_codes": z(cap, W.I // 2, dt=torch.uint8), "h_scales": z(tiled_scale_bytes(cap, W.I), dt=torch.uint8),
             "y": z(cap, W.H),
         }
@@ -363,8 +377,13 @@ def moe_nvfp4_forward(W: MoeWeights, x: torch.Tensor, act_gscale: torch.Tensor, 
                 dbg.stage_events[i] = ev.cuda_event
         dbg_ptr = ctypes.pointer(dbg)
     ws_struct = W.struct()
-    _check(lib.moe_nvfp4_forward(ctypes.byref(ws_struct), _p(x), T, _p(act_gscale), _p(h_gscale), _p(logit_offset),
-                                 _p(out), dbg_ptr, _p(workspace), workspace.numel(), _stream()))
+    if mode == 0:
+        _check(lib.moe_nvfp4_forward(ctypes.byref(ws_struct), _p(x), T, _p(act_gscale), _p(h_gscale),
+                                     _p(logit_offset), _p(out), dbg_ptr, _p(workspace), workspace.numel(), _stream()))
+    else:
+        _check(lib.moe_nvfp4_forward_scaled(ctypes.byref(ws_struct), _p(x), T, mode, _p(act_gscale), _p(h_gscale),
+                                            _p(logit_offset), _p(out), dbg_ptr, _p(workspace), workspace.numel(),
+                                            _stream()))
     if debug:
         dbg_tensors["workspace"] = workspace
         return out, dbg_tensors

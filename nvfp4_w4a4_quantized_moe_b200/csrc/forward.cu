@@ -15,42 +15,120 @@ namespace nvfp4moe {
 // Quantises token t's row once under g1 and writes it to each of its k
 // permuted rows: packed codes and tiled scales.  One thread per 16-element
 // block; groups of four lanes assemble a 32-bit scale word.
+// Activation global-scale modes (NVFP4_ACT_SCALE_*): bit 0 = one scale per
+// expert, bit 1 = g1 derived on the device from the batch amax.
+constexpr int kActPerExpert = 1, kActDynamic = 2;
+
+// g1 of the batch (dynamic modes): the weight rule, fl32(amax / 2688).
+NVDEV float dynamic_gscale(uint32_t amax_bits) { return __fdiv_rn(__uint_as_float(amax_bits), 2688.0f); }
+
+// Quantise x into its k permuted rows.  With one g1 for the tensor a block is
+// quantised once and written k times; with one per expert each copy is
+// quantised under its own expert's g1.  In the dynamic modes g1 comes from
+// amax_bits ([0]: batch, [1 + e]: expert e) and block (0, 0) publishes it in
+// act_gscale.
+template <int MODE>
 __global__ void __launch_bounds__(128) quantize_scatter_kernel(const uint4* __restrict__ x, int T, int H,
-                                                               const float* __restrict__ gscale,
-                                                               const int32_t* __restrict__ inv_perm, int k,
+                                                               float* __restrict__ act_gscale,
+                                                               const uint32_t* __restrict__ amax_bits,
+                                                               const int32_t* __restrict__ inv_perm,
+                                                               const int32_t* __restrict__ topk_idx, int k, int E,
                                                                uint2* __restrict__ a_codes,
                                                                uint8_t* __restrict__ a_scales) {
   // block (t, by): token t, 16-element blocks [128 by, 128 by + 128) of its row
   __shared__ int32_t rows[16];
+  __shared__ float gs[16];
   griddep_wait();
   griddep_launch();
   const int t = blockIdx.x;
-  if (threadIdx.x < k) rows[threadIdx.x] = inv_perm[(size_t)t * k + threadIdx.x];
+  if (threadIdx.x < k) {
+    rows[threadIdx.x] = inv_perm[(size_t)t * k + threadIdx.x];
+    if (MODE & kActPerExpert) {
+      const int e = topk_idx[(size_t)t * k + threadIdx.x];
+      gs[threadIdx.x] = (MODE & kActDynamic) ? dynamic_gscale(amax_bits[1 + e]) : act_gscale[e];
+    }
+  }
+  if ((MODE & kActDynamic) && blockIdx.x == 0 && blockIdx.y == 0) {
+    if (MODE & kActPerExpert) {
+      for (int e = threadIdx.x; e < E; e += blockDim.x) act_gscale[e] = dynamic_gscale(amax_bits[1 + e]);
+    } else if (threadIdx.x == 0) {
+      act_gscale[0] = dynamic_gscale(amax_bits[0]);
+    }
+  }
   __syncthreads();
-  const float g = *gscale;
-  const float d = __fmul_rn(6.0f, g);
   const int nblk = H / kQBlock;
   const int lane = threadIdx.x & 31;
   const int kb = blockIdx.y * blockDim.x + threadIdx.x;
   const bool valid = kb < nblk;
-  uint2 c = make_uint2(0, 0);
-  uint32_t s = 0;
+  uint4 u0 = make_uint4(0, 0, 0, 0), u1 = u0;
   if (valid) {
     const uint4* src = x + ((size_t)t * H + (size_t)kb * kQBlock) / 8;
-    s = quant_block16_bf16(__ldg(src), __ldg(src + 1), g, d, c);
+    u0 = __ldg(src);
+    u1 = __ldg(src + 1);
   }
-  const uint32_t w1 = __shfl_down_sync(0xffffffffu, s, 1);
-  const uint32_t w2 = __shfl_down_sync(0xffffffffu, s, 2);
-  const uint32_t w3 = __shfl_down_sync(0xffffffffu, s, 3);
-  const uint32_t word = s | (w1 << 8) | (w2 << 16) | (w3 << 24);
-  if (valid) {
-    for (int j = 0; j < k; ++j) {
-      const int row = rows[j];
+  auto write = [&](int row, const uint2& c, uint32_t s) {
+    const uint32_t w1 = __shfl_down_sync(0xffffffffu, s, 1);
+    const uint32_t w2 = __shfl_down_sync(0xffffffffu, s, 2);
+    const uint32_t w3 = __shfl_down_sync(0xffffffffu, s, 3);
+    const uint32_t word = s | (w1 << 8) | (w2 << 16) | (w3 << 24);
+    if (valid) {
       a_codes[(size_t)row * nblk + kb] = c;
-      if ((lane & 3) == 0)
-        *reinterpret_cast<uint32_t*>(a_scales + tiled_scale_offset(row, kb, nblk >> 2)) = word;
+      if ((lane & 3) == 0) *reinterpret_cast<uint32_t*>(a_scales + tiled_scale_offset(row, kb, nblk >> 2)) = word;
     }
+  };
+  if (MODE & kActPerExpert) {
+    for (int j = 0; j < k; ++j) {
+      const float g = gs[j];
+      uint2 c = make_uint2(0, 0);
+      uint32_t s = 0;
+      if (valid) s = quant_block16_bf16(u0, u1, g, __fmul_rn(6.0f, g), c);
+      write(rows[j], c, s);
+    }
+  } else {
+    const float g = (MODE & kActDynamic) ? dynamic_gscale(amax_bits[0]) : act_gscale[0];
+    uint2 c = make_uint2(0, 0);
+    uint32_t s = 0;
+    if (valid) s = quant_block16_bf16(u0, u1, g, __fmul_rn(6.0f, g), c);
+    for (int j = 0; j < k; ++j) write(rows[j], c, s);
   }
+}
+
+// amax |x| of every token (exact, on packed bf16 pairs) into tok_amax[t] and
+// the batch amax into amax_bits[0].  Non-negative floats order like their
+// bits, so the maxima are integer atomics.
+__global__ void __launch_bounds__(256) token_amax_kernel(const uint4* __restrict__ x, int H,
+                                                         uint32_t* __restrict__ tok_amax,
+                                                         uint32_t* __restrict__ amax_bits) {
+  const int t = blockIdx.x;
+  const int vpr = H / 8;
+  __nv_bfloat162 m2 = __floats2bfloat162_rn(0.0f, 0.0f);
+  for (int c = threadIdx.x; c < vpr; c += blockDim.x) {
+    const uint4 u = __ldg(x + (size_t)t * vpr + c);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) m2 = __hmax2(m2, __habs2(*reinterpret_cast<const __nv_bfloat162*>(&w[j])));
+  }
+  uint32_t mb = __float_as_uint(fmaxf(__low2float(m2), __high2float(m2)));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, o));
+  __shared__ uint32_t red[8];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mb;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int i = 1; i < (int)(blockDim.x >> 5); ++i) mb = max(mb, red[i]);
+    tok_amax[t] = mb;
+    atomicMax(amax_bits, mb);
+  }
+}
+
+// amax of the tokens routed to each expert: amax_bits[1 + e].
+__global__ void __launch_bounds__(256) expert_amax_kernel(const int32_t* __restrict__ topk_idx, int T, int k,
+                                                          const uint32_t* __restrict__ tok_amax,
+                                                          uint32_t* __restrict__ amax_bits) {
+  griddep_wait();
+  griddep_launch();
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < T * k) atomicMax(amax_bits + 1 + topk_idx[i], tok_amax[i / k]);
 }
 
 // out[t] = bf16( sum_j y[inv_perm[t, j]] ), fp32 sum in slot order.  The
@@ -103,6 +181,8 @@ struct ForwardScratch {
   uint8_t* h_codes;
   uint8_t* h_scales;
   uint16_t* y;
+  uint32_t* amax_bits;      // [E + 1] batch amax, then per expert (dynamic modes)
+  uint32_t* tok_amax;       // [T]
 };
 
 static ForwardScratch carve_forward(Carver& c, int T, int E, int H, int I, int k) {
@@ -120,6 +200,8 @@ static ForwardScratch carve_forward(Carver& c, int T, int E, int H, int I, int k
   f.h_codes = c.take<uint8_t>((size_t)cap * I / 2);
   f.h_scales = c.take<uint8_t>((size_t)cap * I / 16);
   f.y = c.take<uint16_t>((size_t)cap * H);
+  f.amax_bits = c.take<uint32_t>((size_t)E + 1);
+  f.tok_amax = c.take<uint32_t>((size_t)T);
   return f;
 }
 
@@ -144,11 +226,21 @@ extern "C" size_t moe_nvfp4_workspace_size(int T, int E, int H, int I, int k) {
   return c.size();
 }
 
-extern "C" nvfp4_status moe_nvfp4_forward(const moe_nvfp4_weights* W, const void* x_bf16, int T,
-                                          const float* act_gscale, const float* h_gscale, const float* logit_offset,
-                                          void* out_bf16, const moe_nvfp4_debug* dbg, void* ws, size_t ws_bytes,
-                                          void* stream) {
+template <int MODE>
+static nvfp4_status launch_quantize_scatter(const ForwardScratch& f, const void* x_bf16, int T, int H, int E, int k,
+                                            float* act_gscale, cudaStream_t s) {
+  return launch_dependent("quantize_scatter_kernel", quantize_scatter_kernel<MODE>,
+                          dim3(T, (H / kQBlock + 127) / 128), dim3(128), 0, s, static_cast<const uint4*>(x_bf16), T,
+                          H, act_gscale, (const uint32_t*)f.amax_bits, (const int32_t*)f.inv_perm,
+                          (const int32_t*)f.topk_idx, k, E, reinterpret_cast<uint2*>(f.a_codes), f.a_scales);
+}
+
+static nvfp4_status forward_impl(const moe_nvfp4_weights* W, const void* x_bf16, int T, int mode, float* act_gscale,
+                                 const float* h_gscale, const float* logit_offset, void* out_bf16,
+                                 const moe_nvfp4_debug* dbg, void* ws, size_t ws_bytes, void* stream) {
   NV_CHECK(nvfp4moe_check_weights(W));
+  NV_REQUIRE(mode >= NVFP4_ACT_SCALE_TENSOR && mode <= NVFP4_ACT_SCALE_DYNAMIC_EXPERT, NVFP4_ERR_INVALID_ARG,
+             "moe_nvfp4_forward: unknown activation scale mode %d", mode);
   NV_REQUIRE(x_bf16 && act_gscale && h_gscale && out_bf16, NVFP4_ERR_INVALID_ARG,
              "moe_nvfp4_forward: x, act_gscale, h_gscale and out are required");
   NV_REQUIRE(W->router_weight && W->bias && W->gate_codes && W->gate_scales && W->gate_gscale && W->up_codes &&
@@ -173,6 +265,12 @@ extern "C" nvfp4_status moe_nvfp4_forward(const moe_nvfp4_weights* W, const void
 
   NV_CHECK(check_cuda(cudaMemsetAsync(f.route.status, 0, sizeof(uint32_t), s), "clear status word"));
   NV_CHECK(mark(dbg, 0, s));
+  if (mode & kActDynamic) {
+    // 0: amax of every token and of the batch
+    NV_CHECK(check_cuda(cudaMemsetAsync(f.amax_bits, 0, sizeof(uint32_t) * (size_t)(E + 1), s), "clear amax"));
+    token_amax_kernel<<<T, 256, 0, s>>>(static_cast<const uint4*>(x_bf16), H, f.tok_amax, f.amax_bits);
+    NV_CHECK(check_launch("token_amax_kernel"));
+  }
   // 1-3: router, top-k, permutation
   RouteArgs ra;
   ra.x = x_bf16;
@@ -186,12 +284,19 @@ extern "C" nvfp4_status moe_nvfp4_forward(const moe_nvfp4_weights* W, const void
   NV_CHECK(launch_route(ra, f.route, s));
   NV_CHECK(mark(dbg, 1, s));
 
-  // 4: quantise x once per token into its k permuted rows.  Padding rows are
-  // left as they are: an MMA row only feeds the same output row, and the
-  // epilogues skip padding rows.
-  NV_CHECK(launch_dependent("quantize_scatter_kernel", quantize_scatter_kernel, dim3(T, (H / kQBlock + 127) / 128),
-                            dim3(128), 0, s, static_cast<const uint4*>(x_bf16), T, H, act_gscale,
-                            (const int32_t*)f.inv_perm, k, reinterpret_cast<uint2*>(f.a_codes), f.a_scales));
+  // 4: quantise x into its k permuted rows (under the batch's or each
+  // expert's g1).  Padding rows are left as they are: an MMA row only feeds
+  // the same output row, and the epilogues skip padding rows.
+  if (mode == NVFP4_ACT_SCALE_DYNAMIC_EXPERT) {
+    NV_CHECK(launch_dependent("expert_amax_kernel", expert_amax_kernel, dim3((T * k + 255) / 256), dim3(256), 0, s,
+                              (const int32_t*)f.topk_idx, T, k, (const uint32_t*)f.tok_amax, f.amax_bits));
+  }
+  switch (mode) {
+    case NVFP4_ACT_SCALE_TENSOR: NV_CHECK(launch_quantize_scatter<0>(f, x_bf16, T, H, E, k, act_gscale, s)); break;
+    case NVFP4_ACT_SCALE_EXPERT: NV_CHECK(launch_quantize_scatter<1>(f, x_bf16, T, H, E, k, act_gscale, s)); break;
+    case NVFP4_ACT_SCALE_DYNAMIC: NV_CHECK(launch_quantize_scatter<2>(f, x_bf16, T, H, E, k, act_gscale, s)); break;
+    default: NV_CHECK(launch_quantize_scatter<3>(f, x_bf16, T, H, E, k, act_gscale, s)); break;
+  }
   NV_CHECK(mark(dbg, 2, s));
 
   // 5-6: gate/up GEMM with SiLU*up and requantisation
@@ -208,6 +313,7 @@ extern "C" nvfp4_status moe_nvfp4_forward(const moe_nvfp4_weights* W, const void
   g1.h_gscale = h_gscale; g1.h_codes = f.h_codes; g1.h_scales = f.h_scales;
   g1.h_f32 = dbg ? dbg->h : nullptr;
   g1.h_amax = dbg ? dbg->h_amax : nullptr;
+  g1.per_expert_scales = (mode & kActPerExpert) != 0;
   g1.status = f.route.status;
   NV_CHECK(launch_grouped_gemm(g1, s));
   NV_CHECK(mark(dbg, 3, s));
@@ -223,6 +329,7 @@ extern "C" nvfp4_status moe_nvfp4_forward(const moe_nvfp4_weights* W, const void
   g2.tile_expert = f.route.tile_expert; g2.num_mtiles = f.route.num_mtiles;
   g2.expert_offsets = f.offsets; g2.expert_counts = f.route.counts;
   g2.row_w = f.route.row_w; g2.y_bf16 = f.y; g2.y_f32 = dbg ? dbg->y : nullptr;
+  g2.per_expert_scales = (mode & kActPerExpert) != 0;
   g2.status = f.route.status;
   NV_CHECK(launch_grouped_gemm(g2, s));
   NV_CHECK(mark(dbg, 4, s));
@@ -248,4 +355,22 @@ extern "C" nvfp4_status moe_nvfp4_forward(const moe_nvfp4_weights* W, const void
     NV_CHECK(copy_out(dbg->h_scales, f.h_scales, (size_t)cap * I / 16, s));
   }
   return NVFP4_OK;
+}
+
+extern "C" nvfp4_status moe_nvfp4_forward(const moe_nvfp4_weights* W, const void* x_bf16, int T,
+                                          const float* act_gscale, const float* h_gscale, const float* logit_offset,
+                                          void* out_bf16, const moe_nvfp4_debug* dbg, void* ws, size_t ws_bytes,
+                                          void* stream) {
+  // the tensor mode only reads act_gscale
+  return forward_impl(W, x_bf16, T, NVFP4_ACT_SCALE_TENSOR, const_cast<float*>(act_gscale), h_gscale, logit_offset,
+                      out_bf16, dbg, ws, ws_bytes, stream);
+}
+
+extern "C" nvfp4_status moe_nvfp4_forward_scaled(const moe_nvfp4_weights* W, const void* x_bf16, int T,
+                                                 int act_scale_mode, float* act_gscale, const float* h_gscale,
+                                                 const float* logit_offset, void* out_bf16,
+                                                 const moe_nvfp4_debug* dbg, void* ws, size_t ws_bytes,
+                                                 void* stream) {
+  return forward_impl(W, x_bf16, T, act_scale_mode, act_gscale, h_gscale, logit_offset, out_bf16, dbg, ws, ws_bytes,
+                      stream);
 }

@@ -80,6 +80,7 @@ struct GemmParams {
   uint16_t* y_bf16;
   float* y_f32;
   int H;
+  int per_expert;       // g_act, g_h and h_amax are [E] arrays
   uint32_t* status;
 };
 
@@ -285,7 +286,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int half = (warp - 2) >> 2;
     const int row_in_tile = quad * 32 + lane;
     const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16);
-    const float g_act = *p.g_act;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
       const int mt = t / p.n_tiles, nt = t % p.n_tiles;
@@ -297,6 +297,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
+      const int se = p.per_expert ? e : 0;                  // index of this tile's scales
+      const float g_act = p.g_act[se];
       if (EPI == kEpiGateUp) {
         const float sg = __fmul_rn(g_act, p.g_b0[e]);
         const float su = __fmul_rn(g_act, p.g_b1[e]);
@@ -322,7 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float up = __fmul_rn(__uint_as_float(ru[i]), su);
             h[i] = __fmul_rn(silu(gate), up);
           }
-          const float g2 = *p.g_h;
+          const float g2 = p.g_h[se];
           const float d2 = __fmul_rn(6.0f, g2);
           uint2 c0, c1, c2, c3;
           const uint32_t s0 = quant_block16(h, g2, d2, c0);
@@ -341,7 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             float m = 0.0f;
 #pragma unroll
             for (int i = 0; i < 64; ++i) m = fmaxf(m, fabsf(h[i]));
-            atomicMax(reinterpret_cast<unsigned int*>(p.h_amax), __float_as_uint(m));
+            atomicMax(reinterpret_cast<unsigned int*>(p.h_amax + se), __float_as_uint(m));
           }
         }
         uint4* cdst = reinterpret_cast<uint4*>(p.h_codes + (size_t)grow * (p.I / 2) + hcol0 / 2);
@@ -469,6 +471,7 @@ nvfp4_status launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t s) {
   p.y_bf16 = static_cast<uint16_t*>(a.y_bf16);
   p.y_f32 = a.y_f32;
   p.H = a.H;
+  p.per_expert = a.per_expert_scales ? 1 : 0;
   p.status = a.status;
   const int max_tiles = a.rows_capacity / kBM * p.n_tiles;
   const int grid = std::max(1, std::min(sms, max_tiles));

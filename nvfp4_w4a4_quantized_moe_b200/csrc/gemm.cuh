@@ -24,6 +24,9 @@ struct GroupedGemmArgs {
   const uint8_t* b1_scales = nullptr;
   const float* b1_gscale = nullptr;
   const float* act_gscale = nullptr;        // g1 (gate/up) or g2 (down)
+  // act_gscale, h_gscale and h_amax hold one value per expert (indexed by the
+  // tile's expert) instead of one for the tensor
+  bool per_expert_scales = false;
   // row grouping
   const int32_t* tile_expert = nullptr;
   const int32_t* num_mtiles = nullptr;
