@@ -260,7 +260,38 @@ def moe_layer(x, router_weight, bias, k, rsf, experts, g1, g2,
             y_all[(int(tok[ti[r]]), int(sj[r]))] = y[r]
     return {"out": nvfp4.bf16_round(out), "out_f64": out, "topk_idx": topk_idx,
             "topk_w": topk_w, "logits": logits, "h": h_all, "y": y_all,
-            "a_codes": a_codes, "a_scales": a_scales, "g1": g1, "g2": g2}
+            "a_codes": a_codes, "a_scales": a_scales, "g1": g1, "g2": g2, "tokens": tok}
+
+
+def reap_saliency(result: dict, num_experts: int):
+    """REAP saliency accumulators of one batch ("K-EXAONE-152B-A23B-REAP-80E-BF16"
+    model card, "Pruning Setup": saliency = mean(topk_weight * ||f_e(x)||_2)
+    over routed tokens, with the real sigmoid-and-bias routing weights and the
+    routed_scaling_factor included).  From a ``moe_layer`` result: f_e(x) is
+    the expert's down-projection output y (before the routing weight) and
+    topk_weight the routing weight w (which carries rsf).  Returns
+    (sum [E] fp64 of w * ||y||_2, count [E]); the saliency is sum / count over
+    all calibration batches (0 where count is 0)."""
+    total = np.zeros(num_experts, np.float64)
+    count = np.zeros(num_experts, np.int64)
+    idx, w = result["topk_idx"], result["topk_w"]
+    row_of = {int(t): n for n, t in enumerate(result["tokens"])}
+    for (t, j), y in result["y"].items():
+        n = row_of[t]
+        e = int(idx[n, j])
+        total[e] += float(w[n, j]) * float(np.sqrt(np.sum(np.asarray(y, np.float64) ** 2)))
+        count[e] += 1
+    return total, count
+
+
+def reap_keep(saliency: np.ndarray, keep: int) -> np.ndarray:
+    """Experts retained by REAP pruning: the ``keep`` highest saliencies (ties
+    to the lower index), returned in their original order so that the sliced
+    gate.weight / e_score_correction_bias / expert tensors keep their relative
+    order ("gate.weight sliced according to retained experts")."""
+    s = np.asarray(saliency, np.float64)
+    order = sorted(range(s.size), key=lambda e: (-s[e], e))
+    return np.array(sorted(order[:keep]), dtype=np.int64)
 
 
 def dense_moe_layer(x, router_weight, bias, k, rsf, experts_bf16,

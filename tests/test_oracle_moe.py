@@ -252,3 +252,45 @@ def test_dynamic_expert_scales_bound_the_dynamic_scale():
     sub = moe.moe_layer(x, wg, bias, cfg.k, cfg.rsf, lambda e: q[e], "dynamic_expert", np.full(cfg.E, F32(4e-4)),
                         tokens=[1, 9])
     np.testing.assert_array_equal(sub["out"], res["out"][[1, 9]])
+
+
+# --- REAP saliency ("Pruning Setup" of the BF16 model card) ---
+
+def test_reap_saliency_scales_with_the_down_global_scale():
+    """f_e(x) is linear in the down projection's global scale: doubling one
+    expert's g_down doubles exactly that expert's saliency and no other."""
+    cfg, x, wg, bias, bf, q = _tiny_layer()
+    g1, g2 = F32(0.003), F32(0.0005)
+    base = moe.moe_layer(x, wg, bias, cfg.k, cfg.rsf, lambda e: q[e], g1, g2)
+    q2 = dict(q)
+    dc, ds, dg = q[3][2]
+    q2[3] = (q[3][0], q[3][1], (dc, ds, F32(dg * 2)))
+    doubled = moe.moe_layer(x, wg, bias, cfg.k, cfg.rsf, lambda e: q2[e], g1, g2)
+    s0, n0 = moe.reap_saliency(base, cfg.E)
+    s1, n1 = moe.reap_saliency(doubled, cfg.E)
+    np.testing.assert_array_equal(n0, n1)
+    assert s1[3] == 2 * s0[3]
+    other = np.arange(cfg.E) != 3
+    np.testing.assert_array_equal(s1[other], s0[other])
+
+
+def test_reap_saliency_bounds_the_output_norm():
+    """sum_e saliency_sum_e = sum_t sum_j ||w_tj y_tj|| >= sum_t ||out_t|| (the
+    triangle inequality on the combine), with the counts summing to T k."""
+    cfg, x, wg, bias, bf, q = _tiny_layer()
+    res = moe.moe_layer(x, wg, bias, cfg.k, cfg.rsf, lambda e: q[e], F32(0.003), F32(0.0005))
+    s, n = moe.reap_saliency(res, cfg.E)
+    assert n.sum() == cfg.T * cfg.k
+    assert s.sum() >= np.linalg.norm(res["out_f64"], axis=1).sum() * (1 - 1e-12)
+    # a token subset gives the part of the accumulators its slots contribute
+    sub = moe.moe_layer(x, wg, bias, cfg.k, cfg.rsf, lambda e: q[e], F32(0.003), F32(0.0005), tokens=[0, 5])
+    ss, ns = moe.reap_saliency(sub, cfg.E)
+    assert ns.sum() == 2 * cfg.k and np.all(ss <= s + 1e-15)
+
+
+def test_reap_keep_takes_the_highest_saliencies_in_expert_order():
+    s = np.array([0.5, 0.1, 0.9, 0.5, 0.0, 0.7])
+    np.testing.assert_array_equal(moe.reap_keep(s, 3), [0, 2, 5])   # 0.9, 0.7, then 0.5 of the lower index
+    # ties go to the lower expert index
+    np.testing.assert_array_equal(moe.reap_keep(np.array([1.0, 2.0, 1.0, 1.0]), 2), [0, 1])
+    np.testing.assert_array_equal(moe.reap_keep(s, 6), np.arange(6))
