@@ -207,6 +207,15 @@ typedef struct moe_nvfp4_debug {
    * permutation, 2 quantise x, 3 gate/up GEMM, 4 down GEMM, 5 combine), so a
    * caller can time every stage of a call on the device. */
   void* stage_events[6];
+  /* REAP saliency accumulators ("K-EXAONE-152B-A23B-REAP-80E-BF16" card,
+   * "Pruning Setup": saliency = mean(topk_weight * ||f_e(x)||_2) over routed
+   * tokens).  Nullable, [E] each, owned and zeroed by the caller; every call
+   * ADDS its batch: saliency_sum[e] += sum over the (token, slot) pairs routed
+   * to e of w * ||y||_2, with y the expert's fp32 down output before the
+   * routing weight w; saliency_count[e] += their number.  Sum over
+   * calibration batches, then divide.  Deterministic: fixed reduction order. */
+  double* saliency_sum;
+  unsigned long long* saliency_count;
 } moe_nvfp4_debug;
 
 NVFP4_API size_t moe_nvfp4_workspace_size(int T, int E, int H, int I, int k);

@@ -55,7 +55,8 @@ N_STAGE_EVENTS = 6
 
 
 class MoeDebugStruct(ctypes.Structure):
-    _fields_ = [(n, _vp) for n in DEBUG_FIELDS] + [("stage_events", _vp * N_STAGE_EVENTS)]
+    _fields_ = ([(n, _vp) for n in DEBUG_FIELDS] + [("stage_events", _vp * N_STAGE_EVENTS)] +
+                [("saliency_sum", _vp), ("saliency_count", _vp)])
 
 
 def _declare(name, restype, *argtypes):
@@ -321,6 +322,38 @@ class MoeWeights:
                    _cuda(bias, torch.float32, "bias"), gc, gs, gg, uc, us, ug, dc, ds, dg)
 
 
+def reap_keep(saliency_sum: torch.Tensor, saliency_count: torch.Tensor, keep: int) -> torch.Tensor:
+    """Experts retained by REAP pruning ("Pruning Setup": the lowest-saliency
+    routed experts are removed): the ``keep`` highest mean saliencies
+    (sum / count, 0 for an expert never routed), ties to the lower index,
+    returned in expert order."""
+    s = (saliency_sum.double().cpu() / saliency_count.cpu().clamp(min=1).double()).tolist()
+    order = sorted(range(len(s)), key=lambda e: (-s[e], e))
+    return torch.tensor(sorted(order[:keep]), dtype=torch.int64)
+
+
+def select_experts(W: "MoeWeights", keep: torch.Tensor) -> "MoeWeights":
+    """The layer restricted to the experts ``keep`` (in that order): gate.weight
+    rows and e_score_correction_bias sliced as the pruned checkpoint does, and
+    each retained expert's codes, tiled scales and global scales copied over
+    (an expert's I or H rows are whole 128-row scale tiles, so its scales are
+    one contiguous range)."""
+    idx = keep.to(W.router_weight.device)
+    E2 = int(idx.numel())
+
+    def rows(t, per):
+        return t.reshape(W.E, per).index_select(0, idx).reshape(-1).contiguous()
+
+    def codes(t):
+        return t.reshape(W.E, -1).index_select(0, idx).reshape(E2, *t.shape[1:]).contiguous()
+
+    return MoeWeights(E2, W.H, W.I, W.k, W.rsf, W.router_weight.index_select(0, idx).contiguous(),
+                      W.bias.index_select(0, idx).contiguous(),
+                      codes(W.gate_codes), rows(W.gate_scales, W.I * W.H // 16), W.gate_gscale.index_select(0, idx),
+                      codes(W.up_codes), rows(W.up_scales, W.I * W.H // 16), W.up_gscale.index_select(0, idx),
+                      codes(W.down_codes), rows(W.down_scales, W.H * W.I // 16), W.down_gscale.index_select(0, idx))
+
+
 def moe_nvfp4_workspace_size(T: int, E: int, H: int, I: int, k: int) -> int:
     return lib.moe_nvfp4_workspace_size(T, E, H, I, k)
 
@@ -332,15 +365,20 @@ ACT_SCALE_MODES = {"tensor": 0, "expert": 1, "dynamic": 2, "dynamic_expert": 3}
 def moe_nvfp4_forward(W: MoeWeights, x: torch.Tensor, act_gscale: torch.Tensor, h_gscale: torch.Tensor,
                       logit_offset: torch.Tensor | None = None, debug: bool = False,
                       out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
-                      stage_events=None, act_scale_mode: str = "tensor"):
+                      stage_events=None, act_scale_mode: str = "tensor", saliency=None):
     """out [T, H] bf16; with debug=True also a dict of intermediate results.
     ``act_scale_mode`` is one of ACT_SCALE_MODES: in "tensor" act_gscale and
     h_gscale hold one fp32 each, in "expert" E each; in "dynamic" and
     "dynamic_expert" the library writes g1 into act_gscale ([1] or [E]).
     ``stage_events``: optional list of 6 torch.cuda.Event(enable_timing=True),
     each already recorded once (torch creates the CUDA event lazily), which
-    the library records again between the stages of the layer."""
+    the library records again between the stages of the layer.
+    ``saliency``: optional (sum float64 [E], count int64 [E]) REAP saliency
+    accumulators on the device that the call adds this batch to."""
     mode = ACT_SCALE_MODES[act_scale_mode]
+    if saliency is not None:
+        _cuda(saliency[0], torch.float64, "saliency sum")
+        _cuda(saliency[1], torch.int64, "saliency count")
     _cuda(x, torch.bfloat16, "x")
     _cuda(act_gscale, torch.float32, "act_gscale")
     _cuda(h_gscale, torch.float32, "h_gscale")
@@ -365,8 +403,11 @@ def moe_nvfp4_forward(W: MoeWeights, x: torch.Tensor, act_gscale: torch.Tensor, 
             "h_codes": z(cap, W.I // 2, dt=torch.uint8), "h_scales": z(tiled_scale_bytes(cap, W.I), dt=torch.uint8),
             "y": z(cap, W.H),
         }
-    if debug or stage_events is not None:
+    if debug or stage_events is not None or saliency is not None:
         dbg = MoeDebugStruct()
+        if saliency is not None:
+            dbg.saliency_sum = saliency[0].data_ptr()
+            dbg.saliency_count = saliency[1].data_ptr()
         if debug:
             for n in DEBUG_FIELDS:
                 setattr(dbg, n, dbg_tensors[n].data_ptr())

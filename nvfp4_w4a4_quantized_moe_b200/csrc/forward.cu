@@ -121,6 +121,39 @@ __global__ void __launch_bounds__(256) token_amax_kernel(const uint4* __restrict
   }
 }
 
+// REAP saliency of one batch ("Pruning Setup" of the BF16 model card): for
+// expert e, the sum over its real rows of ||w y||_2 = w ||y||_2, from the
+// down epilogue's per-thread sums of squares, in a fixed order (one block
+// per expert, rows strided over threads, then a fixed tree), added to the
+// caller's accumulators together with the row count.
+constexpr int kSalThreads = 256;
+__global__ void __launch_bounds__(kSalThreads) reap_saliency_kernel(const float* __restrict__ y_sq_part, int parts,
+                                                                    const int32_t* __restrict__ offsets,
+                                                                    const int32_t* __restrict__ counts,
+                                                                    double* __restrict__ saliency_sum,
+                                                                    unsigned long long* __restrict__ saliency_count) {
+  const int e = blockIdx.x;
+  const int r0 = offsets[e], n = counts[e];
+  double acc = 0.0;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const float* p = y_sq_part + (size_t)(r0 + i) * parts;
+    double ss = 0.0;
+    for (int c = 0; c < parts; ++c) ss += (double)p[c];
+    acc += sqrt(ss);
+  }
+  __shared__ double red[kSalThreads];
+  red[threadIdx.x] = acc;
+  __syncthreads();
+  for (int o = kSalThreads / 2; o > 0; o >>= 1) {
+    if (threadIdx.x < o) red[threadIdx.x] += red[threadIdx.x + o];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    saliency_sum[e] += red[0];
+    saliency_count[e] += (unsigned long long)n;
+  }
+}
+
 // amax of the tokens routed to each expert: amax_bits[1 + e].
 __global__ void __launch_bounds__(256) expert_amax_kernel(const int32_t* __restrict__ topk_idx, int T, int k,
                                                           const uint32_t* __restrict__ tok_amax,
@@ -183,6 +216,7 @@ struct ForwardScratch {
   uint16_t* y;
   uint32_t* amax_bits;      // [E + 1] batch amax, then per expert (dynamic modes)
   uint32_t* tok_amax;       // [T]
+  float* y_sq_part;         // [rows][H/128] (saliency requested)
 };
 
 static ForwardScratch carve_forward(Carver& c, int T, int E, int H, int I, int k) {
@@ -202,6 +236,7 @@ static ForwardScratch carve_forward(Carver& c, int T, int E, int H, int I, int k
   f.y = c.take<uint16_t>((size_t)cap * H);
   f.amax_bits = c.take<uint32_t>((size_t)E + 1);
   f.tok_amax = c.take<uint32_t>((size_t)T);
+  f.y_sq_part = c.take<float>((size_t)cap * (H / 128));
   return f;
 }
 
@@ -330,6 +365,8 @@ static nvfp4_status forward_impl(const moe_nvfp4_weights* W, const void* x_bf16,
   g2.expert_offsets = f.offsets; g2.expert_counts = f.route.counts;
   g2.row_w = f.route.row_w; g2.y_bf16 = f.y; g2.y_f32 = dbg ? dbg->y : nullptr;
   g2.per_expert_scales = (mode & kActPerExpert) != 0;
+  const bool saliency = dbg && dbg->saliency_sum && dbg->saliency_count;
+  g2.y_sq_part = saliency ? f.y_sq_part : nullptr;
   g2.status = f.route.status;
   NV_CHECK(launch_grouped_gemm(g2, s));
   NV_CHECK(mark(dbg, 4, s));
@@ -341,6 +378,11 @@ static nvfp4_status forward_impl(const moe_nvfp4_weights* W, const void* x_bf16,
                             reinterpret_cast<const uint4*>(f.y), (const int32_t*)f.inv_perm, T, H, k,
                             static_cast<uint4*>(out_bf16)));
   NV_CHECK(mark(dbg, 5, s));
+  if (saliency) {
+    reap_saliency_kernel<<<E, kSalThreads, 0, s>>>(f.y_sq_part, H / 128, f.offsets, f.route.counts,
+                                                  dbg->saliency_sum, dbg->saliency_count);
+    NV_CHECK(check_launch("reap_saliency_kernel"));
+  }
 
   if (dbg) {
     NV_CHECK(copy_out(dbg->logits, f.logits, sizeof(float) * (size_t)T * E, s));

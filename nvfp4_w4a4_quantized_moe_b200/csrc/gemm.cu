@@ -79,6 +79,7 @@ struct GemmParams {
   const float* row_w;
   uint16_t* y_bf16;
   float* y_f32;
+  float* y_sq_part;
   int H;
   int per_expert;       // g_act, g_h and h_amax are [E] arrays
   uint32_t* status;
@@ -370,6 +371,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                                  __fmul_rn(__uint_as_float(r[4 * i + 2]), scale),
                                  __fmul_rn(__uint_as_float(r[4 * i + 3]), scale));
         }
+        if (real && p.y_sq_part) {
+          float ss = 0.0f;
+#pragma unroll
+          for (int i = 0; i < 128; ++i) {
+            const float v = __fmul_rn(__uint_as_float(r[i]), scale);
+            ss = fmaf(v, v, ss);
+          }
+          p.y_sq_part[(size_t)grow * (p.H / 128) + nt * 2 + half] = ss;
+        }
         // scaled and packed to bf16 pairs right away, which frees r
         uint32_t yw[64];
 #pragma unroll
@@ -470,6 +480,7 @@ nvfp4_status launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t s) {
   p.row_w = a.row_w;
   p.y_bf16 = static_cast<uint16_t*>(a.y_bf16);
   p.y_f32 = a.y_f32;
+  p.y_sq_part = a.y_sq_part;
   p.H = a.H;
   p.per_expert = a.per_expert_scales ? 1 : 0;
   p.status = a.status;

@@ -42,6 +42,9 @@ struct GroupedGemmArgs {
   const float* row_w = nullptr;
   void* y_bf16 = nullptr;
   float* y_f32 = nullptr;
+  // nullable [rows][H/128]: sum of squares of each thread's 128 scaled y
+  // values (the REAP saliency's row norms are finished from these)
+  float* y_sq_part = nullptr;
   uint32_t* status = nullptr;
 };
 
