@@ -35,6 +35,12 @@ R16 activation global scales, beyond R8 (the extension "per-expert
     with the weight rule R1, g1 = fl32(amax / 2688), over the whole batch x
     ("dynamic") or over the tokens routed to each expert ("dynamic_expert";
     an expert without tokens gets 0).  h keeps a caller-supplied g2.
+R19 the shared expert (the model cards keep "shared experts" in BF16; their
+    size is not on the pages): one SiLU-gated MLP of the routed experts'
+    shape, bf16 weights gate_s, up_s [I_s, H] and down_s [H, I_s], applied to
+    every token: y_s = down_s (bf16(silu(gate_s x) * up_s x)), the
+    intermediate rounded once to bf16 (the operand of a bf16 matmul); the
+    layer output is bf16(y_s + sum_j w_j y_j).
 """
 from __future__ import annotations
 
@@ -206,8 +212,17 @@ def _scale_of(g, e):
     return F32(g[e]) if np.ndim(g) else F32(g)
 
 
+def shared_expert(x, shared) -> np.ndarray:
+    """R19: y_s [N, H] fp64 for rows x [N, H]; ``shared`` = (gate [I_s, H],
+    up [I_s, H], down [H, I_s]) holding bf16 values."""
+    gate, up, down = (np.asarray(t, np.float64) for t in shared)
+    xd = np.asarray(x, np.float64)
+    h = silu(xd @ gate.T) * (xd @ up.T)
+    return nvfp4.bf16_round(h).astype(np.float64) @ down.T
+
+
 def moe_layer(x, router_weight, bias, k, rsf, experts, g1, g2,
-              logit_offset=None, tokens=None, logits=None, topk_idx_all=None):
+              logit_offset=None, tokens=None, logits=None, topk_idx_all=None, shared=None):
     """The NVFP4 W4A4 routed-expert layer for the tokens ``tokens`` (all if None).
 
     ``experts(e)`` returns ((gate codes, scales, g), (up ...), (down ...)) for
@@ -220,7 +235,7 @@ def moe_layer(x, router_weight, bias, k, rsf, experts, g1, g2,
     Because routing is per token, evaluating a subset of tokens is exact; the
     dynamic modes take their amax over the whole batch ``x``, and
     "dynamic_expert" needs the routing of every token (``topk_idx_all``,
-    computed here when not given)."""
+    computed here when not given).  ``shared`` adds the shared expert (R19)."""
     x = np.asarray(x, F32)
     T, H = x.shape
     tok = np.arange(T) if tokens is None else np.asarray(tokens)
@@ -258,6 +273,8 @@ def moe_layer(x, router_weight, bias, k, rsf, experts, g1, g2,
             out[ti[r]] += float(topk_w[ti[r], sj[r]]) * y[r]
             h_all[(int(tok[ti[r]]), int(sj[r]))] = h[r]
             y_all[(int(tok[ti[r]]), int(sj[r]))] = y[r]
+    if shared is not None:
+        out += shared_expert(x[tok], shared)
     return {"out": nvfp4.bf16_round(out), "out_f64": out, "topk_idx": topk_idx,
             "topk_w": topk_w, "logits": logits, "h": h_all, "y": y_all,
             "a_codes": a_codes, "a_scales": a_scales, "g1": g1, "g2": g2, "tokens": tok}

@@ -294,3 +294,38 @@ def test_reap_keep_takes_the_highest_saliencies_in_expert_order():
     # ties go to the lower expert index
     np.testing.assert_array_equal(moe.reap_keep(np.array([1.0, 2.0, 1.0, 1.0]), 2), [0, 1])
     np.testing.assert_array_equal(moe.reap_keep(s, 6), np.arange(6))
+
+
+# --- the shared BF16 expert (reading R19) ---
+
+def _shared(cfg, seed=3):
+    gen = torch.Generator().manual_seed(seed)
+    mk = lambda *s: (torch.randn(*s, generator=gen) * 0.02).to(torch.bfloat16).float().numpy()  # noqa: E731
+    return mk(cfg.I, cfg.H), mk(cfg.I, cfg.H), mk(cfg.H, cfg.I)
+
+
+def test_shared_expert_alone_is_torchs_mlp():
+    """With every routed expert zeroed, the layer is bf16 of the shared MLP;
+    torch's fp64 matmuls and SiLU give the same numbers."""
+    cfg, x, wg, bias, bf, q = _tiny_layer()
+    sh = _shared(cfg)
+    zero = {e: tuple((np.zeros_like(c), np.zeros_like(s), g) for c, s, g in q[e]) for e in range(cfg.E)}
+    res = moe.moe_layer(x, wg, bias, cfg.k, cfg.rsf, lambda e: zero[e], F32(0.003), F32(0.0005), shared=sh)
+    xt = torch.from_numpy(x).double()
+    g, u, d = (torch.from_numpy(t).double() for t in sh)
+    h = torch.nn.functional.silu(xt @ g.T) * (xt @ u.T)
+    ref = (h.to(torch.bfloat16).double() @ d.T).to(torch.bfloat16).float().numpy()
+    np.testing.assert_array_equal(res["out"], ref)
+
+
+def test_shared_expert_adds_to_the_routed_layer():
+    cfg, x, wg, bias, bf, q = _tiny_layer()
+    sh = _shared(cfg)
+    routed = moe.moe_layer(x, wg, bias, cfg.k, cfg.rsf, lambda e: q[e], F32(0.003), F32(0.0005))
+    both = moe.moe_layer(x, wg, bias, cfg.k, cfg.rsf, lambda e: q[e], F32(0.003), F32(0.0005), shared=sh)
+    np.testing.assert_allclose(both["out_f64"] - moe.shared_expert(x, sh), routed["out_f64"], rtol=0,
+                               atol=1e-12 * np.abs(both["out_f64"]).max())
+    zeros = tuple(np.zeros_like(t) for t in sh)
+    np.testing.assert_array_equal(
+        moe.moe_layer(x, wg, bias, cfg.k, cfg.rsf, lambda e: q[e], F32(0.003), F32(0.0005), shared=zeros)["out"],
+        routed["out"])
