@@ -183,6 +183,14 @@ typedef struct moe_nvfp4_weights {
   const uint8_t* down_codes;      /* [E][H][I/2]                                 */
   const uint8_t* down_scales;     /* TILED, E*H rows x I cols                    */
   const float* down_gscale;       /* [E]                                         */
+  /* The shared expert, kept BF16 (NVFP4 card, "Quantization Setup"; its size
+   * is not on the pages): out += down_s(silu(gate_s x) * up_s x) for every
+   * token, the intermediate rounded to bf16.  NULL pointers and I_shared 0:
+   * no shared expert.  I_shared % 128 == 0. */
+  const void* shared_gate;        /* bf16 [I_shared][H]                          */
+  const void* shared_up;          /* bf16 [I_shared][H]                          */
+  const void* shared_down;        /* bf16 [H][I_shared]                          */
+  int I_shared;
 } moe_nvfp4_weights;
 
 /* Optional copies of intermediate results (every pointer nullable; device
@@ -219,13 +227,18 @@ typedef struct moe_nvfp4_debug {
 } moe_nvfp4_debug;
 
 NVFP4_API size_t moe_nvfp4_workspace_size(int T, int E, int H, int I, int k);
+/* The same with a shared expert of intermediate size I_shared (0: none). */
+NVFP4_API size_t moe_nvfp4_workspace_size_shared(int T, int E, int H, int I, int k, int I_shared);
 
-/* out[T][H] bf16 = sum_j w_j * down_e( quant_g2( silu(gate_e(xq)) * up_e(xq) ) )
+/* out[T][H] bf16 = [shared(x) +] sum_j w_j * down_e( quant_g2( silu(gate_e(xq)) * up_e(xq) ) )
  * with xq = x quantised under act_gscale (g1) and the intermediate quantised
  * under h_gscale (g2), both one fp32 in device memory.  Steps: router GEMM ->
  * top-k -> permutation -> quantise x into permuted rows -> grouped FP4 GEMM
  * gate/up with SiLU*up and requantisation fused -> grouped FP4 GEMM down with
- * g2 * g_down * w_j fused -> combine in slot order (fp32 sum, bf16 out).
+ * g2 * g_down * w_j fused -> [shared expert: bf16 GEMMs gate/up with SiLU*up,
+ * then down] -> combine: fp32 sum of the shared row and the k rows in slot
+ * order, bf16 out.  With a shared expert the workspace comes from
+ * moe_nvfp4_workspace_size_shared.
  * Needs H % 256 == 0, I % 128 == 0, 1 <= k <= 16, k <= E <= 256, T >= 1. */
 NVFP4_API nvfp4_status moe_nvfp4_forward(const moe_nvfp4_weights* W, const void* x_bf16, int T,
                                const float* act_gscale, const float* h_gscale, const float* logit_offset,

@@ -11,6 +11,7 @@ loudly when it has not been built.
 from __future__ import annotations
 
 import ctypes
+import dataclasses
 import os
 from dataclasses import dataclass
 
@@ -46,7 +47,8 @@ class MoeWeightsStruct(ctypes.Structure):
                 ("router_weight", _vp), ("bias", _vp),
                 ("gate_codes", _vp), ("gate_scales", _vp), ("gate_gscale", _vp),
                 ("up_codes", _vp), ("up_scales", _vp), ("up_gscale", _vp),
-                ("down_codes", _vp), ("down_scales", _vp), ("down_gscale", _vp)]
+                ("down_codes", _vp), ("down_scales", _vp), ("down_gscale", _vp),
+                ("shared_gate", _vp), ("shared_up", _vp), ("shared_down", _vp), ("I_shared", _i)]
 
 
 DEBUG_FIELDS = ("logits", "topk_idx", "topk_w", "expert_offsets", "perm", "inv_perm", "a_codes", "a_scales", "h",
@@ -78,6 +80,7 @@ _declare("moe_route_workspace_size", _sz, _i, _i, _i)
 _declare("moe_route", _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
          _vp)
 _declare("moe_nvfp4_workspace_size", _sz, _i, _i, _i, _i, _i)
+_declare("moe_nvfp4_workspace_size_shared", _sz, _i, _i, _i, _i, _i, _i)
 _declare("moe_nvfp4_forward", _i, ctypes.POINTER(MoeWeightsStruct), _vp, _i, _vp, _vp, _vp, _vp,
          ctypes.POINTER(MoeDebugStruct), _vp, _sz, _vp)
 _declare("moe_nvfp4_forward_scaled", _i, ctypes.POINTER(MoeWeightsStruct), _vp, _i, _i, _vp, _vp, _vp, _vp,
@@ -100,7 +103,8 @@ EXPORTS = ("nvfp4_last_error", "nvfp4_abi_version", "nvfp4_workspace_status",
            "nvfp4_quantize_weights_workspace_size", "nvfp4_quantize_weights", "nvfp4_quantize_weights_noalloc",
            "nvfp4_quantize_act",
            "moe_route_rows_capacity", "moe_route_workspace_size", "moe_route", "moe_nvfp4_workspace_size",
-           "moe_nvfp4_forward", "moe_nvfp4_forward_scaled", "moe_nvfp4_gemm_workspace_size", "moe_nvfp4_gate_up",
+           "moe_nvfp4_forward", "moe_nvfp4_forward_scaled", "moe_nvfp4_workspace_size_shared",
+           "moe_nvfp4_gemm_workspace_size", "moe_nvfp4_gate_up",
            "moe_nvfp4_down",
            "nvfp4_block_stats_compute",
            "nvfp4_test_e2m1", "nvfp4_test_e2m1_sweep", "nvfp4_test_e4m3", "nvfp4_test_sigmoid",
@@ -303,12 +307,27 @@ class MoeWeights:
     down_codes: torch.Tensor         # u8 [E, H, I/2]
     down_scales: torch.Tensor
     down_gscale: torch.Tensor
+    # the shared expert, bf16 (None: none): gate, up [I_s, H], down [H, I_s]
+    shared_gate: torch.Tensor | None = None
+    shared_up: torch.Tensor | None = None
+    shared_down: torch.Tensor | None = None
+
+    @property
+    def I_shared(self) -> int:
+        return 0 if self.shared_gate is None else int(self.shared_gate.shape[0])
+
+    def with_shared(self, gate: torch.Tensor, up: torch.Tensor, down: torch.Tensor) -> "MoeWeights":
+        """This layer plus a shared bf16 expert."""
+        for n, t in (("shared gate", gate), ("shared up", up), ("shared down", down)):
+            _cuda(t, torch.bfloat16, n)
+        return dataclasses.replace(self, shared_gate=gate, shared_up=up, shared_down=down)
 
     def struct(self) -> MoeWeightsStruct:
         return MoeWeightsStruct(self.E, self.H, self.I, self.k, float(self.rsf), _p(self.router_weight),
                                 _p(self.bias), _p(self.gate_codes), _p(self.gate_scales), _p(self.gate_gscale),
                                 _p(self.up_codes), _p(self.up_scales), _p(self.up_gscale), _p(self.down_codes),
-                                _p(self.down_scales), _p(self.down_gscale))
+                                _p(self.down_scales), _p(self.down_gscale), _p(self.shared_gate),
+                                _p(self.shared_up), _p(self.shared_down), self.I_shared)
 
     @classmethod
     def quantize(cls, gate, up, down, router_weight, bias, k: int, rsf: float) -> "MoeWeights":
@@ -351,11 +370,12 @@ def select_experts(W: "MoeWeights", keep: torch.Tensor) -> "MoeWeights":
                       W.bias.index_select(0, idx).contiguous(),
                       codes(W.gate_codes), rows(W.gate_scales, W.I * W.H // 16), W.gate_gscale.index_select(0, idx),
                       codes(W.up_codes), rows(W.up_scales, W.I * W.H // 16), W.up_gscale.index_select(0, idx),
-                      codes(W.down_codes), rows(W.down_scales, W.H * W.I // 16), W.down_gscale.index_select(0, idx))
+                      codes(W.down_codes), rows(W.down_scales, W.H * W.I // 16), W.down_gscale.index_select(0, idx),
+                      W.shared_gate, W.shared_up, W.shared_down)
 
 
-def moe_nvfp4_workspace_size(T: int, E: int, H: int, I: int, k: int) -> int:
-    return lib.moe_nvfp4_workspace_size(T, E, H, I, k)
+def moe_nvfp4_workspace_size(T: int, E: int, H: int, I: int, k: int, I_shared: int = 0) -> int:
+    return lib.moe_nvfp4_workspace_size_shared(T, E, H, I, k, I_shared)
 
 
 #: Activation global-scale modes of moe_nvfp4_forward_scaled (NVFP4_ACT_SCALE_*).
@@ -389,7 +409,7 @@ def moe_nvfp4_forward(W: MoeWeights, x: torch.Tensor, act_gscale: torch.Tensor, 
     dev = x.device
     out = torch.empty((T, H), dtype=torch.bfloat16, device=dev) if out is None else _cuda(out, torch.bfloat16, "out")
     if workspace is None:
-        workspace = _workspace(moe_nvfp4_workspace_size(T, W.E, W.H, W.I, W.k), dev)
+        workspace = _workspace(moe_nvfp4_workspace_size(T, W.E, W.H, W.I, W.k, W.I_shared), dev)
     dbg_tensors = None
     dbg_ptr = None
     if debug:

@@ -154,6 +154,19 @@ __global__ void __launch_bounds__(kSalThreads) reap_saliency_kernel(const float*
   }
 }
 
+// The shared expert's dense "grouping": one expert holding rows [0, T).
+__global__ void dense_tiles_kernel(int T, int32_t* __restrict__ tile_expert, int32_t* __restrict__ num_mtiles,
+                                   int32_t* __restrict__ offsets, int32_t* __restrict__ counts) {
+  const int mt = (T + kRowTile - 1) / kRowTile;
+  for (int i = threadIdx.x; i < mt; i += blockDim.x) tile_expert[i] = 0;
+  if (threadIdx.x == 0) {
+    *num_mtiles = mt;
+    offsets[0] = 0;
+    offsets[1] = mt * kRowTile;
+    counts[0] = T;
+  }
+}
+
 // amax of the tokens routed to each expert: amax_bits[1 + e].
 __global__ void __launch_bounds__(256) expert_amax_kernel(const int32_t* __restrict__ topk_idx, int T, int k,
                                                           const uint32_t* __restrict__ tok_amax,
@@ -164,8 +177,9 @@ __global__ void __launch_bounds__(256) expert_amax_kernel(const int32_t* __restr
   if (i < T * k) atomicMax(amax_bits + 1 + topk_idx[i], tok_amax[i / k]);
 }
 
-// out[t] = bf16( sum_j y[inv_perm[t, j]] ), fp32 sum in slot order.  The
-// routing weight is already folded into y by the down-projection epilogue.
+// out[t] = bf16( [y_shared[t] +] sum_j y[inv_perm[t, j]] ), fp32 sum, shared
+// row first, then slot order.  The routing weight is already folded into y by
+// the down-projection epilogue.
 // Block (t, by) covers token t's 8-column groups by*blockDim.x + i*gridDim.y*
 // blockDim.x (+ threadIdx.x): a small batch spreads a row over several
 // blocks, a large one keeps whole rows in one block for long contiguous
@@ -173,6 +187,7 @@ __global__ void __launch_bounds__(256) expert_amax_kernel(const int32_t* __restr
 constexpr int kCombineThreads = 256;
 
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const uint4* __restrict__ y,
+                                                                  const uint4* __restrict__ y_shared,
                                                                   const int32_t* __restrict__ inv_perm, int T, int H,
                                                                   int k, uint4* __restrict__ out) {
   __shared__ int32_t rows[16];
@@ -187,6 +202,7 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const uint4* _
     for (int j = 0; j < 16; ++j)
       if (j < k) v[j] = __ldg(y + (size_t)rows[j] * vpr + c);
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    if (y_shared) unpack_bf16x8(__ldg(y_shared + (size_t)t * vpr + c), acc);   // the shared expert's row first
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       if (j < k) {
@@ -217,9 +233,16 @@ struct ForwardScratch {
   uint32_t* amax_bits;      // [E + 1] batch amax, then per expert (dynamic modes)
   uint32_t* tok_amax;       // [T]
   float* y_sq_part;         // [rows][H/128] (saliency requested)
+  // shared expert (I_shared > 0)
+  uint16_t* sh_h;           // bf16 [T_pad][I_shared]
+  uint16_t* sh_y;           // bf16 [T_pad][H]
+  int32_t* sh_tiles;        // [T_pad / 128]
+  int32_t* sh_ntiles;       // [1]
+  int32_t* sh_offsets;      // [2]
+  int32_t* sh_counts;       // [1]
 };
 
-static ForwardScratch carve_forward(Carver& c, int T, int E, int H, int I, int k) {
+static ForwardScratch carve_forward(Carver& c, int T, int E, int H, int I, int k, int I_shared) {
   ForwardScratch f;
   const int cap = route_rows_capacity(T, E, k);
   f.route = carve_route_scratch(c, T, E, k);
@@ -237,6 +260,17 @@ static ForwardScratch carve_forward(Carver& c, int T, int E, int H, int I, int k
   f.amax_bits = c.take<uint32_t>((size_t)E + 1);
   f.tok_amax = c.take<uint32_t>((size_t)T);
   f.y_sq_part = c.take<float>((size_t)cap * (H / 128));
+  f.sh_h = f.sh_y = nullptr;
+  f.sh_tiles = f.sh_ntiles = f.sh_offsets = f.sh_counts = nullptr;
+  if (I_shared > 0) {
+    const size_t tp = (size_t)(T + kRowTile - 1) / kRowTile * kRowTile;
+    f.sh_h = c.take<uint16_t>(tp * I_shared);
+    f.sh_y = c.take<uint16_t>(tp * H);
+    f.sh_tiles = c.take<int32_t>(tp / kRowTile);
+    f.sh_ntiles = c.take<int32_t>(1);
+    f.sh_offsets = c.take<int32_t>(2);
+    f.sh_counts = c.take<int32_t>(1);
+  }
   return f;
 }
 
@@ -254,11 +288,15 @@ static nvfp4_status copy_out(void* dst, const void* src, size_t bytes, cudaStrea
 
 using namespace nvfp4moe;
 
-extern "C" size_t moe_nvfp4_workspace_size(int T, int E, int H, int I, int k) {
-  if (T < 0 || E < 0 || H < 0 || I < 0 || k < 0) return 0;
+extern "C" size_t moe_nvfp4_workspace_size_shared(int T, int E, int H, int I, int k, int I_shared) {
+  if (T < 0 || E < 0 || H < 0 || I < 0 || k < 0 || I_shared < 0) return 0;
   Carver c(nullptr);
-  carve_forward(c, T, E, H, I, k);
+  carve_forward(c, T, E, H, I, k, I_shared);
   return c.size();
+}
+
+extern "C" size_t moe_nvfp4_workspace_size(int T, int E, int H, int I, int k) {
+  return moe_nvfp4_workspace_size_shared(T, E, H, I, k, 0);
 }
 
 template <int MODE>
@@ -288,18 +326,24 @@ static nvfp4_status forward_impl(const moe_nvfp4_weights* W, const void* x_bf16,
                  aligned(W->gate_scales, 16) && aligned(W->up_scales, 16) && aligned(W->down_scales, 16),
              NVFP4_ERR_INVALID_ARG, "moe_nvfp4_forward: tensors need 16-byte alignment");
   const int E = W->E, H = W->H, I = W->I, k = W->k;
-  const size_t need = moe_nvfp4_workspace_size(T, E, H, I, k);
+  const int I_s = W->I_shared;
+  const bool shared = I_s > 0;
+  const size_t need = moe_nvfp4_workspace_size_shared(T, E, H, I, k, I_s);
   NV_REQUIRE(ws && ws_bytes >= need && aligned(ws, 256), NVFP4_ERR_WORKSPACE,
              "moe_nvfp4_forward: needs a 256-byte aligned workspace of %zu bytes", need);
   int sms = 0;
   NV_CHECK(device_sm_count(&sms));
   cudaStream_t s = as_stream(stream);
   Carver c(ws);
-  ForwardScratch f = carve_forward(c, T, E, H, I, k);
+  ForwardScratch f = carve_forward(c, T, E, H, I, k, I_s);
   const int cap = route_rows_capacity(T, E, k);
 
   NV_CHECK(check_cuda(cudaMemsetAsync(f.route.status, 0, sizeof(uint32_t), s), "clear status word"));
   NV_CHECK(mark(dbg, 0, s));
+  if (shared) {
+    dense_tiles_kernel<<<1, 128, 0, s>>>(T, f.sh_tiles, f.sh_ntiles, f.sh_offsets, f.sh_counts);
+    NV_CHECK(check_launch("dense_tiles_kernel"));
+  }
   if (mode & kActDynamic) {
     // 0: amax of every token and of the batch
     NV_CHECK(check_cuda(cudaMemsetAsync(f.amax_bits, 0, sizeof(uint32_t) * (size_t)(E + 1), s), "clear amax"));
@@ -371,12 +415,43 @@ static nvfp4_status forward_impl(const moe_nvfp4_weights* W, const void* x_bf16,
   NV_CHECK(launch_grouped_gemm(g2, s));
   NV_CHECK(mark(dbg, 4, s));
 
+  // the shared expert (bf16): gate/up with SiLU*up, then down; its y goes
+  // into the combine
+  if (shared) {
+    const int tp = (T + kRowTile - 1) / kRowTile * kRowTile;
+    GroupedGemmArgs s1;
+    s1.epi = kEpiSharedGateUp;
+    s1.E = 1; s1.H = H; s1.I = I_s;
+    s1.rows_capacity = tp;
+    s1.a_rows = T;
+    s1.a_codes = static_cast<const uint8_t*>(x_bf16);
+    s1.b0_codes = static_cast<const uint8_t*>(W->shared_gate);
+    s1.b1_codes = static_cast<const uint8_t*>(W->shared_up);
+    s1.tile_expert = f.sh_tiles; s1.num_mtiles = f.sh_ntiles;
+    s1.expert_offsets = f.sh_offsets; s1.expert_counts = f.sh_counts;
+    s1.h_bf16 = f.sh_h;
+    s1.status = f.route.status;
+    NV_CHECK(launch_grouped_gemm(s1, s));
+    GroupedGemmArgs s2;
+    s2.epi = kEpiSharedDown;
+    s2.E = 1; s2.H = H; s2.I = I_s;
+    s2.rows_capacity = tp;
+    s2.a_codes = reinterpret_cast<const uint8_t*>(f.sh_h);
+    s2.b0_codes = static_cast<const uint8_t*>(W->shared_down);
+    s2.tile_expert = f.sh_tiles; s2.num_mtiles = f.sh_ntiles;
+    s2.expert_offsets = f.sh_offsets; s2.expert_counts = f.sh_counts;
+    s2.y_bf16 = f.sh_y;
+    s2.status = f.route.status;
+    NV_CHECK(launch_grouped_gemm(s2, s));
+  }
+
   // 8: combine
   // below about two waves of whole-row blocks, split rows across blocks
   const int row_blocks = T >= 2 * sms ? 1 : (H / 8 + kCombineThreads - 1) / kCombineThreads;
   NV_CHECK(launch_dependent("combine_kernel", combine_kernel, dim3(T, row_blocks), dim3(kCombineThreads), 0, s,
-                            reinterpret_cast<const uint4*>(f.y), (const int32_t*)f.inv_perm, T, H, k,
-                            static_cast<uint4*>(out_bf16)));
+                            reinterpret_cast<const uint4*>(f.y),
+                            shared ? reinterpret_cast<const uint4*>(f.sh_y) : (const uint4*)nullptr,
+                            (const int32_t*)f.inv_perm, T, H, k, static_cast<uint4*>(out_bf16)));
   NV_CHECK(mark(dbg, 5, s));
   if (saliency) {
     reap_saliency_kernel<<<E, kSalThreads, 0, s>>>(f.y_sq_part, H / 128, f.offsets, f.route.counts,

@@ -38,14 +38,25 @@ constexpr int kSfbBytes = kBN * kBK / kQBlock;   // 4 KiB (8 scale atoms)
 constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
 constexpr int kThreads = 320;
 constexpr int kEpiWarps = 8;
-// Pipeline stages: the gate/up GEMM keeps four; the down GEMM gives one up
-// for the shared-memory buffer its epilogue stages y through, 32 rows x 64
-// bf16 columns (4 KiB) per warp at a time.
+// Operand kinds: FP4 stages hold 256 K elements (128-byte rows) plus their
+// scale atoms; bf16 stages hold 64 K elements in the same 128-byte rows and
+// no scales, so the MMA descriptors advance identically (32 bytes per MMA).
+template <int EPI> __host__ __device__ constexpr bool is_bf16() { return EPI >= kEpiSharedGateUp; }
+template <int EPI> __host__ __device__ constexpr bool is_gate_up() {
+  return EPI == kEpiGateUp || EPI == kEpiSharedGateUp;
+}
+template <int EPI> __host__ __device__ constexpr int stage_bytes_of() {
+  return is_bf16<EPI>() ? kABytes + kBBytes : kStageBytes;
+}
+template <int EPI> __host__ __device__ constexpr int bk_of() { return is_bf16<EPI>() ? 64 : kBK; }
+// Pipeline stages: the gate/up GEMMs keep four; the down GEMMs stage y in
+// shared memory, 32 rows x 64 bf16 columns (4 KiB) per warp at a time, which
+// costs the FP4 down GEMM one of its stages.
 template <int EPI> __host__ __device__ constexpr int stages_of() { return EPI == kEpiDown ? 3 : 4; }
 constexpr int kYPassCols = 64;
 constexpr int kYStageBytes = 32 * kYPassCols * 2;
 template <int EPI> __host__ __device__ constexpr int smem_bytes_of() {
-  return stages_of<EPI>() * kStageBytes + 1024 + (EPI == kEpiDown ? kEpiWarps * kYStageBytes : 0);
+  return stages_of<EPI>() * stage_bytes_of<EPI>() + 1024 + (is_gate_up<EPI>() ? 0 : kEpiWarps * kYStageBytes);
 }
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCol = 0;                  // 256 fp32 accumulator columns
@@ -80,6 +91,7 @@ struct GemmParams {
   uint16_t* y_bf16;
   float* y_f32;
   float* y_sq_part;
+  uint16_t* h_bf16;
   int H;
   int per_expert;       // g_act, g_h and h_amax are [E] arrays
   uint32_t* status;
@@ -99,6 +111,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   constexpr int kStages = stages_of<EPI>();
+  constexpr bool kBf16 = is_bf16<EPI>();
+  constexpr bool kGateUp = is_gate_up<EPI>();
+  constexpr int kSB = stage_bytes_of<EPI>();
   __shared__ __align__(8) uint64_t full_bar[kStages];
   __shared__ __align__(8) uint64_t empty_bar[kStages];
   __shared__ __align__(8) uint64_t acc_full_bar;
@@ -123,7 +138,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB0);
-    if (EPI == kEpiGateUp) prefetch_tmap(&tmB1);
+    if (kGateUp) prefetch_tmap(&tmB1);
   }
   if (warp == 1) {
     tmem_alloc(&tmem_base_s, kTmemCols);
@@ -138,8 +153,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   griddep_launch();
 
   const int num_tiles = (*p.num_mtiles) * p.n_tiles;
-  const int KT = (p.K + kBK - 1) / kBK;
-  const int nblk4 = p.K / 64;                    // scale atoms per 128-row tile
+  const int KT = (p.K + bk_of<EPI>() - 1) / bk_of<EPI>();
+  const int nblk4 = p.K / 64;                    // FP4: scale atoms per 128-row tile
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -156,11 +171,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int mt = t / p.n_tiles, nt = t % p.n_tiles;
       const int e = min(max(p.tile_expert[mt], 0), p.E - 1);
       const int arow = mt * kBM;
-      const int brow = e * p.Nw + nt * (EPI == kEpiGateUp ? 128 : kBN);
-      const uint8_t* asf = p.a_sf + (size_t)mt * tile_sf_bytes;
-      const uint8_t* bsf0 = p.b0_sf + (size_t)(brow / kRowTile) * tile_sf_bytes;
-      const uint8_t* bsf1 = (EPI == kEpiGateUp ? p.b1_sf + (size_t)(brow / kRowTile) * tile_sf_bytes
-                                               : bsf0 + tile_sf_bytes);
+      const int brow = e * p.Nw + nt * (kGateUp ? 128 : kBN);
+      const uint8_t* asf = kBf16 ? nullptr : p.a_sf + (size_t)mt * tile_sf_bytes;
+      const uint8_t* bsf0 = kBf16 ? nullptr : p.b0_sf + (size_t)(brow / kRowTile) * tile_sf_bytes;
+      const uint8_t* bsf1 = kBf16 ? nullptr
+                                  : (kGateUp ? p.b1_sf + (size_t)(brow / kRowTile) * tile_sf_bytes
+                                             : bsf0 + tile_sf_bytes);
       for (int kt = 0; kt < KT; ++kt) {
         ok = __all_sync(0xffffffffu, mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag));
         if (!ok) {
@@ -168,21 +184,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         if (leader) {
-          uint8_t* sA = st0 + stage * kStageBytes;
+          uint8_t* sA = st0 + stage * kSB;
           uint8_t* sB = sA + kABytes;
-          uint8_t* sSFA = sB + kBBytes;
-          uint8_t* sSFB = sSFA + kSfaBytes;
-          const int katoms = min(4, (p.K - kt * kBK) / 64);
-          const uint32_t sf_bytes = (uint32_t)katoms * kAtomBytes;
-          const int x = kt * kBKBytes;
-          const size_t sf_off = (size_t)kt * 4 * kAtomBytes;
-          mbar_arrive_expect_tx(&full_bar[stage], kABytes + kBBytes + 3 * sf_bytes);
+          // x in tensor-map elements: 128 bytes of K per stage either way
+          const int x = kt * (kBf16 ? 64 : kBKBytes);
+          if (kBf16) {
+            mbar_arrive_expect_tx(&full_bar[stage], kABytes + kBBytes);
+          } else {
+            const int katoms = min(4, (p.K - kt * kBK) / 64);
+            const uint32_t sf_bytes = (uint32_t)katoms * kAtomBytes;
+            mbar_arrive_expect_tx(&full_bar[stage], kABytes + kBBytes + 3 * sf_bytes);
+            uint8_t* sSFA = sB + kBBytes;
+            uint8_t* sSFB = sSFA + kSfaBytes;
+            const size_t sf_off = (size_t)kt * 4 * kAtomBytes;
+            bulk_load(sSFA, asf + sf_off, sf_bytes, &full_bar[stage]);
+            bulk_load(sSFB, bsf0 + sf_off, sf_bytes, &full_bar[stage]);
+            bulk_load(sSFB + kSfbBytes / 2, bsf1 + sf_off, sf_bytes, &full_bar[stage]);
+          }
           tma_load_2d(sA, &tmA, x, arow, &full_bar[stage]);
           tma_load_2d(sB, &tmB0, x, brow, &full_bar[stage]);
-          if (EPI == kEpiGateUp) tma_load_2d(sB + kBBytes / 2, &tmB1, x, brow, &full_bar[stage]);
-          bulk_load(sSFA, asf + sf_off, sf_bytes, &full_bar[stage]);
-          bulk_load(sSFB, bsf0 + sf_off, sf_bytes, &full_bar[stage]);
-          bulk_load(sSFB + kSfbBytes / 2, bsf1 + sf_off, sf_bytes, &full_bar[stage]);
+          if (kGateUp) tma_load_2d(sB + kBBytes / 2, &tmB1, x, brow, &full_bar[stage]);
         }
         __syncwarp();
         filled |= 1u << stage;
@@ -207,12 +228,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // slowly to keep the tensor pipe busy.  Shared-memory descriptors are
     // built once; a stage only adds constant offsets to their address fields.
     const uint32_t leader = elect_one();
-    const uint32_t idesc = idesc_fp4(kBM, kBN);
+    const uint32_t idesc = kBf16 ? idesc_bf16(kBM, kBN) : idesc_fp4(kBM, kBN);
     const uint32_t s0 = smem_u32(smem);
     const uint64_t a0 = sdesc_sw128(s0), b0 = sdesc_sw128(s0 + kABytes);
     const uint64_t sfa0 = sdesc_scale_atom(s0 + kABytes + kBBytes);
     const uint64_t sfb0 = sdesc_scale_atom(s0 + kABytes + kBBytes + kSfaBytes);
-    constexpr uint64_t kStageStep = kStageBytes >> 4;          // start address is in 16-byte units
+    constexpr uint64_t kStageStep = kSB >> 4;                  // start address is in 16-byte units
     constexpr uint64_t kAtomStep = kAtomBytes >> 4;
     constexpr uint64_t kSfbHalfStep = (kSfbBytes / 2) >> 4;
     const uint32_t sfa_t = tmem + kSfCol + kSfaOff, sfb_t = tmem + kSfCol + kSfbOff;
@@ -237,8 +258,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         const uint64_t d = (uint64_t)stage * kStageStep;
-        const int katoms = min(4, (p.K - kt * kBK) / 64);
-        if (leader) {
+        const int katoms = kBf16 ? 4 : min(4, (p.K - kt * kBK) / 64);
+        if (leader && kBf16) {
+          // 4 x (K = 16 bf16 = 32 bytes) per 128-byte stage row
+#pragma unroll
+          for (int j = 0; j < 4; ++j) mma_bf16(acc_t, a0 + d + 2 * j, b0 + d + 2 * j, idesc, accumulate | j);
+          tc_commit(&empty_bar[stage]);
+        } else if (leader) {
           if (katoms == 4) {
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -299,8 +325,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const int se = p.per_expert ? e : 0;                  // index of this tile's scales
-      const float g_act = p.g_act[se];
-      if (EPI == kEpiGateUp) {
+      const float g_act = kBf16 ? 1.0f : p.g_act[se];
+      if (EPI == kEpiSharedGateUp) {
+        // bf16 operands, no global scales: h = silu(gate) * up, stored bf16
+        uint32_t rg[64], ru[64];
+        tmem_ld32(tbase + kAccCol + half * 64, rg);
+        tmem_ld32(tbase + kAccCol + half * 64 + 32, rg + 32);
+        tmem_ld32(tbase + kAccCol + 128 + half * 64, ru);
+        tmem_ld32(tbase + kAccCol + 128 + half * 64 + 32, ru + 32);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty_bar);
+        if (real) {
+          uint4* dst = reinterpret_cast<uint4*>(p.h_bf16 + (size_t)grow * p.I + nt * 128 + half * 64);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            uint32_t w[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int c = 8 * i + 2 * q;
+              w[q] = pack_bf16x2(__fmul_rn(silu(__uint_as_float(rg[c])), __uint_as_float(ru[c])),
+                                 __fmul_rn(silu(__uint_as_float(rg[c + 1])), __uint_as_float(ru[c + 1])));
+            }
+            dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      } else if (EPI == kEpiGateUp) {
         const float sg = __fmul_rn(g_act, p.g_b0[e]);
         const float su = __fmul_rn(g_act, p.g_b1[e]);
         // drain this thread's 64 gate and 64 up columns, then hand the
@@ -352,7 +403,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         cdst[1] = cw1;
         *reinterpret_cast<uint32_t*>(p.h_sf + tiled_scale_offset(grow, hcol0 / kQBlock, p.I / 64)) = sw;
       } else {
-        const float scale = __fmul_rn(__fmul_rn(g_act, p.g_b0[e]), p.row_w ? p.row_w[grow] : 1.0f);
+        const float scale =
+            kBf16 ? 1.0f : __fmul_rn(__fmul_rn(g_act, p.g_b0[e]), p.row_w ? p.row_w[grow] : 1.0f);
         const int col0 = nt * kBN + half * 128;
         // drain this thread's 128 columns, then hand the accumulator back
         uint32_t r[128];
@@ -391,7 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // hit 32 rows per instruction, so the warp stages 64 columns of its
           // 32 rows in shared memory (16-byte chunks XOR-swizzled by row) and
           // writes them back four whole 128-byte row segments per instruction.
-          uint4* ybuf = reinterpret_cast<uint4*>(smem + kStages * kStageBytes + (warp - 2) * kYStageBytes);
+          uint4* ybuf = reinterpret_cast<uint4*>(smem + kStages * kSB + (warp - 2) * kYStageBytes);
           const int row0 = mt * kBM + quad * 32;
 #pragma unroll
           for (int pass = 0; pass < 2; ++pass) {
@@ -426,7 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // Opts a kernel into the large dynamic shared memory once per device.
 static nvfp4_status set_smem_attr(const void* fn, int which, int smem) {
   static std::mutex mu;
-  static bool done[2][64] = {};
+  static bool done[4][64] = {};
   int dev = 0;
   NV_CHECK(check_cuda(cudaGetDevice(&dev), "cudaGetDevice"));
   if (dev < 0 || dev >= 64) dev = 63;
@@ -442,17 +494,21 @@ static nvfp4_status set_smem_attr(const void* fn, int which, int smem) {
 nvfp4_status launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t s) {
   int sms = 0;
   NV_CHECK(device_sm_count(&sms));
-  const bool gu = a.epi == kEpiGateUp;
+  const bool gu = a.epi == kEpiGateUp || a.epi == kEpiSharedGateUp;
+  const bool bf = a.epi == kEpiSharedGateUp || a.epi == kEpiSharedDown;
   const int K = gu ? a.H : a.I;
   const int Nw = gu ? a.I : a.H;
+  // 128-byte K boxes: 128 packed FP4 bytes, or 64 bf16 elements
+  const CUtensorMapDataType dt = bf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  const uint64_t inner = bf ? (uint64_t)K : (uint64_t)K / 2;       // elements per row
+  const uint64_t pitch = bf ? (uint64_t)K * 2 : (uint64_t)K / 2;   // bytes per row
+  const uint32_t box = bf ? 64 : kBKBytes;
   CUtensorMap tmA, tmB0, tmB1;
-  NV_CHECK(make_tmap_2d(&tmA, a.a_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, (uint64_t)K / 2, (uint64_t)a.rows_capacity,
-                        (uint64_t)K / 2, kBKBytes, kBM));
-  NV_CHECK(make_tmap_2d(&tmB0, a.b0_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, (uint64_t)K / 2, (uint64_t)a.E * Nw,
-                        (uint64_t)K / 2, kBKBytes, gu ? 128 : kBN));
+  NV_CHECK(make_tmap_2d(&tmA, a.a_codes, dt, inner, (uint64_t)(a.a_rows > 0 ? a.a_rows : a.rows_capacity), pitch, box,
+                        kBM));
+  NV_CHECK(make_tmap_2d(&tmB0, a.b0_codes, dt, inner, (uint64_t)a.E * Nw, pitch, box, gu ? 128 : kBN));
   if (gu) {
-    NV_CHECK(make_tmap_2d(&tmB1, a.b1_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, (uint64_t)K / 2, (uint64_t)a.E * Nw,
-                          (uint64_t)K / 2, kBKBytes, 128));
+    NV_CHECK(make_tmap_2d(&tmB1, a.b1_codes, dt, inner, (uint64_t)a.E * Nw, pitch, box, 128));
   } else {
     tmB1 = tmB0;
   }
@@ -481,19 +537,32 @@ nvfp4_status launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t s) {
   p.y_bf16 = static_cast<uint16_t*>(a.y_bf16);
   p.y_f32 = a.y_f32;
   p.y_sq_part = a.y_sq_part;
+  p.h_bf16 = static_cast<uint16_t*>(a.h_bf16);
   p.H = a.H;
   p.per_expert = a.per_expert_scales ? 1 : 0;
   p.status = a.status;
   const int max_tiles = a.rows_capacity / kBM * p.n_tiles;
   const int grid = std::max(1, std::min(sms, max_tiles));
-  if (gu) {
-    NV_CHECK(set_smem_attr((const void*)grouped_fp4_gemm_kernel<kEpiGateUp>, 0, smem_bytes_of<kEpiGateUp>()));
-    return launch_dependent("grouped_fp4_gemm_kernel<gate_up>", grouped_fp4_gemm_kernel<kEpiGateUp>, dim3(grid),
-                            dim3(kThreads), smem_bytes_of<kEpiGateUp>(), s, tmA, tmB0, tmB1, p);
+  switch (a.epi) {
+    case kEpiGateUp:
+      NV_CHECK(set_smem_attr((const void*)grouped_fp4_gemm_kernel<kEpiGateUp>, 0, smem_bytes_of<kEpiGateUp>()));
+      return launch_dependent("grouped_fp4_gemm_kernel<gate_up>", grouped_fp4_gemm_kernel<kEpiGateUp>, dim3(grid),
+                              dim3(kThreads), smem_bytes_of<kEpiGateUp>(), s, tmA, tmB0, tmB1, p);
+    case kEpiDown:
+      NV_CHECK(set_smem_attr((const void*)grouped_fp4_gemm_kernel<kEpiDown>, 1, smem_bytes_of<kEpiDown>()));
+      return launch_dependent("grouped_fp4_gemm_kernel<down>", grouped_fp4_gemm_kernel<kEpiDown>, dim3(grid),
+                              dim3(kThreads), smem_bytes_of<kEpiDown>(), s, tmA, tmB0, tmB1, p);
+    case kEpiSharedGateUp:
+      NV_CHECK(set_smem_attr((const void*)grouped_fp4_gemm_kernel<kEpiSharedGateUp>, 2,
+                             smem_bytes_of<kEpiSharedGateUp>()));
+      return launch_dependent("grouped_fp4_gemm_kernel<shared_gate_up>", grouped_fp4_gemm_kernel<kEpiSharedGateUp>,
+                              dim3(grid), dim3(kThreads), smem_bytes_of<kEpiSharedGateUp>(), s, tmA, tmB0, tmB1, p);
+    default:
+      NV_CHECK(set_smem_attr((const void*)grouped_fp4_gemm_kernel<kEpiSharedDown>, 3,
+                             smem_bytes_of<kEpiSharedDown>()));
+      return launch_dependent("grouped_fp4_gemm_kernel<shared_down>", grouped_fp4_gemm_kernel<kEpiSharedDown>,
+                              dim3(grid), dim3(kThreads), smem_bytes_of<kEpiSharedDown>(), s, tmA, tmB0, tmB1, p);
   }
-  NV_CHECK(set_smem_attr((const void*)grouped_fp4_gemm_kernel<kEpiDown>, 1, smem_bytes_of<kEpiDown>()));
-  return launch_dependent("grouped_fp4_gemm_kernel<down>", grouped_fp4_gemm_kernel<kEpiDown>, dim3(grid),
-                          dim3(kThreads), smem_bytes_of<kEpiDown>(), s, tmA, tmB0, tmB1, p);
 }
 
 // Builds the m-tile -> expert map from caller-supplied segment offsets,
@@ -532,6 +601,14 @@ static nvfp4_status check_weights(const moe_nvfp4_weights* W) {
              W->H);
   NV_REQUIRE(W->I > 0 && W->I % 128 == 0, NVFP4_ERR_UNSUPPORTED_SHAPE, "I=%d must be a positive multiple of 128",
              W->I);
+  const bool any_shared = W->shared_gate || W->shared_up || W->shared_down || W->I_shared;
+  NV_REQUIRE(!any_shared || (W->shared_gate && W->shared_up && W->shared_down && W->I_shared > 0 &&
+                             W->I_shared % 128 == 0),
+             NVFP4_ERR_INVALID_ARG, "shared expert: all three weights and I_shared %% 128 == 0 (I_shared=%d)",
+             W->I_shared);
+  NV_REQUIRE(!any_shared || (aligned(W->shared_gate, 16) && aligned(W->shared_up, 16) &&
+                             aligned(W->shared_down, 16)),
+             NVFP4_ERR_INVALID_ARG, "shared expert weights need 16-byte alignment");
   return NVFP4_OK;
 }
 

@@ -5,7 +5,9 @@
 
 namespace nvfp4moe {
 
-enum GemmEpilogue { kEpiGateUp = 0, kEpiDown = 1 };
+// 0/1: the routed experts' block-scaled FP4 GEMMs; 2/3: the same tiles on
+// bf16 operands for the shared expert (dense, no scale factors)
+enum GemmEpilogue { kEpiGateUp = 0, kEpiDown = 1, kEpiSharedGateUp = 2, kEpiSharedDown = 3 };
 
 // One grouped GEMM over the permuted rows: row tile m (128 rows) belongs to
 // expert tile_expert[m]; m-tiles beyond *num_mtiles are not computed.
@@ -13,6 +15,7 @@ struct GroupedGemmArgs {
   int epi = kEpiGateUp;
   int E = 0, H = 0, I = 0;
   int rows_capacity = 0;
+  int a_rows = 0;            // rows the A tensor map covers (0: rows_capacity); TMA reads zeros past them
   // A operand: packed codes [rows][K/2], tiled scales
   const uint8_t* a_codes = nullptr;
   const uint8_t* a_scales = nullptr;
@@ -45,6 +48,8 @@ struct GroupedGemmArgs {
   // nullable [rows][H/128]: sum of squares of each thread's 128 scaled y
   // values (the REAP saliency's row norms are finished from these)
   float* y_sq_part = nullptr;
+  // kEpiSharedGateUp output: silu(gate) * up as bf16 [rows][I]
+  void* h_bf16 = nullptr;
   uint32_t* status = nullptr;
 };
 
