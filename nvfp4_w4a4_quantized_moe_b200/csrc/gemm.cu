@@ -49,15 +49,19 @@ template <int EPI> __host__ __device__ constexpr int stage_bytes_of() {
   return is_bf16<EPI>() ? kABytes + kBBytes : kStageBytes;
 }
 template <int EPI> __host__ __device__ constexpr int bk_of() { return is_bf16<EPI>() ? 64 : kBK; }
-// Pipeline stages: the gate/up GEMMs keep four; the down GEMMs stage y in
-// shared memory, 32 rows x 64 bf16 columns (4 KiB) per warp at a time, which
-// costs the FP4 down GEMM one of its stages.
-template <int EPI> __host__ __device__ constexpr int stages_of() { return EPI == kEpiDown ? 3 : 4; }
-constexpr int kYPassCols = 64;
-constexpr int kYStageBytes = 32 * kYPassCols * 2;
+// Pipeline stages: four in every kind.  The down GEMMs stage y in shared
+// memory, 32 rows x y_pass_cols_of() bf16 columns per warp at a time: 64 columns
+// (4 KiB) for the bf16 kind, 16 (1 KiB) for the FP4 kind, whose four 54 KiB
+// stages leave no room for more.
+template <int EPI> __host__ __device__ constexpr int stages_of() { return 4; }
+template <int EPI> __host__ __device__ constexpr int y_pass_cols_of() { return EPI == kEpiDown ? 16 : 64; }
+template <int EPI> __host__ __device__ constexpr int y_stage_bytes_of() { return 32 * y_pass_cols_of<EPI>() * 2; }
 template <int EPI> __host__ __device__ constexpr int smem_bytes_of() {
-  return stages_of<EPI>() * stage_bytes_of<EPI>() + 1024 + (is_gate_up<EPI>() ? 0 : kEpiWarps * kYStageBytes);
+  return stages_of<EPI>() * stage_bytes_of<EPI>() + 1024 + (is_gate_up<EPI>() ? 0 : kEpiWarps * y_stage_bytes_of<EPI>());
 }
+static_assert(smem_bytes_of<kEpiDown>() <= 232448 - 256, "FP4 down GEMM shared memory");
+static_assert(smem_bytes_of<kEpiGateUp>() <= 232448 - 256, "FP4 gate/up GEMM shared memory");
+static_assert(smem_bytes_of<kEpiSharedDown>() <= 232448 - 256, "bf16 down GEMM shared memory");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCol = 0;                  // 256 fp32 accumulator columns
 // Scale factors of one stage: 4 MMA k-steps x (4 SFA + 8 SFB) columns.  The
@@ -440,25 +444,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t real_mask = __ballot_sync(0xffffffffu, real);
         if (p.y_bf16 && real_mask != 0) {
           // Each lane holds one row.  Stores straight from registers would
-          // hit 32 rows per instruction, so the warp stages 64 columns of its
-          // 32 rows in shared memory (16-byte chunks XOR-swizzled by row) and
-          // writes them back four whole 128-byte row segments per instruction.
-          uint4* ybuf = reinterpret_cast<uint4*>(smem + kStages * kSB + (warp - 2) * kYStageBytes);
+          // hit 32 rows per instruction, so the warp stages kYCols columns of
+          // its 32 rows in shared memory and writes them back as whole row
+          // segments (kYCols * 2 bytes), 32 / kCh rows per instruction.  The
+          // 16-byte chunks are XOR-swizzled by row so that every 8-lane phase
+          // of a 16-byte access covers the 32 banks once, in both directions.
+          constexpr int kYCols = y_pass_cols_of<EPI>(), kCh = kYCols / 8, kRowsPer = 32 / kCh;
+          uint4* ybuf = reinterpret_cast<uint4*>(smem + kStages * kSB + (warp - 2) * y_stage_bytes_of<EPI>());
           const int row0 = mt * kBM + quad * 32;
+          auto swz = [](int r) { return (r / (8 / kCh)) % kCh; };
 #pragma unroll
-          for (int pass = 0; pass < 2; ++pass) {
+          for (int pass = 0; pass < 128 / kYCols; ++pass) {
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-              ybuf[lane * 8 + (ch ^ (lane & 7))] = make_uint4(yw[pass * 32 + ch * 4], yw[pass * 32 + ch * 4 + 1],
-                                                              yw[pass * 32 + ch * 4 + 2], yw[pass * 32 + ch * 4 + 3]);
+            for (int ch = 0; ch < kCh; ++ch) {
+              const int w = pass * (kYCols / 2) + ch * 4;
+              ybuf[lane * kCh + (ch ^ swz(lane))] = make_uint4(yw[w], yw[w + 1], yw[w + 2], yw[w + 3]);
             }
             __syncwarp();
 #pragma unroll
-            for (int it = 0; it < 8; ++it) {
-              const int rr = it * 4 + (lane >> 3), ch = lane & 7;
-              const uint4 v = ybuf[rr * 8 + (ch ^ (rr & 7))];
+            for (int it = 0; it < kCh; ++it) {
+              const int rr = it * kRowsPer + lane / kCh, ch = lane % kCh;
+              const uint4 v = ybuf[rr * kCh + (ch ^ swz(rr))];
               if ((real_mask >> rr) & 1u)
-                *reinterpret_cast<uint4*>(p.y_bf16 + (size_t)(row0 + rr) * p.H + col0 + pass * kYPassCols + ch * 8) = v;
+                *reinterpret_cast<uint4*>(p.y_bf16 + (size_t)(row0 + rr) * p.H + col0 + pass * kYCols + ch * 8) = v;
             }
             __syncwarp();
           }
