@@ -34,13 +34,14 @@ static inline int router_n_mma(int E) { return (E + 15) / 16 * 16; }
 static inline int router_stage_bytes(int E) { return kRAbytes + (router_n_mma(E) * 128 + 1023) / 1024 * 1024; }
 static inline int router_smem_bytes(int E) { return kRStages * router_stage_bytes(E) + 1024; }
 
-// Split count: enough CTAs to cover the SMs of a B200 (148) with at least
-// four K stages each.  A function of the shape only, so results are the same
-// on every device.
+// Split count: as many CTAs as fit on the SMs of a B200 (148) at one per SM,
+// with at least four K stages each; rounding up instead (a second CTA on
+// some SMs) measured slower.  A function of the shape only, so results are
+// the same on every device.
 int router_splits(int T, int H) {
   const int mt = (T + kRBM - 1) / kRBM;
   const int kt = H / kRBK;
-  int sp = (148 + mt - 1) / mt;
+  int sp = 148 / mt;
   sp = std::min(sp, std::max(1, kt / 4));
   return std::max(1, sp);
 }
@@ -185,34 +186,25 @@ __global__ void __launch_bounds__(kRThreads, 1)
 constexpr int kMaxE = 256, kMaxK = 16;
 
 // Logit of (token t, expert e).  With splits > 0 it is the split-ordered sum
-// of the router GEMM's partial sums (plus the optional offset), with up to
-// sixteen loads in flight, and is written to `logits`; with splits == 0 `src`
-// already holds the logits, and with splits < 0 it holds logits that this
-// kernel wrote itself.
+// of the router GEMM's partial sums (plus the optional offset), loaded eight
+// at a time so that they are in flight together, and is written to
+// `logits`; with splits == 0 `src` already holds the logits, and with
+// splits < 0 it holds logits that this kernel wrote itself.
 NVDEV float token_logit(const float* __restrict__ src, int splits, const float* __restrict__ offset,
                         float* __restrict__ logits, int T, int E, int t, int e) {
   const float* p = src + (size_t)t * E + e;
   if (splits == 0) return *p;
   if (splits < 0) return __ldcg(p);      // written earlier by this kernel: read through L2
   const size_t stride = (size_t)T * E;
-  float l = p[0];
-  int q = 1;
-  for (; q + 16 <= splits; q += 16) {
-    float v[16];
-#pragma unroll
-    for (int u = 0; u < 16; ++u) v[u] = p[(size_t)(q + u) * stride];
-#pragma unroll
-    for (int u = 0; u < 16; ++u) l = __fadd_rn(l, v[u]);
-  }
-  if (q + 8 <= splits) {
+  float l = 0.0f;
+  for (int q0 = 0; q0 < splits; q0 += 8) {
     float v[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) v[u] = p[(size_t)(q + u) * stride];
+    for (int u = 0; u < 8; ++u) v[u] = (q0 + u < splits) ? p[(size_t)(q0 + u) * stride] : 0.0f;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) l = __fadd_rn(l, v[u]);
-    q += 8;
+    for (int u = 0; u < 8; ++u)
+      if (q0 + u < splits) l = (q0 + u == 0) ? v[u] : __fadd_rn(l, v[u]);
   }
-  for (; q < splits; ++q) l = __fadd_rn(l, p[(size_t)q * stride]);
   if (offset) l = __fadd_rn(l, offset[e]);
   logits[(size_t)t * E + e] = l;
   return l;
@@ -226,12 +218,45 @@ NVDEV void topk_token(const float* __restrict__ src, int splits, const float* __
                       int t, int lane, int& out_idx, float& out_w) {
   float sig[kMaxE / 32], c[kMaxE / 32];
   const int per = (E + 31) >> 5;
+  // every slot's logit first, then the sigmoids.  With up to eight splits
+  // (large batches) all of the lane's partial sums are loaded before any is
+  // added, so their latencies overlap; the sums keep split order.
+  float lg[kMaxE / 32];
+  if (splits > 0 && splits <= 8) {
+    const size_t stride = (size_t)T * E;
+    float v[kMaxE / 32][8];
+#pragma unroll
+    for (int i = 0; i < kMaxE / 32; ++i) {
+      const int e = lane + 32 * i;
+      const float* p = src + (size_t)t * E + e;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[i][u] = (i < per && e < E && u < splits) ? p[(size_t)u * stride] : 0.0f;
+    }
+#pragma unroll
+    for (int i = 0; i < kMaxE / 32; ++i) {
+      const int e = lane + 32 * i;
+      float l = v[i][0];
+#pragma unroll
+      for (int u = 1; u < 8; ++u)
+        if (u < splits) l = __fadd_rn(l, v[i][u]);
+      if (i < per && e < E) {
+        if (offset) l = __fadd_rn(l, offset[e]);
+        logits[(size_t)t * E + e] = l;
+      }
+      lg[i] = l;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < kMaxE / 32; ++i) {
+      const int e = lane + 32 * i;
+      lg[i] = (i < per && e < E) ? token_logit(src, splits, offset, logits, T, E, t, e) : 0.0f;   // splits < 0: no write
+    }
+  }
 #pragma unroll
   for (int i = 0; i < kMaxE / 32; ++i) {
     const int e = lane + 32 * i;
     if (i < per && e < E) {
-      const float l = token_logit(src, splits, offset, logits, T, E, t, e);   // splits < 0: no write
-      sig[i] = sigmoid_fixed(l);
+      sig[i] = sigmoid_fixed(lg[i]);
       c[i] = __fadd_rn(sig[i], bias[e]);
     } else {
       sig[i] = 0.0f;
@@ -284,6 +309,8 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ src
                                                    const float* __restrict__ offset, float* __restrict__ logits,
                                                    const float* __restrict__ bias, int T, int E, int k, float rsf,
                                                    int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
+  griddep_wait();
+  griddep_launch();
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;
@@ -312,9 +339,18 @@ NVDEV void build_bitmap(uint32_t (*bm)[kChunk / 32], const int32_t* topk_idx, in
   __syncthreads();
 }
 
+// Also fills perm with -1 and row_w with 0 over the padded capacity; the
+// scatter, two launches later, overwrites the real rows.
 __global__ void __launch_bounds__(kChunk) perm_count_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
-                                                            int32_t* __restrict__ chunk_counts) {
+                                                            int32_t* __restrict__ chunk_counts, int cap,
+                                                            int32_t* __restrict__ perm, float* __restrict__ row_w) {
   __shared__ uint32_t bm[kMaxE][kChunk / 32];
+  griddep_wait();
+  griddep_launch();
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < cap; i += gridDim.x * blockDim.x) {
+    perm[i] = -1;
+    row_w[i] = 0.0f;
+  }
   build_bitmap(bm, topk_idx, T, E, k, blockIdx.x * kChunk + threadIdx.x);
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     int n = 0;
@@ -332,6 +368,8 @@ __global__ void __launch_bounds__(256) perm_scan_kernel(int32_t* __restrict__ ch
                                                         int32_t* __restrict__ tile_expert,
                                                         int32_t* __restrict__ num_mtiles) {
   __shared__ int32_t sp[256];
+  griddep_wait();
+  griddep_launch();
   const int e = threadIdx.x;
   int total = 0;
   if (e < E)
@@ -370,6 +408,8 @@ __global__ void __launch_bounds__(kChunk) perm_scatter_kernel(const int32_t* __r
                                                               int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm,
                                                               float* __restrict__ row_w) {
   __shared__ uint32_t bm[kMaxE][kChunk / 32];
+  griddep_wait();
+  griddep_launch();
   const int t = blockIdx.x * kChunk + threadIdx.x;
   build_bitmap(bm, topk_idx, T, E, k, t);
   if (t >= T) return;
@@ -523,19 +563,18 @@ nvfp4_status launch_route(const RouteArgs& a, const RouteScratch& r, cudaStream_
                             a.T, a.E, a.k, a.rsf, cap, a.topk_idx, a.topk_w, r.counts, a.expert_offsets,
                             r.tile_expert, r.num_mtiles, a.perm, a.inv_perm, r.row_w);
   }
-  NV_CHECK(check_cuda(cudaMemsetAsync(a.perm, 0xFF, sizeof(int32_t) * (size_t)cap, s), "memset perm"));
-  NV_CHECK(check_cuda(cudaMemsetAsync(r.row_w, 0, sizeof(float) * (size_t)cap, s), "memset row_w"));
-  topk_kernel<<<(a.T + 7) / 8, 256, 0, s>>>(splits ? r.partial : a.logits, splits, a.logit_offset, a.logits, a.bias,
-                                            a.T, a.E, a.k, a.rsf, a.topk_idx, a.topk_w);
-  NV_CHECK(check_launch("topk_kernel"));
-  perm_count_kernel<<<nchunks, kChunk, 0, s>>>(a.topk_idx, a.T, a.E, a.k, r.chunk_counts);
-  NV_CHECK(check_launch("perm_count_kernel"));
-  perm_scan_kernel<<<1, 256, 0, s>>>(r.chunk_counts, nchunks, a.E, r.counts, a.expert_offsets, r.tile_expert,
-                                     r.num_mtiles);
-  NV_CHECK(check_launch("perm_scan_kernel"));
-  perm_scatter_kernel<<<nchunks, kChunk, 0, s>>>(a.topk_idx, a.topk_w, a.T, a.E, a.k, r.chunk_counts, a.perm,
-                                                 a.inv_perm, r.row_w);
-  return check_launch("perm_scatter_kernel");
+  // each kernel waits for its predecessor's results (griddepcontrol.wait) as
+  // its first step, so programmatic launch only hides the launch latency
+  NV_CHECK(launch_dependent("topk_kernel", topk_kernel, dim3((a.T + 7) / 8), dim3(256), 0, s,
+                            (const float*)(splits ? r.partial : a.logits), splits, a.logit_offset, a.logits, a.bias,
+                            a.T, a.E, a.k, a.rsf, a.topk_idx, a.topk_w));
+  NV_CHECK(launch_dependent("perm_count_kernel", perm_count_kernel, dim3(nchunks), dim3(kChunk), 0, s,
+                            (const int32_t*)a.topk_idx, a.T, a.E, a.k, r.chunk_counts, cap, a.perm, r.row_w));
+  NV_CHECK(launch_dependent("perm_scan_kernel", perm_scan_kernel, dim3(1), dim3(256), 0, s, r.chunk_counts, nchunks,
+                            a.E, r.counts, a.expert_offsets, r.tile_expert, r.num_mtiles));
+  return launch_dependent("perm_scatter_kernel", perm_scatter_kernel, dim3(nchunks), dim3(kChunk), 0, s,
+                          (const int32_t*)a.topk_idx, (const float*)a.topk_w, a.T, a.E, a.k,
+                          (const int32_t*)r.chunk_counts, a.perm, a.inv_perm, r.row_w);
 }
 
 nvfp4_status check_route_shape(int T, int H, int E, int k) {
