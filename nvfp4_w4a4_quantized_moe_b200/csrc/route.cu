@@ -186,10 +186,11 @@ __global__ void __launch_bounds__(kRThreads, 1)
 constexpr int kMaxE = 256, kMaxK = 16;
 
 // Logit of (token t, expert e).  With splits > 0 it is the split-ordered sum
-// of the router GEMM's partial sums (plus the optional offset), loaded eight
+// of the router GEMM's partial sums (plus the optional offset), loaded kBatch
 // at a time so that they are in flight together, and is written to
 // `logits`; with splits == 0 `src` already holds the logits, and with
 // splits < 0 it holds logits that this kernel wrote itself.
+template <int kBatch = 8>
 NVDEV float token_logit(const float* __restrict__ src, int splits, const float* __restrict__ offset,
                         float* __restrict__ logits, int T, int E, int t, int e) {
   const float* p = src + (size_t)t * E + e;
@@ -197,12 +198,12 @@ NVDEV float token_logit(const float* __restrict__ src, int splits, const float* 
   if (splits < 0) return __ldcg(p);      // written earlier by this kernel: read through L2
   const size_t stride = (size_t)T * E;
   float l = 0.0f;
-  for (int q0 = 0; q0 < splits; q0 += 8) {
-    float v[8];
+  for (int q0 = 0; q0 < splits; q0 += kBatch) {
+    float v[kBatch];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) v[u] = (q0 + u < splits) ? p[(size_t)(q0 + u) * stride] : 0.0f;
+    for (int u = 0; u < kBatch; ++u) v[u] = (q0 + u < splits) ? p[(size_t)(q0 + u) * stride] : 0.0f;
 #pragma unroll
-    for (int u = 0; u < 8; ++u)
+    for (int u = 0; u < kBatch; ++u)
       if (q0 + u < splits) l = (q0 + u == 0) ? v[u] : __fadd_rn(l, v[u]);
   }
   if (offset) l = __fadd_rn(l, offset[e]);
@@ -263,42 +264,42 @@ NVDEV void topk_token(const float* __restrict__ src, int splits, const float* __
       c[i] = -INFINITY;
     }
   }
-  uint32_t taken = 0;
+  // Selection keys: sigma + bias mapped to unsigned integers in the same
+  // order (sign bit flipped for non-negative values, all bits for negative
+  // ones; sigma > 0, so the sum is never -0), 0 for an absent or taken
+  // expert.  Each round is a warp max of the keys, then a warp min of the
+  // expert ids that reach it: the largest score, ties to the lower expert.
+  uint32_t key[kMaxE / 32];
+#pragma unroll
+  for (int i = 0; i < kMaxE / 32; ++i) {
+    const uint32_t u = __float_as_uint(c[i]);
+    key[i] = (i < per && lane + 32 * i < E) ? ((u & 0x80000000u) ? ~u : (u | 0x80000000u)) : 0u;
+  }
   float sum = 0.0f, my_sig = 0.0f;
   int my_idx = 0;
   for (int j = 0; j < k; ++j) {
-    float bc = -INFINITY;
-    int be = 0x7fffffff;
+    uint32_t bk = 0u, be = 0xffffffffu;
 #pragma unroll
-    for (int i = 0; i < kMaxE / 32; ++i) {
-      const int e = lane + 32 * i;
-      if (i < per && e < E && !((taken >> i) & 1u) && (c[i] > bc || (c[i] == bc && e < be))) {
-        bc = c[i];
-        be = e;
+    for (int i = 0; i < kMaxE / 32; ++i)       // ascending i: a tie keeps the lower expert
+      if (key[i] > bk) {
+        bk = key[i];
+        be = (uint32_t)(lane + 32 * i);
       }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float oc = __shfl_xor_sync(0xffffffffu, bc, o);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-      if (oc > bc || (oc == bc && oe < be)) {
-        bc = oc;
-        be = oe;
-      }
-    }
+    const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
+    const int win = (int)__reduce_min_sync(0xffffffffu, bk == m ? be : 0xffffffffu);
     // the owner lane marks the winner and broadcasts its sigma
     float s_own = 0.0f;
 #pragma unroll
     for (int i = 0; i < kMaxE / 32; ++i)
-      if (lane + 32 * i == be) {
+      if (lane + 32 * i == win) {
         s_own = sig[i];
-        taken |= 1u << i;
+        key[i] = 0u;
       }
-    const float s_sel = __shfl_sync(0xffffffffu, s_own, be & 31);
+    const float s_sel = __shfl_sync(0xffffffffu, s_own, win & 31);
     sum = __fadd_rn(sum, s_sel);
     if (lane == j) {
       my_sig = s_sel;
-      my_idx = be;
+      my_idx = win;
     }
   }
   out_idx = my_idx;
@@ -330,6 +331,28 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ src
 // counts into row bases.  Everything is integer and order-independent.
 // ---------------------------------------------------------------------------
 constexpr int kChunk = 256;
+
+// In-place exclusive scan of sp[0..256) by warp 0 of the block (eight entries
+// per lane, then a shuffle scan of the lane sums); the caller synchronises
+// the block before and after.
+NVDEV void warp0_exclusive_scan256(int32_t* sp) {
+  if ((threadIdx.x >> 5) != 0) return;
+  const int lane = threadIdx.x & 31;
+  int ex[8], run = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    ex[j] = run;
+    run += sp[lane * 8 + j];
+  }
+  int inc = run;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += y;
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) sp[lane * 8 + j] = inc - run + ex[j];
+}
 
 NVDEV void build_bitmap(uint32_t (*bm)[kChunk / 32], const int32_t* topk_idx, int T, int E, int k, int t) {
   for (int i = threadIdx.x; i < E * (kChunk / 32); i += blockDim.x) bm[i / (kChunk / 32)][i % (kChunk / 32)] = 0;
@@ -377,14 +400,9 @@ __global__ void __launch_bounds__(256) perm_scan_kernel(int32_t* __restrict__ ch
   const int padded = (total + kRowTile - 1) / kRowTile * kRowTile;
   sp[e] = (e < E) ? padded : 0;
   __syncthreads();
-  // inclusive scan (Hillis-Steele) over 256 entries
-  for (int o = 1; o < 256; o <<= 1) {
-    const int v = (e >= o) ? sp[e - o] : 0;
-    __syncthreads();
-    sp[e] += v;
-    __syncthreads();
-  }
-  const int start = sp[e] - ((e < E) ? padded : 0);
+  warp0_exclusive_scan256(sp);
+  __syncthreads();
+  const int start = sp[e];
   if (e < E) {
     offsets[e] = start;
     counts[e] = total;
@@ -429,8 +447,8 @@ __global__ void __launch_bounds__(kChunk) perm_scatter_kernel(const int32_t* __r
 // ---------------------------------------------------------------------------
 // Routing of a small batch (T <= 256) in one block: top-k, per-expert counts,
 // the padded scan, and the scatter, with the padding fill of perm and row_w
-// that the large-batch path leaves to memsets.  The arithmetic is the same
-// (topk_token) and so is every integer result.
+// that the large-batch path does in its count kernel.  The arithmetic is the
+// same (topk_token) and so is every integer result.
 // ---------------------------------------------------------------------------
 constexpr int kSmallT = 256;
 constexpr int kSmallThreads = 1024;
@@ -458,7 +476,8 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
   // all logits first, one (token, expert) per thread, so that every thread's
   // partial-sum loads are in flight at once
   if (splits > 0) {
-    for (int i = tid; i < T * E; i += blockDim.x) token_logit(src, splits, offset, logits, T, E, i / E, i % E);
+    // the decode shape has 24 splits: one batch of loads per pair
+    for (int i = tid; i < T * E; i += blockDim.x) token_logit<24>(src, splits, offset, logits, T, E, i / E, i % E);
     src = logits;
     splits = -1;
   }
@@ -481,14 +500,10 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
   padded = (total + kRowTile - 1) / kRowTile * kRowTile;
   if (tid < 256) sp[tid] = tid < E ? padded : 0;
   __syncthreads();
-  for (int o = 1; o < 256; o <<= 1) {
-    const int v = (tid < 256 && tid >= o) ? sp[tid - o] : 0;
-    __syncthreads();
-    if (tid < 256) sp[tid] += v;
-    __syncthreads();
-  }
+  warp0_exclusive_scan256(sp);
+  __syncthreads();
   if (tid < E) {
-    const int start = sp[tid] - padded;
+    const int start = sp[tid];
     base[tid] = start;
     offsets[tid] = start;
     counts[tid] = total;

@@ -62,7 +62,10 @@ def test_skewed_loads_and_empty_experts():
 @pytest.mark.parametrize("name,T,H,E,k,offset_std", [("tiny", 32, 256, 8, 2, 0.0),
                                                      ("mid", 1000, 1024, 80, 8, 0.5),
                                                      ("decode", 16, 6144, 80, 8, 0.0),
-                                                     ("prefill", 8192, 6144, 80, 8, 0.5)])
+                                                     ("prefill", 8192, 6144, 80, 8, 0.5),
+                                                     # router split counts 1 and 24 on the large-batch path
+                                                     ("one_split", 9600, 512, 80, 8, 0.0),
+                                                     ("many_splits", 600, 6144, 80, 8, 0.0)])
 def test_route_from_hidden_states(name, T, H, E, k, offset_std):
     """Logits match fp64 within the fp32 summation bound; top-k sets match
     wherever the oracle's k-th and (k+1)-th biased scores are apart by more
