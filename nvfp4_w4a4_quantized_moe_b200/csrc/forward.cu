@@ -38,9 +38,27 @@ __global__ void __launch_bounds__(128) quantize_scatter_kernel(const uint4* __re
   // block (t, by): token t, 16-element blocks [128 by, 128 by + 128) of its row
   __shared__ int32_t rows[16];
   __shared__ float gs[16];
+  const int t = blockIdx.x;
+  const int nblk = H / kQBlock;
+  const int lane = threadIdx.x & 31;
+  const int kb = blockIdx.y * blockDim.x + threadIdx.x;
+  const bool valid = kb < nblk;
+  // x is the caller's input, so it is read before waiting for the routing;
+  // with the tensor's own g1 (also an input) it is quantised there as well
+  uint4 u0 = make_uint4(0, 0, 0, 0), u1 = u0;
+  if (valid) {
+    const uint4* src = x + ((size_t)t * H + (size_t)kb * kQBlock) / 8;
+    u0 = __ldg(src);
+    u1 = __ldg(src + 1);
+  }
+  uint2 c0 = make_uint2(0, 0);
+  uint32_t s0 = 0;
+  if (MODE == 0 && valid) {
+    const float g = act_gscale[0];
+    s0 = quant_block16_bf16(u0, u1, g, __fmul_rn(6.0f, g), c0);
+  }
   griddep_wait();
   griddep_launch();
-  const int t = blockIdx.x;
   if (threadIdx.x < k) {
     rows[threadIdx.x] = inv_perm[(size_t)t * k + threadIdx.x];
     if (MODE & kActPerExpert) {
@@ -56,16 +74,6 @@ __global__ void __launch_bounds__(128) quantize_scatter_kernel(const uint4* __re
     }
   }
   __syncthreads();
-  const int nblk = H / kQBlock;
-  const int lane = threadIdx.x & 31;
-  const int kb = blockIdx.y * blockDim.x + threadIdx.x;
-  const bool valid = kb < nblk;
-  uint4 u0 = make_uint4(0, 0, 0, 0), u1 = u0;
-  if (valid) {
-    const uint4* src = x + ((size_t)t * H + (size_t)kb * kQBlock) / 8;
-    u0 = __ldg(src);
-    u1 = __ldg(src + 1);
-  }
   auto write = [&](int row, const uint2& c, uint32_t s) {
     const uint32_t w1 = __shfl_down_sync(0xffffffffu, s, 1);
     const uint32_t w2 = __shfl_down_sync(0xffffffffu, s, 2);
@@ -85,11 +93,11 @@ __global__ void __launch_bounds__(128) quantize_scatter_kernel(const uint4* __re
       write(rows[j], c, s);
     }
   } else {
-    const float g = (MODE & kActDynamic) ? dynamic_gscale(amax_bits[0]) : act_gscale[0];
-    uint2 c = make_uint2(0, 0);
-    uint32_t s = 0;
-    if (valid) s = quant_block16_bf16(u0, u1, g, __fmul_rn(6.0f, g), c);
-    for (int j = 0; j < k; ++j) write(rows[j], c, s);
+    if (MODE & kActDynamic) {
+      const float g = dynamic_gscale(amax_bits[0]);
+      if (valid) s0 = quant_block16_bf16(u0, u1, g, __fmul_rn(6.0f, g), c0);
+    }
+    for (int j = 0; j < k; ++j) write(rows[j], c0, s0);
   }
 }
 
