@@ -453,13 +453,14 @@ def run_ours(args, cfg):
 
     # offline weight quantiser over the full layer (the quantiser workload)
     qws = torch.empty(c.lib.nvfp4_quantize_weights_workspace_size(cfg.E), dtype=torch.uint8, device=dev)
+    qlayout = "staged" if W.codes_layout == c.LAYOUT_STAGED else "tiled"     # what the layer's weights use
     qbytes = 0
     for w in (gate, up, down):
         n = w.numel()
         qbytes += 2 * n + n // 2 + n // 16 + 4 * w.shape[0]
     for _ in range(3):
         for w in (gate, up, down):
-            c.nvfp4_quantize_weights(w, "tiled", workspace=qws)
+            c.nvfp4_quantize_weights(w, qlayout, workspace=qws)
     torch.cuda.synchronize()
     dist.barrier()
     q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -467,7 +468,7 @@ def run_ours(args, cfg):
     q0.record(stream)
     for _ in range(qsteps):
         for w in (gate, up, down):
-            c.nvfp4_quantize_weights(w, "tiled", workspace=qws)
+            c.nvfp4_quantize_weights(w, qlayout, workspace=qws)
     q1.record(stream)
     torch.cuda.synchronize()
     q_ms = dist.max(q0.elapsed_time(q1)) / qsteps
@@ -556,12 +557,13 @@ def block_stats_report(c, cfg, bf16_weights, W, stream, dist, peaks):
     and bandwidth of the statistics kernel (2.5625 bytes read per element)."""
     enc = ((W.gate_codes, W.gate_scales, W.gate_gscale), (W.up_codes, W.up_scales, W.up_gscale),
            (W.down_codes, W.down_scales, W.down_gscale))
+    layout = "staged" if W.codes_layout == c.LAYOUT_STAGED else "tiled"
     bufs = [torch.empty((w.shape[0], len(c.BLOCK_STATS_FIELDS)), dtype=torch.int64, device=w.device)
             for w in bf16_weights]
 
     def run():
         for w, (cd, sc, g), b in zip(bf16_weights, enc, bufs):
-            c.nvfp4_block_stats_compute(w, cd, sc, g, "tiled", 0.1, stats=b)
+            c.nvfp4_block_stats_compute(w, cd, sc, g, layout, 0.1, stats=b)
 
     run()
     torch.cuda.synchronize()

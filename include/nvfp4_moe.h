@@ -35,6 +35,19 @@
  *       major, and inside an atom row r (0..127), block b (0..3) sits at byte
  *       (r % 32) * 16 + (r / 32) * 4 + b.  The buffer holds
  *       ceil(rows/128) * 128 * cols / 16 bytes; needs cols % 64 == 0.
+ *   - Weight code layouts (the packed codes of a weight matrix, rows x cols):
+ *       NVFP4_LAYOUT_CANONICAL / NVFP4_LAYOUT_TILED: [rows][cols/2] row-major.
+ *       NVFP4_LAYOUT_STAGED (scales TILED as above): the bytes the GEMM
+ *       copies to shared memory for one 128-row x 256-column K stage are one
+ *       contiguous, pre-swizzled 16 KiB tile.  Tile (i, j) covers rows
+ *       [128 i, 128 i + 128) and columns [256 j, 256 j + 256) and starts at
+ *       byte (i * cols/256 + j) * 16384.  Inside it, row r (0..127) fills
+ *       bytes [128 r, 128 r + 128), and the 16 bytes of its columns
+ *       [256 j + 32 c, 256 j + 32 c + 32) sit at byte 128 r + 16 (c ^ (r % 8)):
+ *       the image a 128-byte-swizzled TMA box leaves in shared memory.  The
+ *       buffer has the canonical size; needs rows % 128 == 0 and
+ *       cols % 256 == 0.  Streaming a stage then reads one contiguous range
+ *       instead of 128 rows of 128 bytes.
  *   - Workspace: calls that take (ws, ws_bytes) need at least the size their
  *     *_workspace_size() function returns, 256-byte aligned.  Its first word
  *     is a status word: each call clears it when it starts and a device-side
@@ -66,7 +79,7 @@ typedef enum nvfp4_status {
   NVFP4_ERR_DEVICE = 6             /* the current device is not an sm_100 GPU */
 } nvfp4_status;
 
-enum { NVFP4_LAYOUT_CANONICAL = 0, NVFP4_LAYOUT_TILED = 1 };
+enum { NVFP4_LAYOUT_CANONICAL = 0, NVFP4_LAYOUT_TILED = 1, NVFP4_LAYOUT_STAGED = 2 };
 
 /* Message for the last failed call on this host thread ("" if none). */
 NVFP4_API const char* nvfp4_last_error(void);
@@ -88,11 +101,14 @@ NVFP4_API nvfp4_status nvfp4_workspace_status(void* ws, void* stream);
  * of a row: s = E4M3(amax_block / (6 g)), S = s * g, codes = E2M1(x * (1/S))
  * with round-to-nearest-even and saturation; a zero block or matrix gives
  * scale 0 and codes +-0.
- *   codes        [n_mats][rows][cols/2]
+ *   codes        [n_mats][rows][cols/2]; STAGED: each matrix's codes in the
+ *                staged layout (its n_mats * rows * cols / 2 bytes)
  *   scales       CANONICAL: [n_mats][rows][cols/16];
- *                TILED: n_mats * rows rows in the tiled layout (rows % 128 == 0)
+ *                TILED, STAGED: n_mats * rows rows in the tiled layout
+ *                (rows % 128 == 0)
  *   global_scale [n_mats] fp32
- * Needs cols % 32 == 0 (TILED: cols % 64 == 0, rows % 128 == 0).
+ * Needs cols % 32 == 0 (TILED: cols % 64 == 0, rows % 128 == 0; STAGED:
+ * cols % 256 == 0, rows % 128 == 0).
  * Each matrix is read twice (amax pass, then quantise pass) with the second
  * read scheduled while the matrix is still in L2.
  * ---------------------------------------------------------------------- */
@@ -191,6 +207,10 @@ typedef struct moe_nvfp4_weights {
   const void* shared_up;          /* bf16 [I_shared][H]                          */
   const void* shared_down;        /* bf16 [H][I_shared]                          */
   int I_shared;
+  /* Layout of gate_codes, up_codes and down_codes: NVFP4_LAYOUT_CANONICAL
+   * (0, row-major as above) or NVFP4_LAYOUT_STAGED (needs H % 256 == 0 and
+   * I % 256 == 0).  The scales are TILED either way. */
+  int codes_layout;
 } moe_nvfp4_weights;
 
 /* Optional copies of intermediate results (every pointer nullable; device
@@ -307,8 +327,8 @@ NVFP4_API nvfp4_status moe_nvfp4_down(const moe_nvfp4_weights* W, const uint8_t*
  * weights of their block).
  *
  * For each of n_mats matrices w[m] ([rows][cols] bf16) and its NVFP4 encoding
- * (codes [n_mats][rows][cols/2], scales in `layout` as the weight quantiser
- * writes them, global_scale[n_mats]), stats[m] receives:
+ * (codes and scales in `layout` as the weight quantiser writes them,
+ * global_scale[n_mats]), stats[m] receives:
  *   elements, outliers            elements; elements with |w| > threshold
  *   blocks, outlier_blocks        16-element blocks; blocks holding an outlier
  *   zero_scale_blocks             blocks with scale code 0
@@ -323,8 +343,9 @@ NVFP4_API nvfp4_status moe_nvfp4_down(const moe_nvfp4_weights* W, const uint8_t*
  * Counts are exact.  The sums are taken in fp32 within a block and in fp64
  * across blocks, which keeps them within about 1e-6 relative.  `stats`
  * is device memory of n_mats entries; the call overwrites it.  Needs
- * cols % 16 == 0 (TILED: cols % 64 == 0, rows % 128 == 0), w 16-byte and
- * codes and stats 8-byte aligned.  Reads 2.5625 bytes per element.
+ * cols % 16 == 0 (TILED: cols % 64 == 0, rows % 128 == 0; STAGED:
+ * cols % 256 == 0, rows % 128 == 0), w 16-byte and codes and stats 8-byte
+ * aligned.  Reads 2.5625 bytes per element.
  * ---------------------------------------------------------------------- */
 typedef struct {
   uint64_t elements, outliers, blocks, outlier_blocks, zero_scale_blocks, subnormal_scale_blocks,

@@ -21,7 +21,8 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnvfp4moe
 
 LAYOUT_CANONICAL = 0
 LAYOUT_TILED = 1
-_LAYOUTS = {"canonical": LAYOUT_CANONICAL, "tiled": LAYOUT_TILED}
+LAYOUT_STAGED = 2          # weight codes in K-stage tiles, scales tiled
+_LAYOUTS = {"canonical": LAYOUT_CANONICAL, "tiled": LAYOUT_TILED, "staged": LAYOUT_STAGED}
 
 STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED_SHAPE", 3: "CUDA", 4: "TIMEOUT", 5: "WORKSPACE",
                 6: "DEVICE"}
@@ -48,7 +49,8 @@ class MoeWeightsStruct(ctypes.Structure):
                 ("gate_codes", _vp), ("gate_scales", _vp), ("gate_gscale", _vp),
                 ("up_codes", _vp), ("up_scales", _vp), ("up_gscale", _vp),
                 ("down_codes", _vp), ("down_scales", _vp), ("down_gscale", _vp),
-                ("shared_gate", _vp), ("shared_up", _vp), ("shared_down", _vp), ("I_shared", _i)]
+                ("shared_gate", _vp), ("shared_up", _vp), ("shared_down", _vp), ("I_shared", _i),
+                ("codes_layout", _i)]
 
 
 DEBUG_FIELDS = ("logits", "topk_idx", "topk_w", "expert_offsets", "perm", "inv_perm", "a_codes", "a_scales", "h",
@@ -168,7 +170,7 @@ def nvfp4_quantize_weights(w: torch.Tensor, layout: str = "tiled", workspace: to
     n, rows, cols = w.shape
     lay = _LAYOUTS[layout]
     codes = torch.empty((n, rows, cols // 2), dtype=torch.uint8, device=w.device)
-    if lay == LAYOUT_TILED:
+    if lay != LAYOUT_CANONICAL:
         scales = torch.empty(tiled_scale_bytes(n * rows, cols), dtype=torch.uint8, device=w.device)
     else:
         scales = torch.empty((n, rows, cols // 16), dtype=torch.uint8, device=w.device)
@@ -192,7 +194,8 @@ def nvfp4_quantize_weights_noalloc(w: torch.Tensor, layout: str = "tiled", out=N
     if out is None:
         codes = torch.empty((n, rows, cols // 2), dtype=torch.uint8, device=w.device)
         scales = (torch.empty(tiled_scale_bytes(n * rows, cols), dtype=torch.uint8, device=w.device)
-                  if lay == LAYOUT_TILED else torch.empty((n, rows, cols // 16), dtype=torch.uint8, device=w.device))
+                  if lay != LAYOUT_CANONICAL else torch.empty((n, rows, cols // 16), dtype=torch.uint8,
+                                                              device=w.device))
         gscale = torch.empty(n, dtype=torch.float32, device=w.device)
     else:
         codes, scales, gscale = out
@@ -290,7 +293,8 @@ def moe_route(x, router_weight, bias, k: int, rsf: float, logit_offset=None, log
 
 @dataclass
 class MoeWeights:
-    """Device tensors of one NVFP4 MoE layer (scales in the tiled layout)."""
+    """Device tensors of one NVFP4 MoE layer (scales in the tiled layout; codes
+    row-major or, with ``codes_layout`` = LAYOUT_STAGED, in K-stage tiles)."""
     E: int
     H: int
     I: int
@@ -311,6 +315,7 @@ class MoeWeights:
     shared_gate: torch.Tensor | None = None
     shared_up: torch.Tensor | None = None
     shared_down: torch.Tensor | None = None
+    codes_layout: int = LAYOUT_CANONICAL
 
     @property
     def I_shared(self) -> int:
@@ -327,18 +332,25 @@ class MoeWeights:
                                 _p(self.bias), _p(self.gate_codes), _p(self.gate_scales), _p(self.gate_gscale),
                                 _p(self.up_codes), _p(self.up_scales), _p(self.up_gscale), _p(self.down_codes),
                                 _p(self.down_scales), _p(self.down_gscale), _p(self.shared_gate),
-                                _p(self.shared_up), _p(self.shared_down), self.I_shared)
+                                _p(self.shared_up), _p(self.shared_down), self.I_shared, int(self.codes_layout))
 
     @classmethod
-    def quantize(cls, gate, up, down, router_weight, bias, k: int, rsf: float) -> "MoeWeights":
+    def quantize(cls, gate, up, down, router_weight, bias, k: int, rsf: float,
+                 codes_layout: str | None = None) -> "MoeWeights":
         """RTN-quantise bf16 expert weights (gate/up [E, I, H], down [E, H, I])
-        with the library's weight quantiser, tiled scales."""
+        with the library's weight quantiser, tiled scales.  The codes are
+        staged when H and I are multiples of 256 (``codes_layout`` None), else
+        row-major; "staged" or "canonical" forces one."""
         E, I, H = gate.shape
-        gc, gs, gg = nvfp4_quantize_weights(gate, "tiled")
-        uc, us, ug = nvfp4_quantize_weights(up, "tiled")
-        dc, ds, dg = nvfp4_quantize_weights(down, "tiled")
+        if codes_layout is None:
+            codes_layout = "staged" if H % 256 == 0 and I % 256 == 0 else "canonical"
+        lay = "staged" if codes_layout == "staged" else "tiled"
+        gc, gs, gg = nvfp4_quantize_weights(gate, lay)
+        uc, us, ug = nvfp4_quantize_weights(up, lay)
+        dc, ds, dg = nvfp4_quantize_weights(down, lay)
         return cls(E, H, I, k, rsf, _cuda(router_weight, torch.bfloat16, "router_weight"),
-                   _cuda(bias, torch.float32, "bias"), gc, gs, gg, uc, us, ug, dc, ds, dg)
+                   _cuda(bias, torch.float32, "bias"), gc, gs, gg, uc, us, ug, dc, ds, dg,
+                   codes_layout=LAYOUT_STAGED if lay == "staged" else LAYOUT_CANONICAL)
 
 
 def reap_keep(saliency_sum: torch.Tensor, saliency_count: torch.Tensor, keep: int) -> torch.Tensor:
@@ -355,8 +367,8 @@ def select_experts(W: "MoeWeights", keep: torch.Tensor) -> "MoeWeights":
     """The layer restricted to the experts ``keep`` (in that order): gate.weight
     rows and e_score_correction_bias sliced as the pruned checkpoint does, and
     each retained expert's codes, tiled scales and global scales copied over
-    (an expert's I or H rows are whole 128-row scale tiles, so its scales are
-    one contiguous range)."""
+    (an expert's I or H rows are whole 128-row tiles, so its scales and its
+    codes, row-major or staged, are contiguous ranges)."""
     idx = keep.to(W.router_weight.device)
     E2 = int(idx.numel())
 
@@ -371,7 +383,7 @@ def select_experts(W: "MoeWeights", keep: torch.Tensor) -> "MoeWeights":
                       codes(W.gate_codes), rows(W.gate_scales, W.I * W.H // 16), W.gate_gscale.index_select(0, idx),
                       codes(W.up_codes), rows(W.up_scales, W.I * W.H // 16), W.up_gscale.index_select(0, idx),
                       codes(W.down_codes), rows(W.down_scales, W.H * W.I // 16), W.down_gscale.index_select(0, idx),
-                      W.shared_gate, W.shared_up, W.shared_down)
+                      W.shared_gate, W.shared_up, W.shared_down, W.codes_layout)
 
 
 def moe_nvfp4_workspace_size(T: int, E: int, H: int, I: int, k: int, I_shared: int = 0) -> int:

@@ -170,6 +170,20 @@ NVDEV size_t tiled_scale_offset(int row, int kb, int nblk4) {
   return atom * kAtomBytes + (row & 31) * 16 + ((row >> 5) & 3) * 4 + (kb & 3);
 }
 
+// Staged code layout (NVFP4_LAYOUT_STAGED): the 8-byte unit that holds the
+// codes of 16-element block kb of `row` (nblk blocks per row, a multiple of
+// 16).  128 rows by one 256-element K stage form a 16 KiB tile; tiles are
+// stage-major within a row tile.  Inside a tile, row r fills bytes
+// [128 r, 128 r + 128) and its 16-byte chunk c (blocks 2c and 2c + 1) sits at
+// chunk c ^ (r % 8): the image a 128-byte-swizzled TMA box leaves in shared
+// memory, so that one plain bulk copy of a tile is an MMA operand.
+constexpr int kStagedTileBytes = 16384;
+NVDEV size_t staged_code_unit(size_t row, int kb, int nblk) {
+  const size_t tile = (row >> 7) * (size_t)(nblk >> 4) + (size_t)(kb >> 4);
+  const int r = (int)(row & 127), c = (kb & 15) >> 1;
+  return tile * (kStagedTileBytes / 8) + (size_t)r * 16 + (size_t)(((c ^ (r & 7)) << 1) | (kb & 1));
+}
+
 // ---------------------------------------------------------------------------
 // Shared memory, mbarriers, TMA
 // ---------------------------------------------------------------------------

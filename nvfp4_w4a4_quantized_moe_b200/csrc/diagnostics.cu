@@ -93,6 +93,10 @@ __global__ void __launch_bounds__(kDThreads) block_stats_kernel(const uint4* __r
       sum[5] += e2;
     }
   };
+  auto code_unit = [&](long long b) -> size_t {
+    if (layout != NVFP4_LAYOUT_STAGED) return (size_t)mat * blocks + b;
+    return (size_t)mat * blocks + staged_code_unit((size_t)(b / nblk), (int)(b % nblk), nblk);
+  };
   auto scale_of = [&](long long b) -> uint32_t {
     const int row = (int)(b / nblk), kb = (int)(b % nblk);
     const int srow = mat * rows + row;
@@ -107,7 +111,7 @@ __global__ void __launch_bounds__(kDThreads) block_stats_kernel(const uint4* __r
     const long long gb = (long long)mat * blocks + b, gb2 = (long long)mat * blocks + (two ? b2 : b);
     const uint4 u0 = __ldg(w + 2 * gb), u1 = __ldg(w + 2 * gb + 1);
     const uint4 v0 = __ldg(w + 2 * gb2), v1 = __ldg(w + 2 * gb2 + 1);
-    const uint2 c = __ldg(codes + gb), c2 = __ldg(codes + gb2);
+    const uint2 c = __ldg(codes + code_unit(b)), c2 = __ldg(codes + code_unit(two ? b2 : b));
     const uint32_t s = scale_of(b), s2 = scale_of(two ? b2 : b);
     account(u0, u1, c, s);
     if (two) account(v0, v1, c2, s2);
@@ -159,9 +163,10 @@ extern "C" nvfp4_status nvfp4_block_stats_compute(const void* w_bf16, const uint
              "nvfp4_block_stats_compute: a pointer argument is NULL");
   NV_REQUIRE(n_mats >= 1 && rows >= 1 && cols >= 1, NVFP4_ERR_INVALID_ARG,
              "nvfp4_block_stats_compute: n_mats=%d rows=%d cols=%d", n_mats, rows, cols);
-  NV_REQUIRE(layout == NVFP4_LAYOUT_CANONICAL || layout == NVFP4_LAYOUT_TILED, NVFP4_ERR_INVALID_ARG,
-             "nvfp4_block_stats_compute: unknown layout %d", layout);
-  NV_REQUIRE(cols % 16 == 0 && (layout == NVFP4_LAYOUT_CANONICAL || (cols % 64 == 0 && rows % 128 == 0)),
+  NV_REQUIRE(layout == NVFP4_LAYOUT_CANONICAL || layout == NVFP4_LAYOUT_TILED || layout == NVFP4_LAYOUT_STAGED,
+             NVFP4_ERR_INVALID_ARG, "nvfp4_block_stats_compute: unknown layout %d", layout);
+  NV_REQUIRE(cols % 16 == 0 && (layout == NVFP4_LAYOUT_CANONICAL || (cols % 64 == 0 && rows % 128 == 0)) &&
+                 (layout != NVFP4_LAYOUT_STAGED || cols % 256 == 0),
              NVFP4_ERR_UNSUPPORTED_SHAPE, "nvfp4_block_stats_compute: cols=%d rows=%d do not fit the layout", cols,
              rows);
   NV_REQUIRE(n_mats <= 65535, NVFP4_ERR_UNSUPPORTED_SHAPE, "nvfp4_block_stats_compute: n_mats=%d > 65535",

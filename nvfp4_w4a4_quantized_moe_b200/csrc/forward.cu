@@ -394,6 +394,7 @@ static nvfp4_status forward_impl(const moe_nvfp4_weights* W, const void* x_bf16,
   g1.a_codes = f.a_codes; g1.a_scales = f.a_scales;
   g1.b0_codes = W->gate_codes; g1.b0_scales = W->gate_scales; g1.b0_gscale = W->gate_gscale;
   g1.b1_codes = W->up_codes; g1.b1_scales = W->up_scales; g1.b1_gscale = W->up_gscale;
+  g1.b_staged = W->codes_layout == NVFP4_LAYOUT_STAGED;
   g1.act_gscale = act_gscale;
   g1.tile_expert = f.route.tile_expert; g1.num_mtiles = f.route.num_mtiles;
   g1.expert_offsets = f.offsets; g1.expert_counts = f.route.counts;
@@ -412,6 +413,7 @@ static nvfp4_status forward_impl(const moe_nvfp4_weights* W, const void* x_bf16,
   g2.rows_capacity = cap;
   g2.a_codes = f.h_codes; g2.a_scales = f.h_scales;
   g2.b0_codes = W->down_codes; g2.b0_scales = W->down_scales; g2.b0_gscale = W->down_gscale;
+  g2.b_staged = W->codes_layout == NVFP4_LAYOUT_STAGED;
   g2.act_gscale = h_gscale;
   g2.tile_expert = f.route.tile_expert; g2.num_mtiles = f.route.num_mtiles;
   g2.expert_offsets = f.offsets; g2.expert_counts = f.route.counts;

@@ -98,6 +98,11 @@ struct GemmParams {
   uint16_t* h_bf16;
   int H;
   int per_expert;       // g_act, g_h and h_amax are [E] arrays
+  // B codes in the staged layout: each 128-row group of a stage is one
+  // contiguous 16 KiB tile, fetched with a plain bulk copy instead of TMA
+  int b_staged;
+  const uint8_t* b0_codes;
+  const uint8_t* b1_codes;
   uint32_t* status;
 };
 
@@ -206,8 +211,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             bulk_load(sSFB + kSfbBytes / 2, bsf1 + sf_off, sf_bytes, &full_bar[stage]);
           }
           tma_load_2d(sA, &tmA, x, arow, &full_bar[stage]);
-          tma_load_2d(sB, &tmB0, x, brow, &full_bar[stage]);
-          if (kGateUp) tma_load_2d(sB + kBBytes / 2, &tmB1, x, brow, &full_bar[stage]);
+          if (!kBf16 && p.b_staged) {
+            // gate/up: the gate and up tiles of rows [brow, brow + 128);
+            // down: the tiles of rows [brow, brow + 128) and the next 128
+            const size_t ks = (size_t)(p.K / kBK);
+            const size_t t0 = ((size_t)(brow / kRowTile) * ks + kt) * kStagedTileBytes;
+            bulk_load(sB, p.b0_codes + t0, kStagedTileBytes, &full_bar[stage]);
+            bulk_load(sB + kBBytes / 2, kGateUp ? p.b1_codes + t0 : p.b0_codes + t0 + ks * kStagedTileBytes,
+                      kStagedTileBytes, &full_bar[stage]);
+          } else {
+            tma_load_2d(sB, &tmB0, x, brow, &full_bar[stage]);
+            if (kGateUp) tma_load_2d(sB + kBBytes / 2, &tmB1, x, brow, &full_bar[stage]);
+          }
         }
         __syncwarp();
         filled |= 1u << stage;
@@ -548,6 +563,9 @@ nvfp4_status launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t s) {
   p.h_bf16 = static_cast<uint16_t*>(a.h_bf16);
   p.H = a.H;
   p.per_expert = a.per_expert_scales ? 1 : 0;
+  p.b_staged = a.b_staged ? 1 : 0;
+  p.b0_codes = a.b0_codes;
+  p.b1_codes = a.b1_codes;
   p.status = a.status;
   const int max_tiles = a.rows_capacity / kBM * p.n_tiles;
   const int grid = std::max(1, std::min(sms, max_tiles));
@@ -609,6 +627,11 @@ static nvfp4_status check_weights(const moe_nvfp4_weights* W) {
              W->H);
   NV_REQUIRE(W->I > 0 && W->I % 128 == 0, NVFP4_ERR_UNSUPPORTED_SHAPE, "I=%d must be a positive multiple of 128",
              W->I);
+  NV_REQUIRE(W->codes_layout == NVFP4_LAYOUT_CANONICAL || W->codes_layout == NVFP4_LAYOUT_STAGED,
+             NVFP4_ERR_INVALID_ARG, "codes_layout=%d: expected NVFP4_LAYOUT_CANONICAL or NVFP4_LAYOUT_STAGED",
+             W->codes_layout);
+  NV_REQUIRE(W->codes_layout != NVFP4_LAYOUT_STAGED || W->I % 256 == 0, NVFP4_ERR_UNSUPPORTED_SHAPE,
+             "staged codes need I %% 256 == 0 (I=%d)", W->I);
   const bool any_shared = W->shared_gate || W->shared_up || W->shared_down || W->I_shared;
   NV_REQUIRE(!any_shared || (W->shared_gate && W->shared_up && W->shared_down && W->I_shared > 0 &&
                              W->I_shared % 128 == 0),
@@ -673,6 +696,7 @@ extern "C" nvfp4_status moe_nvfp4_gate_up(const moe_nvfp4_weights* W, const uint
   a.a_codes = a_codes; a.a_scales = a_scales;
   a.b0_codes = W->gate_codes; a.b0_scales = W->gate_scales; a.b0_gscale = W->gate_gscale;
   a.b1_codes = W->up_codes; a.b1_scales = W->up_scales; a.b1_gscale = W->up_gscale;
+  a.b_staged = W->codes_layout == NVFP4_LAYOUT_STAGED;
   a.act_gscale = act_gscale;
   a.tile_expert = g.tile_expert; a.num_mtiles = g.num_mtiles;
   a.expert_offsets = expert_offsets; a.expert_counts = expert_counts;
@@ -707,6 +731,7 @@ extern "C" nvfp4_status moe_nvfp4_down(const moe_nvfp4_weights* W, const uint8_t
   a.rows_capacity = rows_capacity;
   a.a_codes = h_codes; a.a_scales = h_scales;
   a.b0_codes = W->down_codes; a.b0_scales = W->down_scales; a.b0_gscale = W->down_gscale;
+  a.b_staged = W->codes_layout == NVFP4_LAYOUT_STAGED;
   a.act_gscale = h_gscale;
   a.tile_expert = g.tile_expert; a.num_mtiles = g.num_mtiles;
   a.expert_offsets = expert_offsets; a.expert_counts = expert_counts;

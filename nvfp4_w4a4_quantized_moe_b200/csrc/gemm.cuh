@@ -19,7 +19,9 @@ struct GroupedGemmArgs {
   // A operand: packed codes [rows][K/2], tiled scales
   const uint8_t* a_codes = nullptr;
   const uint8_t* a_scales = nullptr;
-  // B operands (gate and up for kEpiGateUp; down for kEpiDown)
+  // B operands (gate and up for kEpiGateUp; down for kEpiDown); b_staged:
+  // the FP4 codes are in the staged layout (NVFP4_LAYOUT_STAGED)
+  bool b_staged = false;
   const uint8_t* b0_codes = nullptr;
   const uint8_t* b0_scales = nullptr;
   const float* b0_gscale = nullptr;

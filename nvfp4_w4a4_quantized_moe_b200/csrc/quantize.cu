@@ -401,7 +401,9 @@ __global__ void __launch_bounds__(kWThreads, 1) quantize_weights_kernel(
             y[2 * i] = lo_f32(r);
             y[2 * i + 1] = hi_f32(r);
           }
-          codes[(long long)mat * blocks + c0 + j] = make_uint2(e2m1x8_hw(y), e2m1x8_hw(y + 8));
+          codes[(long long)mat * blocks +
+                (layout == NVFP4_LAYOUT_STAGED ? (long long)staged_code_unit(row, kb, nblk) : c0 + j)] =
+              make_uint2(e2m1x8_hw(y), e2m1x8_hw(y + 8));
           const int srow = mat * rows + row;
           scales[layout == NVFP4_LAYOUT_CANONICAL ? (size_t)srow * nblk + kb
                                                   : tiled_scale_offset(srow, kb, nblk >> 2)] = (uint8_t)sc;
@@ -512,6 +514,19 @@ extern "C" nvfp4_status nvfp4_quantize_act(const void* x_bf16, int rows, int col
   return NVFP4_OK;
 }
 
+// Layout and shape checks shared by both weight-quantiser entry points.
+static nvfp4_status check_weight_layout(const char* fn, int layout, int rows, int cols) {
+  NV_REQUIRE(layout == NVFP4_LAYOUT_CANONICAL || layout == NVFP4_LAYOUT_TILED || layout == NVFP4_LAYOUT_STAGED,
+             NVFP4_ERR_INVALID_ARG, "%s: unknown layout %d", fn, layout);
+  NV_REQUIRE(cols % 32 == 0, NVFP4_ERR_UNSUPPORTED_SHAPE, "%s: cols=%d must be a multiple of 32", fn, cols);
+  NV_REQUIRE(layout == NVFP4_LAYOUT_CANONICAL || (cols % 64 == 0 && rows % 128 == 0), NVFP4_ERR_UNSUPPORTED_SHAPE,
+             "%s: the tiled and staged layouts need rows %% 128 == 0 and cols %% 64 == 0 (got %d x %d)", fn, rows,
+             cols);
+  NV_REQUIRE(layout != NVFP4_LAYOUT_STAGED || cols % 256 == 0, NVFP4_ERR_UNSUPPORTED_SHAPE,
+             "%s: the staged layout needs cols %% 256 == 0 (got %d)", fn, cols);
+  return NVFP4_OK;
+}
+
 extern "C" size_t nvfp4_quantize_weights_workspace_size(int n_mats) {
   if (n_mats < 0) return 0;
   Carver c(nullptr);
@@ -528,13 +543,7 @@ extern "C" nvfp4_status nvfp4_quantize_weights(const void* w_bf16, int n_mats, i
              "nvfp4_quantize_weights: a pointer argument is NULL");
   NV_REQUIRE(n_mats >= 0 && rows >= 0 && cols > 0, NVFP4_ERR_INVALID_ARG,
              "nvfp4_quantize_weights: n_mats=%d rows=%d cols=%d", n_mats, rows, cols);
-  NV_REQUIRE(layout == NVFP4_LAYOUT_CANONICAL || layout == NVFP4_LAYOUT_TILED, NVFP4_ERR_INVALID_ARG,
-             "nvfp4_quantize_weights: unknown layout %d", layout);
-  NV_REQUIRE(cols % 32 == 0, NVFP4_ERR_UNSUPPORTED_SHAPE, "nvfp4_quantize_weights: cols=%d must be a multiple of 32",
-             cols);
-  NV_REQUIRE(layout == NVFP4_LAYOUT_CANONICAL || (cols % 64 == 0 && rows % 128 == 0), NVFP4_ERR_UNSUPPORTED_SHAPE,
-             "nvfp4_quantize_weights: the tiled layout needs rows %% 128 == 0 and cols %% 64 == 0 (got %d x %d)", rows,
-             cols);
+  NV_CHECK(check_weight_layout("nvfp4_quantize_weights", layout, rows, cols));
   NV_REQUIRE((long long)rows * cols / 16 < (1ll << 24) && n_mats < (1 << 24),
              NVFP4_ERR_UNSUPPORTED_SHAPE, "nvfp4_quantize_weights: too many elements");
   const size_t need = nvfp4_quantize_weights_workspace_size(n_mats);
@@ -606,12 +615,7 @@ extern "C" nvfp4_status nvfp4_quantize_weights_noalloc(const void* w_bf16, int n
              "nvfp4_quantize_weights_noalloc: n_mats=%d exceeds the built-in scratch limit of %d matrices per call "
              "(use nvfp4_quantize_weights with a workspace, or split the call)",
              n_mats, kStaticMaxMats);
-  NV_REQUIRE(layout == NVFP4_LAYOUT_CANONICAL || layout == NVFP4_LAYOUT_TILED, NVFP4_ERR_INVALID_ARG,
-             "nvfp4_quantize_weights_noalloc: unknown layout %d", layout);
-  NV_REQUIRE(cols % 32 == 0, NVFP4_ERR_UNSUPPORTED_SHAPE,
-             "nvfp4_quantize_weights_noalloc: cols=%d must be a multiple of 32", cols);
-  NV_REQUIRE(layout == NVFP4_LAYOUT_CANONICAL || (cols % 64 == 0 && rows % 128 == 0), NVFP4_ERR_UNSUPPORTED_SHAPE,
-             "nvfp4_quantize_weights_noalloc: the tiled layout needs rows %% 128 == 0 and cols %% 64 == 0");
+  NV_CHECK(check_weight_layout("nvfp4_quantize_weights_noalloc", layout, rows, cols));
   NV_REQUIRE((long long)rows * cols / 16 < (1ll << 24) && n_mats < (1 << 24),
              NVFP4_ERR_UNSUPPORTED_SHAPE, "nvfp4_quantize_weights_noalloc: too many elements");
   NV_REQUIRE(aligned(w_bf16, 16) && aligned(codes, 16) && aligned(scales, 4), NVFP4_ERR_INVALID_ARG,

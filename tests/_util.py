@@ -79,3 +79,30 @@ def host(t: torch.Tensor) -> np.ndarray:
     if t.dtype == torch.bfloat16:
         t = t.float()
     return t.detach().cpu().numpy()
+
+
+# --- staged weight-code layout (one contiguous 16 KiB tile per 128 rows x
+# 256 columns, 16-byte chunks swizzled by row; see the library header) --------
+
+def staged_unit_index(rows: int, cols: int) -> np.ndarray:
+    """idx[r, b] = index of the 8-byte unit that holds the codes of (row r,
+    16-element block b) of one matrix in the staged layout."""
+    nb = cols // 16
+    r = np.arange(rows)[:, None]
+    b = np.arange(nb)[None, :]
+    tile = (r // 128) * (nb // 16) + b // 16
+    chunk = (b % 16) // 2
+    return tile * 2048 + (r % 128) * 16 + (chunk ^ (r % 8)) * 2 + b % 2
+
+
+def staged_to_canonical(codes, rows: int, cols: int) -> np.ndarray:
+    """Row-major codes [rows, cols/2] of one matrix read out of its staged bytes."""
+    units = np.asarray(codes).reshape(-1, 8)
+    return units[staged_unit_index(rows, cols)].reshape(rows, cols // 2)
+
+
+def canonical_to_staged(codes, rows: int, cols: int) -> np.ndarray:
+    """The staged bytes of one matrix from its row-major codes [rows, cols/2]."""
+    out = np.empty((rows * cols // 16, 8), dtype=np.uint8)
+    out[staged_unit_index(rows, cols)] = np.asarray(codes, dtype=np.uint8).reshape(rows, cols // 16, 8)
+    return out.reshape(rows, cols // 2)

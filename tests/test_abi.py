@@ -23,7 +23,7 @@ def test_library_exports_every_declared_function():
 
 def test_abi_version_and_sizes():
     c = capi()
-    assert c.abi_version() == 3
+    assert c.abi_version() == 4
     assert c.moe_route_rows_capacity(8192, 80, 8) == 75776
     assert c.moe_route_rows_capacity(16, 80, 8) % 128 == 0
     assert c.lib.moe_nvfp4_workspace_size(16, 80, 6144, 2048, 8) > 0
@@ -41,6 +41,9 @@ def test_host_side_argument_checks():
     assert lib.nvfp4_quantize_act(fake, 4, 48, fake, 0, fake, fake, None) == 2
     assert lib.nvfp4_quantize_act(fake, 4, 64, fake, 7, fake, fake, None) == 1
     assert lib.nvfp4_quantize_weights(fake, 1, 100, 64, 1, fake, fake, fake, fake, 1 << 20, None) == 2
+    # the staged code layout needs cols % 256 == 0
+    assert lib.nvfp4_quantize_weights(fake, 1, 128, 128, 2, fake, fake, fake, fake, 1 << 20, None) == 2
+    assert lib.nvfp4_quantize_weights(fake, 1, 128, 64, 3, fake, fake, fake, fake, 1 << 20, None) == 1
     # workspace too small
     assert lib.nvfp4_quantize_weights(fake, 1, 128, 64, 1, fake, fake, fake, fake, 8, None) == 5
     # routing shapes
@@ -52,4 +55,11 @@ def test_host_side_argument_checks():
     W = c.MoeWeightsStruct(8, 192, 128, 2, 2.5, *([fake] * 11))
     assert lib.moe_nvfp4_forward(ctypes.byref(W), fake, 4, fake, fake, None, fake, None, fake, 1 << 30, None) == 2
     W = c.MoeWeightsStruct(8, 256, 128, 2, 2.5, *([fake] * 11))
+    assert lib.moe_nvfp4_forward(ctypes.byref(W), fake, 4, fake, fake, None, fake, None, fake, 16, None) == 5
+    # codes layout: only row-major or staged, and staged needs I % 256 == 0
+    W.codes_layout = 1
+    assert lib.moe_nvfp4_forward(ctypes.byref(W), fake, 4, fake, fake, None, fake, None, fake, 1 << 30, None) == 1
+    W.codes_layout = 2
+    assert lib.moe_nvfp4_forward(ctypes.byref(W), fake, 4, fake, fake, None, fake, None, fake, 1 << 30, None) == 2
+    W = c.MoeWeightsStruct(8, 256, 256, 2, 2.5, *([fake] * 11), None, None, None, 0, 2)
     assert lib.moe_nvfp4_forward(ctypes.byref(W), fake, 4, fake, fake, None, fake, None, fake, 16, None) == 5

@@ -8,7 +8,7 @@ import numpy as np
 import pytest
 import torch
 
-from _util import capi, host, rel_l2, require_cuda, tiled_rows
+from _util import capi, host, rel_l2, require_cuda, staged_to_canonical, tiled_rows
 from nvfp4_w4a4_quantized_moe_b200 import workloads
 from oracle import moe, nvfp4
 
@@ -99,6 +99,32 @@ def test_forward_matches_oracle(name):
     assert flips <= 0.001 * total, f"{flips}/{total} requantised codes differ"
     err = rel_l2(host(out)[same], ref["out"][same])
     assert err <= 1e-2, err
+
+
+def test_staged_and_row_major_codes_give_identical_layers():
+    """The staged code layout only moves bytes: the quantiser's staged codes
+    read back as its row-major codes, and the layer's output is bit-identical
+    with either (gate/up and down both fetch staged tiles)."""
+    require_cuda()
+    cfg = CASES["mid_skewed"]
+    c = capi()
+    x = workloads.hidden_states(cfg, device="cpu").cuda()
+    wg, bias, off = workloads.router_params(cfg, device="cpu")
+    gate, up, down = (t.cuda() for t in workloads.stacked_expert_weights(cfg, device="cpu"))
+    Ws = c.MoeWeights.quantize(gate, up, down, wg.cuda(), bias.cuda(), cfg.k, cfg.rsf, codes_layout="staged")
+    Wc = c.MoeWeights.quantize(gate, up, down, wg.cuda(), bias.cuda(), cfg.k, cfg.rsf, codes_layout="canonical")
+    assert Ws.codes_layout == c.LAYOUT_STAGED and Wc.codes_layout == c.LAYOUT_CANONICAL
+    for s, r, (rows, cols) in ((Ws.gate_codes, Wc.gate_codes, (cfg.I, cfg.H)), (Ws.up_codes, Wc.up_codes, (cfg.I, cfg.H)),
+                               (Ws.down_codes, Wc.down_codes, (cfg.H, cfg.I))):
+        hs, hr = host(s), host(r)
+        for e in (0, cfg.E - 1):
+            np.testing.assert_array_equal(staged_to_canonical(hs[e], rows, cols), hr[e])
+    g1 = torch.tensor([float(x.float().abs().max()) / 2688.0]).cuda()
+    g2 = torch.tensor([0.002]).cuda()
+    off_d = off.cuda() if off is not None else None
+    os_ = c.moe_nvfp4_forward(Ws, x, g1, g2, logit_offset=off_d)
+    oc = c.moe_nvfp4_forward(Wc, x, g1, g2, logit_offset=off_d)
+    assert torch.equal(os_, oc)
 
 
 def test_forward_status_word_is_clear_and_repeatable():

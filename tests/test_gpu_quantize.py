@@ -6,7 +6,7 @@ import numpy as np
 import pytest
 import torch
 
-from _util import capi, host, require_cuda, tiled_rows, tiled_to_canonical
+from _util import capi, host, require_cuda, staged_to_canonical, tiled_rows, tiled_to_canonical
 from nvfp4_w4a4_quantized_moe_b200 import workloads
 from oracle import nvfp4
 
@@ -59,7 +59,7 @@ def test_activation_quantiser_hand_examples():
         assert host(scales)[0, : len(case["scales_hex"][0]) // 2].tobytes().hex() == case["scales_hex"][0]
 
 
-@pytest.mark.parametrize("layout", ["canonical", "tiled"])
+@pytest.mark.parametrize("layout", ["canonical", "tiled", "staged"])
 def test_weight_quantiser_matches_oracle(layout):
     require_cuda()
     c = capi()
@@ -72,8 +72,9 @@ def test_weight_quantiser_matches_oracle(layout):
     for m in range(4):
         rc, rs, rg = nvfp4.quantize_weight(wf[m])
         assert host(g)[m].view(np.uint32) == np.float32(rg).view(np.uint32), m
-        np.testing.assert_array_equal(host(codes)[m], rc)
-        if layout == "tiled":
+        got = staged_to_canonical(host(codes)[m], 256, 512) if layout == "staged" else host(codes)[m]
+        np.testing.assert_array_equal(got, rc)
+        if layout != "canonical":
             np.testing.assert_array_equal(tiled_to_canonical(sc, 4 * 256, 512)[m * 256:(m + 1) * 256], rs)
         else:
             np.testing.assert_array_equal(sc[m], rs)
@@ -97,15 +98,15 @@ def test_weight_quantiser_tiny_layer():
 
 def test_weight_quantiser_full_layer_sampled():
     """The offline quantiser on the full 80-expert layer (3.0e9 parameters),
-    as the benchmark runs it: every global scale checked, and 16 rows of six
-    matrices compared code by code."""
+    as the benchmark runs it (staged codes, tiled scales): every global scale
+    checked, and 16 rows of six matrices compared code by code."""
     require_cuda()
     c = capi()
     cfg = workloads.CONFIGS["quantiser"]
     gate, up, down = workloads.stacked_expert_weights(cfg, device="cuda")
     rng = np.random.default_rng(0)
     for name, w in (("gate", gate), ("up", up), ("down", down)):
-        codes, scales, g = c.nvfp4_quantize_weights(w, "tiled")
+        codes, scales, g = c.nvfp4_quantize_weights(w, "staged")
         torch.cuda.synchronize()
         n, rows, cols = w.shape
         amax = w.abs().amax(dim=(1, 2)).float().cpu().numpy()       # exact (a max of bf16 values)
@@ -114,7 +115,7 @@ def test_weight_quantiser_full_layer_sampled():
         for m in rng.choice(n, 2, replace=False):
             r = np.sort(rng.choice(rows, 16, replace=False))
             rc, rs = nvfp4.quantize(w[m, r].float().cpu().numpy(), ref_g[m])
-            np.testing.assert_array_equal(host(codes[m, r]), rc)
+            np.testing.assert_array_equal(staged_to_canonical(host(codes[m]), rows, cols)[r], rc)
             sc = tiled_rows(host(scales), m * rows + r, cols)
             np.testing.assert_array_equal(sc, rs)
         del codes, scales

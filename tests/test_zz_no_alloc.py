@@ -25,7 +25,7 @@ def _weights(seed, n, rows, cols):
     return w.to(torch.bfloat16).cuda()
 
 
-@pytest.mark.parametrize("layout", ["tiled", "canonical"])
+@pytest.mark.parametrize("layout", ["tiled", "canonical", "staged"])
 def test_noalloc_matches_workspace_form_on_consecutive_calls(layout):
     require_cuda()
     c = capi()
