@@ -14,9 +14,11 @@
 //            so one tile yields 128 columns of h = silu(gate) * up, which the
 //            epilogue re-quantises to NVFP4 (16-column blocks stay in-thread).
 //   down:    256 output columns, scaled by g2 * g_down[e] * w(row).
-// Warp roles (320 threads): warp 0 issues TMA loads, warp 1 owns tensor memory
-// and issues MMAs, warps 2..9 drain the accumulator (warp w reads TMEM lanes
-// 32*(w%4).., columns split in two halves).  The grid is persistent: one CTA
+// Warp roles (320 threads): warp 0 issues the loads (TMA for A and row-major
+// weight codes, plain bulk copies for staged weight codes and the scale
+// atoms), warp 1 owns tensor memory and issues MMAs, warps 2..9 drain the
+// accumulator (warp w reads TMEM lanes 32*(w%4).., columns split in two
+// halves).  The grid is persistent: one CTA
 // per SM walks the (m-tile, n-tile) list, whose length is read on the device.
 // Every wait is bounded in time; a wait that gives up sets the workspace
 // status word and the CTA winds down after its outstanding copies land.
@@ -115,7 +117,8 @@ NVDEV float silu(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 
 template <int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
-    grouped_fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+    grouped_fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA32,
+                            const __grid_constant__ CUtensorMap tmB0,
                             const __grid_constant__ CUtensorMap tmB1, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -146,6 +149,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmA);
+    prefetch_tmap(&tmA32);
     prefetch_tmap(&tmB0);
     if (kGateUp) prefetch_tmap(&tmB1);
   }
@@ -186,6 +190,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint8_t* bsf1 = kBf16 ? nullptr
                                   : (kGateUp ? p.b1_sf + (size_t)(brow / kRowTile) * tile_sf_bytes
                                              : bsf0 + tile_sf_bytes);
+      // A rows to load: the tile's data rows rounded up to 32-row boxes (a
+      // decode tile holds a handful of tokens).  Rows past them keep stale
+      // shared memory; they only feed accumulator rows the epilogue never
+      // stores.
+      int a_boxes = 4;
+      if (p.expert_counts) {
+        const int real = p.expert_counts[e] - (arow - p.expert_offsets[e]);
+        a_boxes = min(4, max(1, (real + 31) / 32));
+      }
+      const uint32_t a_bytes = (uint32_t)a_boxes * (kABytes / 4);
       for (int kt = 0; kt < KT; ++kt) {
         ok = __all_sync(0xffffffffu, mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag));
         if (!ok) {
@@ -198,11 +212,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           // x in tensor-map elements: 128 bytes of K per stage either way
           const int x = kt * (kBf16 ? 64 : kBKBytes);
           if (kBf16) {
-            mbar_arrive_expect_tx(&full_bar[stage], kABytes + kBBytes);
+            mbar_arrive_expect_tx(&full_bar[stage], a_bytes + kBBytes);
           } else {
             const int katoms = min(4, (p.K - kt * kBK) / 64);
             const uint32_t sf_bytes = (uint32_t)katoms * kAtomBytes;
-            mbar_arrive_expect_tx(&full_bar[stage], kABytes + kBBytes + 3 * sf_bytes);
+            mbar_arrive_expect_tx(&full_bar[stage], a_bytes + kBBytes + 3 * sf_bytes);
             uint8_t* sSFA = sB + kBBytes;
             uint8_t* sSFB = sSFA + kSfaBytes;
             const size_t sf_off = (size_t)kt * 4 * kAtomBytes;
@@ -210,7 +224,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             bulk_load(sSFB, bsf0 + sf_off, sf_bytes, &full_bar[stage]);
             bulk_load(sSFB + kSfbBytes / 2, bsf1 + sf_off, sf_bytes, &full_bar[stage]);
           }
-          tma_load_2d(sA, &tmA, x, arow, &full_bar[stage]);
+          if (a_boxes == 4) {
+            tma_load_2d(sA, &tmA, x, arow, &full_bar[stage]);
+          } else {
+            for (int i = 0; i < a_boxes; ++i)
+              tma_load_2d(sA + i * (kABytes / 4), &tmA32, x, arow + 32 * i, &full_bar[stage]);
+          }
           if (!kBf16 && p.b_staged) {
             // gate/up: the gate and up tiles of rows [brow, brow + 128);
             // down: the tiles of rows [brow, brow + 128) and the next 128
@@ -269,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       uint32_t accumulate = 0;
       for (int kt = 0; kt < KT; ++kt) {
-        // TMA wrote this stage through the async proxy that the MMAs read
+        // the copies wrote this stage through the async proxy that the MMAs read
         // through; the completed barrier phase is all the ordering needed
         ok = __all_sync(0xffffffffu, mbar_wait(&full_bar[stage], phase, abort_flag));
         if (!ok) {
@@ -526,9 +545,10 @@ nvfp4_status launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t s) {
   const uint64_t inner = bf ? (uint64_t)K : (uint64_t)K / 2;       // elements per row
   const uint64_t pitch = bf ? (uint64_t)K * 2 : (uint64_t)K / 2;   // bytes per row
   const uint32_t box = bf ? 64 : kBKBytes;
-  CUtensorMap tmA, tmB0, tmB1;
-  NV_CHECK(make_tmap_2d(&tmA, a.a_codes, dt, inner, (uint64_t)(a.a_rows > 0 ? a.a_rows : a.rows_capacity), pitch, box,
-                        kBM));
+  CUtensorMap tmA, tmA32, tmB0, tmB1;
+  const uint64_t a_rows = (uint64_t)(a.a_rows > 0 ? a.a_rows : a.rows_capacity);
+  NV_CHECK(make_tmap_2d(&tmA, a.a_codes, dt, inner, a_rows, pitch, box, kBM));
+  NV_CHECK(make_tmap_2d(&tmA32, a.a_codes, dt, inner, a_rows, pitch, box, 32));
   NV_CHECK(make_tmap_2d(&tmB0, a.b0_codes, dt, inner, (uint64_t)a.E * Nw, pitch, box, gu ? 128 : kBN));
   if (gu) {
     NV_CHECK(make_tmap_2d(&tmB1, a.b1_codes, dt, inner, (uint64_t)a.E * Nw, pitch, box, 128));
@@ -573,21 +593,21 @@ nvfp4_status launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t s) {
     case kEpiGateUp:
       NV_CHECK(set_smem_attr((const void*)grouped_fp4_gemm_kernel<kEpiGateUp>, 0, smem_bytes_of<kEpiGateUp>()));
       return launch_dependent("grouped_fp4_gemm_kernel<gate_up>", grouped_fp4_gemm_kernel<kEpiGateUp>, dim3(grid),
-                              dim3(kThreads), smem_bytes_of<kEpiGateUp>(), s, tmA, tmB0, tmB1, p);
+                              dim3(kThreads), smem_bytes_of<kEpiGateUp>(), s, tmA, tmA32, tmB0, tmB1, p);
     case kEpiDown:
       NV_CHECK(set_smem_attr((const void*)grouped_fp4_gemm_kernel<kEpiDown>, 1, smem_bytes_of<kEpiDown>()));
       return launch_dependent("grouped_fp4_gemm_kernel<down>", grouped_fp4_gemm_kernel<kEpiDown>, dim3(grid),
-                              dim3(kThreads), smem_bytes_of<kEpiDown>(), s, tmA, tmB0, tmB1, p);
+                              dim3(kThreads), smem_bytes_of<kEpiDown>(), s, tmA, tmA32, tmB0, tmB1, p);
     case kEpiSharedGateUp:
       NV_CHECK(set_smem_attr((const void*)grouped_fp4_gemm_kernel<kEpiSharedGateUp>, 2,
                              smem_bytes_of<kEpiSharedGateUp>()));
       return launch_dependent("grouped_fp4_gemm_kernel<shared_gate_up>", grouped_fp4_gemm_kernel<kEpiSharedGateUp>,
-                              dim3(grid), dim3(kThreads), smem_bytes_of<kEpiSharedGateUp>(), s, tmA, tmB0, tmB1, p);
+                              dim3(grid), dim3(kThreads), smem_bytes_of<kEpiSharedGateUp>(), s, tmA, tmA32, tmB0, tmB1, p);
     default:
       NV_CHECK(set_smem_attr((const void*)grouped_fp4_gemm_kernel<kEpiSharedDown>, 3,
                              smem_bytes_of<kEpiSharedDown>()));
       return launch_dependent("grouped_fp4_gemm_kernel<shared_down>", grouped_fp4_gemm_kernel<kEpiSharedDown>,
-                              dim3(grid), dim3(kThreads), smem_bytes_of<kEpiSharedDown>(), s, tmA, tmB0, tmB1, p);
+                              dim3(grid), dim3(kThreads), smem_bytes_of<kEpiSharedDown>(), s, tmA, tmA32, tmB0, tmB1, p);
   }
 }
 

@@ -5,7 +5,7 @@ import numpy as np
 import pytest
 import torch
 
-from _util import canonical_to_tiled, capi, host, rel_l2, require_cuda, tiled_to_canonical
+from _util import canonical_to_staged, canonical_to_tiled, capi, host, rel_l2, require_cuda, tiled_to_canonical
 from nvfp4_w4a4_quantized_moe_b200 import workloads
 from oracle import moe, nvfp4
 
@@ -45,13 +45,21 @@ class Problem:
         self.g1 = F32(0.013)
         self.g2 = F32(0.021)
 
-    def weights(self, c):
+    def weights(self, c, layout="canonical"):
+        """The weights on the device; with layout "staged" the codes are
+        rearranged into the staged layout (scales are tiled either way)."""
         cu = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()  # noqa: E731
         tiled = lambda s: cu(canonical_to_tiled(s.reshape(-1, s.shape[-1])))  # noqa: E731
+
+        def codes(a):
+            if layout != "staged":
+                return cu(a)
+            return cu(np.stack([canonical_to_staged(m, m.shape[0], 2 * m.shape[1]) for m in a]))
         return c.MoeWeights(self.E, self.H, self.I, 1, 1.0, torch.zeros((self.E, self.H), dtype=torch.bfloat16).cuda(),
-                            torch.zeros(self.E).cuda(), cu(self.gate[0]), tiled(self.gate[1]), cu(self.g["gate"]),
-                            cu(self.up[0]), tiled(self.up[1]), cu(self.g["up"]), cu(self.down[0]),
-                            tiled(self.down[1]), cu(self.g["down"]))
+                            torch.zeros(self.E).cuda(), codes(self.gate[0]), tiled(self.gate[1]), cu(self.g["gate"]),
+                            codes(self.up[0]), tiled(self.up[1]), cu(self.g["up"]), codes(self.down[0]),
+                            tiled(self.down[1]), cu(self.g["down"]),
+                            codes_layout=c.LAYOUT_STAGED if layout == "staged" else c.LAYOUT_CANONICAL)
 
     def segments(self):
         for e in range(self.E):
@@ -73,12 +81,23 @@ PROBLEMS = {
 }
 
 
-@pytest.mark.parametrize("name", list(PROBLEMS))
-def test_gate_up_matches_oracle(name):
+def _layout_params():
+    """(problem, codes layout) pairs: every problem with row-major codes, and
+    with staged codes where H and I are multiples of 256."""
+    out = []
+    for n, p in PROBLEMS.items():
+        out.append((n, "canonical"))
+        if p["H"] % 256 == 0 and p["I"] % 256 == 0:
+            out.append((n, "staged"))
+    return out
+
+
+@pytest.mark.parametrize("name,layout", _layout_params())
+def test_gate_up_matches_oracle(name, layout):
     require_cuda()
     c = capi()
     P = Problem(**PROBLEMS[name])
-    W = P.weights(c)
+    W = P.weights(c, layout)
     cu = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()  # noqa: E731
     res = c.moe_nvfp4_gate_up(W, cu(P.a_codes), cu(canonical_to_tiled(P.a_scales)), cu(P.offsets), cu(P.counts),
                               cu(np.array([P.g1])), cu(np.array([P.g2])), want_h=True, want_amax=True)
@@ -123,13 +142,13 @@ def _diagnose_down(P, y, e, r0, n, weighted):
     return "\n".join(out)
 
 
-@pytest.mark.parametrize("name", list(PROBLEMS))
+@pytest.mark.parametrize("name,layout", _layout_params())
 @pytest.mark.parametrize("weighted", [False, True])
-def test_down_matches_oracle(name, weighted):
+def test_down_matches_oracle(name, layout, weighted):
     require_cuda()
     c = capi()
     P = Problem(**PROBLEMS[name])
-    W = P.weights(c)
+    W = P.weights(c, layout)
     cu = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()  # noqa: E731
     rw = P.row_w if weighted else np.ones_like(P.row_w)
     res = c.moe_nvfp4_down(W, cu(P.h_codes), cu(canonical_to_tiled(P.h_scales)), cu(P.offsets), cu(P.counts),
