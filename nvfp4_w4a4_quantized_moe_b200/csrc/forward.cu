@@ -200,6 +200,7 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const uint4* _
                                                                   int k, uint4* __restrict__ out) {
   __shared__ int32_t rows[16];
   griddep_wait();
+  griddep_launch();
   const int t = blockIdx.x;
   if (threadIdx.x < k) rows[threadIdx.x] = inv_perm[(size_t)t * k + threadIdx.x];
   __syncthreads();
@@ -346,7 +347,12 @@ static nvfp4_status forward_impl(const moe_nvfp4_weights* W, const void* x_bf16,
   ForwardScratch f = carve_forward(c, T, E, H, I, k, I_s);
   const int cap = route_rows_capacity(T, E, k);
 
-  NV_CHECK(check_cuda(cudaMemsetAsync(f.route.status, 0, sizeof(uint32_t), s), "clear status word"));
+  // The status word is cleared by the first kernel when that is the router
+  // GEMM (a memset would stop it from starting early behind the previous
+  // kernel on the stream), else by a memset.
+  const bool router_first = !shared && !(mode & kActDynamic);
+  if (!router_first)
+    NV_CHECK(check_cuda(cudaMemsetAsync(f.route.status, 0, sizeof(uint32_t), s), "clear status word"));
   NV_CHECK(mark(dbg, 0, s));
   if (shared) {
     dense_tiles_kernel<<<1, 128, 0, s>>>(T, f.sh_tiles, f.sh_ntiles, f.sh_offsets, f.sh_counts);
@@ -368,6 +374,7 @@ static nvfp4_status forward_impl(const moe_nvfp4_weights* W, const void* x_bf16,
   ra.logits = f.logits;
   ra.topk_idx = f.topk_idx; ra.topk_w = f.topk_w; ra.expert_offsets = f.offsets;
   ra.perm = f.perm; ra.inv_perm = f.inv_perm;
+  ra.clear_status = router_first;
   NV_CHECK(launch_route(ra, f.route, s));
   NV_CHECK(mark(dbg, 1, s));
 

@@ -25,7 +25,7 @@ constexpr int kRThreads = 192;
 constexpr int kRAbytes = kRBM * kRBK * 2;     // 16 KiB
 
 struct RouterGemmParams {
-  int T, E, H, n_mma, kt_per_split, splits;
+  int T, E, H, n_mma, kt_per_split, splits, clear_status;
   float* partial;
   uint32_t* status;
 };
@@ -88,6 +88,9 @@ __global__ void __launch_bounds__(kRThreads, 1)
   const uint32_t tmem = tmem_base_s;
   griddep_wait();
   griddep_launch();
+  // first kernel of a call: the status word is cleared here, after the
+  // stream's previous work, and before any wait of this call can give up
+  if (p.clear_status && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *p.status = 0u;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -563,14 +566,16 @@ nvfp4_status launch_route(const RouteArgs& a, const RouteScratch& r, cudaStream_
     p.T = a.T; p.E = a.E; p.H = a.H; p.n_mma = n_mma;
     p.kt_per_split = (a.H / kRBK + splits - 1) / splits;
     p.splits = splits;
+    p.clear_status = a.clear_status ? 1 : 0;
     p.partial = r.partial;
     p.status = r.status;
     const int smem = router_smem_bytes(a.E);
     NV_CHECK(check_cuda(cudaFuncSetAttribute(router_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
                         "cudaFuncSetAttribute"));
     dim3 grid((a.T + kRBM - 1) / kRBM, splits);
-    router_gemm_kernel<<<grid, kRThreads, smem, s>>>(tmX, tmW, p);
-    NV_CHECK(check_launch("router_gemm_kernel"));
+    // a programmatic dependent too: its setup overlaps the previous kernel on
+    // the stream, and it waits for that kernel before reading x
+    NV_CHECK(launch_dependent("router_gemm_kernel", router_gemm_kernel, grid, dim3(kRThreads), smem, s, tmX, tmW, p));
   }
   if (a.T <= kSmallT) {
     return launch_dependent("route_small_kernel", route_small_kernel, dim3(1), dim3(kSmallThreads), 0, s,

@@ -18,6 +18,9 @@ struct RouteArgs {
   int32_t* expert_offsets = nullptr;    // [E+1]
   int32_t* perm = nullptr;              // [capacity]
   int32_t* inv_perm = nullptr;          // [T][k]
+  // the router GEMM clears the status word once the previous work on the
+  // stream has finished (the caller then issues no memset before it)
+  bool clear_status = false;
 };
 
 struct RouteScratch {

@@ -137,3 +137,21 @@ def test_forward_status_word_is_clear_and_repeatable():
     o2 = c.moe_nvfp4_forward(W, x.cuda(), g, g, workspace=ws)
     c.nvfp4_workspace_status(ws)
     assert torch.equal(o1, o2)        # deterministic: no atomics in the value path
+
+
+@pytest.mark.parametrize("mode", ["tensor", "dynamic"])
+def test_each_call_clears_the_status_word(mode):
+    """A call starts by clearing the workspace's status word: with the
+    tensor-wide scale the router kernel does it (no memset ahead of it), in
+    the dynamic mode a memset does.  A stale non-zero word from an earlier
+    call must not survive a successful one."""
+    require_cuda()
+    cfg = CASES["mid_skewed"]
+    c, x, wg, bias, off, W, q = _setup(cfg)
+    ws = torch.empty(c.moe_nvfp4_workspace_size(cfg.T, cfg.E, cfg.H, cfg.I, cfg.k), dtype=torch.uint8, device="cuda")
+    g = torch.tensor([0.01]).cuda() if mode == "tensor" else torch.zeros(1).cuda()
+    for _ in range(2):
+        ws[:4].view(torch.int32).fill_(4)          # NVFP4_ERR_TIMEOUT left behind
+        c.moe_nvfp4_forward(W, x.cuda(), g, torch.tensor([0.01]).cuda(), workspace=ws, act_scale_mode=mode,
+                            logit_offset=off.cuda() if off is not None else None)
+        c.nvfp4_workspace_status(ws)               # raises on a non-zero word
