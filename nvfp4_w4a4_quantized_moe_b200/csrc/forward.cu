@@ -192,13 +192,16 @@ __global__ void __launch_bounds__(256) expert_amax_kernel(const int32_t* __restr
 // blockDim.x (+ threadIdx.x): a small batch spreads a row over several
 // blocks, a large one keeps whole rows in one block for long contiguous
 // reads.  A thread issues all k row loads of a column group before adding.
+// KMAX bounds k at compile time: the common k <= 8 keeps half the registers
+// of k <= 16, so twice the blocks (and loads in flight) fit on an SM.
 constexpr int kCombineThreads = 256;
 
+template <int KMAX>
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const uint4* __restrict__ y,
                                                                   const uint4* __restrict__ y_shared,
                                                                   const int32_t* __restrict__ inv_perm, int T, int H,
                                                                   int k, uint4* __restrict__ out) {
-  __shared__ int32_t rows[16];
+  __shared__ int32_t rows[KMAX];
   griddep_wait();
   griddep_launch();
   const int t = blockIdx.x;
@@ -206,14 +209,14 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const uint4* _
   __syncthreads();
   const int vpr = H / 8;
   for (int c = blockIdx.y * blockDim.x + threadIdx.x; c < vpr; c += gridDim.y * blockDim.x) {
-    uint4 v[16];
+    uint4 v[KMAX];
 #pragma unroll
-    for (int j = 0; j < 16; ++j)
+    for (int j = 0; j < KMAX; ++j)
       if (j < k) v[j] = __ldg(y + (size_t)rows[j] * vpr + c);
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     if (y_shared) unpack_bf16x8(__ldg(y_shared + (size_t)t * vpr + c), acc);   // the shared expert's row first
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
+    for (int j = 0; j < KMAX; ++j) {
       if (j < k) {
         float f[8];
         unpack_bf16x8(v[j], f);
@@ -465,8 +468,8 @@ static nvfp4_status forward_impl(const moe_nvfp4_weights* W, const void* x_bf16,
   // 8: combine
   // below about two waves of whole-row blocks, split rows across blocks
   const int row_blocks = T >= 2 * sms ? 1 : (H / 8 + kCombineThreads - 1) / kCombineThreads;
-  NV_CHECK(launch_dependent("combine_kernel", combine_kernel, dim3(T, row_blocks), dim3(kCombineThreads), 0, s,
-                            reinterpret_cast<const uint4*>(f.y),
+  NV_CHECK(launch_dependent("combine_kernel", k <= 8 ? combine_kernel<8> : combine_kernel<16>, dim3(T, row_blocks),
+                            dim3(kCombineThreads), 0, s, reinterpret_cast<const uint4*>(f.y),
                             shared ? reinterpret_cast<const uint4*>(f.sh_y) : (const uint4*)nullptr,
                             (const int32_t*)f.inv_perm, T, H, k, static_cast<uint4*>(out_bf16)));
   NV_CHECK(mark(dbg, 5, s));

@@ -20,6 +20,8 @@ CASES = {
     "mid_skewed": workloads.LayerConfig("mid", T=300, H=1024, I=512, E=16, k=4, x_outlier_p=0.001,
                                         logit_offset_std=0.5),
     "ragged_small": workloads.LayerConfig("rs", T=3, H=512, I=256, E=6, k=3),
+    # k > 8 takes the combine kernel's wide variant
+    "wide_k": workloads.LayerConfig("wk", T=40, H=512, I=256, E=12, k=10),
 }
 
 
@@ -155,3 +157,34 @@ def test_each_call_clears_the_status_word(mode):
         c.moe_nvfp4_forward(W, x.cuda(), g, torch.tensor([0.01]).cuda(), workspace=ws, act_scale_mode=mode,
                             logit_offset=off.cuda() if off is not None else None)
         c.nvfp4_workspace_status(ws)               # raises on a non-zero word
+
+
+@pytest.mark.parametrize("name", ["tiny", "mid_skewed"])
+def test_forward_replays_from_a_cuda_graph(name):
+    """The forward queues kernels only (no allocation, no host sync, every
+    launch a programmatic dependent), so a serving loop can capture it once
+    and replay it: the replayed output is bit-identical to the eager one."""
+    require_cuda()
+    cfg = CASES[name]
+    c, x, wg, bias, off, W, q = _setup(cfg)
+    xd = x.cuda()
+    off_d = off.cuda() if off is not None else None
+    g1 = torch.tensor([float(xd.float().abs().max()) / 2688.0]).cuda()
+    g2 = torch.tensor([0.002]).cuda()
+    ws = torch.empty(c.moe_nvfp4_workspace_size(cfg.T, cfg.E, cfg.H, cfg.I, cfg.k), dtype=torch.uint8, device="cuda")
+    out = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16, device="cuda")
+    ref = c.moe_nvfp4_forward(W, xd, g1, g2, logit_offset=off_d, workspace=ws).clone()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        c.moe_nvfp4_forward(W, xd, g1, g2, logit_offset=off_d, out=out, workspace=ws)
+    torch.cuda.current_stream().wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        c.moe_nvfp4_forward(W, xd, g1, g2, logit_offset=off_d, out=out, workspace=ws)
+    for _ in range(2):
+        out.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref)
+    c.nvfp4_workspace_status(ws)
