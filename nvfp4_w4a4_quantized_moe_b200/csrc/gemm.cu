@@ -357,13 +357,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int e = min(max(p.tile_expert[mt], 0), p.E - 1);
       const int grow = mt * kBM + row_in_tile;
       const bool real = p.expert_counts ? (grow - p.expert_offsets[e] < p.expert_counts[e]) : true;
+      // the tile's scalars are loaded before the accumulator is ready, so that
+      // no global load sits between the accumulator-full wait and the hand-back
+      const int se = p.per_expert ? e : 0;                  // index of this tile's scales
+      const float g_act = kBf16 ? 1.0f : p.g_act[se];
+      const float g_b0 = kBf16 ? 1.0f : p.g_b0[e];
+      const float g_b1 = kBf16 || !kGateUp ? 1.0f : p.g_b1[e];
+      const float g_h = EPI == kEpiGateUp ? p.g_h[se] : 1.0f;
+      const float w_row = EPI == kEpiDown && p.row_w ? p.row_w[grow] : 1.0f;
       if (!mbar_wait(&acc_full_bar, acc_phase, abort_flag)) {
         give_up(p.status, abort_flag);
         break;
       }
       tc_fence_after();
-      const int se = p.per_expert ? e : 0;                  // index of this tile's scales
-      const float g_act = kBf16 ? 1.0f : p.g_act[se];
       if (EPI == kEpiSharedGateUp) {
         // bf16 operands, no global scales: h = silu(gate) * up, stored bf16
         uint32_t rg[64], ru[64];
@@ -390,8 +396,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       } else if (EPI == kEpiGateUp) {
-        const float sg = __fmul_rn(g_act, p.g_b0[e]);
-        const float su = __fmul_rn(g_act, p.g_b1[e]);
+        const float sg = __fmul_rn(g_act, g_b0);
+        const float su = __fmul_rn(g_act, g_b1);
         // drain this thread's 64 gate and 64 up columns, then hand the
         // accumulator back before any arithmetic
         uint32_t rg[64], ru[64];
@@ -414,7 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float up = __fmul_rn(__uint_as_float(ru[i]), su);
             h[i] = __fmul_rn(silu(gate), up);
           }
-          const float g2 = p.g_h[se];
+          const float g2 = g_h;
           const float d2 = __fmul_rn(6.0f, g2);
           uint2 c0, c1, c2, c3;
           const uint32_t s0 = quant_block16(h, g2, d2, c0);
@@ -441,8 +447,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         cdst[1] = cw1;
         *reinterpret_cast<uint32_t*>(p.h_sf + tiled_scale_offset(grow, hcol0 / kQBlock, p.I / 64)) = sw;
       } else {
-        const float scale =
-            kBf16 ? 1.0f : __fmul_rn(__fmul_rn(g_act, p.g_b0[e]), p.row_w ? p.row_w[grow] : 1.0f);
+        const float scale = kBf16 ? 1.0f : __fmul_rn(__fmul_rn(g_act, g_b0), w_row);
         const int col0 = nt * kBN + half * 128;
         // drain this thread's 128 columns, then hand the accumulator back
         uint32_t r[128];
