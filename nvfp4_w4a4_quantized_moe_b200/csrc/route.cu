@@ -2,6 +2,8 @@
 // section "Pruning Setup", "Routing behavior": renormalised sigmoid routing,
 // sigmoid-and-bias selection, routed_scaling_factor; the router stays BF16 per
 // the NVFP4 model card's "Quantization Setup").
+#include <mutex>
+
 #include "common.cuh"
 #include "host.cuh"
 #include "route.cuh"
@@ -214,15 +216,64 @@ NVDEV float token_logit(const float* __restrict__ src, int splits, const float* 
   return l;
 }
 
+// Score of one (token, expert) logit: sigma, and the selection key of
+// sigma + bias mapped to an unsigned integer in the same order (sign bit
+// flipped for non-negative values, all bits for negative ones; sigma > 0, so
+// the sum is never -0).
+NVDEV void expert_score(float l, float b, float& sig, uint32_t& key) {
+  sig = sigmoid_fixed(l);
+  const uint32_t u = __float_as_uint(__fadd_rn(sig, b));
+  key = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// The k selection rounds of one token by one warp, from each lane's scores
+// of experts lane, lane+32, ... (key 0 for an absent expert).  Each round is
+// a warp max of the keys, then a warp min of the expert ids that reach it:
+// the largest score, ties to the lower expert.  Lane j < k returns slot j's
+// expert and weight (sigma / sum of the selected sigmas, times rsf; the sum
+// in slot order).
+NVDEV void select_topk(const float* sig, uint32_t* key, int k, float rsf, int lane, int& out_idx, float& out_w) {
+  float sum = 0.0f, my_sig = 0.0f;
+  int my_idx = 0;
+  for (int j = 0; j < k; ++j) {
+    uint32_t bk = 0u, be = 0xffffffffu;
+#pragma unroll
+    for (int i = 0; i < kMaxE / 32; ++i)       // ascending i: a tie keeps the lower expert
+      if (key[i] > bk) {
+        bk = key[i];
+        be = (uint32_t)(lane + 32 * i);
+      }
+    const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
+    const int win = (int)__reduce_min_sync(0xffffffffu, bk == m ? be : 0xffffffffu);
+    // the owner lane marks the winner and broadcasts its sigma
+    float s_own = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kMaxE / 32; ++i)
+      if (lane + 32 * i == win) {
+        s_own = sig[i];
+        key[i] = 0u;
+      }
+    const float s_sel = __shfl_sync(0xffffffffu, s_own, win & 31);
+    sum = __fadd_rn(sum, s_sel);
+    if (lane == j) {
+      my_sig = s_sel;
+      my_idx = win;
+    }
+  }
+  out_idx = my_idx;
+  out_w = __fmul_rn(__fdiv_rn(my_sig, sum), rsf);
+}
+
 // Top-k of token t by one warp.  Lane l holds experts l, l+32, ...; each of
 // the k rounds is a warp-wide argmax of sigma + bias (ties to the lower
 // expert).  Lane j < k returns slot j's expert and weight.
 NVDEV void topk_token(const float* __restrict__ src, int splits, const float* __restrict__ offset,
                       float* __restrict__ logits, const float* __restrict__ bias, int T, int E, int k, float rsf,
                       int t, int lane, int& out_idx, float& out_w) {
-  float sig[kMaxE / 32], c[kMaxE / 32];
+  float sig[kMaxE / 32];
+  uint32_t key[kMaxE / 32];
   const int per = (E + 31) >> 5;
-  // every slot's logit first, then the sigmoids.  With up to eight splits
+  // every slot's logit first, then the scores.  With up to eight splits
   // (large batches) all of the lane's partial sums are loaded before any is
   // added, so their latencies overlap; the sums keep split order.
   float lg[kMaxE / 32];
@@ -259,54 +310,11 @@ NVDEV void topk_token(const float* __restrict__ src, int splits, const float* __
 #pragma unroll
   for (int i = 0; i < kMaxE / 32; ++i) {
     const int e = lane + 32 * i;
-    if (i < per && e < E) {
-      sig[i] = sigmoid_fixed(lg[i]);
-      c[i] = __fadd_rn(sig[i], bias[e]);
-    } else {
-      sig[i] = 0.0f;
-      c[i] = -INFINITY;
-    }
+    sig[i] = 0.0f;
+    key[i] = 0u;
+    if (i < per && e < E) expert_score(lg[i], bias[e], sig[i], key[i]);
   }
-  // Selection keys: sigma + bias mapped to unsigned integers in the same
-  // order (sign bit flipped for non-negative values, all bits for negative
-  // ones; sigma > 0, so the sum is never -0), 0 for an absent or taken
-  // expert.  Each round is a warp max of the keys, then a warp min of the
-  // expert ids that reach it: the largest score, ties to the lower expert.
-  uint32_t key[kMaxE / 32];
-#pragma unroll
-  for (int i = 0; i < kMaxE / 32; ++i) {
-    const uint32_t u = __float_as_uint(c[i]);
-    key[i] = (i < per && lane + 32 * i < E) ? ((u & 0x80000000u) ? ~u : (u | 0x80000000u)) : 0u;
-  }
-  float sum = 0.0f, my_sig = 0.0f;
-  int my_idx = 0;
-  for (int j = 0; j < k; ++j) {
-    uint32_t bk = 0u, be = 0xffffffffu;
-#pragma unroll
-    for (int i = 0; i < kMaxE / 32; ++i)       // ascending i: a tie keeps the lower expert
-      if (key[i] > bk) {
-        bk = key[i];
-        be = (uint32_t)(lane + 32 * i);
-      }
-    const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
-    const int win = (int)__reduce_min_sync(0xffffffffu, bk == m ? be : 0xffffffffu);
-    // the owner lane marks the winner and broadcasts its sigma
-    float s_own = 0.0f;
-#pragma unroll
-    for (int i = 0; i < kMaxE / 32; ++i)
-      if (lane + 32 * i == win) {
-        s_own = sig[i];
-        key[i] = 0u;
-      }
-    const float s_sel = __shfl_sync(0xffffffffu, s_own, win & 31);
-    sum = __fadd_rn(sum, s_sel);
-    if (lane == j) {
-      my_sig = s_sel;
-      my_idx = win;
-    }
-  }
-  out_idx = my_idx;
-  out_w = __fmul_rn(__fdiv_rn(my_sig, sum), rsf);
+  select_topk(sig, key, k, rsf, lane, out_idx, out_w);
 }
 
 __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ src, int splits,
@@ -450,22 +458,35 @@ __global__ void __launch_bounds__(kChunk) perm_scatter_kernel(const int32_t* __r
 // ---------------------------------------------------------------------------
 // Routing of a small batch (T <= 256) in one block: top-k, per-expert counts,
 // the padded scan, and the scatter, with the padding fill of perm and row_w
-// that the large-batch path does in its count kernel.  The arithmetic is the
-// same (topk_token) and so is every integer result.
+// that the large-batch path does in its count kernel.  The scores (sigma and
+// the selection key) are computed one (token, expert) per thread and kept in
+// shared memory, so a token's warp only runs the selection rounds.  The
+// arithmetic is the same as topk_token's (expert_score, select_topk) and so
+// is every integer result.
 // ---------------------------------------------------------------------------
 constexpr int kSmallT = 256;
 constexpr int kSmallThreads = 1024;
 
+// Dynamic shared memory of the small-batch kernel: the scores of a chunk of
+// tokens between the two phases, sigma (fp32) and the selection key (u32) of
+// each (token, expert), then every token's top-k ids and weights.
+constexpr int kScoreSmemBytes = 64 * 1024;
+int route_small_chunk_tokens(int T, int E) { return std::min(T, kScoreSmemBytes / (8 * E)); }
+int route_small_smem_bytes(int T, int E, int k) { return route_small_chunk_tokens(T, E) * E * 8 + T * k * 8; }
+
 __global__ void __launch_bounds__(kSmallThreads, 1)
     route_small_kernel(const float* __restrict__ src, int splits, const float* __restrict__ offset,
                        float* __restrict__ logits, const float* __restrict__ bias, int T, int E, int k, float rsf,
-                       int cap, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
+                       int cap, int chunk_t, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
                        int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                        int32_t* __restrict__ tile_expert, int32_t* __restrict__ num_mtiles,
                        int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm, float* __restrict__ row_w) {
   __shared__ uint32_t bm[kMaxE][kSmallT / 32];
   __shared__ int32_t sp[256];
   __shared__ int32_t base[kMaxE];
+  extern __shared__ uint32_t s_score[];          // [chunk_t * E] sigma bits, then [chunk_t * E] keys
+  int32_t* s_idx = reinterpret_cast<int32_t*>(s_score + 2 * chunk_t * E);   // [T * k]
+  float* s_w = reinterpret_cast<float*>(s_idx + T * k);                     // [T * k]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   // the router GEMM before this kernel writes none of these, so the fill
   // overlaps it
@@ -476,26 +497,47 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
   }
   griddep_wait();
   griddep_launch();
-  // all logits first, one (token, expert) per thread, so that every thread's
-  // partial-sum loads are in flight at once
-  if (splits > 0) {
-    // the decode shape has 24 splits: one batch of loads per pair
-    for (int i = tid; i < T * E; i += blockDim.x) token_logit<24>(src, splits, offset, logits, T, E, i / E, i % E);
-    src = logits;
-    splits = -1;
-  }
-  __syncthreads();
-  for (int t = warp; t < T; t += blockDim.x >> 5) {
-    int idx;
-    float w;
-    topk_token(src, splits, offset, logits, bias, T, E, k, rsf, t, lane, idx, w);
-    if (lane < k) {
-      topk_idx[(size_t)t * k + lane] = idx;
-      topk_w[(size_t)t * k + lane] = w;
-      atomicOr(&bm[idx][t >> 5], 1u << (t & 31));
+  const int per = (E + 31) >> 5;
+  for (int t0 = 0; t0 < T; t0 += chunk_t) {
+    const int nt = min(chunk_t, T - t0);
+    // every (token, expert) of the chunk, one per thread: the logit (the
+    // split-ordered sum of the partials; the decode shape has 24 splits, all
+    // loaded in one batch), then sigma and the selection key
+    for (int i = tid; i < nt * E; i += blockDim.x) {
+      const int t = t0 + i / E, e = i % E;
+      const float l = splits > 0 ? token_logit<24>(src, splits, offset, logits, T, E, t, e) : src[(size_t)t * E + e];
+      float sig;
+      uint32_t key;
+      expert_score(l, bias[e], sig, key);
+      s_score[i] = __float_as_uint(sig);
+      s_score[chunk_t * E + i] = key;
     }
+    __syncthreads();
+    // top-k, one warp per token
+    for (int tt = warp; tt < nt; tt += blockDim.x >> 5) {
+      const int t = t0 + tt;
+      float sig[kMaxE / 32];
+      uint32_t key[kMaxE / 32];
+#pragma unroll
+      for (int i = 0; i < kMaxE / 32; ++i) {
+        const int e = lane + 32 * i;
+        const bool here = i < per && e < E;
+        sig[i] = here ? __uint_as_float(s_score[tt * E + e]) : 0.0f;
+        key[i] = here ? s_score[chunk_t * E + tt * E + e] : 0u;
+      }
+      int idx;
+      float w;
+      select_topk(sig, key, k, rsf, lane, idx, w);
+      if (lane < k) {
+        topk_idx[(size_t)t * k + lane] = idx;
+        topk_w[(size_t)t * k + lane] = w;
+        s_idx[t * k + lane] = idx;
+        s_w[t * k + lane] = w;
+        atomicOr(&bm[idx][t >> 5], 1u << (t & 31));
+      }
+    }
+    __syncthreads();
   }
-  __syncthreads();
   // per-expert totals, 128-row padding, exclusive scan (threads 0..255)
   int total = 0, padded = 0;
   if (tid < E)
@@ -520,14 +562,32 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
   // stable scatter: rank of token t among the tokens of expert e
   for (int i = tid; i < T * k; i += blockDim.x) {
     const int t = i / k;
-    const int e = topk_idx[i];
+    const int e = s_idx[i];
     int rank = __popc(bm[e][t >> 5] & ((1u << (t & 31)) - 1u));
     for (int w = 0; w < (t >> 5); ++w) rank += __popc(bm[e][w]);
     const int row = base[e] + rank;
     perm[row] = t;
     inv_perm[i] = row;
-    row_w[row] = topk_w[i];
+    row_w[row] = s_w[i];
   }
+}
+
+// Opts the small-batch kernel into its largest dynamic shared memory, once
+// per device.
+static nvfp4_status allow_route_small_smem() {
+  static std::mutex mu;
+  static bool done[64] = {};
+  int dev = 0;
+  NV_CHECK(check_cuda(cudaGetDevice(&dev), "cudaGetDevice"));
+  if (dev < 0 || dev >= 64) dev = 63;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!done[dev]) {
+    NV_CHECK(check_cuda(cudaFuncSetAttribute(route_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kScoreSmemBytes + kSmallT * kMaxK * 8),
+                        "cudaFuncSetAttribute"));
+    done[dev] = true;
+  }
+  return NVFP4_OK;
 }
 
 RouteScratch carve_route_scratch(Carver& c, int T, int E, int k) {
@@ -578,9 +638,12 @@ nvfp4_status launch_route(const RouteArgs& a, const RouteScratch& r, cudaStream_
     NV_CHECK(launch_dependent("router_gemm_kernel", router_gemm_kernel, grid, dim3(kRThreads), smem, s, tmX, tmW, p));
   }
   if (a.T <= kSmallT) {
-    return launch_dependent("route_small_kernel", route_small_kernel, dim3(1), dim3(kSmallThreads), 0, s,
+    const int chunk_t = route_small_chunk_tokens(a.T, a.E);
+    const int smem = route_small_smem_bytes(a.T, a.E, a.k);
+    NV_CHECK(allow_route_small_smem());
+    return launch_dependent("route_small_kernel", route_small_kernel, dim3(1), dim3(kSmallThreads), smem, s,
                             (const float*)(splits ? r.partial : a.logits), splits, a.logit_offset, a.logits, a.bias,
-                            a.T, a.E, a.k, a.rsf, cap, a.topk_idx, a.topk_w, r.counts, a.expert_offsets,
+                            a.T, a.E, a.k, a.rsf, cap, chunk_t, a.topk_idx, a.topk_w, r.counts, a.expert_offsets,
                             r.tile_expert, r.num_mtiles, a.perm, a.inv_perm, r.row_w);
   }
   // each kernel waits for its predecessor's results (griddepcontrol.wait) as
