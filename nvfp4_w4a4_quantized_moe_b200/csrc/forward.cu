@@ -378,6 +378,13 @@ static nvfp4_status forward_impl(const moe_nvfp4_weights* W, const void* x_bf16,
   ra.topk_idx = f.topk_idx; ra.topk_w = f.topk_w; ra.expert_offsets = f.offsets;
   ra.perm = f.perm; ra.inv_perm = f.inv_perm;
   ra.clear_status = router_first;
+  // small batches with the tensor's own g1: the routing kernel quantises x
+  // and fills the permuted rows itself, one kernel fewer in the chain
+  const bool fused_x = mode == NVFP4_ACT_SCALE_TENSOR && route_fuses_x_quantise(T, H, k);
+  ra.quant_x = fused_x;
+  ra.act_gscale = act_gscale;
+  ra.a_codes = f.a_codes;
+  ra.a_scales = f.a_scales;
   NV_CHECK(launch_route(ra, f.route, s));
   NV_CHECK(mark(dbg, 1, s));
 
@@ -388,7 +395,8 @@ static nvfp4_status forward_impl(const moe_nvfp4_weights* W, const void* x_bf16,
     NV_CHECK(launch_dependent("expert_amax_kernel", expert_amax_kernel, dim3((T * k + 255) / 256), dim3(256), 0, s,
                               (const int32_t*)f.topk_idx, T, k, (const uint32_t*)f.tok_amax, f.amax_bits));
   }
-  switch (mode) {
+  switch (fused_x ? -1 : mode) {
+    case -1: break;
     case NVFP4_ACT_SCALE_TENSOR: NV_CHECK(launch_quantize_scatter<0>(f, x_bf16, T, H, E, k, act_gscale, s)); break;
     case NVFP4_ACT_SCALE_EXPERT: NV_CHECK(launch_quantize_scatter<1>(f, x_bf16, T, H, E, k, act_gscale, s)); break;
     case NVFP4_ACT_SCALE_DYNAMIC: NV_CHECK(launch_quantize_scatter<2>(f, x_bf16, T, H, E, k, act_gscale, s)); break;

@@ -469,10 +469,27 @@ constexpr int kSmallThreads = 1024;
 
 // Dynamic shared memory of the small-batch kernel: the scores of a chunk of
 // tokens between the two phases, sigma (fp32) and the selection key (u32) of
-// each (token, expert), then every token's top-k ids and weights.
+// each (token, expert); every pair's top-k id, weight and permuted row; and,
+// when the kernel also quantises x, each token's codes and scale bytes.
 constexpr int kScoreSmemBytes = 64 * 1024;
-int route_small_chunk_tokens(int T, int E) { return std::min(T, kScoreSmemBytes / (8 * E)); }
-int route_small_smem_bytes(int T, int E, int k) { return route_small_chunk_tokens(T, E) * E * 8 + T * k * 8; }
+constexpr int kRouteSmallMaxDyn = 200 * 1024;
+__host__ __device__ inline int route_small_chunk_tokens(int T, int E) { return min(T, kScoreSmemBytes / (8 * E)); }
+__host__ __device__ inline int route_small_xq_offset(int T, int E, int k) {   // bytes before x's codes, 16-byte aligned
+  return (route_small_chunk_tokens(T, E) * E * 8 + T * k * 12 + 15) / 16 * 16;
+}
+int route_small_smem_bytes(int T, int E, int k, int H, bool quant_x) {
+  return quant_x ? route_small_xq_offset(T, E, k) + T * (H / 2 + H / kQBlock) : route_small_chunk_tokens(T, E) * E * 8 + T * k * 12;
+}
+// Every permuted row of x then leaves through this one block.  Measured on
+// B200: at 16 tokens x 8 slots of H = 6144 (442 KB of rows) the fused kernel
+// took 39.6 us against 18.5 + 8.1 us for routing plus the separate quantise
+// kernel, while at 32 x 2 slots of H = 256 (9 KB) the layer's step went down
+// by 7 %.  So the fusion is kept to 64 KiB of rows.
+constexpr long long kFusedXRowBytes = 64 * 1024;
+bool route_fuses_x_quantise(int T, int H, int k) {
+  return T <= kSmallT && (long long)T * k * (H / 2 + H / kQBlock) <= kFusedXRowBytes &&
+         route_small_xq_offset(T, kMaxE, k) + T * (H / 2 + H / kQBlock) <= kRouteSmallMaxDyn;
+}
 
 __global__ void __launch_bounds__(kSmallThreads, 1)
     route_small_kernel(const float* __restrict__ src, int splits, const float* __restrict__ offset,
@@ -480,13 +497,20 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
                        int cap, int chunk_t, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
                        int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                        int32_t* __restrict__ tile_expert, int32_t* __restrict__ num_mtiles,
-                       int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm, float* __restrict__ row_w) {
+                       int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm, float* __restrict__ row_w,
+                       int quant_x, const uint4* __restrict__ x, int H, const float* __restrict__ act_gscale,
+                       uint8_t* __restrict__ a_codes, uint8_t* __restrict__ a_scales) {
   __shared__ uint32_t bm[kMaxE][kSmallT / 32];
   __shared__ int32_t sp[256];
   __shared__ int32_t base[kMaxE];
   extern __shared__ uint32_t s_score[];          // [chunk_t * E] sigma bits, then [chunk_t * E] keys
   int32_t* s_idx = reinterpret_cast<int32_t*>(s_score + 2 * chunk_t * E);   // [T * k]
   float* s_w = reinterpret_cast<float*>(s_idx + T * k);                     // [T * k]
+  int32_t* s_row = reinterpret_cast<int32_t*>(s_w + T * k);                 // [T * k]
+  // quantised x: [T][H/2] codes, then [T][H/16] scale bytes
+  uint8_t* xq_c = reinterpret_cast<uint8_t*>(s_score) + (quant_x ? route_small_xq_offset(T, E, k) : 0);
+  uint8_t* xq_s = xq_c + (size_t)T * (H / 2);
+  const int nblk = H / kQBlock;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   // the router GEMM before this kernel writes none of these, so the fill
   // overlaps it
@@ -494,6 +518,20 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
   for (int i = tid; i < cap; i += blockDim.x) {
     perm[i] = -1;
     row_w[i] = 0.0f;
+  }
+  if (quant_x) {
+    // x and g1 are the layer's inputs, complete once the router GEMM ahead of
+    // this kernel has started (it waited for their producer), so they are
+    // quantised here, before the wait, exactly as the quantise-scatter kernel
+    // does: one 16-element block per thread and step, read through L2
+    const float g = act_gscale[0];
+    const float d = __fmul_rn(6.0f, g);
+    for (int b = tid; b < T * nblk; b += blockDim.x) {
+      uint2 c;
+      const uint32_t sc = quant_block16_bf16(__ldcg(x + (size_t)b * 2), __ldcg(x + (size_t)b * 2 + 1), g, d, c);
+      reinterpret_cast<uint2*>(xq_c)[b] = c;
+      xq_s[b] = (uint8_t)sc;
+    }
   }
   griddep_wait();
   griddep_launch();
@@ -569,6 +607,24 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
     perm[row] = t;
     inv_perm[i] = row;
     row_w[row] = s_w[i];
+    s_row[i] = row;
+  }
+  if (quant_x) {
+    // each token's codes and scales to its k rows: 16-byte code chunks, and
+    // the tiled scale layout's 4-block words
+    __syncthreads();
+    const int cpr = H / 32;
+    for (int i = tid; i < T * k * cpr; i += blockDim.x) {
+      const int pair = i / cpr, ch = i % cpr;
+      reinterpret_cast<uint4*>(a_codes + (size_t)s_row[pair] * (H / 2))[ch] =
+          reinterpret_cast<const uint4*>(xq_c + (size_t)(pair / k) * (H / 2))[ch];
+    }
+    const int wpr = nblk / 4;
+    for (int i = tid; i < T * k * wpr; i += blockDim.x) {
+      const int pair = i / wpr, w = i % wpr;
+      *reinterpret_cast<uint32_t*>(a_scales + tiled_scale_offset(s_row[pair], 4 * w, nblk >> 2)) =
+          *reinterpret_cast<const uint32_t*>(xq_s + (size_t)(pair / k) * nblk + 4 * w);
+    }
   }
 }
 
@@ -583,7 +639,7 @@ static nvfp4_status allow_route_small_smem() {
   std::lock_guard<std::mutex> lock(mu);
   if (!done[dev]) {
     NV_CHECK(check_cuda(cudaFuncSetAttribute(route_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             kScoreSmemBytes + kSmallT * kMaxK * 8),
+                                             kRouteSmallMaxDyn),
                         "cudaFuncSetAttribute"));
     done[dev] = true;
   }
@@ -639,12 +695,14 @@ nvfp4_status launch_route(const RouteArgs& a, const RouteScratch& r, cudaStream_
   }
   if (a.T <= kSmallT) {
     const int chunk_t = route_small_chunk_tokens(a.T, a.E);
-    const int smem = route_small_smem_bytes(a.T, a.E, a.k);
+    const bool qx = a.quant_x && route_fuses_x_quantise(a.T, a.H, a.k);
+    const int smem = route_small_smem_bytes(a.T, a.E, a.k, a.H, qx);
     NV_CHECK(allow_route_small_smem());
     return launch_dependent("route_small_kernel", route_small_kernel, dim3(1), dim3(kSmallThreads), smem, s,
                             (const float*)(splits ? r.partial : a.logits), splits, a.logit_offset, a.logits, a.bias,
                             a.T, a.E, a.k, a.rsf, cap, chunk_t, a.topk_idx, a.topk_w, r.counts, a.expert_offsets,
-                            r.tile_expert, r.num_mtiles, a.perm, a.inv_perm, r.row_w);
+                            r.tile_expert, r.num_mtiles, a.perm, a.inv_perm, r.row_w, qx ? 1 : 0,
+                            static_cast<const uint4*>(a.x), a.H, a.act_gscale, a.a_codes, a.a_scales);
   }
   // each kernel waits for its predecessor's results (griddepcontrol.wait) as
   // its first step, so programmatic launch only hides the launch latency

@@ -21,7 +21,20 @@ struct RouteArgs {
   // the router GEMM clears the status word once the previous work on the
   // stream has finished (the caller then issues no memset before it)
   bool clear_status = false;
+  // Optional, for small batches (route_fuses_x_quantise): the routing kernel
+  // also quantises x under the tensor's g1 (act_gscale[0]) and writes each
+  // token's codes and tiled scales to its k permuted rows of a_codes [rows]
+  // [H/2] / a_scales, the work the layer's quantise-scatter kernel does
+  bool quant_x = false;
+  const float* act_gscale = nullptr;
+  uint8_t* a_codes = nullptr;
+  uint8_t* a_scales = nullptr;
 };
+
+// Whether the single-block routing kernel also quantises x and writes it to
+// the permuted rows: only for small volumes, since those writes all go
+// through one SM (route.cu gives the measured bound).
+bool route_fuses_x_quantise(int T, int H, int k);
 
 struct RouteScratch {
   uint32_t* status = nullptr;           // device status word (start of the workspace)
