@@ -389,8 +389,9 @@ static nvfp4_status forward_impl(const moe_nvfp4_weights* W, const void* x_bf16,
   NV_CHECK(mark(dbg, 1, s));
 
   // 4: quantise x into its k permuted rows (under the batch's or each
-  // expert's g1).  Padding rows are left as they are: an MMA row only feeds
-  // the same output row, and the epilogues skip padding rows.
+  // expert's g1); the routing kernel has done it already when fused_x.
+  // Padding rows are left as they are: an MMA row only feeds the same output
+  // row, and the epilogues skip padding rows.
   if (mode == NVFP4_ACT_SCALE_DYNAMIC_EXPERT) {
     NV_CHECK(launch_dependent("expert_amax_kernel", expert_amax_kernel, dim3((T * k + 255) / 256), dim3(256), 0, s,
                               (const int32_t*)f.topk_idx, T, k, (const uint32_t*)f.tok_amax, f.amax_bits));
