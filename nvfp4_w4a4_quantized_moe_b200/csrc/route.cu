@@ -22,19 +22,26 @@ namespace nvfp4moe {
 // ---------------------------------------------------------------------------
 constexpr int kRBM = 128;
 constexpr int kRBK = 64;                      // bf16 elements of K per stage
-constexpr int kRStages = 4;
+// Up to eight stages, as many as fit (router_stages): at 8192 tokens each CTA
+// streams 1.3 MB of x and W_g, and four stages kept too few bytes in flight
+// to cover the load latency.
+constexpr int kRStages = 8;
 constexpr int kRThreads = 192;
 constexpr int kRAbytes = kRBM * kRBK * 2;     // 16 KiB
 
 struct RouterGemmParams {
   int T, E, H, n_mma, kt_per_split, splits, clear_status;
+  int stages;            // pipeline depth used (<= kRStages)
   float* partial;
   uint32_t* status;
 };
 
 static inline int router_n_mma(int E) { return (E + 15) / 16 * 16; }
 static inline int router_stage_bytes(int E) { return kRAbytes + (router_n_mma(E) * 128 + 1023) / 1024 * 1024; }
-static inline int router_smem_bytes(int E) { return kRStages * router_stage_bytes(E) + 1024; }
+static inline int router_stages(int E) {
+  return std::max(2, std::min(kRStages, (227 * 1024 - 1024) / router_stage_bytes(E)));
+}
+static inline int router_smem_bytes(int E) { return router_stages(E) * router_stage_bytes(E) + 1024; }
 
 // Split count: as many CTAs as fit on the SMs of a B200 (148) at one per SM,
 // with at least four K stages each; rounding up instead (a second CTA on
@@ -68,7 +75,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
   const int kt1 = min(kt0 + p.kt_per_split, KT);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kRStages; ++s) {
+    for (int s = 0; s < p.stages; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
     }
@@ -112,14 +119,14 @@ __global__ void __launch_bounds__(kRThreads, 1)
         tma_load_2d(sA + kRAbytes, &tmW, kt * kRBK, 0, &full_bar[stage]);
         filled |= 1u << stage;
         fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
-        if (++stage == kRStages) {
+        if (++stage == p.stages) {
           stage = 0;
           phase ^= 1u;
         }
       }
       if (!ok) {
         volatile int never = 0;
-        for (int s = 0; s < kRStages; ++s)
+        for (int s = 0; s < p.stages; ++s)
           if ((filled >> s) & 1u) mbar_wait(&full_bar[s], (fill_parity >> s) & 1u, &never);
       }
     }
@@ -143,7 +150,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
         for (int j = 0; j < 4; ++j)      // 16 bf16 = 32 bytes of K per MMA
           mma_bf16(tmem, adesc + 2 * j, bdesc + 2 * j, idesc, (kt > kt0 || j > 0) ? 1u : 0u);
         tc_commit(&empty_bar[stage]);
-        if (++stage == kRStages) {
+        if (++stage == p.stages) {
           stage = 0;
           phase ^= 1u;
         }
@@ -683,6 +690,7 @@ nvfp4_status launch_route(const RouteArgs& a, const RouteScratch& r, cudaStream_
     p.kt_per_split = (a.H / kRBK + splits - 1) / splits;
     p.splits = splits;
     p.clear_status = a.clear_status ? 1 : 0;
+    p.stages = router_stages(a.E);
     p.partial = r.partial;
     p.status = r.status;
     const int smem = router_smem_bytes(a.E);
