@@ -38,21 +38,12 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 FP4_OVER_BF16 = 4.0            # nominal dense ratio (9 vs 2.25 PFLOP/s)
 
 
-def fuses_x_quantise(T: int, H: int, k: int) -> bool:
-    """Whether the library's routing kernel also quantises x (tensor-wide g1):
-    up to 256 tokens and at most 64 KiB of permuted rows of codes and scales.
-    Host-side accounting only; the library decides the same way."""
-    return T <= 256 and T * k * (H // 2 + H // 16) <= 64 * 1024
-
-
-def kernels_per_step(T: int, H: int, k: int) -> int:
-    """Kernels one forward launches: router GEMM, routing (one single-block
-    kernel up to 256 tokens, else top-k and three permutation kernels),
-    quantise-scatter (folded into the routing kernel for small layers), the
-    two GEMMs and the combine."""
-    if T > 256:
-        return 9
-    return 5 if fuses_x_quantise(T, H, k) else 6
+def kernels_per_step(c, cfg) -> int:
+    """Kernels one forward launches, as the library counts them: router GEMM,
+    routing (one single-block kernel up to 256 tokens, else top-k and three
+    permutation kernels), quantise-scatter (folded into the routing kernel
+    for small layers), the two GEMMs and the combine."""
+    return c.moe_nvfp4_forward_launches(cfg.T, cfg.E, cfg.H, cfg.I, cfg.k)
 NVFP4_BYTES_PER_ELEM = 0.5 + 1.0 / 16
 
 
@@ -549,7 +540,7 @@ def run_ours(args, cfg):
                       "frac": q_gbs / peaks["hbm_gbs"]},
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": x.numel() * 2, "d2h_bytes_per_step": out.numel() * 2},
-        "gpu_launches": kernels_per_step(cfg.T, cfg.H, cfg.k) * args.steps,
+        "gpu_launches": kernels_per_step(c, cfg) * args.steps,
         "clocks": clocks,
         "cpu_baseline": cpu,
     }

@@ -294,6 +294,15 @@ NVFP4_API nvfp4_status moe_nvfp4_forward_scaled(const moe_nvfp4_weights* W, cons
                                                 const moe_nvfp4_debug* dbg, void* ws, size_t ws_bytes,
                                                 void* stream);
 
+/* Number of kernels one moe_nvfp4_forward_scaled call (act_scale_mode; mode 0
+ * is moe_nvfp4_forward) queues for this shape, without the REAP saliency
+ * kernel that the debug struct can add; memsets are not kernels.  It depends
+ * on the shape only: small batches route in one kernel, and small layers
+ * quantise x inside it.  Host-only arithmetic, no CUDA call.  Returns -1 for
+ * a shape or mode the forward rejects.  This has no counterpart on the pages:
+ * it lets a caller account for the launches it measures. */
+NVFP4_API int moe_nvfp4_forward_launches(int T, int E, int H, int I, int k, int I_shared, int act_scale_mode);
+
 /* ------------------------------------------------------------------------
  * The two grouped GEMMs on caller-supplied quantised operands (the same
  * kernels moe_nvfp4_forward runs).  Rows are grouped by expert_offsets

@@ -83,6 +83,7 @@ _declare("moe_route", _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _vp,
          _vp)
 _declare("moe_nvfp4_workspace_size", _sz, _i, _i, _i, _i, _i)
 _declare("moe_nvfp4_workspace_size_shared", _sz, _i, _i, _i, _i, _i, _i)
+_declare("moe_nvfp4_forward_launches", _i, _i, _i, _i, _i, _i, _i, _i)
 _declare("moe_nvfp4_forward", _i, ctypes.POINTER(MoeWeightsStruct), _vp, _i, _vp, _vp, _vp, _vp,
          ctypes.POINTER(MoeDebugStruct), _vp, _sz, _vp)
 _declare("moe_nvfp4_forward_scaled", _i, ctypes.POINTER(MoeWeightsStruct), _vp, _i, _i, _vp, _vp, _vp, _vp,
@@ -106,6 +107,7 @@ EXPORTS = ("nvfp4_last_error", "nvfp4_abi_version", "nvfp4_workspace_status",
            "nvfp4_quantize_act",
            "moe_route_rows_capacity", "moe_route_workspace_size", "moe_route", "moe_nvfp4_workspace_size",
            "moe_nvfp4_forward", "moe_nvfp4_forward_scaled", "moe_nvfp4_workspace_size_shared",
+           "moe_nvfp4_forward_launches",
            "moe_nvfp4_gemm_workspace_size", "moe_nvfp4_gate_up",
            "moe_nvfp4_down",
            "nvfp4_block_stats_compute",
@@ -384,6 +386,15 @@ def select_experts(W: "MoeWeights", keep: torch.Tensor) -> "MoeWeights":
                       codes(W.up_codes), rows(W.up_scales, W.I * W.H // 16), W.up_gscale.index_select(0, idx),
                       codes(W.down_codes), rows(W.down_scales, W.H * W.I // 16), W.down_gscale.index_select(0, idx),
                       W.shared_gate, W.shared_up, W.shared_down, W.codes_layout)
+
+
+def moe_nvfp4_forward_launches(T: int, E: int, H: int, I: int, k: int, I_shared: int = 0,
+                               act_scale_mode: str = "tensor") -> int:
+    """Kernels one forward call queues for this shape (host arithmetic only)."""
+    n = lib.moe_nvfp4_forward_launches(T, E, H, I, k, I_shared, ACT_SCALE_MODES[act_scale_mode])
+    if n < 0:
+        raise ValueError(f"unsupported forward shape T={T} E={E} H={H} I={I} k={k} I_shared={I_shared}")
+    return n
 
 
 def moe_nvfp4_workspace_size(T: int, E: int, H: int, I: int, k: int, I_shared: int = 0) -> int:

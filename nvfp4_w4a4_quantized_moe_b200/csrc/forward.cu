@@ -311,6 +311,21 @@ extern "C" size_t moe_nvfp4_workspace_size(int T, int E, int H, int I, int k) {
   return moe_nvfp4_workspace_size_shared(T, E, H, I, k, 0);
 }
 
+// Mirrors the launch sequence of forward_impl below.
+extern "C" int moe_nvfp4_forward_launches(int T, int E, int H, int I, int k, int I_shared, int mode) {
+  if (T < 1 || H <= 0 || H % 256 != 0 || I <= 0 || I % 128 != 0 || k < 1 || k > 16 || k > E || E > 256 ||
+      I_shared < 0 || I_shared % 128 != 0 || mode < NVFP4_ACT_SCALE_TENSOR || mode > NVFP4_ACT_SCALE_DYNAMIC_EXPERT)
+    return -1;
+  int n = 0;
+  if (I_shared > 0) n += 1 + 2;                                    // dense tile map, shared gate/up and down
+  if (mode & kActDynamic) n += 1;                                   // token amax
+  n += 1 + (T <= 256 ? 1 : 4);                                      // router GEMM, routing
+  if (mode == NVFP4_ACT_SCALE_DYNAMIC_EXPERT) n += 1;               // expert amax
+  if (!(mode == NVFP4_ACT_SCALE_TENSOR && route_fuses_x_quantise(T, H, k))) n += 1;   // quantise-scatter
+  n += 2 + 1;                                                       // gate/up, down, combine
+  return n;
+}
+
 template <int MODE>
 static nvfp4_status launch_quantize_scatter(const ForwardScratch& f, const void* x_bf16, int T, int H, int E, int k,
                                             float* act_gscale, cudaStream_t s) {

@@ -30,6 +30,29 @@ def test_abi_version_and_sizes():
     assert c.lib.nvfp4_quantize_weights_workspace_size(240) >= 256
 
 
+def test_forward_launch_count_follows_the_shape():
+    """The host-only launch count of the forward: router GEMM, routing (one
+    kernel up to 256 tokens, else four), quantise-scatter (inside the routing
+    kernel when at most 64 KiB of permuted rows), gate/up, down, combine, plus
+    the shared expert's three kernels and the dynamic modes' amax kernels."""
+    c = capi()
+    n = c.moe_nvfp4_forward_launches
+    assert n(32, 8, 256, 128, 2) == 5          # tiny layer: 32 x 2 rows of 144 bytes
+    assert n(16, 80, 6144, 2048, 8) == 6       # decode: 442 KB of rows, a separate quantise kernel
+    assert n(256, 80, 6144, 2048, 8) == 6
+    assert n(257, 80, 6144, 2048, 8) == 9      # multi-kernel routing above 256 tokens
+    assert n(8192, 80, 6144, 2048, 8) == 9
+    assert n(16, 80, 6144, 2048, 8, I_shared=2048) == 9
+    assert n(32, 8, 256, 128, 2, act_scale_mode="expert") == 6     # per-expert g1: no fused quantisation
+    assert n(16, 80, 6144, 2048, 8, act_scale_mode="dynamic") == 7
+    assert n(16, 80, 6144, 2048, 8, act_scale_mode="dynamic_expert") == 8
+    # the 64 KiB bound of the fused path: 227 rows of 288 bytes fit, 228 do not
+    assert n(227, 8, 512, 256, 1) == 5 and n(228, 8, 512, 256, 1) == 6
+    with pytest.raises(ValueError):
+        n(16, 80, 6000, 2048, 8)                # H % 256 != 0
+    assert c.lib.moe_nvfp4_forward_launches(16, 80, 6144, 2048, 8, 0, 7) == -1
+
+
 def test_host_side_argument_checks():
     c = capi()
     lib = c.lib
