@@ -1,0 +1,157 @@
+"""The oracle's NVFP4 readings against two library implementations of the
+format, on CPU.
+
+The NVFP4 model card ("K-EXAONE-152B-A23B-REAP-80E-NVFP4", "Quantization
+Setup") quantises its weights with llmcompressor's NVFP4 scheme, stored in the
+compressed-tensors format, and serves the checkpoint with vLLM.  Both
+libraries are in this image and hold plain-PyTorch references of the format:
+compressed-tensors' weight quantisation (global scale 2688/amax, block scale
+amax/6 times it, elements divided by block/global) and vLLM's activation
+reference (block scale global * (amax * 1/6), elements multiplied by the
+reciprocal of block/global).
+
+What agrees, exactly: the element format (E2M1 magnitudes, round to nearest
+with ties to the even code, saturation at 6, the sign of a negative that
+rounds to zero; the libraries' own E2M1 casts are compared value by value),
+the block-scale format (E4M3,
+round to nearest even, at most 448), the global scale (the libraries store the
+reciprocal of this library's g), and, with vLLM, a zero scale for an all-zero
+block.  What differs is the order of the fp32 roundings (reading R2 of the
+design notes): it only shows where the exact value sits on a rounding
+midpoint, and then the two results are neighbouring codes.  These tests pin
+exactly that, and two small convention differences: compressed-tensors gives
+an all-zero block the E4M3 scale eps (0.125) where this library gives 0
+(reading R7), and an input of exactly -0.0 becomes +0 in the libraries, -0
+here (reading R5).
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import nvfp4
+
+E2M1_MIDPOINTS = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+E4M3_VALUES = np.array([nvfp4.e4m3_decode(np.array([c], np.uint8))[0] for c in range(0x7F)], np.float64)
+E4M3_MIDPOINTS = (E4M3_VALUES[1:] + E4M3_VALUES[:-1]) / 2
+
+
+def _near(v, points, rel=1e-5):
+    v = np.abs(np.asarray(v, np.float64))[..., None]
+    return np.any(np.abs(v - points) <= rel * np.maximum(points, 1e-30), axis=-1)
+
+
+def _values(codes):
+    c = np.stack([codes & 0xF, codes >> 4], -1).reshape(codes.shape[0], -1)
+    return nvfp4.e2m1_decode(c).astype(np.float64), c & 0x7
+
+
+def _magnitude_code(v):
+    return np.searchsorted(np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6]), np.abs(v))
+
+
+def _check_against(x, g, ours_codes, ours_scales, lib_values, lib_scale_codes, zero_scale_code):
+    """Exact agreement up to neighbouring codes at rounding midpoints."""
+    rows, nblk = ours_scales.shape
+    xb = x.astype(np.float64).reshape(rows, nblk, 16)
+    amax_b = np.abs(xb).max(-1)
+    zero = amax_b == 0
+    # all-zero blocks: the libraries' convention, then nothing else to compare
+    assert np.all(lib_scale_codes[zero] == zero_scale_code) and np.all(ours_scales[zero] == 0)
+    # block scales: equal, or neighbours where the exact value amax_b / (6 g) is a midpoint
+    diff = (lib_scale_codes != ours_scales) & ~zero
+    assert diff.sum() <= 0.005 * (~zero).sum()
+    assert np.all(np.abs(lib_scale_codes[diff].astype(int) - ours_scales[diff].astype(int)) == 1)
+    assert np.all(_near(amax_b[diff] / (6.0 * float(g)), E4M3_MIDPOINTS))
+    # elements, in blocks whose scales agree
+    ours_v, _ = _values(ours_codes)
+    same = np.repeat(~diff, 16, axis=1)
+    ev = (ours_v != lib_values) & same
+    # bf16 inputs put many elements exactly on a midpoint; where the two
+    # sequences' effective scales differ by an ulp those land on either side
+    assert ev.sum() <= 0.01 * same.sum()
+    assert np.all(np.abs(_magnitude_code(ours_v[ev]) - _magnitude_code(lib_values[ev])) == 1)
+    s_val = nvfp4.e4m3_decode(ours_scales).astype(np.float64)
+    with np.errstate(divide="ignore", invalid="ignore"):        # all-zero blocks have no y
+        y = x.astype(np.float64) / (np.repeat(s_val, 16, axis=1) * float(g))
+    assert np.all(_near(y[ev], E2M1_MIDPOINTS, rel=1e-4))
+    return int(diff.sum()), int(ev.sum())
+
+
+def _e2m1_probe_values():
+    """Every E2M1 midpoint and grid point, their fp32 neighbours, saturation,
+    signed zeros and random magnitudes, positive and negative."""
+    base = np.concatenate([E2M1_MIDPOINTS, [0.0, 0.5, 1, 1.5, 2, 3, 4, 6, 6.5, 7, 100.0, 1e-30]]).astype(np.float32)
+    near = np.concatenate([np.nextafter(base, np.float32(np.inf)), np.nextafter(base, np.float32(0))])
+    rnd = np.random.default_rng(0).uniform(0, 7, 4096).astype(np.float32)
+    v = np.concatenate([base, near, rnd])
+    return np.concatenate([v, -v]).astype(np.float32)
+
+
+@pytest.mark.parametrize("lib", ["compressed_tensors", "vllm"])
+def test_e2m1_rounding_matches_the_libraries(lib, monkeypatch):
+    """Round to nearest, ties to the even code, saturation at 6, the sign of
+    zero kept: the libraries' E2M1 casts give the oracle's values exactly."""
+    if lib == "compressed_tensors":
+        qa = pytest.importorskip("compressed_tensors.quantization.quant_args")
+        monkeypatch.setattr(torch._dynamo.config, "disable", True)     # eager: the same arithmetic
+        cast = qa.FP4_E2M1_DATA.cast_to_fp4
+    else:
+        cast = pytest.importorskip("vllm.model_executor.layers.quantization.utils.nvfp4_emulation_utils").cast_to_fp4
+    y = _e2m1_probe_values()
+    got = cast(torch.from_numpy(y.copy()).clamp(-6.0, 6.0)).numpy()
+    ours = nvfp4.e2m1_decode(nvfp4.e2m1_encode(y))
+    np.testing.assert_array_equal(got, ours)
+    # the sign of zero agrees (tiny negatives give -0 on both sides) except for
+    # an input of exactly -0.0: the libraries take its sign as 0 and return +0,
+    # this library keeps -0 (code 8, reading R5)
+    neg_zero = (y == 0) & np.signbit(y)
+    assert np.array_equal(np.signbit(got)[~neg_zero], np.signbit(ours)[~neg_zero])
+    assert neg_zero.any() and not np.signbit(got[neg_zero]).any() and np.signbit(ours[neg_zero]).all()
+
+
+def _weights(seed, rows=128, cols=1024):
+    gen = torch.Generator().manual_seed(seed)
+    w = torch.randn(rows, cols, generator=gen) * 0.02
+    w[torch.rand(rows, cols, generator=gen) < 0.01] *= 20          # outliers
+    w[seed % 4] = 0.0                                              # an all-zero row
+    return w.to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_weight_quantiser_matches_compressed_tensors(seed, monkeypatch):
+    ct = pytest.importorskip("compressed_tensors.quantization")
+    from compressed_tensors.quantization.lifecycle.forward_helpers import _quantize
+    from compressed_tensors.quantization.utils.helpers import calculate_qparams, calculate_range, generate_gparam
+    monkeypatch.setattr(torch._dynamo.config, "disable", True)   # its E2M1 cast is torch.compile'd; eager is the same
+    w = _weights(seed)
+    args = ct.QuantizationArgs(num_bits=4, type="float", strategy="tensor_group", group_size=16, symmetric=True,
+                               dynamic=False, scale_dtype=torch.float8_e4m3fn)
+    x = w.float()
+    gs = generate_gparam(x.min(), x.max())
+    xb = x.unflatten(-1, (x.shape[-1] // 16, 16))
+    scale, _ = calculate_qparams(xb.amin(-1), xb.amax(-1), args, global_scale=gs)
+    q_min, q_max = calculate_range(args, "cpu")
+    lib_v = _quantize(xb, scale.unsqueeze(-1), None, q_min, q_max, args, global_scale=gs).flatten(-2)
+    lib_s = scale.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    codes, scales, g = nvfp4.quantize_weight(x.numpy())
+    # the global scale: reciprocals of each other, to fp32 rounding
+    assert abs(float(gs) * float(g) - 1.0) <= 2.0 ** -22
+    eps_code = int(torch.tensor([torch.finfo(torch.float8_e4m3fn).eps]).to(torch.float8_e4m3fn).view(torch.uint8))
+    _check_against(x.numpy(), g, codes, scales, lib_v.numpy().astype(np.float64), lib_s, eps_code)
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_activation_quantiser_matches_vllm_reference(seed):
+    ref = pytest.importorskip("vllm.model_executor.layers.quantization.utils.nvfp4_emulation_utils")
+    gen = torch.Generator().manual_seed(100 + seed)
+    x = torch.randn(64, 2048, generator=gen)
+    x[torch.rand(64, 2048, generator=gen) < 0.001] *= 20
+    x[seed % 3, :48] = 0.0                                          # three all-zero blocks
+    x = x.to(torch.bfloat16).float()
+    amax = np.float32(x.abs().max())
+    g = np.float32(amax / np.float32(2688))                         # calibrated g1 of this library
+    gs = torch.tensor([2688.0]) / torch.tensor([float(amax)])       # the same calibration, stored inverted
+    lib_v, lib_scale = ref.ref_nvfp4_quant(x, gs, 16)
+    lib_s = lib_scale.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    codes, scales = nvfp4.quantize(x.numpy(), g)
+    _check_against(x.numpy(), g, codes, scales, lib_v.numpy().astype(np.float64), lib_s, 0)
