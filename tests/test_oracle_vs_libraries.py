@@ -155,3 +155,21 @@ def test_activation_quantiser_matches_vllm_reference(seed):
     lib_s = lib_scale.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
     codes, scales = nvfp4.quantize(x.numpy(), g)
     _check_against(x.numpy(), g, codes, scales, lib_v.numpy().astype(np.float64), lib_s, 0)
+
+
+@pytest.mark.parametrize("rows,nblk", [(256, 24), (200, 8), (128, 4), (300, 16)])
+def test_tiled_scale_layout_is_the_swizzled_layout_of_vllm(rows, nblk, monkeypatch):
+    """NVFP4_LAYOUT_TILED (the scale layout the tensor-core MMA reads) is
+    byte for byte the block-scale layout vLLM prepares for the CUTLASS and
+    FlashInfer FP4 kernels (swizzle_blockscale), zero padding rows included.
+    The GPU tests check that the library writes the layout of tiled_index."""
+    mod = pytest.importorskip("vllm.model_executor.layers.quantization.utils.nvfp4_utils")
+    from _util import tiled_index
+    monkeypatch.setattr(torch.Tensor, "cuda", lambda self, *a, **k: self)   # its last step moves to the GPU
+    sc = np.random.default_rng(rows + nblk).integers(0, 0x7F, size=(rows, nblk), dtype=np.uint8)
+    swizzled = mod.swizzle_blockscale(torch.from_numpy(sc).view(torch.float8_e4m3fn))
+    swizzled = swizzled.view(torch.uint8).numpy().reshape(-1)
+    rows_padded = (rows + 127) // 128 * 128
+    ours = np.zeros(rows_padded * nblk, np.uint8)
+    ours[tiled_index(rows_padded, nblk * 16)[:rows].reshape(-1)] = sc.reshape(-1)
+    np.testing.assert_array_equal(swizzled, ours)
