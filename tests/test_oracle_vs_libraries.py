@@ -173,3 +173,15 @@ def test_tiled_scale_layout_is_the_swizzled_layout_of_vllm(rows, nblk, monkeypat
     ours = np.zeros(rows_padded * nblk, np.uint8)
     ours[tiled_index(rows_padded, nblk * 16)[:rows].reshape(-1)] = sc.reshape(-1)
     np.testing.assert_array_equal(swizzled, ours)
+
+
+def test_code_packing_is_the_compressed_tensors_packing():
+    """Codes and nibble order (readings R5, R6): compressed-tensors' packer,
+    given the oracle's quantised values, writes the oracle's bytes: magnitude
+    index 0..7, the sign in bit 3, the even-indexed element in the low
+    nibble."""
+    helpers = pytest.importorskip("compressed_tensors.compressors.nvfp4.helpers")
+    codes, _, _ = nvfp4.quantize_weight(_weights(7, rows=64, cols=512).float().numpy())
+    values, _ = _values(codes)
+    packed = helpers.pack_fp4_to_uint8(torch.from_numpy(values.astype(np.float32)))
+    np.testing.assert_array_equal(packed.numpy(), codes)
