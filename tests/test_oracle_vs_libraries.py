@@ -185,3 +185,35 @@ def test_code_packing_is_the_compressed_tensors_packing():
     values, _ = _values(codes)
     packed = helpers.pack_fp4_to_uint8(torch.from_numpy(values.astype(np.float32)))
     np.testing.assert_array_equal(packed.numpy(), codes)
+
+
+def test_routing_matches_vllms_grouped_topk_with_one_group():
+    """Reading R9 against vLLM's router for this model family (exaone_moe:
+    grouped top-k, sigmoid scores, e_score_correction_bias, renormalised,
+    routed_scaling_factor), in its CPU form with one expert group, i.e.
+    without group-limited routing: the bias only selects, the weights are the
+    unbiased sigmoids renormalised over the k chosen, then scaled.  The
+    sigmoid and the sum order differ (torch.sigmoid, torch.sum), so the chosen
+    sets are compared where the k-th and (k+1)-th biased scores are apart, and
+    the weights to a few ulps."""
+    cpu_moe = pytest.importorskip("vllm.model_executor.layers.fused_moe.cpu_fused_moe")
+    from oracle import moe
+    T, E, k, rsf = 512, 80, 8, 2.5
+    rng = np.random.default_rng(5)
+    logits = rng.normal(0, 1.5, (T, E)).astype(np.float32)
+    bias = rng.normal(0, 0.01, E).astype(np.float32)
+    w_lib, idx_lib = cpu_moe.grouped_topk(torch.zeros(T, 1), torch.from_numpy(logits), k, True, num_expert_group=1,
+                                          topk_group=1, scoring_func="sigmoid", routed_scaling_factor=rsf,
+                                          e_score_correction_bias=torch.from_numpy(bias))
+    idx, w = moe.route(logits, bias, k, rsf)
+    c = np.sort(moe.sigmoid_f32(logits).astype(np.float64) + bias, axis=1)[:, ::-1]
+    apart = (c[:, k - 1] - c[:, k]) > 1e-5
+    assert apart.mean() > 0.95
+    lib_i, lib_w = idx_lib.numpy(), w_lib.numpy()
+    for t in np.nonzero(apart)[0]:
+        o_l, o_m = np.argsort(lib_i[t]), np.argsort(idx[t])
+        np.testing.assert_array_equal(lib_i[t][o_l], idx[t][o_m])
+        np.testing.assert_allclose(lib_w[t][o_l], w[t][o_m], rtol=2e-6)
+    # our slots come in descending order of the biased score
+    sel = np.take_along_axis(moe.sigmoid_f32(logits).astype(np.float64) + bias, idx.astype(np.int64), axis=1)
+    assert np.all(np.diff(sel, axis=1) <= 0)
