@@ -469,7 +469,9 @@ __global__ void __launch_bounds__(kChunk) perm_scatter_kernel(const int32_t* __r
 // the selection key) are computed one (token, expert) per thread and kept in
 // shared memory, so a token's warp only runs the selection rounds.  The
 // arithmetic is the same as topk_token's (expert_score, select_topk) and so
-// is every integer result.
+// is every integer result.  For small layers (route_fuses_x_quantise) the
+// kernel also quantises x and writes it to the permuted rows, the work of the
+// layer's quantise-scatter kernel, with the same bits.
 // ---------------------------------------------------------------------------
 constexpr int kSmallT = 256;
 constexpr int kSmallThreads = 1024;
