@@ -86,3 +86,18 @@ def test_host_side_argument_checks():
     assert lib.moe_nvfp4_forward(ctypes.byref(W), fake, 4, fake, fake, None, fake, None, fake, 1 << 30, None) == 2
     W = c.MoeWeightsStruct(8, 256, 256, 2, 2.5, *([fake] * 11), None, None, None, 0, 2)
     assert lib.moe_nvfp4_forward(ctypes.byref(W), fake, 4, fake, fake, None, fake, None, fake, 16, None) == 5
+
+
+@pytest.mark.parametrize("header", ["nvfp4_moe.h", "nvfp4_moe_testing.h"])
+@pytest.mark.parametrize("lang", [("c", "-std=c99"), ("c++", "-std=c++17")])
+def test_headers_compile_as_plain_c_and_cpp(header, lang):
+    """The boundary is a C ABI: its headers need no CUDA or torch headers and
+    compile warning-free as C99 and as C++17."""
+    import os
+    import shutil
+    cc = shutil.which("gcc" if lang[0] == "c" else "g++")
+    if cc is None:
+        pytest.skip("no host compiler")
+    r = subprocess.run([cc, "-fsyntax-only", lang[1], "-Wall", "-Wextra", "-Werror", "-x", lang[0],
+                        os.path.join(ROOT, "include", header)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
