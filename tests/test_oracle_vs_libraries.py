@@ -217,3 +217,41 @@ def test_routing_matches_vllms_grouped_topk_with_one_group():
     # our slots come in descending order of the biased score
     sel = np.take_along_axis(moe.sigmoid_f32(logits).astype(np.float64) + bias, idx.astype(np.int64), axis=1)
     assert np.all(np.diff(sel, axis=1) <= 0)
+
+
+def test_layer_composition_matches_vllms_cpu_moe(monkeypatch):
+    """The layer's composition (readings R10, R12) against vLLM's plain-torch
+    MoE loop (cpu_fused_moe_torch), both in fp64 and without quantisation:
+    gate rows before up rows in the fused gate/up projection, SiLU of the gate
+    half times the up half, the down projection, then each expert output
+    times its routing weight, summed over the k slots.  The routing itself is
+    the oracle's, pinned separately."""
+    cm = pytest.importorskip("vllm.model_executor.layers.fused_moe.cpu_fused_moe")
+    from vllm.model_executor.layers.activation import SiluAndMul
+    from vllm.model_executor.layers.fused_moe.activation import MoEActivation
+    from oracle import moe
+    # the library's own SiLU-and-mul, called without building a vLLM config
+    monkeypatch.setitem(cm._CPU_MOE_ACT_FN, MoEActivation.SILU, SiluAndMul.forward_native)
+    rng = np.random.default_rng(3)
+    T, H, I, E, k, rsf = 24, 64, 32, 6, 2, 2.5
+    x = rng.normal(0, 1, (T, H)).astype(np.float32)
+    wg = rng.normal(0, 0.3, (E, H)).astype(np.float32)
+    bias = rng.normal(0, 0.01, E).astype(np.float32)
+    gate, up, down = rng.normal(0, 0.1, (E, I, H)), rng.normal(0, 0.1, (E, I, H)), rng.normal(0, 0.1, (E, H, I))
+    dense = moe.dense_moe_layer(x, wg, bias, k, rsf, lambda e: (gate[e], up[e], down[e]))
+    idx, w = moe.route(moe.router_logits(x, wg), bias, k, rsf)
+
+    class Experts:                       # what the vLLM loop reads from its layer
+        gate_up_linear = [(lambda t, m=torch.from_numpy(np.concatenate([gate[e], up[e]])): t @ m.T) for e in range(E)]
+        down_linear = [(lambda t, m=torch.from_numpy(down[e]): t @ m.T) for e in range(E)]
+
+    layer = Experts()
+    key = id(layer)
+    monkeypatch.setitem(cm._CPU_MOE_LAYER_CACHE, key, lambda: layer)
+    out = torch.zeros(T, H, dtype=torch.float64)
+    cm.cpu_fused_moe_torch(key, out, torch.from_numpy(x.astype(np.float64)), torch.from_numpy(w.astype(np.float64)),
+                           torch.from_numpy(idx.astype(np.int64)), "silu", global_num_experts=E)
+    np.testing.assert_allclose(out.numpy(), dense, rtol=1e-12, atol=1e-12 * np.abs(dense).max())
+    # a swapped gate/up order would not agree
+    swapped = moe.dense_moe_layer(x, wg, bias, k, rsf, lambda e: (up[e], gate[e], down[e]))
+    assert np.abs(out.numpy() - swapped).max() > 1e-3 * np.abs(dense).max()
