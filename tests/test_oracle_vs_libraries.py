@@ -255,3 +255,28 @@ def test_layer_composition_matches_vllms_cpu_moe(monkeypatch):
     # a swapped gate/up order would not agree
     swapped = moe.dense_moe_layer(x, wg, bias, k, rsf, lambda e: (up[e], gate[e], down[e]))
     assert np.abs(out.numpy() - swapped).max() > 1e-3 * np.abs(dense).max()
+
+
+def test_dequantisation_matches_vllms_dequantiser_on_tiled_scales():
+    """vLLM's dequantiser, given the oracle's packed codes, its scales in this
+    library's tiled layout and the oracle's g, returns the oracle's
+    dequantised values: low nibble first, sign in bit 3, the tiled layout
+    undone by vLLM's own un-swizzle, x = E2M1 * E4M3 * g.  The two orders of
+    the products (here (v*s)*g, exact in its first step; there v*(s*g)) can
+    differ by one ulp, only when v is not a power of two (1.5, 3 or 6)."""
+    ref = pytest.importorskip("vllm.model_executor.layers.quantization.utils.nvfp4_emulation_utils")
+    from _util import tiled_index
+    w = _weights(11, rows=200, cols=512).float().numpy()          # ragged: 200 rows, 2 row tiles
+    codes, scales, g = nvfp4.quantize_weight(w)
+    rows_padded = 256
+    tiled = np.zeros(rows_padded * scales.shape[1], np.uint8)
+    tiled[tiled_index(rows_padded, 512)[:200].reshape(-1)] = scales.reshape(-1)
+    got = ref.dequantize_to_dtype(torch.from_numpy(codes), torch.from_numpy(tiled), torch.tensor(float(g)),
+                                  torch.float32, 16, swizzle=True).numpy()
+    ours = nvfp4.dequantize(codes, scales, g)
+    assert got.shape == ours.shape
+    vals, _ = _values(codes)
+    exact = ~np.isin(np.abs(vals), (1.5, 3.0, 6.0))
+    np.testing.assert_array_equal(got[exact], ours[exact])
+    ulp = np.spacing(np.abs(ours[~exact]).astype(np.float32))
+    assert np.all(np.abs(got[~exact] - ours[~exact]) <= ulp)
