@@ -79,7 +79,9 @@ class Dist:
     over gloo for the multi-process tests.  Only a barrier and a max of the
     ranks' times cross ranks; the layer itself has no collective."""
 
-    def __init__(self, backend: str | None = None):
+    def __init__(self, backend: str | None = None, timeout_s: float = 300.0):
+        """timeout_s bounds every collective: a rank whose peer died or stopped
+        answering gets an error instead of waiting for good."""
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -93,7 +95,7 @@ class Dist:
             import datetime
             import torch.distributed as dist
             kw = {"device_id": torch.device("cuda", self.local)} if backend == "nccl" else {}
-            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300), **kw)
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
             self.pg = dist
 
     def barrier(self):

@@ -55,3 +55,47 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch):
     class A:
         steps, warmup, seed = 1, 1, 0
     assert bench.run_reference(A(), bench.workloads.CONFIGS["tiny"]) == 0
+
+
+def _failing_rank_main(rank, world, port, q, mode):
+    import sys
+    import time
+    sys.path.insert(0, ROOT)
+    os.environ.update(RANK=str(rank), LOCAL_RANK=str(rank), WORLD_SIZE=str(world), MASTER_ADDR="127.0.0.1",
+                      MASTER_PORT=str(port))
+    import bench
+    d = bench.Dist(backend="gloo", timeout_s=5)
+    if rank == 1:
+        if mode == "exit":
+            os._exit(0)                  # dies between steps, with nothing in flight
+        time.sleep(60)                   # alive but never reaches the barrier
+        return
+    t0 = time.time()
+    try:
+        d.barrier()
+        d.max(1.0)
+        q.put(("no error", time.time() - t0))
+    except Exception as e:              # the surviving rank learns of it on the host
+        q.put((type(e).__name__, time.time() - t0))
+
+
+@pytest.mark.parametrize("mode", ["exit", "silent"])
+def test_a_lost_rank_ends_the_others_collectives_with_an_error(mode):
+    """A rank that exits, or that stops answering, makes the other rank's next
+    collective raise within the process group's timeout instead of waiting for
+    good (host-side failure detection; no GPU involved)."""
+    port = _free_port()
+    ctx = tmp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_failing_rank_main, args=(r, 2, port, q, mode)) for r in range(2)]
+    for p in procs:
+        p.start()
+    try:
+        what, waited = q.get(timeout=90)
+    finally:
+        for p in procs:
+            if p.is_alive():
+                p.terminate()
+            p.join(timeout=30)
+    assert what != "no error"
+    assert waited < 60
