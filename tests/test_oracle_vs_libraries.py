@@ -1,28 +1,34 @@
-"""The oracle's NVFP4 readings against two library implementations of the
-format, on CPU.
+"""The oracle's readings against the libraries the pages name, on CPU.
 
 The NVFP4 model card ("K-EXAONE-152B-A23B-REAP-80E-NVFP4", "Quantization
 Setup") quantises its weights with llmcompressor's NVFP4 scheme, stored in the
 compressed-tensors format, and serves the checkpoint with vLLM.  Both
-libraries are in this image and hold plain-PyTorch references of the format:
-compressed-tensors' weight quantisation (global scale 2688/amax, block scale
-amax/6 times it, elements divided by block/global) and vLLM's activation
-reference (block scale global * (amax * 1/6), elements multiplied by the
-reciprocal of block/global).
+libraries are in this image with plain-PyTorch references:
+- compressed-tensors' weight quantisation: global scale 2688/amax, block
+  scale amax/6 times it, elements divided by block/global;
+- vLLM's activation reference: block scale global * (amax * 1/6), elements
+  multiplied by the reciprocal of block/global.
+vLLM also provides its block-scale swizzle and dequantiser, its grouped top-k
+router and its plain-torch MoE loop.
 
-What agrees, exactly: the element format (E2M1 magnitudes, round to nearest
-with ties to the even code, saturation at 6, the sign of a negative that
-rounds to zero; the libraries' own E2M1 casts are compared value by value),
-the block-scale format (E4M3,
-round to nearest even, at most 448), the global scale (the libraries store the
-reciprocal of this library's g), and, with vLLM, a zero scale for an all-zero
-block.  What differs is the order of the fp32 roundings (reading R2 of the
-design notes): it only shows where the exact value sits on a rounding
-midpoint, and then the two results are neighbouring codes.  These tests pin
-exactly that, and two small convention differences: compressed-tensors gives
-an all-zero block the E4M3 scale eps (0.125) where this library gives 0
-(reading R7), and an input of exactly -0.0 becomes +0 in the libraries, -0
-here (reading R5).
+Exact agreement, pinned here:
+- the E2M1 rounding: the libraries' own casts, value by value (ties to the
+  even code, saturation at 6, a negative that rounds to zero stays -0);
+- the E4M3 scale rounding;
+- the global scale, which the libraries store inverted;
+- the packed codes and nibble order;
+- the tiled scale layout, which is vLLM's swizzled layout;
+- a zero scale for an all-zero block in vLLM;
+- the router's choices and weights (to a few ulps);
+- the layer's composition.
+
+What differs is the order of the fp32 roundings (reading R2).  It shows only
+where the exact value sits on a rounding midpoint, and the two results are
+then neighbouring codes.  There are also two small convention differences:
+- compressed-tensors gives an all-zero block the E4M3 scale eps (0.125), where
+  this library gives 0 (reading R7);
+- an input of exactly -0.0 becomes +0 in the libraries and -0 here
+  (reading R5).
 """
 import numpy as np
 import pytest
