@@ -126,18 +126,29 @@ NVFP4_API nvfp4_status nvfp4_quantize_weights(const void* w_bf16, int n_mats, in
  * which every GPU that loads the library keeps until the process exits.
  *   - At most 1024 matrices per call; more returns
  *     NVFP4_ERR_UNSUPPORTED_SHAPE (split the call or use the workspace form).
- *   - The first call on a device looks up the array's device address (once,
- *     with that device current); make that first call before any stream
- *     capture on the device.
+ *   - Every call looks up the array's device address in the current context
+ *     (a host-side query, no allocation).  The first call in a context may
+ *     also load the library's device code there, so make it before any
+ *     stream capture on that device.
  *   - Every call shares the one array and clears it when it starts, so calls
  *     whose work overlaps on the GPU (different streams, or different host
  *     threads on one device) race; serialise them on one stream.
- *   - A device-side wait that gives up leaves no status word to read: the
- *     outputs are then undefined, as with the workspace form.
+ *   - A device-side wait that gives up sets the status word at the start of
+ *     the array: read it with nvfp4_quantize_weights_noalloc_status() before
+ *     the next call, which clears it.  The outputs of that call are then
+ *     undefined, as with the workspace form.
  * Arguments, layouts and results are those of nvfp4_quantize_weights. */
 NVFP4_API nvfp4_status nvfp4_quantize_weights_noalloc(const void* w_bf16, int n_mats, int rows, int cols,
                                                       int layout, uint8_t* codes, uint8_t* scales,
                                                       float* global_scale, void* stream);
+
+/* The status of the last nvfp4_quantize_weights_noalloc call on the current
+ * device, the counterpart of nvfp4_workspace_status for the built-in array
+ * (no counterpart on the pages either).  Synchronises `stream` (the stream
+ * that call used), then reads the status word: NVFP4_OK, or
+ * NVFP4_ERR_TIMEOUT if a device-side wait of that call gave up, in which case
+ * the word is reset to 0.  Allocates nothing. */
+NVFP4_API nvfp4_status nvfp4_quantize_weights_noalloc_status(void* stream);
 
 /* ------------------------------------------------------------------------
  * Dynamic activation quantiser ("Quantization Setup": activations dynamically

@@ -76,6 +76,7 @@ _declare("nvfp4_workspace_status", _i, _vp, _vp)
 _declare("nvfp4_quantize_weights_workspace_size", _sz, _i)
 _declare("nvfp4_quantize_weights", _i, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp)
 _declare("nvfp4_quantize_weights_noalloc", _i, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp)
+_declare("nvfp4_quantize_weights_noalloc_status", _i, _vp)
 _declare("nvfp4_quantize_act", _i, _vp, _i, _i, _vp, _i, _vp, _vp, _vp)
 _declare("moe_route_rows_capacity", _i, _i, _i, _i)
 _declare("moe_route_workspace_size", _sz, _i, _i, _i)
@@ -104,7 +105,7 @@ _declare("nvfp4_test_mma_peak", _i, _i, _i, _i, _i, _vp, _vp, _vp)
 # Every symbol the public headers declare (checked by the CPU test suite).
 EXPORTS = ("nvfp4_last_error", "nvfp4_abi_version", "nvfp4_workspace_status",
            "nvfp4_quantize_weights_workspace_size", "nvfp4_quantize_weights", "nvfp4_quantize_weights_noalloc",
-           "nvfp4_quantize_act",
+           "nvfp4_quantize_weights_noalloc_status", "nvfp4_quantize_act",
            "moe_route_rows_capacity", "moe_route_workspace_size", "moe_route", "moe_nvfp4_workspace_size",
            "moe_nvfp4_forward", "moe_nvfp4_forward_scaled", "moe_nvfp4_workspace_size_shared",
            "moe_nvfp4_forward_launches",
@@ -201,9 +202,26 @@ def nvfp4_quantize_weights_noalloc(w: torch.Tensor, layout: str = "tiled", out=N
         gscale = torch.empty(n, dtype=torch.float32, device=w.device)
     else:
         codes, scales, gscale = out
+        _cuda(codes, torch.uint8, "codes")
+        _cuda(scales, torch.uint8, "scales")
+        _cuda(gscale, torch.float32, "gscale")
+        need_scales = tiled_scale_bytes(n * rows, cols) if lay != LAYOUT_CANONICAL else n * rows * (cols // 16)
+        for t, name, need in ((codes, "codes", n * rows * (cols // 2)), (scales, "scales", need_scales),
+                              (gscale, "gscale", n)):
+            if t.device != w.device:
+                raise ValueError(f"{name} must be on {w.device}, got {t.device}")
+            if t.numel() < need:
+                raise ValueError(f"{name} holds {t.numel()} elements; this call writes {need}")
     _check(lib.nvfp4_quantize_weights_noalloc(_p(w), n, rows, cols, lay, _p(codes), _p(scales), _p(gscale),
                                               _stream()))
     return codes, scales, gscale
+
+
+def nvfp4_quantize_weights_noalloc_status():
+    """Raises Nvfp4Error(TIMEOUT) if a device-side wait of the last
+    nvfp4_quantize_weights_noalloc call on this device gave up; synchronises
+    the current stream."""
+    _check(lib.nvfp4_quantize_weights_noalloc_status(_stream()))
 
 
 def nvfp4_quantize_act(x: torch.Tensor, gscale: torch.Tensor, layout: str = "canonical"):

@@ -583,21 +583,15 @@ constexpr size_t kStaticScratchBytes = 256 + 2 * 4 * kStaticMaxMats;   // state,
 
 static __device__ __align__(256) uint8_t g_weight_quant_scratch[kStaticScratchBytes];
 
-// Device address of the scratch array, looked up once per device (the host
-// symbol is only a stand-in and must never be passed to a kernel).
+// Device address of the scratch array in the current context.  The host
+// symbol is only a stand-in and must never be passed to a kernel.  A
+// __device__ array's address belongs to a CUDA context, not to a device (a
+// host may switch between its own contexts on one device, or reset the
+// device), so it is looked up on every call: a cheap host-side query.
 static nvfp4_status static_scratch_address(uint8_t** out) {
-  static std::mutex mu;
-  static uint8_t* addr[64] = {};
-  int dev = 0;
-  NV_CHECK(check_cuda(cudaGetDevice(&dev), "cudaGetDevice"));
-  NV_REQUIRE(dev >= 0 && dev < 64, NVFP4_ERR_DEVICE, "device index %d out of range", dev);
-  std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
-    void* p = nullptr;
-    NV_CHECK(check_cuda(cudaGetSymbolAddress(&p, g_weight_quant_scratch), "cudaGetSymbolAddress"));
-    addr[dev] = static_cast<uint8_t*>(p);
-  }
-  *out = addr[dev];
+  void* p = nullptr;
+  NV_CHECK(check_cuda(cudaGetSymbolAddress(&p, g_weight_quant_scratch), "cudaGetSymbolAddress"));
+  *out = static_cast<uint8_t*>(p);
   return NVFP4_OK;
 }
 
@@ -635,4 +629,22 @@ extern "C" nvfp4_status nvfp4_quantize_weights_noalloc(const void* w_bf16, int n
   NV_CHECK(check_cuda(cudaMemsetAsync(scratch, 0, c.size(), s), "cudaMemsetAsync(static scratch)"));
   return launch_weight_quantiser(w_bf16, n_mats, rows, cols, layout, codes, scales, global_scale, st, amax, done,
                                  sms, s);
+}
+
+extern "C" nvfp4_status nvfp4_quantize_weights_noalloc_status(void* stream) {
+  using namespace nvfp4moe;
+  uint8_t* scratch = nullptr;
+  NV_CHECK(static_scratch_address(&scratch));
+  // the status word is the first word of the scratch array (WeightQuantState)
+  uint32_t word = 0;
+  cudaStream_t s = as_stream(stream);
+  NV_CHECK(check_cuda(cudaMemcpyAsync(&word, scratch, sizeof(word), cudaMemcpyDeviceToHost, s), "read status"));
+  NV_CHECK(check_cuda(cudaStreamSynchronize(s), "cudaStreamSynchronize"));
+  if (word != 0) {
+    NV_CHECK(check_cuda(cudaMemsetAsync(scratch, 0, sizeof(word), s), "reset status"));
+    NV_CHECK(check_cuda(cudaStreamSynchronize(s), "cudaStreamSynchronize"));
+    return set_error(NVFP4_ERR_TIMEOUT, "nvfp4_quantize_weights_noalloc: a device-side wait gave up (status word %u)",
+                     word);
+  }
+  return NVFP4_OK;
 }

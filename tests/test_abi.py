@@ -23,7 +23,7 @@ def test_library_exports_every_declared_function():
 
 def test_abi_version_and_sizes():
     c = capi()
-    assert c.abi_version() == 4
+    assert c.abi_version() == 5
     assert c.moe_route_rows_capacity(8192, 80, 8) == 75776
     assert c.moe_route_rows_capacity(16, 80, 8) % 128 == 0
     assert c.lib.moe_nvfp4_workspace_size(16, 80, 6144, 2048, 8) > 0
