@@ -255,7 +255,23 @@ typedef struct moe_nvfp4_debug {
    * calibration batches, then divide.  Deterministic: fixed reduction order. */
   double* saliency_sum;
   unsigned long long* saliency_count;
+  /* cudaEvent_t (nullable): recorded on `stream` after the shared expert's
+   * GEMMs, when the layer has a shared expert (they run between stage events
+   * 4 and 5, before the combine). */
+  void* shared_event;
 } moe_nvfp4_debug;
+
+/* REAP expert retention ("K-EXAONE-152B-A23B-REAP-80E-BF16" card, "Pruning
+ * Setup": the routed experts with the lowest saliency are dropped, and the
+ * router's gate.weight and e_score_correction_bias are sliced to the ones
+ * kept).  From the accumulators of moe_nvfp4_debug (device, [E] each): the
+ * mean saliency of expert e is saliency_sum[e] / saliency_count[e] in IEEE
+ * fp64 (0 for an expert never routed); the `keep` experts with the highest
+ * means are retained, ties to the lower index, and keep_idx[0..keep) (device
+ * int32) receives their indices in increasing order.  Needs 1 <= E <= 256,
+ * 0 <= keep <= E. */
+NVFP4_API nvfp4_status moe_reap_keep(const double* saliency_sum, const unsigned long long* saliency_count, int E,
+                                     int keep, int32_t* keep_idx, void* stream);
 
 NVFP4_API size_t moe_nvfp4_workspace_size(int T, int E, int H, int I, int k);
 /* The same with a shared expert of intermediate size I_shared (0: none). */

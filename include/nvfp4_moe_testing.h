@@ -58,6 +58,20 @@ NVFP4_API nvfp4_status nvfp4_test_e4m3(const float* s, int n, uint8_t* codes, fl
 NVFP4_API nvfp4_status nvfp4_test_mma_peak(int iters, int n, int with_cp, int ctas, unsigned long long* cycles,
                                            uint32_t* status, void* stream);
 
+/* Makes a bounded device wait run out, to test the give-up path that every
+ * wait of the library shares (no counterpart on the pages: it checks the
+ * status-word contract of nvfp4_moe.h).  One CTA issues a 4 KiB bulk copy
+ * from src (device, 16-byte aligned) and allocates tensor memory, then waits
+ * on a barrier that nothing completes, with the library's bounded wait and
+ * the limit limit_ns (0 < limit_ns <= 1e9).  When the wait gives up it sets
+ * the status word at the start of `ws` (read it with
+ * nvfp4_workspace_status), lets the copy land, drains its tensor-core work
+ * and frees the tensor memory.  elapsed_ns[0] (device) receives how long the
+ * limited wait lasted, elapsed_ns[1] how long a second warp waited before it
+ * saw the abort flag; *copied (device) the XOR of the 1024 copied words. */
+NVFP4_API nvfp4_status nvfp4_test_wait_timeout(const void* src, uint64_t limit_ns, void* ws, size_t ws_bytes,
+                                               unsigned long long* elapsed_ns, uint32_t* copied, void* stream);
+
 /* out[i] = the router's fp32 sigmoid of l[i]. */
 NVFP4_API nvfp4_status nvfp4_test_sigmoid(const float* l, int n, float* out, void* stream);
 

@@ -60,7 +60,7 @@ N_STAGE_EVENTS = 6
 
 class MoeDebugStruct(ctypes.Structure):
     _fields_ = ([(n, _vp) for n in DEBUG_FIELDS] + [("stage_events", _vp * N_STAGE_EVENTS)] +
-                [("saliency_sum", _vp), ("saliency_count", _vp)])
+                [("saliency_sum", _vp), ("saliency_count", _vp), ("shared_event", _vp)])
 
 
 def _declare(name, restype, *argtypes):
@@ -90,6 +90,7 @@ _declare("moe_nvfp4_forward", _i, ctypes.POINTER(MoeWeightsStruct), _vp, _i, _vp
 _declare("moe_nvfp4_forward_scaled", _i, ctypes.POINTER(MoeWeightsStruct), _vp, _i, _i, _vp, _vp, _vp, _vp,
          ctypes.POINTER(MoeDebugStruct), _vp, _sz, _vp)
 _declare("moe_nvfp4_gemm_workspace_size", _sz, _i)
+_declare("moe_reap_keep", _i, _vp, _vp, _i, _i, _vp, _vp)
 _declare("moe_nvfp4_gate_up", _i, ctypes.POINTER(MoeWeightsStruct), _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp,
          _vp, _vp, _vp, _sz, _vp)
 _declare("moe_nvfp4_down", _i, ctypes.POINTER(MoeWeightsStruct), _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp,
@@ -101,6 +102,7 @@ _declare("nvfp4_test_e2m1_sweep", _i, ctypes.c_uint32, ctypes.c_uint64, _vp, _vp
 _declare("nvfp4_test_e4m3", _i, _vp, _i, _vp, _vp, _vp)
 _declare("nvfp4_test_sigmoid", _i, _vp, _i, _vp, _vp)
 _declare("nvfp4_test_mma_peak", _i, _i, _i, _i, _i, _vp, _vp, _vp)
+_declare("nvfp4_test_wait_timeout", _i, _vp, ctypes.c_uint64, _vp, _sz, _vp, _vp, _vp)
 
 # Every symbol the public headers declare (checked by the CPU test suite).
 EXPORTS = ("nvfp4_last_error", "nvfp4_abi_version", "nvfp4_workspace_status",
@@ -110,10 +112,10 @@ EXPORTS = ("nvfp4_last_error", "nvfp4_abi_version", "nvfp4_workspace_status",
            "moe_nvfp4_forward", "moe_nvfp4_forward_scaled", "moe_nvfp4_workspace_size_shared",
            "moe_nvfp4_forward_launches",
            "moe_nvfp4_gemm_workspace_size", "moe_nvfp4_gate_up",
-           "moe_nvfp4_down",
+           "moe_nvfp4_down", "moe_reap_keep",
            "nvfp4_block_stats_compute",
            "nvfp4_test_e2m1", "nvfp4_test_e2m1_sweep", "nvfp4_test_e4m3", "nvfp4_test_sigmoid",
-           "nvfp4_test_mma_peak")
+           "nvfp4_test_mma_peak", "nvfp4_test_wait_timeout")
 
 
 def _check(status: int):
@@ -165,19 +167,39 @@ def moe_route_rows_capacity(T: int, E: int, k: int) -> int:
 # quantisers
 # ---------------------------------------------------------------------------
 
-def nvfp4_quantize_weights(w: torch.Tensor, layout: str = "tiled", workspace: torch.Tensor | None = None):
-    """w [n_mats, rows, cols] bf16 -> (codes [n, rows, cols/2] u8, scales u8, gscale [n] f32)."""
+def _weight_outputs(w: torch.Tensor, lay: int, out):
+    """(codes, scales, gscale) for n_mats [rows, cols] matrices: allocated
+    with torch, or the caller's ``out``, checked for device, dtype and size."""
+    n, rows, cols = w.shape
+    need_scales = tiled_scale_bytes(n * rows, cols) if lay != LAYOUT_CANONICAL else n * rows * (cols // 16)
+    if out is None:
+        codes = torch.empty((n, rows, cols // 2), dtype=torch.uint8, device=w.device)
+        scales = (torch.empty(need_scales, dtype=torch.uint8, device=w.device) if lay != LAYOUT_CANONICAL
+                  else torch.empty((n, rows, cols // 16), dtype=torch.uint8, device=w.device))
+        return codes, scales, torch.empty(n, dtype=torch.float32, device=w.device)
+    codes, scales, gscale = out
+    _cuda(codes, torch.uint8, "codes")
+    _cuda(scales, torch.uint8, "scales")
+    _cuda(gscale, torch.float32, "gscale")
+    for t, name, need in ((codes, "codes", n * rows * (cols // 2)), (scales, "scales", need_scales),
+                          (gscale, "gscale", n)):
+        if t.device != w.device:
+            raise ValueError(f"{name} must be on {w.device}, got {t.device}")
+        if t.numel() < need:
+            raise ValueError(f"{name} holds {t.numel()} elements; this call writes {need}")
+    return codes, scales, gscale
+
+
+def nvfp4_quantize_weights(w: torch.Tensor, layout: str = "tiled", workspace: torch.Tensor | None = None,
+                           out=None):
+    """w [n_mats, rows, cols] bf16 -> (codes [n, rows, cols/2] u8, scales u8, gscale [n] f32).
+    ``out`` = (codes, scales, gscale) to write into instead of new tensors."""
     _cuda(w, torch.bfloat16, "w")
     if w.dim() == 2:
         w = w.unsqueeze(0)
     n, rows, cols = w.shape
     lay = _LAYOUTS[layout]
-    codes = torch.empty((n, rows, cols // 2), dtype=torch.uint8, device=w.device)
-    if lay != LAYOUT_CANONICAL:
-        scales = torch.empty(tiled_scale_bytes(n * rows, cols), dtype=torch.uint8, device=w.device)
-    else:
-        scales = torch.empty((n, rows, cols // 16), dtype=torch.uint8, device=w.device)
-    gscale = torch.empty(n, dtype=torch.float32, device=w.device)
+    codes, scales, gscale = _weight_outputs(w, lay, out)
     need = lib.nvfp4_quantize_weights_workspace_size(n)
     ws = workspace if workspace is not None else _workspace(need, w.device)
     _check(lib.nvfp4_quantize_weights(_p(w), n, rows, cols, lay, _p(codes), _p(scales), _p(gscale), _p(ws),
@@ -194,24 +216,7 @@ def nvfp4_quantize_weights_noalloc(w: torch.Tensor, layout: str = "tiled", out=N
         w = w.unsqueeze(0)
     n, rows, cols = w.shape
     lay = _LAYOUTS[layout]
-    if out is None:
-        codes = torch.empty((n, rows, cols // 2), dtype=torch.uint8, device=w.device)
-        scales = (torch.empty(tiled_scale_bytes(n * rows, cols), dtype=torch.uint8, device=w.device)
-                  if lay != LAYOUT_CANONICAL else torch.empty((n, rows, cols // 16), dtype=torch.uint8,
-                                                              device=w.device))
-        gscale = torch.empty(n, dtype=torch.float32, device=w.device)
-    else:
-        codes, scales, gscale = out
-        _cuda(codes, torch.uint8, "codes")
-        _cuda(scales, torch.uint8, "scales")
-        _cuda(gscale, torch.float32, "gscale")
-        need_scales = tiled_scale_bytes(n * rows, cols) if lay != LAYOUT_CANONICAL else n * rows * (cols // 16)
-        for t, name, need in ((codes, "codes", n * rows * (cols // 2)), (scales, "scales", need_scales),
-                              (gscale, "gscale", n)):
-            if t.device != w.device:
-                raise ValueError(f"{name} must be on {w.device}, got {t.device}")
-            if t.numel() < need:
-                raise ValueError(f"{name} holds {t.numel()} elements; this call writes {need}")
+    codes, scales, gscale = _weight_outputs(w, lay, out)
     _check(lib.nvfp4_quantize_weights_noalloc(_p(w), n, rows, cols, lay, _p(codes), _p(scales), _p(gscale),
                                               _stream()))
     return codes, scales, gscale
@@ -374,17 +379,22 @@ class MoeWeights:
 
 
 def reap_keep(saliency_sum: torch.Tensor, saliency_count: torch.Tensor, keep: int) -> torch.Tensor:
-    """Experts retained by REAP pruning ("Pruning Setup": the lowest-saliency
-    routed experts are removed): the ``keep`` highest mean saliencies
-    (sum / count, 0 for an expert never routed), ties to the lower index,
-    returned in expert order."""
-    s = (saliency_sum.double().cpu() / saliency_count.cpu().clamp(min=1).double()).tolist()
-    order = sorted(range(len(s)), key=lambda e: (-s[e], e))
-    return torch.tensor(sorted(order[:keep]), dtype=torch.int64)
+    """Experts retained by REAP pruning (moe_reap_keep): the ``keep`` highest
+    mean saliencies, ties to the lower index, in expert order.  Returns their
+    indices as int64 on the host."""
+    _cuda(saliency_sum, torch.float64, "saliency sum")
+    _cuda(saliency_count, torch.int64, "saliency count")
+    E = saliency_sum.numel()
+    if saliency_count.numel() != E:
+        raise ValueError("saliency sum and count must have one entry per expert")
+    idx = torch.empty(max(int(keep), 1), dtype=torch.int32, device=saliency_sum.device)
+    _check(lib.moe_reap_keep(_p(saliency_sum), _p(saliency_count), E, int(keep), _p(idx), _stream()))
+    return idx[:keep].cpu().long()
 
 
 def select_experts(W: "MoeWeights", keep: torch.Tensor) -> "MoeWeights":
-    """The layer restricted to the experts ``keep`` (in that order): gate.weight
+    """The layer restricted to the experts ``keep`` (in that order), by byte
+    slicing only (no arithmetic): gate.weight
     rows and e_score_correction_bias sliced as the pruned checkpoint does, and
     each retained expert's codes, tiled scales and global scales copied over
     (an expert's I or H rows are whole 128-row tiles, so its scales and its
@@ -426,7 +436,7 @@ ACT_SCALE_MODES = {"tensor": 0, "expert": 1, "dynamic": 2, "dynamic_expert": 3}
 def moe_nvfp4_forward(W: MoeWeights, x: torch.Tensor, act_gscale: torch.Tensor, h_gscale: torch.Tensor,
                       logit_offset: torch.Tensor | None = None, debug: bool = False,
                       out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
-                      stage_events=None, act_scale_mode: str = "tensor", saliency=None):
+                      stage_events=None, act_scale_mode: str = "tensor", saliency=None, shared_event=None):
     """out [T, H] bf16; with debug=True also a dict of intermediate results.
     ``act_scale_mode`` is one of ACT_SCALE_MODES: in "tensor" act_gscale and
     h_gscale hold one fp32 each, in "expert" E each; in "dynamic" and
@@ -435,7 +445,9 @@ def moe_nvfp4_forward(W: MoeWeights, x: torch.Tensor, act_gscale: torch.Tensor, 
     each already recorded once (torch creates the CUDA event lazily), which
     the library records again between the stages of the layer.
     ``saliency``: optional (sum float64 [E], count int64 [E]) REAP saliency
-    accumulators on the device that the call adds this batch to."""
+    accumulators on the device that the call adds this batch to.
+    ``shared_event``: optional torch.cuda.Event (recorded once already) that
+    the library records after the shared expert's GEMMs."""
     mode = ACT_SCALE_MODES[act_scale_mode]
     if saliency is not None:
         _cuda(saliency[0], torch.float64, "saliency sum")
@@ -464,7 +476,7 @@ def moe_nvfp4_forward(W: MoeWeights, x: torch.Tensor, act_gscale: torch.Tensor, 
             "h_codes": z(cap, W.I // 2, dt=torch.uint8), "h_scales": z(tiled_scale_bytes(cap, W.I), dt=torch.uint8),
             "y": z(cap, W.H),
         }
-    if debug or stage_events is not None or saliency is not None:
+    if debug or stage_events is not None or saliency is not None or shared_event is not None:
         dbg = MoeDebugStruct()
         if saliency is not None:
             dbg.saliency_sum = saliency[0].data_ptr()
@@ -477,6 +489,10 @@ def moe_nvfp4_forward(W: MoeWeights, x: torch.Tensor, act_gscale: torch.Tensor, 
                 if not ev.cuda_event:
                     raise ValueError("stage_events must have been recorded once (so that the CUDA event exists)")
                 dbg.stage_events[i] = ev.cuda_event
+        if shared_event is not None:
+            if not shared_event.cuda_event:
+                raise ValueError("shared_event must have been recorded once (so that the CUDA event exists)")
+            dbg.shared_event = shared_event.cuda_event
         dbg_ptr = ctypes.pointer(dbg)
     ws_struct = W.struct()
     if mode == 0:
@@ -574,3 +590,17 @@ def nvfp4_test_mma_peak(iters: int, n: int = 256, with_cp: int = 0, ctas: int | 
     cyc = cycles.cpu().double()
     flops = iters * 4 * 2.0 * 128 * n * 64
     return flops / cyc, cyc
+
+
+def nvfp4_test_wait_timeout(src: torch.Tensor, limit_ns: int, workspace: torch.Tensor):
+    """Queues the kernel whose bounded wait runs out after limit_ns; returns
+    (elapsed_ns int64 [2], copied int32 [1]) device tensors.  The status word
+    at the start of ``workspace`` is set when the wait gives up."""
+    _cuda(src, torch.uint8, "src")
+    if src.numel() < 4096:
+        raise ValueError("src must hold at least 4096 bytes")
+    elapsed = torch.zeros(2, dtype=torch.int64, device=src.device)
+    copied = torch.zeros(1, dtype=torch.int32, device=src.device)
+    _check(lib.nvfp4_test_wait_timeout(_p(src), int(limit_ns), _p(workspace), workspace.numel(), _p(elapsed),
+                                       _p(copied), _stream()))
+    return elapsed, copied

@@ -244,10 +244,11 @@ NVDEV bool mbar_wait_spin(uint64_t* bar, uint32_t parity, volatile int* abort) {
 }
 
 // Wait for the phase with the given parity to complete.  Gives up (returns
-// false) after kWaitLimitNs or when *abort is set by another warp.  The
-// abort flag and the clock are looked at only every 256 polls, so a phase
-// that completes is seen without the cost of a timer read.
-NVDEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+// false) after limit_ns (kWaitLimitNs unless a test asks for less) or when
+// *abort is set by another warp.  The abort flag and the clock are looked at
+// only every 256 polls, so a phase that completes is seen without the cost
+// of a timer read.
+NVDEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   uint64_t t0 = 0;
   for (uint32_t i = 1;; ++i) {
@@ -257,7 +258,7 @@ NVDEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
       const uint64_t now = globaltimer_ns();
       if (t0 == 0) {
         t0 = now;
-      } else if (now - t0 > kWaitLimitNs) {
+      } else if (now - t0 > limit_ns) {
         return false;
       }
     }

@@ -162,6 +162,35 @@ __global__ void __launch_bounds__(kSalThreads) reap_saliency_kernel(const float*
   }
 }
 
+// REAP retention ("Pruning Setup" of the BF16 model card: the routed experts
+// with the lowest saliency are removed): the mean saliency of expert e is
+// saliency_sum[e] / saliency_count[e] (IEEE fp64 division; 0 for an expert
+// never routed), and the `keep` highest means are retained, ties to the lower
+// index, written in expert order.  One block, one thread per expert: a
+// thread's rank is the number of experts ahead of it.
+__global__ void __launch_bounds__(256) reap_keep_kernel(const double* __restrict__ saliency_sum,
+                                                        const unsigned long long* __restrict__ saliency_count, int E,
+                                                        int keep, int32_t* __restrict__ keep_idx) {
+  __shared__ double mean[256];
+  __shared__ int kept[256];
+  const int e = threadIdx.x;
+  if (e < E) {
+    const unsigned long long n = saliency_count[e];
+    mean[e] = n ? __ddiv_rn(saliency_sum[e], (double)n) : 0.0;
+  }
+  __syncthreads();
+  int rank = 0;
+  if (e < E)
+    for (int j = 0; j < E; ++j) rank += (mean[j] > mean[e]) || (mean[j] == mean[e] && j < e);
+  kept[e] = (e < E && rank < keep) ? 1 : 0;
+  __syncthreads();
+  if (kept[e]) {
+    int pos = 0;
+    for (int j = 0; j < e; ++j) pos += kept[j];
+    keep_idx[pos] = e;
+  }
+}
+
 // The shared expert's dense "grouping": one expert holding rows [0, T).
 __global__ void dense_tiles_kernel(int T, int32_t* __restrict__ tile_expert, int32_t* __restrict__ num_mtiles,
                                    int32_t* __restrict__ offsets, int32_t* __restrict__ counts) {
@@ -487,6 +516,8 @@ static nvfp4_status forward_impl(const moe_nvfp4_weights* W, const void* x_bf16,
     s2.y_bf16 = f.sh_y;
     s2.status = f.route.status;
     NV_CHECK(launch_grouped_gemm(s2, s));
+    if (dbg && dbg->shared_event)
+      NV_CHECK(check_cuda(cudaEventRecord(static_cast<cudaEvent_t>(dbg->shared_event), s), "cudaEventRecord"));
   }
 
   // 8: combine
@@ -534,4 +565,17 @@ extern "C" nvfp4_status moe_nvfp4_forward_scaled(const moe_nvfp4_weights* W, con
                                                  void* stream) {
   return forward_impl(W, x_bf16, T, act_scale_mode, act_gscale, h_gscale, logit_offset, out_bf16, dbg, ws, ws_bytes,
                       stream);
+}
+
+extern "C" nvfp4_status moe_reap_keep(const double* saliency_sum, const unsigned long long* saliency_count, int E,
+                                      int keep, int32_t* keep_idx, void* stream) {
+  NV_REQUIRE(saliency_sum && saliency_count && keep_idx, NVFP4_ERR_INVALID_ARG, "moe_reap_keep: a pointer is NULL");
+  NV_REQUIRE(E >= 1 && E <= 256 && keep >= 0 && keep <= E, NVFP4_ERR_INVALID_ARG,
+             "moe_reap_keep: needs 1 <= E <= 256 and 0 <= keep <= E (E=%d keep=%d)", E, keep);
+  NV_REQUIRE(aligned(saliency_sum, 8) && aligned(saliency_count, 8) && aligned(keep_idx, 4), NVFP4_ERR_INVALID_ARG,
+             "moe_reap_keep: misaligned pointer");
+  int sms = 0;
+  NV_CHECK(device_sm_count(&sms));
+  reap_keep_kernel<<<1, 256, 0, as_stream(stream)>>>(saliency_sum, saliency_count, E, keep, keep_idx);
+  return check_launch("reap_keep_kernel");
 }

@@ -308,6 +308,85 @@ __global__ void __launch_bounds__(128, 1) mma_peak_kernel(int iters, int n, int 
   }
 }
 
+// The give-up path that every bounded wait of the library shares, made to
+// run: one CTA sets up as the GEMMs do (a bulk copy in flight, tensor memory
+// allocated), then its producer warp waits on a barrier that nothing ever
+// completes, with the library's own bounded wait and a caller-chosen limit.
+// When the wait gives up the warp sets the abort flag and the status word and
+// lets its copy land; the MMA-side warp, waiting on the same barrier, leaves
+// on the abort flag, drains its tcgen05 work through a commit and frees the
+// tensor memory.  Nothing traps and the context stays usable.
+__global__ void __launch_bounds__(64, 1)
+    test_wait_timeout_kernel(const uint4* __restrict__ src, uint64_t limit_ns, uint32_t* status,
+                             unsigned long long* elapsed_ns, uint32_t* copied) {
+  constexpr int kWords = 256;                       // 4 KiB copied
+  __shared__ __align__(128) uint4 buf[kWords];
+  __shared__ __align__(8) uint64_t full_bar, never_bar, drain_bar;
+  __shared__ uint32_t tmem_s;
+  __shared__ int abort_s;
+  volatile int* abort_flag = &abort_s;
+  const int warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    mbar_init(&full_bar, 1);
+    mbar_init(&never_bar, 1);
+    mbar_init(&drain_bar, 1);
+    abort_s = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_s, 32);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_s;
+  const uint32_t leader = elect_one();
+  if (warp == 0) {
+    if (leader) {
+      mbar_arrive_expect_tx(&full_bar, sizeof(buf));
+      bulk_load(buf, src, sizeof(buf), &full_bar);
+    }
+    __syncwarp();
+    const uint64_t t0 = globaltimer_ns();
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(&never_bar, 0, abort_flag, limit_ns));
+    const uint64_t t1 = globaltimer_ns();
+    if (!ok && leader) {
+      *abort_flag = 1;
+      atomicExch(status, kDevTimeout);
+      elapsed_ns[0] = t1 - t0;
+      // the issued copy lands before the CTA's shared memory goes away
+      volatile int never = 0;
+      mbar_wait(&full_bar, 0, &never);
+    }
+    __syncwarp();
+  } else {
+    const uint64_t t0 = globaltimer_ns();
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(&never_bar, 0, abort_flag));
+    const uint64_t t1 = globaltimer_ns();
+    if (leader) {
+      if (!ok) elapsed_ns[1] = t1 - t0;
+      // every tcgen05 operation this lane issued completes before the
+      // tensor memory is freed
+      tc_commit(&drain_bar);
+      volatile int never = 0;
+      mbar_wait(&drain_bar, 0, &never);
+    }
+    __syncwarp();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 32);
+  }
+  if (threadIdx.x == 0) {
+    uint32_t x = 0;
+    for (int i = 0; i < kWords; ++i) x ^= buf[i].x ^ buf[i].y ^ buf[i].z ^ buf[i].w;
+    *copied = x;
+  }
+}
+
 }  // namespace nvfp4moe
 
 using namespace nvfp4moe;
@@ -363,4 +442,20 @@ extern "C" nvfp4_status nvfp4_test_sigmoid(const float* l, int n, float* out, vo
   if (n == 0) return NVFP4_OK;
   test_sigmoid_kernel<<<(n + 255) / 256, 256, 0, as_stream(stream)>>>(l, n, out);
   return check_launch("test_sigmoid_kernel");
+}
+
+extern "C" nvfp4_status nvfp4_test_wait_timeout(const void* src, uint64_t limit_ns, void* ws, size_t ws_bytes,
+                                                unsigned long long* elapsed_ns, uint32_t* copied, void* stream) {
+  NV_REQUIRE(src && ws && elapsed_ns && copied, NVFP4_ERR_INVALID_ARG, "nvfp4_test_wait_timeout: a pointer is NULL");
+  NV_REQUIRE(limit_ns > 0 && limit_ns <= 1000000000ull, NVFP4_ERR_INVALID_ARG,
+             "nvfp4_test_wait_timeout: limit_ns=%llu must be in (0, 1e9]", (unsigned long long)limit_ns);
+  NV_REQUIRE(ws_bytes >= 256 && aligned(ws, 256) && aligned(src, 16), NVFP4_ERR_WORKSPACE,
+             "nvfp4_test_wait_timeout: needs a 256-byte aligned workspace of at least 256 bytes and a 16-byte "
+             "aligned source");
+  int sms = 0;
+  NV_CHECK(device_sm_count(&sms));
+  cudaStream_t s = as_stream(stream);
+  test_wait_timeout_kernel<<<1, 64, 0, s>>>(static_cast<const uint4*>(src), limit_ns, static_cast<uint32_t*>(ws),
+                                            elapsed_ns, copied);
+  return check_launch("test_wait_timeout_kernel");
 }

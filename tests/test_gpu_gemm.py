@@ -178,3 +178,63 @@ def test_down_bf16_output_rounds_fp32_result():
     yb = c.moe_nvfp4_down(*args, out_dtype=torch.bfloat16)["y"]
     # internal consistency of the two epilogue outputs (torch does the rounding)
     np.testing.assert_array_equal(host(yb), torch.from_numpy(yf).to(torch.bfloat16).float().numpy())
+
+
+# More tiles than the GPU has SMs (148): 4 experts of 577-612 rows make 20
+# m-tiles, so the gate/up GEMM has 20 x 16 = 320 tiles and the down GEMM
+# 20 x 24 = 480.  Every persistent CTA then walks two to four tiles, which
+# exercises the stage-phase carry-over between tiles, the reuse of the tensor
+# memory accumulator and its hand-back.  Every real row is compared.
+MANY_TILES = dict(E=4, H=6144, I=2048, counts=[600, 577, 612, 590])
+
+
+def _row_rel(got, ref):
+    d = np.linalg.norm(ref.astype(np.float64), axis=1)
+    return np.linalg.norm(got.astype(np.float64) - ref, axis=1) / np.where(d > 0, d, 1.0)
+
+
+@pytest.mark.parametrize("layout", ["canonical", "staged"])
+def test_gate_up_every_row_over_many_tiles(layout):
+    require_cuda()
+    c = capi()
+    P = Problem(**MANY_TILES, seed=3)
+    assert (P.rows // 128) * (P.I // 128) > 2 * 148
+    W = P.weights(c, layout)
+    cu = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()  # noqa: E731
+    res = c.moe_nvfp4_gate_up(W, cu(P.a_codes), cu(canonical_to_tiled(P.a_scales)), cu(P.offsets), cu(P.counts),
+                              cu(np.array([P.g1])), cu(np.array([P.g2])), want_h=True)
+    h = host(res["h"])
+    hc = host(res["h_codes"])
+    hs = tiled_to_canonical(host(res["h_scales"]), P.cap, P.I)
+    flips = total = 0
+    for e, r0, n in P.segments():
+        _, _, ref_h = _oracle_gate_up(P, e, r0, n)
+        rel = _row_rel(h[r0:r0 + n], ref_h)
+        assert rel.max() <= TOL, f"expert {e}: worst row {int(rel.argmax())} rel L2 {rel.max():.3g}"
+        rc, rs = nvfp4.quantize(ref_h, P.g2)
+        flips += int(np.count_nonzero(nvfp4.unpack_codes(hc[r0:r0 + n]) != nvfp4.unpack_codes(rc)))
+        total += ref_h.size
+        # scale bytes: differ only where the row's block amax differs from the oracle's by rounding
+        assert np.count_nonzero(hs[r0:r0 + n] != rs) <= 0.001 * rs.size
+        seg_end = int(P.offsets[e + 1])
+        assert not hc[r0 + n:seg_end].any() and not hs[r0 + n:seg_end].any()
+    assert flips <= 0.001 * total, f"{flips} of {total} requantised codes differ"
+
+
+@pytest.mark.parametrize("layout", ["canonical", "staged"])
+def test_down_every_row_over_many_tiles(layout):
+    require_cuda()
+    c = capi()
+    P = Problem(**MANY_TILES, seed=4)
+    assert (P.rows // 128) * (P.H // 256) > 3 * 148
+    W = P.weights(c, layout)
+    cu = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()  # noqa: E731
+    res = c.moe_nvfp4_down(W, cu(P.h_codes), cu(canonical_to_tiled(P.h_scales)), cu(P.offsets), cu(P.counts),
+                           cu(np.array([P.g2])), cu(P.row_w), out_dtype=torch.float32)
+    y = host(res["y"])
+    for e, r0, n in P.segments():
+        dq = (P.down[0][e], P.down[1][e], P.g["down"][e])
+        ref = moe.expert_down(P.h_codes[r0:r0 + n], P.h_scales[r0:r0 + n], P.g2, dq) * P.row_w[r0:r0 + n, None]
+        rel = _row_rel(y[r0:r0 + n], ref)
+        assert rel.max() <= TOL, f"expert {e}: worst row {int(rel.argmax())} rel L2 {rel.max():.3g}"
+        assert not y[r0 + n:int(P.offsets[e + 1])].any()

@@ -80,3 +80,28 @@ def test_saliency_and_pruned_layer_match_oracle(name, cfg):
     same = np.all(host(dbgp["topk_idx"]) == refp["topk_idx"], axis=1)
     assert same.mean() >= 0.97
     assert rel_l2(host(outp)[same], refp["out"][same]) <= 1e-2
+
+
+def test_library_retention_matches_the_oracle_with_ties_and_unrouted_experts():
+    """moe_reap_keep against the oracle's reap_keep on accumulators with exact
+    ties between means (reached from different sums and counts), experts never
+    routed (mean 0) and every keep count from 0 to E."""
+    require_cuda()
+    c = capi()
+    rng = np.random.default_rng(11)
+    E = 96
+    count = rng.integers(1, 50, E).astype(np.int64)
+    total = rng.uniform(0.0, 10.0, E) * count
+    count[[3, 17, 40]] = 0
+    total[[3, 17, 40]] = 0.0
+    # ties: equal means from different (sum, count) pairs, and duplicated pairs
+    total[[5, 9, 60]] = [3.0, 6.0, 1.5]
+    count[[5, 9, 60]] = [2, 4, 1]
+    total[[70, 71]] = total[20], total[20]
+    count[[70, 71]] = count[20], count[20]
+    mean = np.where(count > 0, total / np.maximum(count, 1), 0.0)
+    st = torch.from_numpy(total).cuda()
+    ct = torch.from_numpy(count).cuda()
+    for keep_n in range(E + 1):
+        got = c.reap_keep(st, ct, keep_n).numpy()
+        np.testing.assert_array_equal(got, moe.reap_keep(mean, keep_n))

@@ -286,3 +286,68 @@ def test_dequantisation_matches_vllms_dequantiser_on_tiled_scales():
     np.testing.assert_array_equal(got[exact], ours[exact])
     ulp = np.spacing(np.abs(ours[~exact]).astype(np.float32))
     assert np.all(np.abs(got[~exact] - ours[~exact]) <= ulp)
+
+
+def test_quantised_layer_matches_vllms_cpu_moe_loop(monkeypatch):
+    """moe_layer itself (not the unquantised dense loop) against vLLM's
+    plain-torch MoE loop (cpu_fused_moe_torch).  The loop is handed the
+    oracle's own quantised expert operations: its gate/up projection
+    quantises the rows of x under g1 and runs expert_gate_up; its down
+    projection rounds h to fp32 (R11), quantises it under g2 and runs
+    expert_down.  The loop then does what the NVFP4 card's per-expert Linears
+    and the BF16 card's routing imply: it gathers each expert's tokens, takes
+    SiLU of the gate half times the up half, weights each expert's output by
+    that slot's routing weight and sums the k slots (R10, R12).  moe_layer's
+    fp64 output must equal the loop's to 1e-12.  So a slot paired with the
+    wrong weight, a dropped slot or an expert fed another expert's rows fails
+    here; the unquantised band of test_oracle_moe could not tell them apart."""
+    cm = pytest.importorskip("vllm.model_executor.layers.fused_moe.cpu_fused_moe")
+    from vllm.model_executor.layers.activation import SiluAndMul
+    from vllm.model_executor.layers.fused_moe.activation import MoEActivation
+    from oracle import moe
+    monkeypatch.setitem(cm._CPU_MOE_ACT_FN, MoEActivation.SILU, SiluAndMul.forward_native)
+    rng = np.random.default_rng(7)
+    T, H, I, E, k, rsf = 40, 128, 64, 6, 3, 2.5
+    x = torch.from_numpy(rng.normal(0, 1, (T, H)).astype(np.float32)).to(torch.bfloat16).float().numpy()
+    wg = rng.normal(0, 0.3, (E, H)).astype(np.float32)
+    bias = rng.normal(0, 0.01, E).astype(np.float32)
+    bf = lambda a: torch.from_numpy(a.astype(np.float32)).to(torch.bfloat16).float().numpy()  # noqa: E731
+    q = {e: tuple(nvfp4.quantize_weight(bf(rng.normal(0, 0.05, s))) for s in ((I, H), (I, H), (H, I)))
+         for e in range(E)}
+    g1 = np.float32(np.float32(np.abs(x).max()) / np.float32(2688))
+    g2 = np.float32(3e-4)
+    ref = moe.moe_layer(x, wg, bias, k, rsf, lambda e: q[e], g1, g2)
+    idx, w = ref["topk_idx"], ref["topk_w"]
+
+    def gate_up(e):
+        def f(t):
+            ac, asc = nvfp4.quantize(t.numpy().astype(np.float32), g1)
+            gate_v, up_v, _ = moe.expert_gate_up(ac, asc, g1, q[e][0], q[e][1])
+            return torch.from_numpy(np.concatenate([gate_v, up_v], axis=1))
+        return f
+
+    def down(e):
+        def f(h):
+            hc, hs = nvfp4.quantize(h.numpy().astype(np.float32), g2)
+            return torch.from_numpy(moe.expert_down(hc, hs, g2, q[e][2]))
+        return f
+
+    class Experts:
+        gate_up_linear = [gate_up(e) for e in range(E)]
+        down_linear = [down(e) for e in range(E)]
+
+    layer = Experts()
+    monkeypatch.setitem(cm._CPU_MOE_LAYER_CACHE, id(layer), lambda: layer)
+    out = torch.zeros(T, H, dtype=torch.float64)
+    cm.cpu_fused_moe_torch(id(layer), out, torch.from_numpy(x.astype(np.float64)),
+                           torch.from_numpy(w.astype(np.float64)), torch.from_numpy(idx.astype(np.int64)), "silu",
+                           global_num_experts=E)
+    got, want = out.numpy(), ref["out_f64"]
+    np.testing.assert_allclose(want, got, rtol=1e-12, atol=1e-12 * np.abs(got).max())
+    # the same loop with every slot given slot 0's weight is far off
+    w0 = np.repeat(w[:, :1], k, axis=1)
+    out0 = torch.zeros(T, H, dtype=torch.float64)
+    cm.cpu_fused_moe_torch(id(layer), out0, torch.from_numpy(x.astype(np.float64)),
+                           torch.from_numpy(w0.astype(np.float64)), torch.from_numpy(idx.astype(np.int64)), "silu",
+                           global_num_experts=E)
+    assert np.abs(out0.numpy() - want).max() > 1e-3 * np.abs(want).max()
