@@ -389,6 +389,80 @@ NVDEV void tmem_ld32(uint32_t taddr, uint32_t* r) {
 }
 NVDEV void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// ---------------------------------------------------------------------------
+// CTA pairs (a cluster of two CTAs sharing one tcgen05 MMA, .cta_group::2).
+// The even CTA of the pair (rank 0) is the leader: it issues the pair's
+// tensor-core copies and MMAs, which read both CTAs' shared memory and write
+// both CTAs' tensor memory at the same addresses.  No load here uses cluster
+// multicast: each CTA loads its own operands.
+// ---------------------------------------------------------------------------
+NVDEV uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Shared::cluster address of the variable at shared::cta address `addr` in
+// the CTA of cluster rank `rank`.
+NVDEV uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+// Every thread of both CTAs: release this CTA's earlier memory operations to
+// the cluster, then wait for the other CTA.
+NVDEV void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Arrive on an mbarrier of either CTA of the pair (shared::cluster address),
+// with the default CTA-scope release: the arrivals that cross to the other
+// CTA only say that tensor-memory reads have finished (tcgen05.wait::ld came
+// first), so no memory write needs to be made visible to it, and a
+// cluster-scope release would stall the thread until its earlier global
+// stores had landed.
+NVDEV void mbar_arrive_remote(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+// TMA tile load into this CTA's shared memory whose completion counts on an
+// mbarrier of either CTA of the pair (`bar`, a shared::cluster address): the
+// leader's stage barrier then covers the bytes of both CTAs.  No multicast.
+NVDEV void tma_load_2d_pair(void* dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+NVDEV void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols));
+}
+NVDEV void tmem_relinquish_pair() { asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;"); }
+NVDEV void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols));
+}
+// Arrive once on `bar` (shared::cluster address, either CTA) when every
+// earlier pair-wide tcgen05 operation of this thread is done.
+NVDEV void tc_commit_pair(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+// The pair's block-scaled FP4 MMA: D (128 rows in each CTA's tensor memory)
+// += A (each CTA's 128 rows) x B (N rows, the first N/2 from the leader's
+// shared memory, the rest from the other CTA's), scales from each CTA's
+// tensor memory.
+NVDEV void mma_fp4_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t sfa_tmem,
+                        uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::
+          "r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem));
+}
+// One scale atom from each CTA's shared memory into its own tensor memory.
+NVDEV void tc_cp_scale_atom_pair(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc));
+}
+
 // Programmatic dependent launch.  griddep_wait() blocks until the previous
 // kernel in the stream has finished and its memory is visible (a no-op for a
 // kernel launched without the attribute); griddep_launch() lets the next

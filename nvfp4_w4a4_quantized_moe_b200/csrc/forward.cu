@@ -466,6 +466,7 @@ static nvfp4_status forward_impl(const moe_nvfp4_weights* W, const void* x_bf16,
   g1.h_amax = dbg ? dbg->h_amax : nullptr;
   g1.per_expert_scales = (mode & kActPerExpert) != 0;
   g1.status = f.route.status;
+  g1.pair = T * k >= kPairMinRows;
   NV_CHECK(launch_grouped_gemm(g1, s));
   NV_CHECK(mark(dbg, 3, s));
 
@@ -485,6 +486,7 @@ static nvfp4_status forward_impl(const moe_nvfp4_weights* W, const void* x_bf16,
   const bool saliency = dbg && dbg->saliency_sum && dbg->saliency_count;
   g2.y_sq_part = saliency ? f.y_sq_part : nullptr;
   g2.status = f.route.status;
+  g2.pair = T * k >= kPairMinRows;
   NV_CHECK(launch_grouped_gemm(g2, s));
   NV_CHECK(mark(dbg, 4, s));
 

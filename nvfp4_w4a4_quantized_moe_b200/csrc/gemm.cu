@@ -43,27 +43,36 @@ constexpr int kEpiWarps = 8;
 // Operand kinds: FP4 stages hold 256 K elements (128-byte rows) plus their
 // scale atoms; bf16 stages hold 64 K elements in the same 128-byte rows and
 // no scales, so the MMA descriptors advance identically (32 bytes per MMA).
+// A CTA pair (PAIR) shares one 256 x 256 MMA: each CTA holds its own 128 A
+// rows, half of the 256 B rows and all of B's scales, 38 KiB a stage.
 template <int EPI> __host__ __device__ constexpr bool is_bf16() { return EPI >= kEpiSharedGateUp; }
 template <int EPI> __host__ __device__ constexpr bool is_gate_up() {
   return EPI == kEpiGateUp || EPI == kEpiSharedGateUp;
 }
-template <int EPI> __host__ __device__ constexpr int stage_bytes_of() {
-  return is_bf16<EPI>() ? kABytes + kBBytes : kStageBytes;
+// B rows one CTA loads per stage: all 256, or its half of the pair's tile
+template <bool PAIR> __host__ __device__ constexpr int b_rows_of() { return PAIR ? kBN / 2 : kBN; }
+template <int EPI, bool PAIR> __host__ __device__ constexpr int stage_bytes_of() {
+  return PAIR ? kABytes + b_rows_of<PAIR>() * kBKBytes + kSfaBytes + kSfbBytes
+              : (is_bf16<EPI>() ? kABytes + kBBytes : kStageBytes);
 }
 template <int EPI> __host__ __device__ constexpr int bk_of() { return is_bf16<EPI>() ? 64 : kBK; }
-// Pipeline stages: four in every kind.  The down GEMMs stage y in shared
-// memory, 32 rows x y_pass_cols_of() bf16 columns per warp at a time: 64 columns
-// (4 KiB) for the bf16 kind, 16 (1 KiB) for the FP4 kind, whose four 54 KiB
-// stages leave no room for more.
-template <int EPI> __host__ __device__ constexpr int stages_of() { return 4; }
+// Pipeline stages: four in every one-CTA kind, five for a CTA pair (38 KiB
+// a stage per CTA).  The down
+// GEMMs stage y in shared memory, 32 rows x y_pass_cols_of() bf16 columns per
+// warp at a time: 64 columns (4 KiB) for the bf16 kind, 16 (1 KiB) for the
+// FP4 kind, whose stages leave no room for more.
+template <int EPI, bool PAIR> __host__ __device__ constexpr int stages_of() { return PAIR ? 5 : 4; }
 template <int EPI> __host__ __device__ constexpr int y_pass_cols_of() { return EPI == kEpiDown ? 16 : 64; }
 template <int EPI> __host__ __device__ constexpr int y_stage_bytes_of() { return 32 * y_pass_cols_of<EPI>() * 2; }
-template <int EPI> __host__ __device__ constexpr int smem_bytes_of() {
-  return stages_of<EPI>() * stage_bytes_of<EPI>() + 1024 + (is_gate_up<EPI>() ? 0 : kEpiWarps * y_stage_bytes_of<EPI>());
+template <int EPI, bool PAIR> __host__ __device__ constexpr int smem_bytes_of() {
+  return stages_of<EPI, PAIR>() * stage_bytes_of<EPI, PAIR>() + 1024 +
+         (is_gate_up<EPI>() ? 0 : kEpiWarps * y_stage_bytes_of<EPI>());
 }
-static_assert(smem_bytes_of<kEpiDown>() <= 232448 - 256, "FP4 down GEMM shared memory");
-static_assert(smem_bytes_of<kEpiGateUp>() <= 232448 - 256, "FP4 gate/up GEMM shared memory");
-static_assert(smem_bytes_of<kEpiSharedDown>() <= 232448 - 256, "bf16 down GEMM shared memory");
+static_assert(smem_bytes_of<kEpiDown, false>() <= 232448 - 256, "FP4 down GEMM shared memory");
+static_assert(smem_bytes_of<kEpiGateUp, false>() <= 232448 - 256, "FP4 gate/up GEMM shared memory");
+static_assert(smem_bytes_of<kEpiSharedDown, false>() <= 232448 - 256, "bf16 down GEMM shared memory");
+static_assert(smem_bytes_of<kEpiDown, true>() <= 232448 - 2048, "FP4 down GEMM (CTA pair) shared memory");
+static_assert(smem_bytes_of<kEpiGateUp, true>() <= 232448 - 2048, "FP4 gate/up GEMM (CTA pair) shared memory");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCol = 0;                  // 256 fp32 accumulator columns
 // Scale factors of one stage: 4 MMA k-steps x (4 SFA + 8 SFB) columns.  The
@@ -71,6 +80,7 @@ constexpr uint32_t kAccCol = 0;                  // 256 fp32 accumulator columns
 // same 48 columns.
 constexpr uint32_t kSfCol = 256;
 constexpr uint32_t kSfaOff = 0, kSfbOff = 16;
+constexpr int kMaxExperts = 256;
 
 struct GemmParams {
   const uint8_t* a_sf;
@@ -80,6 +90,7 @@ struct GemmParams {
   int E;                // experts (tile_expert entries are clamped to [0, E))
   int Nw;               // weight rows per expert in B0 / B1
   int n_tiles;          // n-tiles per m-tile
+  int cap_tiles;        // 128-row tiles in the row capacity (CTA pairs: tiles past it are skipped)
   const int32_t* tile_expert;
   const int32_t* num_mtiles;
   const int32_t* expert_offsets;
@@ -108,24 +119,56 @@ struct GemmParams {
   uint32_t* status;
 };
 
+// Tensor maps only the CTA-pair kernel reads: the scale atoms as rows of 512
+// bytes (A's and B's; b1 is up's for gate/up), loaded by TMA so that their
+// bytes count on the leader CTA's stage barrier.
+struct PairMaps {
+  CUtensorMap sfa, sfb0, sfb1;
+};
+
 NVDEV void give_up(uint32_t* status, volatile int* abort_flag) {
   *abort_flag = 1;
   if (status) atomicExch(status, kDevTimeout);
 }
 
+// A CTA of a pair that gives up also raises the other CTA's abort flag, so
+// that its waits end at once instead of running into their own limits.
+NVDEV void give_up_pair(uint32_t* status, volatile int* abort_flag, uint32_t peer_abort_addr) {
+  give_up(status, abort_flag);
+  asm volatile("st.relaxed.cluster.shared::cluster.u32 [%0], 1;" ::"r"(peer_abort_addr) : "memory");
+}
+
 NVDEV float silu(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
+
+// A tile of the work list: its expert, its 128-row m-tile in this CTA, its
+// n-tile, and whether this CTA stores anything (the second CTA of a pair
+// whose expert has an odd number of m-tiles has no rows of its own).
+struct TileCoord {
+  int e, mt, nt;
+  bool valid;
+};
 
 template <int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA32,
-                            const __grid_constant__ CUtensorMap tmB0,
-                            const __grid_constant__ CUtensorMap tmB1, const GemmParams p) {
+                            const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
+                            const GemmParams p);
+
+// PAIR = false: one CTA per SM, each walking (m-tile, n-tile) tiles of 128 x 256.
+// PAIR = true: clusters of two CTAs; a pair walks (pair of m-tiles of one
+// expert, n-tile) tiles of 256 x 256 with one .cta_group::2 MMA per k-step.
+template <int EPI, bool PAIR>
+NVDEV void gemm_body(const CUtensorMap& tmA, const CUtensorMap& tmA32, const CUtensorMap& tmB0,
+                     const CUtensorMap& tmB1, const PairMaps* pm, const GemmParams& p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  constexpr int kStages = stages_of<EPI>();
+  constexpr int kStages = stages_of<EPI, PAIR>();
   constexpr bool kBf16 = is_bf16<EPI>();
   constexpr bool kGateUp = is_gate_up<EPI>();
-  constexpr int kSB = stage_bytes_of<EPI>();
+  constexpr int kSB = stage_bytes_of<EPI, PAIR>();
+  constexpr int kBRows = b_rows_of<PAIR>();
+  constexpr int kBLoad = kBRows * kBKBytes;                   // B bytes this CTA loads per stage
+  static_assert(!PAIR || !kBf16, "CTA pairs run the FP4 GEMMs only");
   __shared__ __align__(8) uint64_t full_bar[kStages];
   __shared__ __align__(8) uint64_t empty_bar[kStages];
   __shared__ __align__(8) uint64_t acc_full_bar;
@@ -133,16 +176,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ __align__(8) uint64_t drain_bar;
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s;
+  __shared__ int pair_start[PAIR ? kMaxExperts + 1 : 1];   // first pair m-tile of each expert
   volatile int* abort_flag = &abort_s;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
+      // pair: only the leader's producer arrives on the leader's stage
+      // barrier, expecting the bytes of both CTAs
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
     }
     mbar_init(&acc_full_bar, 1);
-    mbar_init(&acc_empty_bar, kEpiWarps);
+    // pair: the leader's accumulator is drained by both CTAs' epilogues
+    mbar_init(&acc_empty_bar, PAIR ? 2 * kEpiWarps : kEpiWarps);
     mbar_init(&drain_bar, 1);
     abort_s = 0;
     fence_barrier_init();
@@ -152,20 +201,91 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tmA32);
     prefetch_tmap(&tmB0);
     if (kGateUp) prefetch_tmap(&tmB1);
+    if constexpr (PAIR) {
+      prefetch_tmap(&pm->sfa);
+      prefetch_tmap(&pm->sfb0);
+      prefetch_tmap(&pm->sfb1);
+    }
   }
   if (warp == 1) {
-    tmem_alloc(&tmem_base_s, kTmemCols);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(&tmem_base_s, kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(&tmem_base_s, kTmemCols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR) {
+    cluster_sync_all();          // both CTAs' barriers exist before either touches the other's
+  } else {
+    __syncthreads();
+  }
   tc_fence_after();
   const uint32_t tmem = tmem_base_s;
+  // shared::cluster addresses of the leader's barriers and of the other CTA's abort flag
+  const uint32_t peer_abort = PAIR ? mapa_shared(smem_u32(&abort_s), rank ^ 1u) : 0u;
   // everything above overlaps the previous kernel; its outputs are read below
   griddep_wait();
   griddep_launch();
 
-  const int num_tiles = (*p.num_mtiles) * p.n_tiles;
+  int num_tiles;
+  if constexpr (PAIR) {
+    // pair m-tiles per expert: ceil(m-tiles / 2); exclusive prefix in shared memory
+    if (warp == 0) {
+      int carry = 0;
+      for (int e0 = 0; e0 < p.E; e0 += 32) {
+        const int e = e0 + lane;
+        int v = 0;
+        if (e < p.E) {
+          const int mt = max(0, (p.expert_offsets[e + 1] - p.expert_offsets[e]) / kBM);
+          v = (mt + 1) >> 1;
+        }
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int u = __shfl_up_sync(0xffffffffu, v, o);
+          if (lane >= o) v += u;
+        }
+        if (e < p.E) pair_start[e + 1] = carry + v;
+        carry += __shfl_sync(0xffffffffu, v, 31);
+      }
+      if (lane == 0) pair_start[0] = 0;
+    }
+    __syncthreads();
+    num_tiles = pair_start[p.E] * p.n_tiles;
+  } else {
+    num_tiles = (*p.num_mtiles) * p.n_tiles;
+  }
+  // tile t of the work list: one-CTA tiles are (m-tile, n-tile); pair tiles
+  // are (pair m-tile, n-tile), this CTA taking the pair's m-tile `rank`
+  auto tile_of = [&](int t) -> TileCoord {
+    TileCoord c;
+    c.nt = t % p.n_tiles;
+    if constexpr (PAIR) {
+      const int pmt = t / p.n_tiles;
+      int lo = 0, hi = p.E - 1;                  // the last expert whose pairs start at or before pmt
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (pair_start[mid] <= pmt) lo = mid; else hi = mid - 1;
+      }
+      c.e = lo;
+      const int j = pmt - pair_start[lo];
+      const int e_mt = (p.expert_offsets[lo + 1] - p.expert_offsets[lo]) / kBM;
+      const int first = p.expert_offsets[lo] / kBM + 2 * j;
+      c.valid = (2 * j + (int)rank < e_mt) && first + (int)rank < p.cap_tiles;
+      // a CTA without rows of its own loads the pair's first m-tile again
+      c.mt = c.valid ? first + (int)rank : min(first, p.cap_tiles - 1);
+    } else {
+      c.mt = t / p.n_tiles;
+      c.e = min(max(p.tile_expert[c.mt], 0), p.E - 1);
+      c.valid = true;
+    }
+    return c;
+  };
+  // each CTA of a pair strides over pair tiles by cluster
+  const int t_first = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int t_step = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
   const int KT = (p.K + bk_of<EPI>() - 1) / bk_of<EPI>();
   const int nblk4 = p.K / 64;                    // FP4: scale atoms per 128-row tile
 
@@ -173,16 +293,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ producer
     // The whole warp runs the loop (waits and bookkeeping stay warp-uniform);
     // one elected lane issues the copies.
-    const uint32_t leader = elect_one();
+    const uint32_t elected = elect_one();
     int stage = 0;
     uint32_t phase = 0;
     uint32_t filled = 0, fill_parity = 0;       // per stage: ever filled / parity of last fill
     bool ok = true;
     uint8_t* const st0 = smem;
     const size_t tile_sf_bytes = (size_t)nblk4 * kAtomBytes;       // one 128-row tile's scales
-    for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
-      const int mt = t / p.n_tiles, nt = t % p.n_tiles;
-      const int e = min(max(p.tile_expert[mt], 0), p.E - 1);
+    for (int t = t_first; ok && t < num_tiles; t += t_step) {
+      const TileCoord tc = tile_of(t);
+      const int e = tc.e, mt = tc.mt, nt = tc.nt;
       const int arow = mt * kBM;
       const int brow = e * p.Nw + nt * (kGateUp ? 128 : kBN);
       const uint8_t* asf = kBf16 ? nullptr : p.a_sf + (size_t)mt * tile_sf_bytes;
@@ -193,9 +313,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // A rows to load: the tile's data rows rounded up to 32-row boxes (a
       // decode tile holds a handful of tokens).  Rows past them keep stale
       // shared memory; they only feed accumulator rows the epilogue never
-      // stores.
+      // stores.  Pairs load whole tiles.
       int a_boxes = 4;
-      if (p.expert_counts) {
+      if (!PAIR && p.expert_counts) {
         const int real = p.expert_counts[e] - (arow - p.expert_offsets[e]);
         a_boxes = min(4, max(1, (real + 31) / 32));
       }
@@ -203,44 +323,79 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int kt = 0; kt < KT; ++kt) {
         ok = __all_sync(0xffffffffu, mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag));
         if (!ok) {
-          if (leader) give_up(p.status, abort_flag);
+          if (elected) {
+            if constexpr (PAIR) give_up_pair(p.status, abort_flag, peer_abort);
+            else give_up(p.status, abort_flag);
+          }
           break;
         }
-        if (leader) {
+        if (elected) {
           uint8_t* sA = st0 + stage * kSB;
           uint8_t* sB = sA + kABytes;
           // x in tensor-map elements: 128 bytes of K per stage either way
           const int x = kt * (kBf16 ? 64 : kBKBytes);
-          if (kBf16) {
-            mbar_arrive_expect_tx(&full_bar[stage], a_bytes + kBBytes);
-          } else {
-            const int katoms = min(4, (p.K - kt * kBK) / 64);
-            const uint32_t sf_bytes = (uint32_t)katoms * kAtomBytes;
-            mbar_arrive_expect_tx(&full_bar[stage], a_bytes + kBBytes + 3 * sf_bytes);
-            uint8_t* sSFA = sB + kBBytes;
+          if constexpr (PAIR) {
+            // every load of both CTAs counts on the leader's stage barrier,
+            // which the leader alone arms with the bytes of both; the other
+            // CTA's bytes may land first (the barrier's phase cannot complete
+            // before the leader's arrival)
+            const uint32_t fb = mapa_shared(smem_u32(&full_bar[stage]), 0);
+            if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2u * (uint32_t)kSB);
+            uint8_t* sSFA = sB + kBLoad;
             uint8_t* sSFB = sSFA + kSfaBytes;
-            const size_t sf_off = (size_t)kt * 4 * kAtomBytes;
-            bulk_load(sSFA, asf + sf_off, sf_bytes, &full_bar[stage]);
-            bulk_load(sSFB, bsf0 + sf_off, sf_bytes, &full_bar[stage]);
-            bulk_load(sSFB + kSfbBytes / 2, bsf1 + sf_off, sf_bytes, &full_bar[stage]);
-          }
-          if (a_boxes == 4) {
-            tma_load_2d(sA, &tmA, x, arow, &full_bar[stage]);
+            // scale atoms: rows of 512 bytes (128 32-bit words), 4 per stage
+            const int ka = kt * 4;
+            tma_load_2d_pair(sSFA, &pm->sfa, 0, mt * nblk4 + ka, fb);
+            tma_load_2d_pair(sSFB, &pm->sfb0, 0, (brow / kRowTile) * nblk4 + ka, fb);
+            if (kGateUp) {
+              tma_load_2d_pair(sSFB + kSfbBytes / 2, &pm->sfb1, 0, (brow / kRowTile) * nblk4 + ka, fb);
+            } else {
+              tma_load_2d_pair(sSFB + kSfbBytes / 2, &pm->sfb0, 0, (brow / kRowTile + 1) * nblk4 + ka, fb);
+            }
+            tma_load_2d_pair(sA, &tmA, x, arow, fb);
+            // B: gate/up - the leader loads the 128 gate rows, the other CTA
+            // the same 128 up rows; down - each CTA 128 of the 256 rows
+            const CUtensorMap* bm = (kGateUp && rank == 1) ? &tmB1 : &tmB0;
+            const int bro = kGateUp ? brow : brow + (int)rank * kRowTile;
+            if (p.b_staged) {
+              // staged tiles viewed as rows of 128 bytes: tile (row group, stage)
+              const int ks = p.K / kBK;
+              tma_load_2d_pair(sB, bm, 0, ((bro / kRowTile) * ks + kt) * kRowTile, fb);
+            } else {
+              tma_load_2d_pair(sB, bm, x, bro, fb);
+            }
           } else {
-            for (int i = 0; i < a_boxes; ++i)
-              tma_load_2d(sA + i * (kABytes / 4), &tmA32, x, arow + 32 * i, &full_bar[stage]);
-          }
-          if (!kBf16 && p.b_staged) {
-            // gate/up: the gate and up tiles of rows [brow, brow + 128);
-            // down: the tiles of rows [brow, brow + 128) and the next 128
-            const size_t ks = (size_t)(p.K / kBK);
-            const size_t t0 = ((size_t)(brow / kRowTile) * ks + kt) * kStagedTileBytes;
-            bulk_load(sB, p.b0_codes + t0, kStagedTileBytes, &full_bar[stage]);
-            bulk_load(sB + kBBytes / 2, kGateUp ? p.b1_codes + t0 : p.b0_codes + t0 + ks * kStagedTileBytes,
-                      kStagedTileBytes, &full_bar[stage]);
-          } else {
-            tma_load_2d(sB, &tmB0, x, brow, &full_bar[stage]);
-            if (kGateUp) tma_load_2d(sB + kBBytes / 2, &tmB1, x, brow, &full_bar[stage]);
+            if (kBf16) {
+              mbar_arrive_expect_tx(&full_bar[stage], a_bytes + kBBytes);
+            } else {
+              const int katoms = min(4, (p.K - kt * kBK) / 64);
+              const uint32_t sf_bytes = (uint32_t)katoms * kAtomBytes;
+              mbar_arrive_expect_tx(&full_bar[stage], a_bytes + kBBytes + 3 * sf_bytes);
+              uint8_t* sSFA = sB + kBBytes;
+              uint8_t* sSFB = sSFA + kSfaBytes;
+              const size_t sf_off = (size_t)kt * 4 * kAtomBytes;
+              bulk_load(sSFA, asf + sf_off, sf_bytes, &full_bar[stage]);
+              bulk_load(sSFB, bsf0 + sf_off, sf_bytes, &full_bar[stage]);
+              bulk_load(sSFB + kSfbBytes / 2, bsf1 + sf_off, sf_bytes, &full_bar[stage]);
+            }
+            if (a_boxes == 4) {
+              tma_load_2d(sA, &tmA, x, arow, &full_bar[stage]);
+            } else {
+              for (int i = 0; i < a_boxes; ++i)
+                tma_load_2d(sA + i * (kABytes / 4), &tmA32, x, arow + 32 * i, &full_bar[stage]);
+            }
+            if (!kBf16 && p.b_staged) {
+              // gate/up: the gate and up tiles of rows [brow, brow + 128);
+              // down: the tiles of rows [brow, brow + 128) and the next 128
+              const size_t ks = (size_t)(p.K / kBK);
+              const size_t t0 = ((size_t)(brow / kRowTile) * ks + kt) * kStagedTileBytes;
+              bulk_load(sB, p.b0_codes + t0, kStagedTileBytes, &full_bar[stage]);
+              bulk_load(sB + kBBytes / 2, kGateUp ? p.b1_codes + t0 : p.b0_codes + t0 + ks * kStagedTileBytes,
+                        kStagedTileBytes, &full_bar[stage]);
+            } else {
+              tma_load_2d(sB, &tmB0, x, brow, &full_bar[stage]);
+              if (kGateUp) tma_load_2d(sB + kBBytes / 2, &tmB1, x, brow, &full_bar[stage]);
+            }
           }
         }
         __syncwarp();
@@ -252,37 +407,47 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    if (!ok && leader) {
+    if (!PAIR && !ok && elected) {
       // let every copy already issued land before the CTA's shared memory goes away
       volatile int never = 0;
       for (int s = 0; s < kStages; ++s)
         if ((filled >> s) & 1u) mbar_wait(&full_bar[s], (fill_parity >> s) & 1u, &never);
     }
     __syncwarp();
-  } else if (warp == 1) {
+  } else if (warp == 1 && leader) {
     // ------------------------------------------------------------ MMA issuer
     // The whole warp runs the loop and one elected lane issues the tcgen05
     // instructions: a loop run by a single divergent lane issues them too
     // slowly to keep the tensor pipe busy.  Shared-memory descriptors are
     // built once; a stage only adds constant offsets to their address fields.
-    const uint32_t leader = elect_one();
-    const uint32_t idesc = kBf16 ? idesc_bf16(kBM, kBN) : idesc_fp4(kBM, kBN);
+    // In a pair only the leader's warp issues; the other CTA's warp 1 only
+    // owns its half of the tensor-memory allocation.
+    const uint32_t elected = elect_one();
+    const uint32_t idesc = kBf16 ? idesc_bf16(kBM, kBN) : idesc_fp4(PAIR ? 2 * kBM : kBM, kBN);
     const uint32_t s0 = smem_u32(smem);
     const uint64_t a0 = sdesc_sw128(s0), b0 = sdesc_sw128(s0 + kABytes);
-    const uint64_t sfa0 = sdesc_scale_atom(s0 + kABytes + kBBytes);
-    const uint64_t sfb0 = sdesc_scale_atom(s0 + kABytes + kBBytes + kSfaBytes);
+    const uint64_t sfa0 = sdesc_scale_atom(s0 + kABytes + kBLoad);
+    const uint64_t sfb0 = sdesc_scale_atom(s0 + kABytes + kBLoad + kSfaBytes);
     constexpr uint64_t kStageStep = kSB >> 4;                  // start address is in 16-byte units
     constexpr uint64_t kAtomStep = kAtomBytes >> 4;
     constexpr uint64_t kSfbHalfStep = (kSfbBytes / 2) >> 4;
     const uint32_t sfa_t = tmem + kSfCol + kSfaOff, sfb_t = tmem + kSfCol + kSfbOff;
     const uint32_t acc_t = tmem + kAccCol;
+    // pair: stage and accumulator releases go to both CTAs' barriers
+    const uint32_t empty_own = PAIR ? mapa_shared(smem_u32(&empty_bar[0]), 0) : 0u;
+    const uint32_t empty_peer = PAIR ? mapa_shared(smem_u32(&empty_bar[0]), 1) : 0u;
+    const uint32_t accf_own = PAIR ? mapa_shared(smem_u32(&acc_full_bar), 0) : 0u;
+    const uint32_t accf_peer = PAIR ? mapa_shared(smem_u32(&acc_full_bar), 1) : 0u;
     int stage = 0;
     uint32_t phase = 0, acc_phase = 0;
     bool ok = true;
-    for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
+    for (int t = t_first; ok && t < num_tiles; t += t_step) {
       ok = __all_sync(0xffffffffu, mbar_wait(&acc_empty_bar, acc_phase ^ 1u, abort_flag));
       if (!ok) {
-        if (leader) give_up(p.status, abort_flag);
+        if (elected) {
+          if constexpr (PAIR) give_up_pair(p.status, abort_flag, peer_abort);
+          else give_up(p.status, abort_flag);
+        }
         break;
       }
       tc_fence_after();
@@ -292,17 +457,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         // through; the completed barrier phase is all the ordering needed
         ok = __all_sync(0xffffffffu, mbar_wait(&full_bar[stage], phase, abort_flag));
         if (!ok) {
-          if (leader) give_up(p.status, abort_flag);
+          if (elected) {
+            if constexpr (PAIR) give_up_pair(p.status, abort_flag, peer_abort);
+            else give_up(p.status, abort_flag);
+          }
           break;
         }
         const uint64_t d = (uint64_t)stage * kStageStep;
         const int katoms = kBf16 ? 4 : min(4, (p.K - kt * kBK) / 64);
-        if (leader && kBf16) {
+        if constexpr (PAIR) {
+          if (elected) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              tc_cp_scale_atom_pair(sfa_t + 4 * j, sfa0 + d + j * kAtomStep);
+              tc_cp_scale_atom_pair(sfb_t + 8 * j, sfb0 + d + j * kAtomStep);
+              tc_cp_scale_atom_pair(sfb_t + 8 * j + 4, sfb0 + d + kSfbHalfStep + j * kAtomStep);
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              mma_fp4_pair(acc_t, a0 + d + 2 * j, b0 + d + 2 * j, idesc, sfa_t + 4 * j, sfb_t + 8 * j,
+                           accumulate | j);
+            tc_commit_pair(empty_own + 8u * stage);
+            tc_commit_pair(empty_peer + 8u * stage);
+          }
+        } else if (elected && kBf16) {
           // 4 x (K = 16 bf16 = 32 bytes) per 128-byte stage row
 #pragma unroll
           for (int j = 0; j < 4; ++j) mma_bf16(acc_t, a0 + d + 2 * j, b0 + d + 2 * j, idesc, accumulate | j);
           tc_commit(&empty_bar[stage]);
-        } else if (leader) {
+        } else if (elected) {
           if (katoms == 4) {
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -334,29 +517,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (!ok) break;
-      if (leader) tc_commit(&acc_full_bar);
+      if (elected) {
+        if constexpr (PAIR) {
+          tc_commit_pair(accf_own);
+          tc_commit_pair(accf_peer);
+        } else {
+          tc_commit(&acc_full_bar);
+        }
+      }
       __syncwarp();
       acc_phase ^= 1u;
     }
     // every MMA issued by the elected lane completes before tensor memory is freed
-    if (leader) {
-      tc_commit(&drain_bar);
+    if (elected) {
+      if constexpr (PAIR) {
+        tc_commit_pair(mapa_shared(smem_u32(&drain_bar), 0));
+      } else {
+        tc_commit(&drain_bar);
+      }
       volatile int never = 0;
       mbar_wait(&drain_bar, 0, &never);
     }
     __syncwarp();
-  } else {
+  } else if (warp >= 2) {
     // ------------------------------------------------------------ epilogue
     const int quad = warp & 3;
     const int half = (warp - 2) >> 2;
     const int row_in_tile = quad * 32 + lane;
     const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16);
+    // pair: the accumulator is handed back to the leader's MMA warp
+    const uint32_t acce_leader = PAIR ? mapa_shared(smem_u32(&acc_empty_bar), 0) : 0u;
+    const uint32_t tacc = tbase + kAccCol;
     uint32_t acc_phase = 0;
-    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
-      const int mt = t / p.n_tiles, nt = t % p.n_tiles;
-      const int e = min(max(p.tile_expert[mt], 0), p.E - 1);
+    for (int t = t_first; t < num_tiles; t += t_step) {
+      const TileCoord tc = tile_of(t);
+      const int e = tc.e, mt = tc.mt, nt = tc.nt;
       const int grow = mt * kBM + row_in_tile;
-      const bool real = p.expert_counts ? (grow - p.expert_offsets[e] < p.expert_counts[e]) : true;
+      const bool real =
+          tc.valid && (p.expert_counts ? (grow - p.expert_offsets[e] < p.expert_counts[e]) : true);
       // the tile's scalars are loaded before the accumulator is ready, so that
       // no global load sits between the accumulator-full wait and the hand-back
       const int se = p.per_expert ? e : 0;                  // index of this tile's scales
@@ -364,19 +562,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float g_b0 = kBf16 ? 1.0f : p.g_b0[e];
       const float g_b1 = kBf16 || !kGateUp ? 1.0f : p.g_b1[e];
       const float g_h = EPI == kEpiGateUp ? p.g_h[se] : 1.0f;
-      const float w_row = EPI == kEpiDown && p.row_w ? p.row_w[grow] : 1.0f;
+      const float w_row = EPI == kEpiDown && p.row_w && real ? p.row_w[grow] : 1.0f;
       if (!mbar_wait(&acc_full_bar, acc_phase, abort_flag)) {
-        give_up(p.status, abort_flag);
+        if constexpr (PAIR) give_up_pair(p.status, abort_flag, peer_abort);
+        else give_up(p.status, abort_flag);
         break;
       }
       tc_fence_after();
       if (EPI == kEpiSharedGateUp) {
         // bf16 operands, no global scales: h = silu(gate) * up, stored bf16
         uint32_t rg[64], ru[64];
-        tmem_ld32(tbase + kAccCol + half * 64, rg);
-        tmem_ld32(tbase + kAccCol + half * 64 + 32, rg + 32);
-        tmem_ld32(tbase + kAccCol + 128 + half * 64, ru);
-        tmem_ld32(tbase + kAccCol + 128 + half * 64 + 32, ru + 32);
+        tmem_ld32(tacc + half * 64, rg);
+        tmem_ld32(tacc + half * 64 + 32, rg + 32);
+        tmem_ld32(tacc + 128 + half * 64, ru);
+        tmem_ld32(tacc + 128 + half * 64 + 32, ru + 32);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
@@ -401,14 +600,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         // drain this thread's 64 gate and 64 up columns, then hand the
         // accumulator back before any arithmetic
         uint32_t rg[64], ru[64];
-        tmem_ld32(tbase + kAccCol + half * 64, rg);
-        tmem_ld32(tbase + kAccCol + half * 64 + 32, rg + 32);
-        tmem_ld32(tbase + kAccCol + 128 + half * 64, ru);
-        tmem_ld32(tbase + kAccCol + 128 + half * 64 + 32, ru + 32);
+        tmem_ld32(tacc + half * 64, rg);
+        tmem_ld32(tacc + half * 64 + 32, rg + 32);
+        tmem_ld32(tacc + 128 + half * 64, ru);
+        tmem_ld32(tacc + 128 + half * 64 + 32, ru + 32);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty_bar);
+        if (lane == 0) {
+          if constexpr (PAIR) mbar_arrive_remote(acce_leader);
+          else mbar_arrive(&acc_empty_bar);
+        }
         const int hcol0 = nt * 128 + half * 64;
         uint4 cw0 = make_uint4(0, 0, 0, 0), cw1 = make_uint4(0, 0, 0, 0);
         uint32_t sw = 0;
@@ -442,21 +644,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             atomicMax(reinterpret_cast<unsigned int*>(p.h_amax + se), __float_as_uint(m));
           }
         }
-        uint4* cdst = reinterpret_cast<uint4*>(p.h_codes + (size_t)grow * (p.I / 2) + hcol0 / 2);
-        cdst[0] = cw0;
-        cdst[1] = cw1;
-        *reinterpret_cast<uint32_t*>(p.h_sf + tiled_scale_offset(grow, hcol0 / kQBlock, p.I / 64)) = sw;
+        // padding rows of a segment get zero codes and scales; a pair CTA
+        // without rows of its own stores nothing
+        if (tc.valid) {
+          uint4* cdst = reinterpret_cast<uint4*>(p.h_codes + (size_t)grow * (p.I / 2) + hcol0 / 2);
+          cdst[0] = cw0;
+          cdst[1] = cw1;
+          *reinterpret_cast<uint32_t*>(p.h_sf + tiled_scale_offset(grow, hcol0 / kQBlock, p.I / 64)) = sw;
+        }
       } else {
         const float scale = kBf16 ? 1.0f : __fmul_rn(__fmul_rn(g_act, g_b0), w_row);
         const int col0 = nt * kBN + half * 128;
         // drain this thread's 128 columns, then hand the accumulator back
         uint32_t r[128];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(tbase + kAccCol + half * 128 + 32 * c, r + 32 * c);
+        for (int c = 0; c < 4; ++c) tmem_ld32(tacc + half * 128 + 32 * c, r + 32 * c);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty_bar);
+        if (lane == 0) {
+          if constexpr (PAIR) mbar_arrive_remote(acce_leader);
+          else mbar_arrive(&acc_empty_bar);
+        }
         if (real && p.y_f32) {
           float4* dst = reinterpret_cast<float4*>(p.y_f32 + (size_t)grow * p.H + col0);
 #pragma unroll
@@ -511,21 +720,50 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      acc_phase ^= 1u;
     }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) {
+    // neither CTA leaves while the other may still arrive on its barriers or
+    // the leader's MMAs may still read its shared memory
+    cluster_sync_all();
+    if (*abort_flag) {
+      // after a give-up, copies issued before it may still be landing in
+      // this CTA's shared memory: they finish within microseconds
+      const uint64_t t0 = globaltimer_ns();
+      while (globaltimer_ns() - t0 < 1000000ull) {
+      }
+    }
+  }
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    if constexpr (PAIR) tmem_dealloc_pair(tmem, kTmemCols);
+    else tmem_dealloc(tmem, kTmemCols);
   }
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA32,
+                            const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
+                            const GemmParams p) {
+  gemm_body<EPI, false>(tmA, tmA32, tmB0, tmB1, nullptr, p);
+}
+
+// The CTA-pair form of the FP4 GEMMs: launched in clusters of two.
+template <int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_fp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+                                 const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ PairMaps pm,
+                                 const GemmParams p) {
+  gemm_body<EPI, true>(tmA, tmA, tmB0, tmB1, &pm, p);
 }
 
 // Opts a kernel into the large dynamic shared memory once per device.
 static nvfp4_status set_smem_attr(const void* fn, int which, int smem) {
   static std::mutex mu;
-  static bool done[4][64] = {};
+  static bool done[6][64] = {};
   int dev = 0;
   NV_CHECK(check_cuda(cudaGetDevice(&dev), "cudaGetDevice"));
   if (dev < 0 || dev >= 64) dev = 63;
@@ -538,6 +776,57 @@ static nvfp4_status set_smem_attr(const void* fn, int which, int smem) {
   return NVFP4_OK;
 }
 
+// Launches the CTA-pair kernel: clusters of two CTAs, as many clusters as can
+// be resident at once (persistent), as a programmatic dependent launch.
+template <int EPI>
+static nvfp4_status launch_pair(const char* what, const CUtensorMap& tmA, const CUtensorMap& tmB0,
+                                const CUtensorMap& tmB1, const PairMaps& pm, const GemmParams& p, int max_pair_tiles,
+                                cudaStream_t s) {
+  constexpr int smem = smem_bytes_of<EPI, true>();
+  NV_CHECK(set_smem_attr((const void*)grouped_fp4_gemm_pair_kernel<EPI>, EPI == kEpiGateUp ? 4 : 5, smem));
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  static std::mutex mu;
+  static int clusters[2][64] = {};
+  int dev = 0;
+  NV_CHECK(check_cuda(cudaGetDevice(&dev), "cudaGetDevice"));
+  if (dev < 0 || dev >= 64) dev = 63;
+  int n = 0;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    n = clusters[EPI == kEpiGateUp ? 0 : 1][dev];
+    if (n == 0) {
+      int sms = 0;
+      NV_CHECK(device_sm_count(&sms));
+      cfg.gridDim = dim3(2 * (sms / 2));
+      NV_CHECK(check_cuda(cudaOccupancyMaxActiveClusters(&n, grouped_fp4_gemm_pair_kernel<EPI>, &cfg),
+                          "cudaOccupancyMaxActiveClusters"));
+      NV_REQUIRE(n >= 1, NVFP4_ERR_CUDA, "%s: no cluster of two CTAs can be resident", what);
+      clusters[EPI == kEpiGateUp ? 0 : 1][dev] = n;
+    }
+  }
+  cfg.gridDim = dim3(2 * std::max(1, std::min(n, max_pair_tiles)));
+  cfg.numAttrs = 2;
+  return check_cuda(cudaLaunchKernelEx(&cfg, grouped_fp4_gemm_pair_kernel<EPI>, tmA, tmB0, tmB1, pm, p), what);
+}
+
+bool gemm_runs_pair(const GroupedGemmArgs& a) {
+  const bool fp4 = a.epi == kEpiGateUp || a.epi == kEpiDown;
+  const int K = a.epi == kEpiGateUp ? a.H : a.I;
+  return a.pair && fp4 && K % kBK == 0;
+}
+
 nvfp4_status launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t s) {
   int sms = 0;
   NV_CHECK(device_sm_count(&sms));
@@ -545,6 +834,8 @@ nvfp4_status launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t s) {
   const bool bf = a.epi == kEpiSharedGateUp || a.epi == kEpiSharedDown;
   const int K = gu ? a.H : a.I;
   const int Nw = gu ? a.I : a.H;
+  // the CTA pair: FP4 kinds with whole 256-element K stages, when asked for
+  const bool pair = gemm_runs_pair(a);
   // 128-byte K boxes: 128 packed FP4 bytes, or 64 bf16 elements
   const CUtensorMapDataType dt = bf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
   const uint64_t inner = bf ? (uint64_t)K : (uint64_t)K / 2;       // elements per row
@@ -553,12 +844,32 @@ nvfp4_status launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t s) {
   CUtensorMap tmA, tmA32, tmB0, tmB1;
   const uint64_t a_rows = (uint64_t)(a.a_rows > 0 ? a.a_rows : a.rows_capacity);
   NV_CHECK(make_tmap_2d(&tmA, a.a_codes, dt, inner, a_rows, pitch, box, kBM));
-  NV_CHECK(make_tmap_2d(&tmA32, a.a_codes, dt, inner, a_rows, pitch, box, 32));
-  NV_CHECK(make_tmap_2d(&tmB0, a.b0_codes, dt, inner, (uint64_t)a.E * Nw, pitch, box, gu ? 128 : kBN));
-  if (gu) {
-    NV_CHECK(make_tmap_2d(&tmB1, a.b1_codes, dt, inner, (uint64_t)a.E * Nw, pitch, box, 128));
+  if (!pair) {
+    NV_CHECK(make_tmap_2d(&tmA32, a.a_codes, dt, inner, a_rows, pitch, box, 32));
+    NV_CHECK(make_tmap_2d(&tmB0, a.b0_codes, dt, inner, (uint64_t)a.E * Nw, pitch, box, gu ? 128 : kBN));
+    if (gu) {
+      NV_CHECK(make_tmap_2d(&tmB1, a.b1_codes, dt, inner, (uint64_t)a.E * Nw, pitch, box, 128));
+    } else {
+      tmB1 = tmB0;
+    }
+  } else if (a.b_staged) {
+    // staged codes as rows of 128 bytes: each 128-row, 256-element K tile is
+    // 128 consecutive rows, already in the swizzled order
+    const uint64_t rows = (uint64_t)a.E * Nw * (K / kBK);
+    NV_CHECK(make_tmap_2d(&tmB0, a.b0_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 128, rows, 128, 128, 128, false));
+    if (gu) {
+      NV_CHECK(make_tmap_2d(&tmB1, a.b1_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 128, rows, 128, 128, 128, false));
+    } else {
+      tmB1 = tmB0;
+    }
   } else {
-    tmB1 = tmB0;
+    // each CTA of the pair loads 128 weight rows
+    NV_CHECK(make_tmap_2d(&tmB0, a.b0_codes, dt, inner, (uint64_t)a.E * Nw, pitch, box, 128));
+    if (gu) {
+      NV_CHECK(make_tmap_2d(&tmB1, a.b1_codes, dt, inner, (uint64_t)a.E * Nw, pitch, box, 128));
+    } else {
+      tmB1 = tmB0;
+    }
   }
   GemmParams p;
   p.a_sf = a.a_scales;
@@ -568,6 +879,7 @@ nvfp4_status launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t s) {
   p.E = a.E;
   p.Nw = Nw;
   p.n_tiles = gu ? a.I / 128 : a.H / kBN;
+  p.cap_tiles = a.rows_capacity / kBM;
   p.tile_expert = a.tile_expert;
   p.num_mtiles = a.num_mtiles;
   p.expert_offsets = a.expert_offsets;
@@ -593,26 +905,47 @@ nvfp4_status launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t s) {
   p.b1_codes = a.b1_codes;
   p.status = a.status;
   const int max_tiles = a.rows_capacity / kBM * p.n_tiles;
+  if (pair) {
+    // scale atoms as rows of 128 32-bit words (512 bytes), four per stage
+    const int nblk4 = K / 64;
+    PairMaps pm;
+    NV_CHECK(make_tmap_2d(&pm.sfa, a.a_scales, CU_TENSOR_MAP_DATA_TYPE_UINT32, 128,
+                          (uint64_t)(a.rows_capacity / kBM) * nblk4, kAtomBytes, 128, 4, false));
+    NV_CHECK(make_tmap_2d(&pm.sfb0, a.b0_scales, CU_TENSOR_MAP_DATA_TYPE_UINT32, 128,
+                          (uint64_t)a.E * Nw / kBM * nblk4, kAtomBytes, 128, 4, false));
+    if (gu) {
+      NV_CHECK(make_tmap_2d(&pm.sfb1, a.b1_scales, CU_TENSOR_MAP_DATA_TYPE_UINT32, 128,
+                            (uint64_t)a.E * Nw / kBM * nblk4, kAtomBytes, 128, 4, false));
+    } else {
+      pm.sfb1 = pm.sfb0;
+    }
+    if (a.epi == kEpiGateUp)
+      return launch_pair<kEpiGateUp>("grouped_fp4_gemm_pair_kernel<gate_up>", tmA, tmB0, tmB1, pm, p, max_tiles, s);
+    return launch_pair<kEpiDown>("grouped_fp4_gemm_pair_kernel<down>", tmA, tmB0, tmB1, pm, p, max_tiles, s);
+  }
   const int grid = std::max(1, std::min(sms, max_tiles));
   switch (a.epi) {
     case kEpiGateUp:
-      NV_CHECK(set_smem_attr((const void*)grouped_fp4_gemm_kernel<kEpiGateUp>, 0, smem_bytes_of<kEpiGateUp>()));
+      NV_CHECK(set_smem_attr((const void*)grouped_fp4_gemm_kernel<kEpiGateUp>, 0,
+                             smem_bytes_of<kEpiGateUp, false>()));
       return launch_dependent("grouped_fp4_gemm_kernel<gate_up>", grouped_fp4_gemm_kernel<kEpiGateUp>, dim3(grid),
-                              dim3(kThreads), smem_bytes_of<kEpiGateUp>(), s, tmA, tmA32, tmB0, tmB1, p);
+                              dim3(kThreads), smem_bytes_of<kEpiGateUp, false>(), s, tmA, tmA32, tmB0, tmB1, p);
     case kEpiDown:
-      NV_CHECK(set_smem_attr((const void*)grouped_fp4_gemm_kernel<kEpiDown>, 1, smem_bytes_of<kEpiDown>()));
+      NV_CHECK(set_smem_attr((const void*)grouped_fp4_gemm_kernel<kEpiDown>, 1, smem_bytes_of<kEpiDown, false>()));
       return launch_dependent("grouped_fp4_gemm_kernel<down>", grouped_fp4_gemm_kernel<kEpiDown>, dim3(grid),
-                              dim3(kThreads), smem_bytes_of<kEpiDown>(), s, tmA, tmA32, tmB0, tmB1, p);
+                              dim3(kThreads), smem_bytes_of<kEpiDown, false>(), s, tmA, tmA32, tmB0, tmB1, p);
     case kEpiSharedGateUp:
       NV_CHECK(set_smem_attr((const void*)grouped_fp4_gemm_kernel<kEpiSharedGateUp>, 2,
-                             smem_bytes_of<kEpiSharedGateUp>()));
+                             smem_bytes_of<kEpiSharedGateUp, false>()));
       return launch_dependent("grouped_fp4_gemm_kernel<shared_gate_up>", grouped_fp4_gemm_kernel<kEpiSharedGateUp>,
-                              dim3(grid), dim3(kThreads), smem_bytes_of<kEpiSharedGateUp>(), s, tmA, tmA32, tmB0, tmB1, p);
+                              dim3(grid), dim3(kThreads), smem_bytes_of<kEpiSharedGateUp, false>(), s, tmA, tmA32,
+                              tmB0, tmB1, p);
     default:
       NV_CHECK(set_smem_attr((const void*)grouped_fp4_gemm_kernel<kEpiSharedDown>, 3,
-                             smem_bytes_of<kEpiSharedDown>()));
+                             smem_bytes_of<kEpiSharedDown, false>()));
       return launch_dependent("grouped_fp4_gemm_kernel<shared_down>", grouped_fp4_gemm_kernel<kEpiSharedDown>,
-                              dim3(grid), dim3(kThreads), smem_bytes_of<kEpiSharedDown>(), s, tmA, tmA32, tmB0, tmB1, p);
+                              dim3(grid), dim3(kThreads), smem_bytes_of<kEpiSharedDown, false>(), s, tmA, tmA32,
+                              tmB0, tmB1, p);
   }
 }
 
@@ -727,6 +1060,7 @@ extern "C" nvfp4_status moe_nvfp4_gate_up(const moe_nvfp4_weights* W, const uint
   a.expert_offsets = expert_offsets; a.expert_counts = expert_counts;
   a.h_gscale = h_gscale; a.h_codes = h_codes; a.h_scales = h_scales; a.h_f32 = h_f32; a.h_amax = h_amax;
   a.status = g.status;
+  a.pair = rows_capacity >= kPairMinRows;
   return launch_grouped_gemm(a, s);
 }
 
@@ -762,5 +1096,6 @@ extern "C" nvfp4_status moe_nvfp4_down(const moe_nvfp4_weights* W, const uint8_t
   a.expert_offsets = expert_offsets; a.expert_counts = expert_counts;
   a.row_w = row_weight; a.y_bf16 = y_bf16; a.y_f32 = y_f32;
   a.status = g.status;
+  a.pair = rows_capacity >= kPairMinRows;
   return launch_grouped_gemm(a, s);
 }

@@ -53,9 +53,19 @@ struct GroupedGemmArgs {
   // kEpiSharedGateUp output: silu(gate) * up as bf16 [rows][I]
   void* h_bf16 = nullptr;
   uint32_t* status = nullptr;
+  // run the FP4 kinds on CTA pairs (clusters of two sharing one 256-row MMA)
+  // when K is a multiple of 256; the caller asks for it on large batches
+  bool pair = false;
 };
 
+// Batches with at least this many (token, expert) rows run the FP4 GEMMs on
+// CTA pairs; smaller ones (decode) on one CTA per tile, which loads only a
+// tile's data rows.
+constexpr int kPairMinRows = 2048;
+
 nvfp4_status launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t s);
+// Whether launch_grouped_gemm runs these arguments on CTA pairs.
+bool gemm_runs_pair(const GroupedGemmArgs& a);
 
 }  // namespace nvfp4moe
 

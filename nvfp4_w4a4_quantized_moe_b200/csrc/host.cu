@@ -65,7 +65,8 @@ static EncodeTiledFn encode_fn() {
 }
 
 nvfp4_status make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, uint64_t inner,
-                          uint64_t outer, uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer) {
+                          uint64_t outer, uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer,
+                          bool swizzle128) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return set_error(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   cuuint64_t dims[2] = {inner, outer};
@@ -73,7 +74,8 @@ nvfp4_status make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataTyp
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t elem_strides[2] = {1, 1};
   CUresult r = fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, elem_strides,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS)
     return set_error(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) for a %llu x %llu tensor", (int)r,

@@ -26,7 +26,8 @@ inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s
 // `outer` rows, a row pitch of `pitch_bytes`, loaded in boxes of
 // box_inner x box_outer with the 128-byte swizzle.
 nvfp4_status make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, uint64_t inner,
-                          uint64_t outer, uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer);
+                          uint64_t outer, uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer,
+                          bool swizzle128 = true);
 
 // Sequential carving of a workspace: every slice 256-byte aligned.
 struct Carver {
