@@ -720,6 +720,7 @@ NVDEV void gemm_body(const CUtensorMap& tmA, const CUtensorMap& tmA32, const CUt
           }
         }
       }
+      acc_phase ^= 1u;
     }
   }
   tc_fence_before();
