@@ -72,6 +72,15 @@ NVFP4_API nvfp4_status nvfp4_test_mma_peak(int iters, int n, int with_cp, int ct
 NVFP4_API nvfp4_status nvfp4_test_wait_timeout(const void* src, uint64_t limit_ns, void* ws, size_t ws_bytes,
                                                unsigned long long* elapsed_ns, uint32_t* copied, void* stream);
 
+/* For each (amax[i] >= 0, g[i] >= 0): q_lib[i] = the block-scale quotient
+ * amax / (6 g) as the quantisers compute it (a three-instruction division by
+ * Markstein's method where 6 g is in range, else IEEE division; quotients of
+ * 464 and more may come out as 464), q_ieee[i] = the same by CUDA's IEEE
+ * division, and code_lib[i], code_ieee[i] = their E4M3 codes. */
+NVFP4_API nvfp4_status nvfp4_test_block_scale_div(const float* amax, const float* g, int n, float* q_lib,
+                                                  float* q_ieee, uint8_t* code_lib, uint8_t* code_ieee,
+                                                  void* stream);
+
 /* out[i] = the router's fp32 sigmoid of l[i]. */
 NVFP4_API nvfp4_status nvfp4_test_sigmoid(const float* l, int n, float* out, void* stream);
 

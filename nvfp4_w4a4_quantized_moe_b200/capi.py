@@ -103,6 +103,7 @@ _declare("nvfp4_test_e4m3", _i, _vp, _i, _vp, _vp, _vp)
 _declare("nvfp4_test_sigmoid", _i, _vp, _i, _vp, _vp)
 _declare("nvfp4_test_mma_peak", _i, _i, _i, _i, _i, _vp, _vp, _vp)
 _declare("nvfp4_test_wait_timeout", _i, _vp, ctypes.c_uint64, _vp, _sz, _vp, _vp, _vp)
+_declare("nvfp4_test_block_scale_div", _i, _vp, _vp, _i, _vp, _vp, _vp, _vp, _vp)
 
 # Every symbol the public headers declare (checked by the CPU test suite).
 EXPORTS = ("nvfp4_last_error", "nvfp4_abi_version", "nvfp4_workspace_status",
@@ -115,7 +116,7 @@ EXPORTS = ("nvfp4_last_error", "nvfp4_abi_version", "nvfp4_workspace_status",
            "moe_nvfp4_down", "moe_reap_keep",
            "nvfp4_block_stats_compute",
            "nvfp4_test_e2m1", "nvfp4_test_e2m1_sweep", "nvfp4_test_e4m3", "nvfp4_test_sigmoid",
-           "nvfp4_test_mma_peak", "nvfp4_test_wait_timeout")
+           "nvfp4_test_mma_peak", "nvfp4_test_wait_timeout", "nvfp4_test_block_scale_div")
 
 
 def _check(status: int):
@@ -604,3 +605,17 @@ def nvfp4_test_wait_timeout(src: torch.Tensor, limit_ns: int, workspace: torch.T
     _check(lib.nvfp4_test_wait_timeout(_p(src), int(limit_ns), _p(workspace), workspace.numel(), _p(elapsed),
                                        _p(copied), _stream()))
     return elapsed, copied
+
+
+def nvfp4_test_block_scale_div(amax: torch.Tensor, g: torch.Tensor):
+    """(q_lib, q_ieee, code_lib, code_ieee) for fp32 amax and g of equal size."""
+    _cuda(amax, torch.float32, "amax")
+    _cuda(g, torch.float32, "g")
+    if amax.numel() != g.numel():
+        raise ValueError("amax and g must have the same size")
+    n = amax.numel()
+    ql, qi = torch.empty_like(amax), torch.empty_like(amax)
+    cl = torch.empty(n, dtype=torch.uint8, device=amax.device)
+    ci = torch.empty_like(cl)
+    _check(lib.nvfp4_test_block_scale_div(_p(amax), _p(g), n, _p(ql), _p(qi), _p(cl), _p(ci), _stream()))
+    return ql, qi, cl, ci

@@ -102,12 +102,52 @@ NVDEV uint64_t pack_f32x2(float lo, float hi) {
 NVDEV float lo_f32(uint64_t p) { return __uint_as_float((uint32_t)p); }
 NVDEV float hi_f32(uint64_t p) { return __uint_as_float((uint32_t)(p >> 32)); }
 
+// The per-tensor constants of the block scale: g, d = 6 g, and RN(1/d) for
+// the division below when d is in the range where it is exact.
+struct BlockScaler {
+  float g, d, rcp_d;
+  bool fast;
+};
+NVDEV BlockScaler make_scaler(float g) {
+  BlockScaler b;
+  b.g = g;
+  b.d = __fmul_rn(6.0f, g);
+  // 2^-60 <= d <= 2^100: the residual below stays a normal number for every
+  // quotient that can give a non-zero scale, and 1/d is normal
+  b.fast = b.d >= 8.673617e-19f && b.d <= 1.2676506e30f;
+  b.rcp_d = b.fast ? __frcp_rn(b.d) : 0.0f;
+  return b;
+}
+// a / d rounded to nearest (IEEE), for 0 <= a and the scaler's fast range,
+// by Markstein's correction of the product with the correctly rounded
+// reciprocal y = RN(1/d): q = RN(a y), r = a - d q (exact, one fused
+// multiply-add), q' = RN(q + r y) is RN(a / d) (P. Markstein, "Computation of
+// elementary functions on the IBM RISC System/6000 processor", IBM J. Res.
+// Dev. 34(1), 1990; the theorem also in Muller et al., "Handbook of
+// Floating-Point Arithmetic", on division by fused multiply-add).  Three
+// instructions instead of a full division.  Only the quotient's E4M3 code is
+// used, and that is always IEEE division's: a quotient of 464 or more (every
+// such value gives the saturated scale 448) may come out as 464 instead, an
+// overflowing product's NaN is mapped there too, and a quotient far below the
+// smallest scale (where subnormal operands void the method's exactness) may
+// differ in its last bit while its code stays 0.  Checked against CUDA's IEEE
+// division by the test hooks.
+NVDEV float div_markstein(float a, const BlockScaler& b) {
+  const float q = __fmul_rn(a, b.rcp_d);
+  const float r = __fmaf_rn(-q, b.d, a);
+  return fminf(__fmaf_rn(r, b.rcp_d, q), 464.0f);
+}
+// s_raw = amax / d (0 if d = 0), rounded to nearest.
+NVDEV float block_scale_raw(float amax, const BlockScaler& b) {
+  if (b.fast) return div_markstein(amax, b);
+  return (b.d == 0.0f) ? 0.0f : __fdiv_rn(amax, b.d);
+}
+
 // The block scale of R2: s = E4M3(amax / d), S = s * g, inv = 1 / S (zero d
 // or S gives s = 0 and inv = 0).
-NVDEV uint32_t block_scale(float amax, float g, float d, float& inv) {
-  const float s_raw = (d == 0.0f) ? 0.0f : __fdiv_rn(amax, d);
-  const uint32_t s = e4m3_code(s_raw);
-  const float S = __fmul_rn(e4m3_value(s), g);
+NVDEV uint32_t block_scale(float amax, const BlockScaler& b, float& inv) {
+  const uint32_t s = e4m3_code(block_scale_raw(amax, b));
+  const float S = __fmul_rn(e4m3_value(s), b.g);
   inv = (S == 0.0f) ? 0.0f : __frcp_rn(S);
   return s;
 }
@@ -116,12 +156,12 @@ NVDEV uint32_t block_scale(float amax, float g, float d, float& inv) {
 // (d = 6 g), one IEEE rounding per step:  s = E4M3(amax / d);  S = s * g;
 // inv = 1 / S;  q_i = E2M1(x_i * inv).  Returns the scale code; writes 8
 // bytes of packed codes.
-NVDEV uint32_t quant_block16(const float* v, float g, float d, uint2& codes) {
+NVDEV uint32_t quant_block16(const float* v, const BlockScaler& b, uint2& codes) {
   float amax = 0.0f;
 #pragma unroll
   for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
   float inv;
-  const uint32_t s = block_scale(amax, g, d, inv);
+  const uint32_t s = block_scale(amax, b, inv);
   const uint64_t inv2 = pack_f32x2(inv, inv);
   float y[16];
 #pragma unroll
@@ -135,19 +175,27 @@ NVDEV uint32_t quant_block16(const float* v, float g, float d, uint2& codes) {
   return s;
 }
 
+// Lane-wise max(|a|, |b|) of two packed bf16 pairs in one instruction; the
+// sign bits of the result are not meaningful (clear them at the end).
+NVDEV uint32_t max_abs_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
 // max |x| of eight packed bf16 pairs (exact: a bf16 maximum), as fp32.
 NVDEV float amax16_bf16(const uint32_t* w) {
-  __nv_bfloat162 m = __habs2(*reinterpret_cast<const __nv_bfloat162*>(&w[0]));
-#pragma unroll
-  for (int i = 1; i < 8; ++i) m = __hmax2(m, __habs2(*reinterpret_cast<const __nv_bfloat162*>(&w[i])));
-  return fmaxf(__low2float(m), __high2float(m));
+  const uint32_t m = max_abs_bf16x2(max_abs_bf16x2(max_abs_bf16x2(w[0], w[1]), max_abs_bf16x2(w[2], w[3])),
+                                    max_abs_bf16x2(max_abs_bf16x2(w[4], w[5]), max_abs_bf16x2(w[6], w[7]))) &
+                     0x7FFF7FFFu;
+  return fmaxf(__uint_as_float(m << 16), __uint_as_float(m & 0xFFFF0000u));
 }
 
 // The same quantisation of a block given as 16 packed bf16 values (32 bytes).
-NVDEV uint32_t quant_block16_bf16(const uint4& u0, const uint4& u1, float g, float d, uint2& codes) {
+NVDEV uint32_t quant_block16_bf16(const uint4& u0, const uint4& u1, const BlockScaler& b, uint2& codes) {
   const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
   float inv;
-  const uint32_t s = block_scale(amax16_bf16(w), g, d, inv);
+  const uint32_t s = block_scale(amax16_bf16(w), b, inv);
   const uint64_t inv2 = pack_f32x2(inv, inv);
   float y[16];
 #pragma unroll

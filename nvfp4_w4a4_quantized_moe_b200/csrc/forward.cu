@@ -54,8 +54,7 @@ __global__ void __launch_bounds__(128) quantize_scatter_kernel(const uint4* __re
   uint2 c0 = make_uint2(0, 0);
   uint32_t s0 = 0;
   if (MODE == 0 && valid) {
-    const float g = act_gscale[0];
-    s0 = quant_block16_bf16(u0, u1, g, __fmul_rn(6.0f, g), c0);
+    s0 = quant_block16_bf16(u0, u1, make_scaler(act_gscale[0]), c0);
   }
   griddep_wait();
   griddep_launch();
@@ -86,16 +85,14 @@ __global__ void __launch_bounds__(128) quantize_scatter_kernel(const uint4* __re
   };
   if (MODE & kActPerExpert) {
     for (int j = 0; j < k; ++j) {
-      const float g = gs[j];
       uint2 c = make_uint2(0, 0);
       uint32_t s = 0;
-      if (valid) s = quant_block16_bf16(u0, u1, g, __fmul_rn(6.0f, g), c);
+      if (valid) s = quant_block16_bf16(u0, u1, make_scaler(gs[j]), c);
       write(rows[j], c, s);
     }
   } else {
     if (MODE & kActDynamic) {
-      const float g = dynamic_gscale(amax_bits[0]);
-      if (valid) s0 = quant_block16_bf16(u0, u1, g, __fmul_rn(6.0f, g), c0);
+      if (valid) s0 = quant_block16_bf16(u0, u1, make_scaler(dynamic_gscale(amax_bits[0])), c0);
     }
     for (int j = 0; j < k; ++j) write(rows[j], c0, s0);
   }

@@ -622,13 +622,12 @@ NVDEV void gemm_body(const CUtensorMap& tmA, const CUtensorMap& tmA32, const CUt
             const float up = __fmul_rn(__uint_as_float(ru[i]), su);
             h[i] = __fmul_rn(silu(gate), up);
           }
-          const float g2 = g_h;
-          const float d2 = __fmul_rn(6.0f, g2);
+          const BlockScaler b2 = make_scaler(g_h);
           uint2 c0, c1, c2, c3;
-          const uint32_t s0 = quant_block16(h, g2, d2, c0);
-          const uint32_t s1 = quant_block16(h + 16, g2, d2, c1);
-          const uint32_t s2 = quant_block16(h + 32, g2, d2, c2);
-          const uint32_t s3 = quant_block16(h + 48, g2, d2, c3);
+          const uint32_t s0 = quant_block16(h, b2, c0);
+          const uint32_t s1 = quant_block16(h + 16, b2, c1);
+          const uint32_t s2 = quant_block16(h + 32, b2, c2);
+          const uint32_t s3 = quant_block16(h + 48, b2, c3);
           cw0 = make_uint4(c0.x, c0.y, c1.x, c1.y);
           cw1 = make_uint4(c2.x, c2.y, c3.x, c3.y);
           sw = s0 | (s1 << 8) | (s2 << 16) | (s3 << 24);

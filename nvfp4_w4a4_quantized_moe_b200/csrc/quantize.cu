@@ -48,8 +48,7 @@ NVDEV void store_scales(uint8_t* scales, int layout, int row, int kb, int nblk, 
 __global__ void __launch_bounds__(256) quantize_act_kernel(const uint4* __restrict__ x, int rows, int cols,
                                                           const float* __restrict__ gscale, int layout,
                                                           uint2* __restrict__ codes, uint8_t* __restrict__ scales) {
-  const float g = *gscale;
-  const float d = __fmul_rn(6.0f, g);
+  const BlockScaler bs = make_scaler(*gscale);
   const int nblk = cols / kQBlock;
   const long long total = (long long)rows * nblk;
   const long long stride = (long long)gridDim.x * blockDim.x;
@@ -65,7 +64,7 @@ __global__ void __launch_bounds__(256) quantize_act_kernel(const uint4* __restri
       kb = (int)(i % nblk);
       const uint4 u0 = __ldg(x + i * 2), u1 = __ldg(x + i * 2 + 1);
       uint2 c;
-      s = quant_block16_bf16(u0, u1, g, d, c);
+      s = quant_block16_bf16(u0, u1, bs, c);
       codes[i] = c;
     }
     store_scales<1>(scales, layout, row, kb, nblk, &s, valid);
@@ -294,8 +293,8 @@ __global__ void __launch_bounds__(kWThreads, 1) quantize_weights_kernel(
     uint32_t phase = 0;
     bool ok = true;
     for (int mat = 0; mat < n_mats; ++mat) {
-      // running max of |x| on packed bf16 pairs (exact)
-      __nv_bfloat162 m2 = __floats2bfloat162_rn(0.0f, 0.0f);
+      // running max of |x| on packed bf16 pairs (exact; sign bits cleared at the end)
+      uint32_t m2 = 0u;
       for (int c = 0; ok && c < n_chunks; ++c) {
         if (!mbar_wait(&full_a[slot], phase, abort_flag)) {
           ok = false;
@@ -311,8 +310,7 @@ __global__ void __launch_bounds__(kWThreads, 1) quantize_weights_kernel(
             const uint4 u = src[v];
             const uint32_t ws[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              m2 = __hmax2(m2, __habs2(*reinterpret_cast<const __nv_bfloat162*>(&ws[j])));
+            for (int j = 0; j < 4; ++j) m2 = max_abs_bf16x2(m2, ws[j]);
           }
         }
         __syncwarp();
@@ -322,7 +320,8 @@ __global__ void __launch_bounds__(kWThreads, 1) quantize_weights_kernel(
           phase ^= 1u;
         }
       }
-      const float m = fmaxf(__low2float(m2), __high2float(m2));
+      m2 &= 0x7FFF7FFFu;
+      const float m = fmaxf(__uint_as_float(m2 << 16), __uint_as_float(m2 & 0xFFFF0000u));
       uint32_t mb = __float_as_uint(m);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, o));
@@ -357,7 +356,8 @@ __global__ void __launch_bounds__(kWThreads, 1) quantize_weights_kernel(
     const int row_t0 = (int)(bt0 / nblk), kb_t0 = (int)(bt0 % nblk);
     const int step_rows = kWChunkBlocks / nblk, step_kb = kWChunkBlocks % nblk;
     for (int mat = 0; ok && mat < n_mats; ++mat) {
-      float g = 0.0f, d = 0.0f;
+      float g = 0.0f;
+      BlockScaler bs = make_scaler(0.0f);
       int row = row_t0, kb = kb_t0;
       float* inv_tab = s_inv[mat & 1];
       for (int c = 0; c < n_chunks; ++c) {
@@ -368,7 +368,7 @@ __global__ void __launch_bounds__(kWThreads, 1) quantize_weights_kernel(
           // Every warp takes part in the barrier, landed or not.
           if (landed) {
             g = __fdiv_rn(s_amax[mat & 3], 2688.0f);
-            d = __fmul_rn(6.0f, g);
+            bs = make_scaler(g);
             if (gt < 256) {
               const float S = __fmul_rn(e4m3_value((uint32_t)gt), g);
               inv_tab[gt] = (S == 0.0f) ? 0.0f : __frcp_rn(S);
@@ -389,9 +389,7 @@ __global__ void __launch_bounds__(kWThreads, 1) quantize_weights_kernel(
         if (j < nb) {
           const uint4 u0 = src[2 * j], u1 = src[2 * j + 1];
           const uint32_t w8[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-          const float amax = amax16_bf16(w8);
-          const float s_raw = (d == 0.0f) ? 0.0f : __fdiv_rn(amax, d);
-          const uint32_t sc = e4m3_code(s_raw);
+          const uint32_t sc = e4m3_code(block_scale_raw(amax16_bf16(w8), bs));
           const float inv = inv_tab[sc];
           const uint64_t inv2 = pack_f32x2(inv, inv);
           float y[16];

@@ -533,11 +533,10 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
     // this kernel has started (it waited for their producer), so they are
     // quantised here, before the wait, exactly as the quantise-scatter kernel
     // does: one 16-element block per thread and step, read through L2
-    const float g = act_gscale[0];
-    const float d = __fmul_rn(6.0f, g);
+    const BlockScaler bs = make_scaler(act_gscale[0]);
     for (int b = tid; b < T * nblk; b += blockDim.x) {
       uint2 c;
-      const uint32_t sc = quant_block16_bf16(__ldcg(x + (size_t)b * 2), __ldcg(x + (size_t)b * 2 + 1), g, d, c);
+      const uint32_t sc = quant_block16_bf16(__ldcg(x + (size_t)b * 2), __ldcg(x + (size_t)b * 2 + 1), bs, c);
       reinterpret_cast<uint2*>(xq_c)[b] = c;
       xq_s[b] = (uint8_t)sc;
     }

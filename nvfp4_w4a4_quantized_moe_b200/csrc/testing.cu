@@ -387,6 +387,21 @@ __global__ void __launch_bounds__(64, 1)
   }
 }
 
+// The block scale's quotient s_raw = amax / (6 g), computed the library's way
+// (block_scale_raw) and with CUDA's IEEE division, with both E4M3 codes.
+__global__ void test_block_scale_div_kernel(const float* amax, const float* g, int n, float* q_lib, float* q_ieee,
+                                            uint8_t* code_lib, uint8_t* code_ieee) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const BlockScaler b = make_scaler(g[i]);
+  const float ql = block_scale_raw(amax[i], b);
+  const float qi = (b.d == 0.0f) ? 0.0f : __fdiv_rn(amax[i], b.d);
+  q_lib[i] = ql;
+  q_ieee[i] = qi;
+  code_lib[i] = (uint8_t)e4m3_code(ql);
+  code_ieee[i] = (uint8_t)e4m3_code(qi);
+}
+
 }  // namespace nvfp4moe
 
 using namespace nvfp4moe;
@@ -458,4 +473,15 @@ extern "C" nvfp4_status nvfp4_test_wait_timeout(const void* src, uint64_t limit_
   test_wait_timeout_kernel<<<1, 64, 0, s>>>(static_cast<const uint4*>(src), limit_ns, static_cast<uint32_t*>(ws),
                                             elapsed_ns, copied);
   return check_launch("test_wait_timeout_kernel");
+}
+
+extern "C" nvfp4_status nvfp4_test_block_scale_div(const float* amax, const float* g, int n, float* q_lib,
+                                                   float* q_ieee, uint8_t* code_lib, uint8_t* code_ieee,
+                                                   void* stream) {
+  NV_REQUIRE(amax && g && q_lib && q_ieee && code_lib && code_ieee && n >= 0, NVFP4_ERR_INVALID_ARG,
+             "nvfp4_test_block_scale_div: bad argument");
+  if (n == 0) return NVFP4_OK;
+  test_block_scale_div_kernel<<<(n + 255) / 256, 256, 0, as_stream(stream)>>>(amax, g, n, q_lib, q_ieee, code_lib,
+                                                                              code_ieee);
+  return check_launch("test_block_scale_div_kernel");
 }
