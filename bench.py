@@ -60,8 +60,13 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["decode", "prefill", "outlier", "tiny", "prefill16"], default="prefill",
-                    help="the headline workload (default: prefill, the largest single-GPU configuration)")
+    ap.add_argument("--workload", choices=["decode", "prefill", "outlier", "tiny", "prefill16", "quantiser"],
+                    default="prefill",
+                    help="the headline workload (default: prefill, the largest single-GPU configuration); "
+                         "quantiser times the offline weight quantiser alone")
+    ap.add_argument("--quantiser-experts", type=int, default=80,
+                    help="experts whose gate, up and down matrices the quantiser workload quantises (default 80, "
+                         "the full layer; a few make a small case for profiler captures)")
     ap.add_argument("--headline-only", action="store_true",
                     help="skip the decode, outlier and tiny sub-records")
     ap.add_argument("--seed", type=int, default=0)
@@ -186,18 +191,30 @@ def gemm_source_sha() -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel: str, workload: str):
-    """dram bytes per launch recorded by ncu for this kernel and workload, or
-    None when no record exists or the kernel source changed since."""
+def recorded_traffic(kernel: str, workload: str, algorithmic_bytes: float | None = None):
+    """(dram bytes per launch, source) recorded by ncu for this kernel and
+    workload, or (None, None) when no record exists or the kernel source
+    changed since.  A record taken on a reduced case of the same layer shape
+    (its line names the workloads it scales to) gives this workload's traffic
+    as its measured-to-algorithmic ratio times this launch's algorithmic
+    bytes."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     if not os.path.exists(path):
-        return None
+        return None, None
     sha = gemm_source_sha()
+    scaled = None
     for line in open(path):
+        if line.startswith("#"):
+            continue
         f = dict(kv.split("=", 1) for kv in line.split() if "=" in kv)
-        if f.get("kernel") == kernel and f.get("workload") == workload and f.get("source_sha") == sha:
-            return float(f["dram_bytes_per_launch"])
-    return None
+        if f.get("kernel") != kernel or f.get("source_sha") != sha:
+            continue
+        if f.get("workload") == workload:
+            return float(f["dram_bytes_per_launch"]), f"ncu capture ({workload})"
+        if algorithmic_bytes and workload in f.get("scale_to", "").split(","):
+            ratio = float(f["dram_bytes_per_launch"]) / float(f["algorithmic_bytes"])
+            scaled = (ratio * algorithmic_bytes, f"ncu capture ({f['workload']}) scaled by algorithmic bytes")
+    return scaled if scaled else (None, None)
 
 
 # ---------------------------------------------------------------------------
@@ -312,6 +329,7 @@ def run_reference(args, cfg):
 # ---------------------------------------------------------------------------
 
 L2_FLUSH_BYTES = 256 << 20          # written between flushed iterations (L2 is 126 MB)
+PAIR_MIN_ROWS = 2048                # the library's threshold for the CTA-pair GEMMs (T * k)
 MMA_FLOP_PER_SM_CLOCK_NOMINAL = 32768.0
 
 
@@ -463,7 +481,9 @@ def gemm_roofline(run, stage_ms, peaks, fp4_peak, fp4_src, kernel_stage):
     intensity is above the ridge, else bytes against HBM."""
     flops, nbytes = run.work()[kernel_stage]
     t = stage_ms[kernel_stage] * 1e-3
-    kname = "grouped_fp4_gemm_kernel<0>" if kernel_stage == "gemm_gate_up" else "grouped_fp4_gemm_kernel<1>"
+    # batches of at least 2048 (token, expert) rows run on CTA pairs
+    base = "grouped_fp4_gemm_pair_kernel" if run.cfg.T * run.cfg.k >= PAIR_MIN_ROWS else "grouped_fp4_gemm_kernel"
+    kname = base + ("<0>" if kernel_stage == "gemm_gate_up" else "<1>")
     if flops / (fp4_peak * 1e12) > nbytes / (peaks["hbm_gbs"] * 1e9):
         roof = {"bound": "tensor", "achieved": flops / t / 1e12, "peak": fp4_peak, "unit": "TFLOP/s",
                 "peak_source": fp4_src}
@@ -471,7 +491,7 @@ def gemm_roofline(run, stage_ms, peaks, fp4_peak, fp4_src, kernel_stage):
         roof = {"bound": "hbm", "achieved": nbytes / t / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "peak_source": "measured copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = recorded_traffic(kname, run.cfg.name)
+    roof["traffic"], roof["traffic_source"] = recorded_traffic(kname, run.cfg.name, nbytes)
     roof["kernel"] = kname
     roof["ms"] = stage_ms[kernel_stage]
     roof["algorithmic"] = {"bytes": nbytes, "flops": flops, "experts_hit": run.hit, "pairs": run.cfg.T * run.cfg.k}
@@ -532,18 +552,23 @@ def sub_record(c, cfg, args, dist, peaks, fp4_peak, fp4_src, flush):
 
 def quantiser_record(c, bf16, dist, peaks, flush, steps, layout):
     """The offline RTN weight quantiser over one full layer (gate, up and down
-    of every expert, back to back), timed back to back and with the L2 flushed
-    before each pass.  Outputs and workspace are allocated once, outside the
-    timed region."""
-    dev = bf16[0].device
-    qws = torch.empty(c.lib.nvfp4_quantize_weights_workspace_size(bf16[0].shape[0]), dtype=torch.uint8, device=dev)
-    outs = [c.nvfp4_quantize_weights(w, layout, workspace=qws) for w in bf16]
+    of every expert), timed back to back and with the L2 flushed before each
+    pass.  Gate and up have the same shape, so they are quantised as one call
+    over the experts' gate matrices followed by their up matrices (the fused
+    gate/up tensor a serving checkpoint keeps), and down as a second call: two
+    calls, each with one ramp and one tail.  Outputs and workspace are
+    allocated once, outside the timed region."""
+    gate, up, down = bf16
+    dev = gate.device
+    mats = (torch.cat([gate, up]), down)
+    qws = torch.empty(c.lib.nvfp4_quantize_weights_workspace_size(mats[0].shape[0]), dtype=torch.uint8, device=dev)
+    outs = [c.nvfp4_quantize_weights(w, layout, workspace=qws) for w in mats]
 
     def run():
-        for w, o in zip(bf16, outs):
+        for w, o in zip(mats, outs):
             c.nvfp4_quantize_weights(w, layout, workspace=qws, out=o)
 
-    qbytes = sum(2 * w.numel() + w.numel() // 2 + w.numel() // 16 + 4 * w.shape[0] for w in bf16)
+    qbytes = sum(2 * w.numel() + w.numel() // 2 + w.numel() // 16 + 4 * w.shape[0] for w in mats)
     for _ in range(3):
         run()
     torch.cuda.synchronize()
@@ -552,8 +577,10 @@ def quantiser_record(c, bf16, dist, peaks, flush, steps, layout):
     msf = time_loop(run, steps, dist, flush=flush)
     c.nvfp4_workspace_status(qws)
     gbs, gbsf = qbytes / (ms * 1e-3) / 1e9, qbytes / (msf * 1e-3) / 1e9
-    n, r, k = bf16[0].shape
+    n, r, k = gate.shape
+    del mats, outs
     return {"workload": f"quantiser: {n} x (gate, up {r}x{k}; down {k}x{r}) bf16 N(0, 0.02)", "layout": layout,
+            "calls": "2: gate and up stacked (2 x {} matrices of {}x{}), then down ({} of {}x{})".format(n, r, k, n, k, r),
             "ms": ms, "gbs": gbs, "ms_l2_flushed": msf, "gbs_l2_flushed": gbsf, "bytes": qbytes,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / peaks["hbm_gbs"], "frac_l2_flushed": gbsf / peaks["hbm_gbs"],
@@ -818,7 +845,38 @@ def main():
     if not torch.cuda.is_available():
         print(json.dumps({"error": "no CUDA device; the layer has no CPU path"}))
         return 1
+    if args.workload == "quantiser":
+        return run_quantiser_only(args)
     return run_ours(args, cfg)
+
+
+def run_quantiser_only(args):
+    """The offline RTN weight quantiser alone, over the gate, up and down
+    matrices of --quantiser-experts experts (bf16 N(0, 0.02), hidden 6144,
+    intermediate 2048): one JSON line with its GB/s against HBM."""
+    from nvfp4_w4a4_quantized_moe_b200 import capi as c
+    dist = Dist()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    peaks, _ = load_peaks()
+    cfg = dataclasses_replace(workloads.CONFIGS["quantiser"], E=args.quantiser_experts)
+    bf16 = workloads.stacked_expert_weights(cfg, args.seed, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    rec = quantiser_record(c, bf16, dist, peaks, flush, args.steps, "staged")
+    line = {"metric": METRIC, "value": rec["gbs"], "unit": "GB/s", "n_gpus": dist.world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": rec["ms"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
+            "config": {"workload": "quantiser", "experts": cfg.E, "H": cfg.H, "I": cfg.I,
+                       "l2": "flushed and back-to-back both reported"},
+            "quantiser": rec, "roofline": rec["roofline"]}
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+    dist.close()
+    return 0
+
+
+def dataclasses_replace(cfg, **kw):
+    import dataclasses
+    return dataclasses.replace(cfg, **kw)
 
 
 if __name__ == "__main__":

@@ -2,6 +2,7 @@
 // weight quantiser ("K-EXAONE-152B-A23B-REAP-80E-NVFP4" model card, section
 // "Quantization Setup").  Both are HBM-bound streams: 128-bit loads of bf16,
 // 64-bit stores of packed codes, one scale byte per 16 elements.
+#include <algorithm>
 #include <mutex>
 
 #include "common.cuh"
@@ -110,10 +111,19 @@ constexpr int kWAmaxConsumers = 192;                     // 8 x 16 bytes of each
 constexpr int kWQuantConsumers = 768;                    // one block of each chunk per thread
 constexpr int kWThreads = 64 + kWAmaxConsumers + kWQuantConsumers;   // + one producer warp per stream
 // The amax stream may start matrix m once this CTA's quantise consumers are
-// no more than kWLagEighths eighths of a matrix behind it: (8 m - kWLag) / 8
-// matrices' worth of chunks done.  The matrices in flight must stay in L2,
+// no more than `lead` eighths of a matrix behind it: (8 m - lead) / 8
+// matrices' worth of chunks done.  The matrices in flight (the lead plus the
+// one being quantised) must stay in L2 for the quantise stream's re-read,
 // and the amax stream should not stall at the end of every quantise pass.
-constexpr int kWLagEighths = 14;
+// The lead is sized from an L2 budget of kWL2BudgetBytes: for 25 MB matrices
+// 20 eighths (2.5 matrices) measured 3 % faster than 14, and 24 or more made
+// the re-read miss L2 and took 20 % longer.
+constexpr long long kWL2BudgetBytes = 84ll << 20;
+constexpr int kWLeadMin = 8, kWLeadMax = 64;
+static int weight_lead_eighths(long long mat_bytes) {
+  const long long lead = 8 * kWL2BudgetBytes / (mat_bytes > 0 ? mat_bytes : 1) - 8;
+  return (int)std::min<long long>(kWLeadMax, std::max<long long>(kWLeadMin, lead));
+}
 constexpr int kWDynSmem = (kWSlotsA + kWSlotsQ) * kWChunkBytes + 128;
 // warp roles
 constexpr int kWAmaxProducer = 0;                        // warp 0
@@ -217,7 +227,7 @@ NVDEV void weight_stream_producer(const uint8_t* w, long long mat_bytes, long lo
 __global__ void __launch_bounds__(kWThreads, 1) quantize_weights_kernel(
     const uint4* __restrict__ w, int n_mats, int rows, int cols, int layout, uint2* __restrict__ codes,
     uint8_t* __restrict__ scales, float* __restrict__ gscale, WeightQuantState* st, uint32_t* amax_bits,
-    uint32_t* done) {
+    uint32_t* done, int lead) {
   extern __shared__ uint8_t wq_smem_raw[];
   uint8_t* ring_a = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(wq_smem_raw) + 127) & ~uintptr_t(127));
   uint8_t* ring_q = ring_a + kWSlotsA * kWChunkBytes;
@@ -258,7 +268,7 @@ __global__ void __launch_bounds__(kWThreads, 1) quantize_weights_kernel(
     // ------------------------------------------------------------ amax producer
     if (lane == 0) {
       auto gate = [&](int mat) {
-        const long long need_eighths = 8ll * mat - kWLagEighths;
+        const long long need_eighths = 8ll * mat - lead;
         if (need_eighths <= 0) return true;
         const long long need = (need_eighths * n_chunks + 7) / 8 * (kWQuantConsumers / 32);
         const uint64_t t0 = globaltimer_ns();
@@ -470,8 +480,9 @@ static nvfp4_status launch_weight_quantiser(const void* w_bf16, int n_mats, int 
   per_sm = 1;
   const uint4* w = static_cast<const uint4*>(w_bf16);
   uint2* c = reinterpret_cast<uint2*>(codes);
+  int lead = weight_lead_eighths((long long)rows * cols * 2);
   void* args[] = {(void*)&w, (void*)&n_mats, (void*)&rows, (void*)&cols, (void*)&layout, (void*)&c,
-                  (void*)&scales, (void*)&global_scale, (void*)&st, (void*)&amax, (void*)&done};
+                  (void*)&scales, (void*)&global_scale, (void*)&st, (void*)&amax, (void*)&done, (void*)&lead};
   return check_cuda(cudaLaunchCooperativeKernel((const void*)quantize_weights_kernel, dim3(sms * per_sm),
                                                 dim3(kWThreads), args, kWDynSmem, s),
                     "cudaLaunchCooperativeKernel(quantize_weights_kernel)");

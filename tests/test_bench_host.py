@@ -42,10 +42,15 @@ def test_recorded_traffic_matches_kernel_workload_and_source_hash():
     sha = bench.gemm_source_sha()
     for ln in rows:
         f = dict(kv.split("=", 1) for kv in ln.split())
-        got = bench.recorded_traffic(f["kernel"], f["workload"])
+        got, src = bench.recorded_traffic(f["kernel"], f["workload"])
         if f["source_sha"] == sha:
-            assert got == float(f["dram_bytes_per_launch"])
-    assert bench.recorded_traffic("grouped_fp4_gemm_kernel<0>", "no-such-workload") is None
+            assert got == float(f["dram_bytes_per_launch"]) and f["workload"] in src
+            # a reduced-case record scales to the workloads it names
+            for w in filter(None, f.get("scale_to", "").split(",")):
+                alg = 2.0 * float(f["algorithmic_bytes"])
+                scaled, src2 = bench.recorded_traffic(f["kernel"], w, alg)
+                assert scaled == pytest.approx(2.0 * float(f["dram_bytes_per_launch"])) and "scaled" in src2
+    assert bench.recorded_traffic("grouped_fp4_gemm_kernel<0>", "no-such-workload") == (None, None)
 
 
 def test_weak_scaling_value_counts_every_rank():
