@@ -22,6 +22,7 @@
 // per SM walks the (m-tile, n-tile) list, whose length is read on the device.
 // Every wait is bounded in time; a wait that gives up sets the workspace
 // status word and the CTA winds down after its outstanding copies land.
+#include <cstring>
 #include <mutex>
 
 #include "common.cuh"
@@ -59,14 +60,18 @@ template <int EPI> __host__ __device__ constexpr int bk_of() { return is_bf16<EP
 // Pipeline stages: four in every one-CTA kind, five for a CTA pair (38 KiB
 // a stage per CTA).  The down
 // GEMMs stage y in shared memory, 32 rows x y_pass_cols_of() bf16 columns per
-// warp at a time: 64 columns (4 KiB) for the bf16 kind, 16 (1 KiB) for the
-// FP4 kind, whose stages leave no room for more.
+// warp at a time: 64 columns (4 KiB) for the bf16 kind and the CTA pair, 16
+// (1 KiB) for the one-CTA FP4 kind, whose four stages leave no room for more.
 template <int EPI, bool PAIR> __host__ __device__ constexpr int stages_of() { return PAIR ? 5 : 4; }
-template <int EPI> __host__ __device__ constexpr int y_pass_cols_of() { return EPI == kEpiDown ? 16 : 64; }
-template <int EPI> __host__ __device__ constexpr int y_stage_bytes_of() { return 32 * y_pass_cols_of<EPI>() * 2; }
+template <int EPI, bool PAIR> __host__ __device__ constexpr int y_pass_cols_of() {
+  return EPI == kEpiDown && !PAIR ? 16 : 64;
+}
+template <int EPI, bool PAIR> __host__ __device__ constexpr int y_stage_bytes_of() {
+  return 32 * y_pass_cols_of<EPI, PAIR>() * 2;
+}
 template <int EPI, bool PAIR> __host__ __device__ constexpr int smem_bytes_of() {
   return stages_of<EPI, PAIR>() * stage_bytes_of<EPI, PAIR>() + 1024 +
-         (is_gate_up<EPI>() ? 0 : kEpiWarps * y_stage_bytes_of<EPI>());
+         (is_gate_up<EPI>() ? 0 : kEpiWarps * y_stage_bytes_of<EPI, PAIR>());
 }
 static_assert(smem_bytes_of<kEpiDown, false>() <= 232448 - 256, "FP4 down GEMM shared memory");
 static_assert(smem_bytes_of<kEpiGateUp, false>() <= 232448 - 256, "FP4 gate/up GEMM shared memory");
@@ -124,6 +129,9 @@ struct GemmParams {
 // bytes count on the leader CTA's stage barrier.
 struct PairMaps {
   CUtensorMap sfa, sfb0, sfb1;
+  // down: y as bf16 [rows][H], boxes of 32 rows x 64 columns, 128-byte
+  // swizzle; written by TMA stores (all zero when y_bf16 is NULL)
+  CUtensorMap y;
 };
 
 NVDEV void give_up(uint32_t* status, volatile int* abort_flag) {
@@ -205,6 +213,7 @@ NVDEV void gemm_body(const CUtensorMap& tmA, const CUtensorMap& tmA32, const CUt
       prefetch_tmap(&pm->sfa);
       prefetch_tmap(&pm->sfb0);
       prefetch_tmap(&pm->sfb1);
+      if (EPI == kEpiDown && p.y_bf16) prefetch_tmap(&pm->y);
     }
   }
   if (warp == 1) {
@@ -689,15 +698,52 @@ NVDEV void gemm_body(const CUtensorMap& tmA, const CUtensorMap& tmA32, const CUt
         for (int i = 0; i < 64; ++i)
           yw[i] = pack_bf16x2(__fmul_rn(__uint_as_float(r[2 * i]), scale), __fmul_rn(__uint_as_float(r[2 * i + 1]), scale));
         const uint32_t real_mask = __ballot_sync(0xffffffffu, real);
-        if (p.y_bf16 && real_mask != 0) {
+        if (PAIR && p.y_bf16 && real_mask != 0) {
+          // Whole 32-row boxes of 64 columns go out by TMA store from a
+          // staging tile in the 128-byte swizzle (16-byte chunk c of row r
+          // at chunk c ^ (r % 8)), which lane r writes without bank
+          // conflicts.  A box holding padding rows is written back by the
+          // warp instead, data rows only, as 128-byte row segments.
+          uint8_t* ybuf = smem + kStages * kSB + (warp - 2) * y_stage_bytes_of<EPI, PAIR>();
+          const int row0 = mt * kBM + quad * 32;
+#pragma unroll
+          for (int b = 0; b < 2; ++b) {
+            if (lane == 0) bulk_wait_read_all();        // the previous box has left ybuf
+            __syncwarp();
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const int w = b * 32 + c * 4;
+              *reinterpret_cast<uint4*>(ybuf + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                  make_uint4(yw[w], yw[w + 1], yw[w + 2], yw[w + 3]);
+            }
+            if (real_mask == 0xffffffffu) {
+              fence_proxy_async();                      // the writes above, before the async proxy reads them
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_2d(&pm->y, ybuf, col0 + b * 64, row0);
+                bulk_commit_group();
+              }
+            } else {
+              __syncwarp();
+#pragma unroll
+              for (int it = 0; it < 8; ++it) {
+                const int rr = it * 4 + (lane >> 3), ch = lane & 7;
+                const uint4 v = *reinterpret_cast<const uint4*>(ybuf + rr * 128 + ((ch ^ (rr & 7)) << 4));
+                if ((real_mask >> rr) & 1u)
+                  *reinterpret_cast<uint4*>(p.y_bf16 + (size_t)(row0 + rr) * p.H + col0 + b * 64 + ch * 8) = v;
+              }
+              __syncwarp();
+            }
+          }
+        } else if (p.y_bf16 && real_mask != 0) {
           // Each lane holds one row.  Stores straight from registers would
           // hit 32 rows per instruction, so the warp stages kYCols columns of
           // its 32 rows in shared memory and writes them back as whole row
           // segments (kYCols * 2 bytes), 32 / kCh rows per instruction.  The
           // 16-byte chunks are XOR-swizzled by row so that every 8-lane phase
           // of a 16-byte access covers the 32 banks once, in both directions.
-          constexpr int kYCols = y_pass_cols_of<EPI>(), kCh = kYCols / 8, kRowsPer = 32 / kCh;
-          uint4* ybuf = reinterpret_cast<uint4*>(smem + kStages * kSB + (warp - 2) * y_stage_bytes_of<EPI>());
+          constexpr int kYCols = y_pass_cols_of<EPI, PAIR>(), kCh = kYCols / 8, kRowsPer = 32 / kCh;
+          uint4* ybuf = reinterpret_cast<uint4*>(smem + kStages * kSB + (warp - 2) * y_stage_bytes_of<EPI, PAIR>());
           const int row0 = mt * kBM + quad * 32;
           auto swz = [](int r) { return (r / (8 / kCh)) % kCh; };
 #pragma unroll
@@ -721,6 +767,8 @@ NVDEV void gemm_body(const CUtensorMap& tmA, const CUtensorMap& tmA32, const CUt
       }
       acc_phase ^= 1u;
     }
+    // the CTA's shared memory outlives every TMA store of y it issued
+    if (PAIR && EPI == kEpiDown && lane == 0) bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();
@@ -919,6 +967,10 @@ nvfp4_status launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t s) {
     } else {
       pm.sfb1 = pm.sfb0;
     }
+    std::memset(&pm.y, 0, sizeof(pm.y));
+    if (!gu && a.y_bf16)
+      NV_CHECK(make_tmap_2d(&pm.y, a.y_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)a.H,
+                            (uint64_t)a.rows_capacity, (uint64_t)a.H * 2, 64, 32, true));
     if (a.epi == kEpiGateUp)
       return launch_pair<kEpiGateUp>("grouped_fp4_gemm_pair_kernel<gate_up>", tmA, tmB0, tmB1, pm, p, max_tiles, s);
     return launch_pair<kEpiDown>("grouped_fp4_gemm_pair_kernel<down>", tmA, tmB0, tmB1, pm, p, max_tiles, s);
