@@ -539,6 +539,8 @@ def sub_record(c, cfg, args, dist, peaks, fp4_peak, fp4_src, flush):
         rec["bound"] = "launch latency (no roofline)"
     rec["e2e"] = run.e2e(steps, dist)
     rec["gpu_launches_per_step"] = kernels_per_step(c, cfg)
+    if cfg.T * cfg.k <= 256 and cfg.H >= 1024:
+        rec["shared_expert"] = shared_expert_record(c, run, cfg, args, dist, peaks)
     c.nvfp4_workspace_status(run.ws)
     diag = None
     if cfg.name == "outlier":
@@ -585,6 +587,48 @@ def quantiser_record(c, bf16, dist, peaks, flush, steps, layout):
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / peaks["hbm_gbs"], "frac_l2_flushed": gbsf / peaks["hbm_gbs"],
                          "kernel": "quantize_weights_kernel"}}
+
+
+def shared_expert_record(c, run, cfg, args, dist, peaks):
+    """The layer with its shared BF16 expert (f1): one SiLU-gated MLP of the
+    routed experts' shape (I_shared = I), bf16 N(0, 0.02) weights.  Its GEMMs
+    (with a split-K reduction after each at small batches) are timed between
+    the library's events after the routed down GEMM and after the shared
+    GEMMs.  Within a step the routed GEMMs stream the expert weights through
+    L2 first, so the shared weights are not L2-resident when read."""
+    dev = run.dev
+    sh = tuple(t.contiguous() for t in workloads.expert_weights(cfg, cfg.E + 7, args.seed, device=dev))
+    Ws = run.W.with_shared(*sh)
+    ws_sh = torch.empty(c.moe_nvfp4_workspace_size(cfg.T, cfg.E, cfg.H, cfg.I, cfg.k, cfg.I), dtype=torch.uint8,
+                        device=dev)
+    fn = lambda: c.moe_nvfp4_forward(Ws, run.x, run.g1, run.g2, logit_offset=run.off, out=run.out,  # noqa: E731
+                                     workspace=ws_sh)
+    for _ in range(3):
+        fn()
+    steps = max(args.steps, 20)
+    sh_step_ms = time_loop(fn, steps, dist)
+    sh_evs = [(events(c.N_STAGE_EVENTS), events(1)[0]) for _ in range(steps)]
+    for st_evs, sh_ev in sh_evs:
+        c.moe_nvfp4_forward(Ws, run.x, run.g1, run.g2, logit_offset=run.off, out=run.out, workspace=ws_sh,
+                            stage_events=st_evs, shared_event=sh_ev)
+    torch.cuda.synchronize()
+    c.nvfp4_workspace_status(ws_sh)
+    sh_ms = dist.max(float(np.mean([st[4].elapsed_time(ev) for st, ev in sh_evs])))
+    sh_flops = 6.0 * cfg.T * cfg.H * cfg.I
+    sh_bytes = 3.0 * cfg.H * cfg.I * 2 + 2.0 * cfg.T * cfg.H * 2 + 2.0 * cfg.T * cfg.I * 2 * 2
+    sh_tf = sh_flops / (sh_ms * 1e-3) / 1e12
+    sh_gbs = sh_bytes / (sh_ms * 1e-3) / 1e9
+    sh_tensor = sh_flops / (peaks["bf16_tflops"] * 1e12) > sh_bytes / (peaks["hbm_gbs"] * 1e9)
+    rec = {"I_shared": cfg.I, "ms_per_step": sh_step_ms, "gemms_ms": sh_ms, "flops": sh_flops,
+           "bytes": sh_bytes, "tflops": sh_tf, "gbs": sh_gbs,
+           "bound": "tensor" if sh_tensor else "hbm",
+           "frac": sh_tf / peaks["bf16_tflops"] if sh_tensor else sh_gbs / peaks["hbm_gbs"],
+           "peak": peaks["bf16_tflops"] if sh_tensor else peaks["hbm_gbs"],
+           "peak_unit": "TFLOP/s (bf16 burst)" if sh_tensor else "GB/s",
+           "gpu_launches_per_step": c.moe_nvfp4_forward_launches(cfg.T, cfg.E, cfg.H, cfg.I, cfg.k, cfg.I)}
+    del Ws, sh, ws_sh
+    torch.cuda.empty_cache()
+    return rec
 
 
 def run_ours(args, cfg):
@@ -637,38 +681,7 @@ def run_ours(args, cfg):
         fn()
     sal_ms = time_loop(fn, args.steps, dist)
     c.nvfp4_workspace_status(run.ws)
-    # the layer with its shared BF16 expert (f1): one SiLU-gated MLP of the
-    # routed experts' shape (I_shared = I), bf16 N(0, 0.02) weights.  Its two
-    # GEMMs are timed between the library's events after the down GEMM and
-    # after the shared GEMMs.
-    sh = tuple(t.contiguous() for t in workloads.expert_weights(cfg, cfg.E + 7, args.seed, device=dev))
-    Ws = run.W.with_shared(*sh)
-    ws_sh = torch.empty(c.moe_nvfp4_workspace_size(cfg.T, cfg.E, cfg.H, cfg.I, cfg.k, cfg.I), dtype=torch.uint8,
-                        device=dev)
-    fn = lambda: c.moe_nvfp4_forward(Ws, run.x, run.g1, run.g2, logit_offset=run.off, out=run.out,  # noqa: E731
-                                     workspace=ws_sh)
-    for _ in range(3):
-        fn()
-    sh_step_ms = time_loop(fn, args.steps, dist)
-    sh_evs = [(events(c.N_STAGE_EVENTS), events(1)[0]) for _ in range(args.steps)]
-    for st_evs, sh_ev in sh_evs:
-        c.moe_nvfp4_forward(Ws, run.x, run.g1, run.g2, logit_offset=run.off, out=run.out, workspace=ws_sh,
-                            stage_events=st_evs, shared_event=sh_ev)
-    torch.cuda.synchronize()
-    c.nvfp4_workspace_status(ws_sh)
-    sh_ms = dist.max(float(np.mean([st[4].elapsed_time(ev) for st, ev in sh_evs])))
-    sh_flops = 6.0 * cfg.T * cfg.H * cfg.I
-    sh_bytes = 3.0 * cfg.H * cfg.I * 2 + 2.0 * cfg.T * cfg.H * 2 + 2.0 * cfg.T * cfg.I * 2 * 2
-    sh_tf = sh_flops / (sh_ms * 1e-3) / 1e12
-    sh_gbs = sh_bytes / (sh_ms * 1e-3) / 1e9
-    sh_tensor = sh_flops / (peaks["bf16_tflops"] * 1e12) > sh_bytes / (peaks["hbm_gbs"] * 1e9)
-    shared_report = {"I_shared": cfg.I, "ms_per_step": sh_step_ms, "gemms_ms": sh_ms, "flops": sh_flops,
-                     "bytes": sh_bytes, "tflops": sh_tf, "gbs": sh_gbs,
-                     "bound": "tensor" if sh_tensor else "hbm",
-                     "frac": sh_tf / peaks["bf16_tflops"] if sh_tensor else sh_gbs / peaks["hbm_gbs"],
-                     "peak": peaks["bf16_tflops"] if sh_tensor else peaks["hbm_gbs"],
-                     "peak_unit": "TFLOP/s (bf16 burst)" if sh_tensor else "GB/s"}
-    del Ws, sh, ws_sh
+    shared_report = shared_expert_record(c, run, cfg, args, dist, peaks)
     e2e = run.e2e(args.steps, dist)
 
     # roofline of the dominant kernel (the gate/up GEMM) and of the down GEMM

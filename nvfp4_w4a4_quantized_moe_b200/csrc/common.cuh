@@ -241,6 +241,8 @@ NVDEV void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
 }
 NVDEV void fence_barrier_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+// SiLU of the gated MLPs: z / (1 + e^-z) with CUDA's fast exponential and division
+NVDEV float silu(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 NVDEV void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 // TMA store of one box from shared memory (bulk async-group completion);
 // x is the innermost coordinate in elements.

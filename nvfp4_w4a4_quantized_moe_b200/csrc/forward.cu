@@ -5,6 +5,8 @@
 // Sources: "K-EXAONE-152B-A23B-REAP-80E-NVFP4" model card ("Quantization
 // Setup"), "K-EXAONE-152B-A23B-REAP-80E-BF16" model card ("Pruning Setup",
 // "Routing behavior").
+#include <algorithm>
+
 #include "common.cuh"
 #include "gemm.cuh"
 #include "host.cuh"
@@ -201,6 +203,74 @@ __global__ void dense_tiles_kernel(int T, int32_t* __restrict__ tile_expert, int
   }
 }
 
+// Split K of the shared expert's bf16 GEMMs.  With few tokens their (m-tile,
+// n-tile) tiles occupy a handful of the 148 SMs (at 16 tokens: 16 gate/up and
+// 24 down tiles), so the weight stream would run on a tenth of the machine.
+// Below half a wave of tiles each tile's K range is split over the largest
+// divisor of its K stages (64 elements each, at most 16 parts) that keeps the
+// CTAs within one wave.  Host arithmetic only, so the workspace size and the
+// launch count follow the shape alone.
+constexpr int kSplitWaveCtas = 148;
+constexpr int kMaxSplit = 16;
+static int shared_ksplit(int T, int n_tiles, int k_stages) {
+  const int tiles = (T + kRowTile - 1) / kRowTile * n_tiles;
+  if (2 * tiles > kSplitWaveCtas) return 1;
+  int best = 1;
+  for (int d = 2; d <= kMaxSplit && d <= k_stages; ++d)
+    if (k_stages % d == 0 && tiles * d <= kSplitWaveCtas) best = d;
+  return best;
+}
+static int shared_ksplit_gate_up(int T, int H, int I_s) { return shared_ksplit(T, I_s / 128, H / 64); }
+static int shared_ksplit_down(int T, int H, int I_s) { return shared_ksplit(T, H / 256, I_s / 64); }
+
+// The split parts of a shared-expert GEMM added in part order, then its
+// epilogue: gate/up h = bf16(silu(gate) * up) ([T][cols], cols = I_shared;
+// each partial row holds the gate sums then the up sums), down y = bf16(sum)
+// ([T][cols], cols = H).  Four columns per thread.
+template <bool kGateUp>
+__global__ void __launch_bounds__(256) shared_split_reduce_kernel(const float* __restrict__ part, int S, int T,
+                                                                  int cols, uint16_t* __restrict__ out) {
+  griddep_wait();
+  griddep_launch();
+  const int ld = kGateUp ? 2 * cols : cols;
+  const size_t slab = (size_t)T * ld;
+  const int q = cols / 4;
+  const size_t n = (size_t)T * q;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+    const int t = (int)(i / q), c = (int)(i % q) * 4;
+    const float* src = part + (size_t)t * ld + c;
+    // every part's values are loaded before the first add (S <= kMaxSplit)
+    float4 g[kMaxSplit], u[kMaxSplit];
+#pragma unroll
+    for (int sp = 0; sp < kMaxSplit; ++sp) {
+      if (sp < S) {
+        g[sp] = __ldcs(reinterpret_cast<const float4*>(src + sp * slab));
+        if (kGateUp) u[sp] = __ldcs(reinterpret_cast<const float4*>(src + sp * slab + cols));
+      }
+    }
+    float4 a = g[0], b = kGateUp ? u[0] : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int sp = 1; sp < kMaxSplit; ++sp) {
+      if (sp < S) {
+        a = make_float4(__fadd_rn(a.x, g[sp].x), __fadd_rn(a.y, g[sp].y), __fadd_rn(a.z, g[sp].z),
+                        __fadd_rn(a.w, g[sp].w));
+        if (kGateUp)
+          b = make_float4(__fadd_rn(b.x, u[sp].x), __fadd_rn(b.y, u[sp].y), __fadd_rn(b.z, u[sp].z),
+                          __fadd_rn(b.w, u[sp].w));
+      }
+    }
+    uint2 w;
+    if (kGateUp) {
+      w.x = pack_bf16x2(__fmul_rn(silu(a.x), b.x), __fmul_rn(silu(a.y), b.y));
+      w.y = pack_bf16x2(__fmul_rn(silu(a.z), b.z), __fmul_rn(silu(a.w), b.w));
+    } else {
+      w.x = pack_bf16x2(a.x, a.y);
+      w.y = pack_bf16x2(a.z, a.w);
+    }
+    *reinterpret_cast<uint2*>(out + (size_t)t * cols + c) = w;
+  }
+}
+
 // amax of the tokens routed to each expert: amax_bits[1 + e].
 __global__ void __launch_bounds__(256) expert_amax_kernel(const int32_t* __restrict__ topk_idx, int T, int k,
                                                           const uint32_t* __restrict__ tok_amax,
@@ -278,6 +348,7 @@ struct ForwardScratch {
   int32_t* sh_ntiles;       // [1]
   int32_t* sh_offsets;      // [2]
   int32_t* sh_counts;       // [1]
+  float* sh_partial;        // split K: fp32 [S][T][2 I_shared] (gate/up), then [S][T][H] (down)
 };
 
 static ForwardScratch carve_forward(Carver& c, int T, int E, int H, int I, int k, int I_shared) {
@@ -300,6 +371,7 @@ static ForwardScratch carve_forward(Carver& c, int T, int E, int H, int I, int k
   f.y_sq_part = c.take<float>((size_t)cap * (H / 128));
   f.sh_h = f.sh_y = nullptr;
   f.sh_tiles = f.sh_ntiles = f.sh_offsets = f.sh_counts = nullptr;
+  f.sh_partial = nullptr;
   if (I_shared > 0) {
     const size_t tp = (size_t)(T + kRowTile - 1) / kRowTile * kRowTile;
     f.sh_h = c.take<uint16_t>(tp * I_shared);
@@ -308,6 +380,9 @@ static ForwardScratch carve_forward(Carver& c, int T, int E, int H, int I, int k
     f.sh_ntiles = c.take<int32_t>(1);
     f.sh_offsets = c.take<int32_t>(2);
     f.sh_counts = c.take<int32_t>(1);
+    const int s1 = shared_ksplit_gate_up(T, H, I_shared), s2 = shared_ksplit_down(T, H, I_shared);
+    const size_t part = std::max(s1 > 1 ? (size_t)s1 * T * 2 * I_shared : 0, s2 > 1 ? (size_t)s2 * T * H : 0);
+    if (part) f.sh_partial = c.take<float>(part);
   }
   return f;
 }
@@ -343,7 +418,10 @@ extern "C" int moe_nvfp4_forward_launches(int T, int E, int H, int I, int k, int
       I_shared < 0 || I_shared % 128 != 0 || mode < NVFP4_ACT_SCALE_TENSOR || mode > NVFP4_ACT_SCALE_DYNAMIC_EXPERT)
     return -1;
   int n = 0;
-  if (I_shared > 0) n += 1 + 2;                                    // dense tile map, shared gate/up and down
+  if (I_shared > 0) {
+    n += 1 + 2;                                                     // dense tile map, shared gate/up and down
+    n += (shared_ksplit_gate_up(T, H, I_shared) > 1) + (shared_ksplit_down(T, H, I_shared) > 1);   // reductions
+  }
   if (mode & kActDynamic) n += 1;                                   // token amax
   n += 1 + (T <= 256 ? 1 : 4);                                      // router GEMM, routing
   if (mode == NVFP4_ACT_SCALE_DYNAMIC_EXPERT) n += 1;               // expert amax
@@ -503,7 +581,18 @@ static nvfp4_status forward_impl(const moe_nvfp4_weights* W, const void* x_bf16,
     s1.expert_offsets = f.sh_offsets; s1.expert_counts = f.sh_counts;
     s1.h_bf16 = f.sh_h;
     s1.status = f.route.status;
+    s1.ksplit = shared_ksplit_gate_up(T, H, I_s);
+    if (s1.ksplit > 1) {
+      s1.h_bf16 = nullptr;
+      s1.partial = f.sh_partial;
+      s1.partial_rows = T;
+    }
     NV_CHECK(launch_grouped_gemm(s1, s));
+    if (s1.ksplit > 1) {
+      NV_CHECK(launch_dependent("shared_split_reduce_kernel<gate_up>", shared_split_reduce_kernel<true>,
+                                dim3((T * I_s / 4 + 255) / 256), dim3(256), 0, s, (const float*)f.sh_partial,
+                                s1.ksplit, T, I_s, f.sh_h));
+    }
     GroupedGemmArgs s2;
     s2.epi = kEpiSharedDown;
     s2.E = 1; s2.H = H; s2.I = I_s;
@@ -514,7 +603,18 @@ static nvfp4_status forward_impl(const moe_nvfp4_weights* W, const void* x_bf16,
     s2.expert_offsets = f.sh_offsets; s2.expert_counts = f.sh_counts;
     s2.y_bf16 = f.sh_y;
     s2.status = f.route.status;
+    s2.ksplit = shared_ksplit_down(T, H, I_s);
+    if (s2.ksplit > 1) {
+      s2.y_bf16 = nullptr;
+      s2.partial = f.sh_partial;
+      s2.partial_rows = T;
+    }
     NV_CHECK(launch_grouped_gemm(s2, s));
+    if (s2.ksplit > 1) {
+      NV_CHECK(launch_dependent("shared_split_reduce_kernel<down>", shared_split_reduce_kernel<false>,
+                                dim3((T * H / 4 + 255) / 256), dim3(256), 0, s, (const float*)f.sh_partial,
+                                s2.ksplit, T, H, f.sh_y));
+    }
     if (dbg && dbg->shared_event)
       NV_CHECK(check_cuda(cudaEventRecord(static_cast<cudaEvent_t>(dbg->shared_event), s), "cudaEventRecord"));
   }

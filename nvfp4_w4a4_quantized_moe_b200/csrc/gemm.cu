@@ -122,6 +122,12 @@ struct GemmParams {
   const uint8_t* b0_codes;
   const uint8_t* b1_codes;
   uint32_t* status;
+  // split K (bf16 kinds): each (m-tile, n-tile) is ksplit tiles over K / ksplit
+  // elements, whose epilogues store fp32 partial sums of their data rows to
+  // partial [ksplit][partial_rows][2I (gate/up: gate then up) or H (down)]
+  int ksplit;
+  int partial_rows;
+  float* partial;
 };
 
 // Tensor maps only the CTA-pair kernel reads: the scale atoms as rows of 512
@@ -146,13 +152,13 @@ NVDEV void give_up_pair(uint32_t* status, volatile int* abort_flag, uint32_t pee
   asm volatile("st.relaxed.cluster.shared::cluster.u32 [%0], 1;" ::"r"(peer_abort_addr) : "memory");
 }
 
-NVDEV float silu(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 
 // A tile of the work list: its expert, its 128-row m-tile in this CTA, its
 // n-tile, and whether this CTA stores anything (the second CTA of a pair
 // whose expert has an odd number of m-tiles has no rows of its own).
 struct TileCoord {
   int e, mt, nt;
+  int ks;               // split-K part (bf16 kinds at small batches; 0 otherwise)
   bool valid;
 };
 
@@ -264,14 +270,15 @@ NVDEV void gemm_body(const CUtensorMap& tmA, const CUtensorMap& tmA32, const CUt
     __syncthreads();
     num_tiles = pair_start[p.E] * p.n_tiles;
   } else {
-    num_tiles = (*p.num_mtiles) * p.n_tiles;
+    num_tiles = (*p.num_mtiles) * p.n_tiles * p.ksplit;
   }
   // tile t of the work list: one-CTA tiles are (m-tile, n-tile); pair tiles
   // are (pair m-tile, n-tile), this CTA taking the pair's m-tile `rank`
   auto tile_of = [&](int t) -> TileCoord {
     TileCoord c;
-    c.nt = t % p.n_tiles;
+    c.ks = 0;
     if constexpr (PAIR) {
+      c.nt = t % p.n_tiles;
       const int pmt = t / p.n_tiles;
       int lo = 0, hi = p.E - 1;                  // the last expert whose pairs start at or before pmt
       while (lo < hi) {
@@ -286,7 +293,11 @@ NVDEV void gemm_body(const CUtensorMap& tmA, const CUtensorMap& tmA32, const CUt
       // a CTA without rows of its own loads the pair's first m-tile again
       c.mt = c.valid ? first + (int)rank : min(first, p.cap_tiles - 1);
     } else {
-      c.mt = t / p.n_tiles;
+      // split K: the ksplit parts of one (m-tile, n-tile) are consecutive tiles
+      const int tt = t / p.ksplit;
+      c.ks = t - tt * p.ksplit;
+      c.nt = tt % p.n_tiles;
+      c.mt = tt / p.n_tiles;
       c.e = min(max(p.tile_expert[c.mt], 0), p.E - 1);
       c.valid = true;
     }
@@ -295,7 +306,8 @@ NVDEV void gemm_body(const CUtensorMap& tmA, const CUtensorMap& tmA32, const CUt
   // each CTA of a pair strides over pair tiles by cluster
   const int t_first = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
   const int t_step = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
-  const int KT = (p.K + bk_of<EPI>() - 1) / bk_of<EPI>();
+  // K stages per tile (a split-K tile covers K / ksplit)
+  const int KT = (p.K + bk_of<EPI>() - 1) / bk_of<EPI>() / p.ksplit;
   const int nblk4 = p.K / 64;                    // FP4: scale atoms per 128-row tile
 
   if (warp == 0) {
@@ -342,7 +354,7 @@ NVDEV void gemm_body(const CUtensorMap& tmA, const CUtensorMap& tmA32, const CUt
           uint8_t* sA = st0 + stage * kSB;
           uint8_t* sB = sA + kABytes;
           // x in tensor-map elements: 128 bytes of K per stage either way
-          const int x = kt * (kBf16 ? 64 : kBKBytes);
+          const int x = (tc.ks * KT + kt) * (kBf16 ? 64 : kBKBytes);
           if constexpr (PAIR) {
             // every load of both CTAs counts on the leader's stage barrier,
             // which the leader alone arms with the bytes of both; the other
@@ -589,7 +601,19 @@ NVDEV void gemm_body(const CUtensorMap& tmA, const CUtensorMap& tmA32, const CUt
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty_bar);
-        if (real) {
+        if (real && p.partial) {
+          // split K: this part's gate and up sums; the reduction applies SiLU * up
+          float4* pg = reinterpret_cast<float4*>(p.partial + ((size_t)tc.ks * p.partial_rows + grow) * (2 * p.I) +
+                                                 nt * 128 + half * 64);
+          float4* pu = pg + p.I / 4;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            pg[i] = make_float4(__uint_as_float(rg[4 * i]), __uint_as_float(rg[4 * i + 1]),
+                                __uint_as_float(rg[4 * i + 2]), __uint_as_float(rg[4 * i + 3]));
+            pu[i] = make_float4(__uint_as_float(ru[4 * i]), __uint_as_float(ru[4 * i + 1]),
+                                __uint_as_float(ru[4 * i + 2]), __uint_as_float(ru[4 * i + 3]));
+          }
+        } else if (real) {
           uint4* dst = reinterpret_cast<uint4*>(p.h_bf16 + (size_t)grow * p.I + nt * 128 + half * 64);
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
@@ -673,6 +697,15 @@ NVDEV void gemm_body(const CUtensorMap& tmA, const CUtensorMap& tmA32, const CUt
         if (lane == 0) {
           if constexpr (PAIR) mbar_arrive_remote(acce_leader);
           else mbar_arrive(&acc_empty_bar);
+        }
+        if (kBf16 && real && p.partial) {
+          // split K: this part's sums (the bf16 kind has no scale); the
+          // reduction adds the parts and rounds to bf16
+          float4* pd = reinterpret_cast<float4*>(p.partial + ((size_t)tc.ks * p.partial_rows + grow) * p.H + col0);
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            pd[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
         }
         if (real && p.y_f32) {
           float4* dst = reinterpret_cast<float4*>(p.y_f32 + (size_t)grow * p.H + col0);
@@ -952,7 +985,13 @@ nvfp4_status launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t s) {
   p.b0_codes = a.b0_codes;
   p.b1_codes = a.b1_codes;
   p.status = a.status;
-  const int max_tiles = a.rows_capacity / kBM * p.n_tiles;
+  p.ksplit = std::max(1, a.ksplit);
+  p.partial_rows = a.partial_rows;
+  p.partial = a.partial;
+  NV_REQUIRE(p.ksplit == 1 || (bf && !pair && a.partial && (K / 64) % p.ksplit == 0 && a.partial_rows > 0),
+             NVFP4_ERR_INVALID_ARG, "split K needs a bf16 kind, a partial buffer and K / 64 divisible by %d",
+             p.ksplit);
+  const int max_tiles = a.rows_capacity / kBM * p.n_tiles * p.ksplit;
   if (pair) {
     // scale atoms as rows of 128 32-bit words (512 bytes), four per stage
     const int nblk4 = K / 64;

@@ -56,6 +56,12 @@ struct GroupedGemmArgs {
   // run the FP4 kinds on CTA pairs (clusters of two sharing one 256-row MMA)
   // when K is a multiple of 256; the caller asks for it on large batches
   bool pair = false;
+  // split K (bf16 kinds only): ksplit CTAs per (m-tile, n-tile), each over
+  // K / ksplit, storing fp32 partial sums of their data rows to partial
+  // [ksplit][partial_rows][2I or H] instead of running the epilogue
+  int ksplit = 1;
+  int partial_rows = 0;
+  float* partial = nullptr;
 };
 
 // Batches with at least this many (token, expert) rows run the FP4 GEMMs on

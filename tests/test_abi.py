@@ -34,7 +34,8 @@ def test_forward_launch_count_follows_the_shape():
     """The host-only launch count of the forward: router GEMM, routing (one
     kernel up to 256 tokens, else four), quantise-scatter (inside the routing
     kernel when at most 64 KiB of permuted rows), gate/up, down, combine, plus
-    the shared expert's three kernels and the dynamic modes' amax kernels."""
+    the shared expert's three kernels (and a reduction after each of its GEMMs
+    when few tokens split their K), and the dynamic modes' amax kernels."""
     c = capi()
     n = c.moe_nvfp4_forward_launches
     assert n(32, 8, 256, 128, 2) == 5          # tiny layer: 32 x 2 rows of 144 bytes
@@ -42,7 +43,9 @@ def test_forward_launch_count_follows_the_shape():
     assert n(256, 80, 6144, 2048, 8) == 6
     assert n(257, 80, 6144, 2048, 8) == 9      # multi-kernel routing above 256 tokens
     assert n(8192, 80, 6144, 2048, 8) == 9
-    assert n(16, 80, 6144, 2048, 8, I_shared=2048) == 9
+    # the shared expert at 16 tokens: both GEMMs split K, each adding a reduction
+    assert n(16, 80, 6144, 2048, 8, I_shared=2048) == 11
+    assert n(8192, 80, 6144, 2048, 8, I_shared=2048) == 12
     assert n(32, 8, 256, 128, 2, act_scale_mode="expert") == 6     # per-expert g1: no fused quantisation
     assert n(16, 80, 6144, 2048, 8, act_scale_mode="dynamic") == 7
     assert n(16, 80, 6144, 2048, 8, act_scale_mode="dynamic_expert") == 8

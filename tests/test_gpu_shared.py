@@ -2,7 +2,9 @@
 the routed experts' shape on every token, intermediate rounded to bf16,
 added before the output's bf16 rounding) against the oracle.  The shared
 expert runs on the same persistent tcgen05 GEMM as the routed experts, with
-bf16 operands (kind::f16) instead of block-scaled FP4."""
+bf16 operands (kind::f16) instead of block-scaled FP4.  Below half a wave of
+tiles (every case here but "long") its K is split over several CTAs whose
+fp32 partial sums a second kernel adds in part order."""
 import numpy as np
 import pytest
 import torch
@@ -18,6 +20,8 @@ CASES = {
     "tiny": workloads.CONFIGS["tiny"],
     "mid": workloads.LayerConfig("mid", T=300, H=1024, I=512, E=16, k=4, x_outlier_p=0.001),
     "ragged_small": workloads.LayerConfig("rs", T=3, H=512, I=256, E=6, k=3),
+    # enough tokens that the shared GEMMs fill half a wave: no split K
+    "long": workloads.LayerConfig("long", T=2560, H=1024, I=512, E=16, k=4),
 }
 
 
