@@ -292,6 +292,39 @@ NVFP4_API nvfp4_status moe_nvfp4_forward(const moe_nvfp4_weights* W, const void*
                                void* out_bf16, const moe_nvfp4_debug* dbg, void* ws, size_t ws_bytes,
                                void* stream);
 
+/* ------------------------------------------------------------------------
+ * The forward on host buffers, for a caller whose tokens live in host memory
+ * (no counterpart on the pages: it is the serving wrapper around the layer).
+ * x_host_bf16 [T][H] and out_host_bf16 [T][H] are host pointers, page-locked
+ * for the copies to run asynchronously.  The call enqueues, and returns
+ * without waiting:
+ *   1. the copy of x into a staging buffer at the end of `ws`, on a copy
+ *      stream of the library's own;
+ *   2. moe_nvfp4_forward (per-tensor scales, no debug outputs) on `stream`,
+ *      reading the staged x and writing a staged out;
+ *   3. the copy of out back to out_host_bf16, on a second copy stream.
+ * Consecutive calls on DIFFERENT workspaces overlap: one call's copies run
+ * while another computes.  A call on the same workspace as an earlier one
+ * waits for that call's copies before it reuses its staging buffers.  The
+ * library keeps three CUDA events per workspace (until
+ * moe_nvfp4_host_release) and two copy streams per device.
+ * out_host_bf16 holds the result once the work that moe_nvfp4_host_join
+ * orders has completed (for example, after join then a synchronize of
+ * `stream`).  x_host_bf16 must not change before the copy in has run.  The
+ * workspace comes from moe_nvfp4_workspace_size_host.  It belongs to one
+ * device, and its status word is read with nvfp4_workspace_status as for
+ * moe_nvfp4_forward. */
+NVFP4_API size_t moe_nvfp4_workspace_size_host(int T, int E, int H, int I, int k, int I_shared);
+NVFP4_API nvfp4_status moe_nvfp4_forward_host(const moe_nvfp4_weights* W, const void* x_host_bf16, int T,
+                                    const float* act_gscale, const float* h_gscale, const float* logit_offset,
+                                    void* out_host_bf16, void* ws, size_t ws_bytes, void* stream);
+/* Makes `stream` wait until the last moe_nvfp4_forward_host call on `ws` has
+ * copied its out back (nothing to wait for: returns at once). */
+NVFP4_API nvfp4_status moe_nvfp4_host_join(const void* ws, void* stream);
+/* Waits for the last call on `ws` to finish its copies, then frees the
+ * library's events for that workspace (call before freeing `ws`). */
+NVFP4_API nvfp4_status moe_nvfp4_host_release(const void* ws);
+
 /* Activation global-scale modes of moe_nvfp4_forward_scaled.  The pages fix
  * one calibrated fp32 global scale per activation tensor ("Quantization
  * Setup"); the other modes are an extension: one scale per expert, and g1

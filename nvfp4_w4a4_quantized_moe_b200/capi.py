@@ -89,6 +89,10 @@ _declare("moe_nvfp4_forward", _i, ctypes.POINTER(MoeWeightsStruct), _vp, _i, _vp
          ctypes.POINTER(MoeDebugStruct), _vp, _sz, _vp)
 _declare("moe_nvfp4_forward_scaled", _i, ctypes.POINTER(MoeWeightsStruct), _vp, _i, _i, _vp, _vp, _vp, _vp,
          ctypes.POINTER(MoeDebugStruct), _vp, _sz, _vp)
+_declare("moe_nvfp4_workspace_size_host", _sz, _i, _i, _i, _i, _i, _i)
+_declare("moe_nvfp4_forward_host", _i, ctypes.POINTER(MoeWeightsStruct), _vp, _i, _vp, _vp, _vp, _vp, _vp, _sz, _vp)
+_declare("moe_nvfp4_host_join", _i, _vp, _vp)
+_declare("moe_nvfp4_host_release", _i, _vp)
 _declare("moe_nvfp4_gemm_workspace_size", _sz, _i)
 _declare("moe_reap_keep", _i, _vp, _vp, _i, _i, _vp, _vp)
 _declare("moe_nvfp4_gate_up", _i, ctypes.POINTER(MoeWeightsStruct), _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp,
@@ -111,7 +115,8 @@ EXPORTS = ("nvfp4_last_error", "nvfp4_abi_version", "nvfp4_workspace_status",
            "nvfp4_quantize_weights_noalloc_status", "nvfp4_quantize_act",
            "moe_route_rows_capacity", "moe_route_workspace_size", "moe_route", "moe_nvfp4_workspace_size",
            "moe_nvfp4_forward", "moe_nvfp4_forward_scaled", "moe_nvfp4_workspace_size_shared",
-           "moe_nvfp4_forward_launches",
+           "moe_nvfp4_forward_launches", "moe_nvfp4_workspace_size_host", "moe_nvfp4_forward_host",
+           "moe_nvfp4_host_join", "moe_nvfp4_host_release",
            "moe_nvfp4_gemm_workspace_size", "moe_nvfp4_gate_up",
            "moe_nvfp4_down", "moe_reap_keep",
            "nvfp4_block_stats_compute",
@@ -507,6 +512,54 @@ def moe_nvfp4_forward(W: MoeWeights, x: torch.Tensor, act_gscale: torch.Tensor, 
         dbg_tensors["workspace"] = workspace
         return out, dbg_tensors
     return out
+
+
+def moe_nvfp4_workspace_size_host(T: int, E: int, H: int, I: int, k: int, I_shared: int = 0) -> int:
+    return lib.moe_nvfp4_workspace_size_host(T, E, H, I, k, I_shared)
+
+
+def _host(t, dtype, name):
+    if not isinstance(t, torch.Tensor) or t.is_cuda:
+        raise ValueError(f"{name} must be a host (CPU) tensor")
+    if t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {dtype} tensor")
+    return t
+
+
+def moe_nvfp4_forward_host(W: MoeWeights, x_host: torch.Tensor, act_gscale: torch.Tensor, h_gscale: torch.Tensor,
+                           out_host: torch.Tensor, workspace: torch.Tensor, logit_offset: torch.Tensor | None = None):
+    """The forward on host buffers (per-tensor scales): enqueues x in, the
+    layer on the current stream and out back, and returns without waiting.
+    x_host and out_host are [T, H] bf16 CPU tensors (pinned for the copies to
+    overlap); the workspace is a CUDA uint8 tensor of at least
+    moe_nvfp4_workspace_size_host bytes.  out_host is complete after
+    moe_nvfp4_host_join(workspace) and a synchronize of the current stream."""
+    _host(x_host, torch.bfloat16, "x_host")
+    _host(out_host, torch.bfloat16, "out_host")
+    _cuda(act_gscale, torch.float32, "act_gscale")
+    _cuda(h_gscale, torch.float32, "h_gscale")
+    _cuda(workspace, torch.uint8, "workspace")
+    T, H = x_host.shape
+    if tuple(out_host.shape) != (T, H):
+        raise ValueError("out_host must have the shape of x_host")
+    ws_struct = W.struct()
+    _check(lib.moe_nvfp4_forward_host(ctypes.byref(ws_struct), ctypes.c_void_p(x_host.data_ptr()), T,
+                                      _p(act_gscale), _p(h_gscale), _p(logit_offset),
+                                      ctypes.c_void_p(out_host.data_ptr()), _p(workspace), workspace.numel(),
+                                      _stream()))
+    return out_host
+
+
+def moe_nvfp4_host_join(workspace: torch.Tensor):
+    """Makes the current stream wait for the last host-buffer call on this
+    workspace to have copied its out back."""
+    _check(lib.moe_nvfp4_host_join(_p(workspace), _stream()))
+
+
+def moe_nvfp4_host_release(workspace: torch.Tensor):
+    """Waits for the workspace's last host-buffer call and frees the
+    library's events for it."""
+    _check(lib.moe_nvfp4_host_release(_p(workspace)))
 
 
 def moe_nvfp4_gate_up(W: MoeWeights, a_codes, a_scales, expert_offsets, expert_counts, act_gscale, h_gscale,

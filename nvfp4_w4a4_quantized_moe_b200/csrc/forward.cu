@@ -6,6 +6,8 @@
 // Setup"), "K-EXAONE-152B-A23B-REAP-80E-BF16" model card ("Pruning Setup",
 // "Routing behavior").
 #include <algorithm>
+#include <mutex>
+#include <unordered_map>
 
 #include "common.cuh"
 #include "gemm.cuh"
@@ -664,6 +666,122 @@ extern "C" nvfp4_status moe_nvfp4_forward_scaled(const moe_nvfp4_weights* W, con
                                                  void* stream) {
   return forward_impl(W, x_bf16, T, act_scale_mode, act_gscale, h_gscale, logit_offset, out_bf16, dbg, ws, ws_bytes,
                       stream);
+}
+
+// ---------------------------------------------------------------------------
+// The forward on host buffers.  x is copied into a staging buffer at the end
+// of the workspace and out back from another, each on a copy stream of the
+// library's own, so that consecutive calls on different workspaces overlap
+// one call's copies with another's compute.  Per workspace the library keeps
+// three events (x landed, forward done, out copied back); a call waits for
+// the previous call on the same workspace before it overwrites that call's
+// staging buffers.
+// ---------------------------------------------------------------------------
+namespace {
+struct HostSlot {
+  cudaEvent_t in = nullptr, done = nullptr, out = nullptr;
+  bool used = false;
+};
+std::mutex g_host_mu;
+std::unordered_map<const void*, HostSlot> g_host_slots;      // keyed by workspace
+cudaStream_t g_copy_in[64], g_copy_out[64];                  // per device
+
+size_t round256(size_t n) { return (n + 255) / 256 * 256; }
+
+nvfp4_status host_slot_and_streams(const void* ws, HostSlot** slot, cudaStream_t* cin, cudaStream_t* cout) {
+  int dev = 0;
+  NV_CHECK(check_cuda(cudaGetDevice(&dev), "cudaGetDevice"));
+  NV_REQUIRE(dev >= 0 && dev < 64, NVFP4_ERR_CUDA, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_host_mu);
+  if (!g_copy_in[dev]) {
+    NV_CHECK(check_cuda(cudaStreamCreateWithFlags(&g_copy_in[dev], cudaStreamNonBlocking), "cudaStreamCreate"));
+    NV_CHECK(check_cuda(cudaStreamCreateWithFlags(&g_copy_out[dev], cudaStreamNonBlocking), "cudaStreamCreate"));
+  }
+  HostSlot& h = g_host_slots[ws];
+  if (!h.in) {
+    NV_CHECK(check_cuda(cudaEventCreateWithFlags(&h.in, cudaEventDisableTiming), "cudaEventCreate"));
+    NV_CHECK(check_cuda(cudaEventCreateWithFlags(&h.done, cudaEventDisableTiming), "cudaEventCreate"));
+    NV_CHECK(check_cuda(cudaEventCreateWithFlags(&h.out, cudaEventDisableTiming), "cudaEventCreate"));
+  }
+  *slot = &h;
+  *cin = g_copy_in[dev];
+  *cout = g_copy_out[dev];
+  return NVFP4_OK;
+}
+}  // namespace
+
+extern "C" size_t moe_nvfp4_workspace_size_host(int T, int E, int H, int I, int k, int I_shared) {
+  if (T < 1 || H < 1) return 0;
+  const size_t base = moe_nvfp4_workspace_size_shared(T, E, H, I, k, I_shared);
+  if (base == 0) return 0;
+  return round256(base) + 2 * round256((size_t)T * H * 2);
+}
+
+extern "C" nvfp4_status moe_nvfp4_forward_host(const moe_nvfp4_weights* W, const void* x_host_bf16, int T,
+                                               const float* act_gscale, const float* h_gscale,
+                                               const float* logit_offset, void* out_host_bf16, void* ws,
+                                               size_t ws_bytes, void* stream) {
+  NV_CHECK(nvfp4moe_check_weights(W));
+  NV_REQUIRE(x_host_bf16 && out_host_bf16 && act_gscale && h_gscale, NVFP4_ERR_INVALID_ARG,
+             "moe_nvfp4_forward_host: a required pointer is NULL");
+  NV_REQUIRE(T >= 1, NVFP4_ERR_INVALID_ARG, "moe_nvfp4_forward_host: T=%d", T);
+  const size_t need = moe_nvfp4_workspace_size_host(T, W->E, W->H, W->I, W->k, W->I_shared);
+  NV_REQUIRE(ws && ws_bytes >= need && aligned(ws, 256), NVFP4_ERR_WORKSPACE,
+             "moe_nvfp4_forward_host: needs a 256-byte aligned workspace of %zu bytes", need);
+  const size_t base = round256(moe_nvfp4_workspace_size_shared(T, W->E, W->H, W->I, W->k, W->I_shared));
+  const size_t io = (size_t)T * W->H * 2;
+  uint8_t* x_dev = static_cast<uint8_t*>(ws) + base;
+  uint8_t* out_dev = x_dev + round256(io);
+  HostSlot* h = nullptr;
+  cudaStream_t cin = nullptr, cout = nullptr;
+  NV_CHECK(host_slot_and_streams(ws, &h, &cin, &cout));
+  cudaStream_t s = as_stream(stream);
+  // x in, once the previous call on this workspace has read its x
+  if (h->used) NV_CHECK(check_cuda(cudaStreamWaitEvent(cin, h->done, 0), "cudaStreamWaitEvent"));
+  NV_CHECK(check_cuda(cudaMemcpyAsync(x_dev, x_host_bf16, io, cudaMemcpyHostToDevice, cin), "copy x in"));
+  NV_CHECK(check_cuda(cudaEventRecord(h->in, cin), "cudaEventRecord"));
+  // the forward on the caller's stream, once x has landed and the previous
+  // call's out has left the staging buffer
+  NV_CHECK(check_cuda(cudaStreamWaitEvent(s, h->in, 0), "cudaStreamWaitEvent"));
+  if (h->used) NV_CHECK(check_cuda(cudaStreamWaitEvent(s, h->out, 0), "cudaStreamWaitEvent"));
+  NV_CHECK(forward_impl(W, x_dev, T, NVFP4_ACT_SCALE_TENSOR, const_cast<float*>(act_gscale), h_gscale,
+                        logit_offset, out_dev, nullptr, ws, base, stream));
+  NV_CHECK(check_cuda(cudaEventRecord(h->done, s), "cudaEventRecord"));
+  // out back
+  NV_CHECK(check_cuda(cudaStreamWaitEvent(cout, h->done, 0), "cudaStreamWaitEvent"));
+  NV_CHECK(check_cuda(cudaMemcpyAsync(out_host_bf16, out_dev, io, cudaMemcpyDeviceToHost, cout), "copy out back"));
+  NV_CHECK(check_cuda(cudaEventRecord(h->out, cout), "cudaEventRecord"));
+  h->used = true;
+  return NVFP4_OK;
+}
+
+extern "C" nvfp4_status moe_nvfp4_host_join(const void* ws, void* stream) {
+  NV_REQUIRE(ws, NVFP4_ERR_INVALID_ARG, "moe_nvfp4_host_join: ws is NULL");
+  cudaEvent_t ev = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_host_mu);
+    auto it = g_host_slots.find(ws);
+    if (it == g_host_slots.end() || !it->second.used) return NVFP4_OK;
+    ev = it->second.out;
+  }
+  return check_cuda(cudaStreamWaitEvent(as_stream(stream), ev, 0), "cudaStreamWaitEvent");
+}
+
+extern "C" nvfp4_status moe_nvfp4_host_release(const void* ws) {
+  NV_REQUIRE(ws, NVFP4_ERR_INVALID_ARG, "moe_nvfp4_host_release: ws is NULL");
+  HostSlot h;
+  {
+    std::lock_guard<std::mutex> lock(g_host_mu);
+    auto it = g_host_slots.find(ws);
+    if (it == g_host_slots.end()) return NVFP4_OK;
+    h = it->second;
+    g_host_slots.erase(it);
+  }
+  if (h.used) NV_CHECK(check_cuda(cudaEventSynchronize(h.out), "cudaEventSynchronize"));
+  cudaEventDestroy(h.in);
+  cudaEventDestroy(h.done);
+  cudaEventDestroy(h.out);
+  return NVFP4_OK;
 }
 
 extern "C" nvfp4_status moe_reap_keep(const double* saliency_sum, const unsigned long long* saliency_count, int E,

@@ -89,7 +89,7 @@ using namespace nvfp4moe;
 
 extern "C" const char* nvfp4_last_error(void) { return g_last_error; }
 
-extern "C" int nvfp4_abi_version(void) { return 5; }
+extern "C" int nvfp4_abi_version(void) { return 6; }
 
 extern "C" nvfp4_status nvfp4_workspace_status(void* ws, void* stream) {
   NV_REQUIRE(ws != nullptr, NVFP4_ERR_INVALID_ARG, "nvfp4_workspace_status: ws is NULL");

@@ -48,7 +48,7 @@ static inline int router_smem_bytes(int E) { return router_stages(E) * router_st
 // some SMs) measured slower.  A function of the shape only, so results are
 // the same on every device.
 int router_splits(int T, int H) {
-  const int mt = (T + kRBM - 1) / kRBM;
+  const int mt = std::max(1, (T + kRBM - 1) / kRBM);
   const int kt = H / kRBK;
   int sp = 148 / mt;
   sp = std::min(sp, std::max(1, kt / 4));
@@ -665,7 +665,8 @@ RouteScratch carve_route_scratch(Carver& c, int T, int E, int k) {
   r.num_mtiles = c.take<int32_t>(1);
   r.row_w = c.take<float>((size_t)cap);
   // router_splits() never exceeds ceil(148 / m-tiles), whatever H is
-  r.partial = c.take<float>((size_t)((148 + (T + kRBM - 1) / kRBM - 1) / ((T + kRBM - 1) / kRBM)) * T * E);
+  const int mt = std::max(1, (T + kRBM - 1) / kRBM);
+  r.partial = c.take<float>((size_t)((148 + mt - 1) / mt) * T * E);
   return r;
 }
 

@@ -23,10 +23,19 @@ def test_library_exports_every_declared_function():
 
 def test_abi_version_and_sizes():
     c = capi()
-    assert c.abi_version() == 5
+    assert c.abi_version() == 6
     assert c.moe_route_rows_capacity(8192, 80, 8) == 75776
     assert c.moe_route_rows_capacity(16, 80, 8) % 128 == 0
     assert c.lib.moe_nvfp4_workspace_size(16, 80, 6144, 2048, 8) > 0
+    # the host-buffer forward: the forward's workspace, then x and out staging
+    r256 = lambda n: (n + 255) // 256 * 256  # noqa: E731
+    for T in (1, 16, 8192):
+        base = c.lib.moe_nvfp4_workspace_size_shared(T, 80, 6144, 2048, 8, 0)
+        assert c.moe_nvfp4_workspace_size_host(T, 80, 6144, 2048, 8) == r256(base) + 2 * r256(T * 6144 * 2)
+    assert c.moe_nvfp4_workspace_size_host(0, 80, 6144, 2048, 8) == 0
+    # zero tokens: the sizes stay defined (no division by the m-tile count)
+    assert c.lib.moe_nvfp4_workspace_size(0, 80, 6144, 2048, 8) > 0
+    assert c.lib.moe_route_workspace_size(0, 80, 8) > 0
     assert c.lib.nvfp4_quantize_weights_workspace_size(240) >= 256
 
 
@@ -89,6 +98,12 @@ def test_host_side_argument_checks():
     assert lib.moe_nvfp4_forward(ctypes.byref(W), fake, 4, fake, fake, None, fake, None, fake, 1 << 30, None) == 2
     W = c.MoeWeightsStruct(8, 256, 256, 2, 2.5, *([fake] * 11), None, None, None, 0, 2)
     assert lib.moe_nvfp4_forward(ctypes.byref(W), fake, 4, fake, fake, None, fake, None, fake, 16, None) == 5
+    # the host-buffer forward: the same shape checks, NULL buffers, its own workspace size
+    assert lib.moe_nvfp4_forward_host(ctypes.byref(W), fake, 4, fake, fake, None, fake, fake, 16, None) == 5
+    assert lib.moe_nvfp4_forward_host(ctypes.byref(W), None, 4, fake, fake, None, fake, fake, 1 << 30, None) == 1
+    W = c.MoeWeightsStruct(8, 192, 128, 2, 2.5, *([fake] * 11))
+    assert lib.moe_nvfp4_forward_host(ctypes.byref(W), fake, 4, fake, fake, None, fake, fake, 1 << 30, None) == 2
+    assert lib.moe_nvfp4_host_join(None, None) == 1 and lib.moe_nvfp4_host_release(None) == 1
 
 
 @pytest.mark.parametrize("header", ["nvfp4_moe.h", "nvfp4_moe_testing.h"])
