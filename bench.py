@@ -182,12 +182,23 @@ class ClockSampler:
 GEMM_SOURCES = ("gemm.cu", "gemm.cuh", "common.cuh")
 
 
+def _code_only(text: str) -> str:
+    """C++ source without its comments and blank lines, so that an edit of a
+    comment does not change the hash (the sources hold no comment markers
+    inside string literals)."""
+    import re
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = (re.sub(r"//.*$", "", ln).rstrip() for ln in text.splitlines())
+    return "\n".join(ln for ln in lines if ln)
+
+
 def gemm_source_sha() -> str:
-    """Hash of the sources the GEMM kernel is compiled from."""
+    """Hash of the code (comments stripped) the GEMM kernel is compiled from."""
     import hashlib
     h = hashlib.sha256()
     for name in GEMM_SOURCES:
-        h.update(open(os.path.join(ROOT, "nvfp4_w4a4_quantized_moe_b200", "csrc", name), "rb").read())
+        src = open(os.path.join(ROOT, "nvfp4_w4a4_quantized_moe_b200", "csrc", name), encoding="utf-8").read()
+        h.update(_code_only(src).encode())
     return h.hexdigest()[:16]
 
 

@@ -20,6 +20,10 @@
 // accumulator (warp w reads TMEM lanes 32*(w%4).., columns split in two
 // halves).  The grid is persistent: one CTA
 // per SM walks the (m-tile, n-tile) list, whose length is read on the device.
+// Batches of at least 2048 rows run the FP4 kinds on CTA pairs (clusters of
+// two sharing one 256-row MMA, each CTA loading half of B), whose down
+// epilogue writes y by TMA tensor stores; at small batches the bf16 kinds of
+// the shared expert split K over several CTAs and store fp32 partial sums.
 // Every wait is bounded in time; a wait that gives up sets the workspace
 // status word and the CTA winds down after its outstanding copies land.
 #include <cstring>

@@ -53,6 +53,13 @@ def test_recorded_traffic_matches_kernel_workload_and_source_hash():
     assert bench.recorded_traffic("grouped_fp4_gemm_kernel<0>", "no-such-workload") == (None, None)
 
 
+def test_source_hash_ignores_comments_but_not_code():
+    src = "int a = 1;  // one\n/* a\n   block */\nint b = 2;\n\n// only a comment\n"
+    assert bench._code_only(src) == "int a = 1;\nint b = 2;"
+    assert bench._code_only(src.replace("// one", "// uno")) == bench._code_only(src)
+    assert bench._code_only(src.replace("2;", "3;")) != bench._code_only(src)
+
+
 def test_weak_scaling_value_counts_every_rank():
     # 16 tokens per rank, 4 ranks, 0.25 ms for the slowest rank's step
     assert bench.weak_scaling_value(16, 4, 0.25) == pytest.approx(16 * 4 / 0.25e-3)
