@@ -22,6 +22,12 @@ CASES = {
     "ragged_small": workloads.LayerConfig("rs", T=3, H=512, I=256, E=6, k=3),
     # k > 8 takes the combine kernel's wide variant
     "wide_k": workloads.LayerConfig("wk", T=40, H=512, I=256, E=12, k=10),
+    # a single token
+    "one_token": workloads.LayerConfig("ot", T=1, H=512, I=256, E=8, k=2),
+    # the largest expert count and top-k the ABI accepts: 9,600 rows run the
+    # CTA-pair GEMMs, most experts hold one (odd) m-tile, so most pairs have a
+    # second CTA without rows, and k = 16 takes the wide combine
+    "max_experts": workloads.LayerConfig("mx", T=600, H=512, I=256, E=256, k=16, logit_offset_std=0.5),
 }
 
 
