@@ -28,6 +28,9 @@ def _layer(cfg):
 @pytest.mark.parametrize("name,cfg", [
     ("tiny", workloads.CONFIGS["tiny"]),
     ("mid", workloads.LayerConfig("mid", T=300, H=1024, I=512, E=16, k=4, logit_offset_std=0.5)),
+    # 2,400 rows: the CTA-pair GEMMs, whose down epilogue both CTAs of a pair
+    # run (sums of squares of their own rows)
+    ("pair", workloads.LayerConfig("pr", T=600, H=1024, I=256, E=16, k=4, logit_offset_std=0.5)),
 ])
 def test_saliency_and_pruned_layer_match_oracle(name, cfg):
     require_cuda()
