@@ -55,6 +55,11 @@ def test_forward_launch_count_follows_the_shape():
     # the shared expert at 16 tokens: both GEMMs split K, each adding a reduction
     assert n(16, 80, 6144, 2048, 8, I_shared=2048) == 11
     assert n(8192, 80, 6144, 2048, 8, I_shared=2048) == 12
+    # the split K of the shared GEMMs starts below half a wave of tiles: 300
+    # tokens are 3 x 4 tiles each (both split), 2560 tokens 20 x 4 (neither)
+    assert n(300, 16, 1024, 512, 4, I_shared=512) == 9 + 3 + 2
+    assert n(2560, 16, 1024, 512, 4, I_shared=512) == 9 + 3
+    assert n(3, 6, 512, 256, 3, I_shared=256) == 5 + 3 + 2
     assert n(32, 8, 256, 128, 2, act_scale_mode="expert") == 6     # per-expert g1: no fused quantisation
     assert n(16, 80, 6144, 2048, 8, act_scale_mode="dynamic") == 7
     assert n(16, 80, 6144, 2048, 8, act_scale_mode="dynamic_expert") == 8
