@@ -47,8 +47,8 @@ FP4_OVER_BF16 = 4.0            # nominal dense ratio (9 vs 2.25 PFLOP/s)
 
 def kernels_per_step(c, cfg) -> int:
     """Kernels one forward launches, as the library counts them: router GEMM,
-    routing (one single-block kernel up to 256 tokens, else top-k and three
-    permutation kernels), quantise-scatter (folded into the routing kernel
+    routing (one single-block kernel up to 256 tokens, else a top-k and a
+    permutation kernel), quantise-scatter (folded into the routing kernel
     for small layers), the two GEMMs and the combine."""
     return c.moe_nvfp4_forward_launches(cfg.T, cfg.E, cfg.H, cfg.I, cfg.k)
 NVFP4_BYTES_PER_ELEM = 0.5 + 1.0 / 16

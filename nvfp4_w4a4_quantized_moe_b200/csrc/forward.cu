@@ -425,7 +425,7 @@ extern "C" int moe_nvfp4_forward_launches(int T, int E, int H, int I, int k, int
     n += (shared_ksplit_gate_up(T, H, I_shared) > 1) + (shared_ksplit_down(T, H, I_shared) > 1);   // reductions
   }
   if (mode & kActDynamic) n += 1;                                   // token amax
-  n += 1 + (T <= 256 ? 1 : 4);                                      // router GEMM, routing
+  n += 1 + (T <= 256 ? 1 : 2);                                      // router GEMM, routing
   if (mode == NVFP4_ACT_SCALE_DYNAMIC_EXPERT) n += 1;               // expert amax
   if (!(mode == NVFP4_ACT_SCALE_TENSOR && route_fuses_x_quantise(T, H, k))) n += 1;   // quantise-scatter
   n += 2 + 1;                                                       // gate/up, down, combine

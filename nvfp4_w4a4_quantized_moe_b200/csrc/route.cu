@@ -192,8 +192,10 @@ __global__ void __launch_bounds__(kRThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// Top-k: one warp per token.  Lane l holds experts l, l+32, ...; each of the k
-// rounds is a warp-wide argmax of sigma + bias (ties to the lower expert).
+// Top-k: the logits (split-ordered sums of the router GEMM's partials), then
+// sigma and the selection key of sigma + bias for every (token, expert), then
+// k selection rounds per token by one warp, each a warp-wide argmax of
+// sigma + bias (ties to the lower expert).
 // ---------------------------------------------------------------------------
 constexpr int kMaxE = 256, kMaxK = 16;
 
@@ -234,18 +236,20 @@ NVDEV void expert_score(float l, float b, float& sig, uint32_t& key) {
 }
 
 // The k selection rounds of one token by one warp, from each lane's scores
-// of experts lane, lane+32, ... (key 0 for an absent expert).  Each round is
-// a warp max of the keys, then a warp min of the expert ids that reach it:
-// the largest score, ties to the lower expert.  Lane j < k returns slot j's
-// expert and weight (sigma / sum of the selected sigmas, times rsf; the sum
-// in slot order).
+// of experts lane, lane+32, ... (PER slots per lane, PER * 32 >= E; key 0
+// for an absent expert).  Each round is a warp max of the keys, then a warp
+// min of the expert ids that reach it: the largest score, ties to the lower
+// expert.  Lane j < k returns slot j's expert and weight (sigma / sum of the
+// selected sigmas, times rsf; the sum in slot order).  An absent expert's
+// key 0 never wins a round, so every PER that covers E gives the same result.
+template <int PER>
 NVDEV void select_topk(const float* sig, uint32_t* key, int k, float rsf, int lane, int& out_idx, float& out_w) {
   float sum = 0.0f, my_sig = 0.0f;
   int my_idx = 0;
   for (int j = 0; j < k; ++j) {
     uint32_t bk = 0u, be = 0xffffffffu;
 #pragma unroll
-    for (int i = 0; i < kMaxE / 32; ++i)       // ascending i: a tie keeps the lower expert
+    for (int i = 0; i < PER; ++i)              // ascending i: a tie keeps the lower expert
       if (key[i] > bk) {
         bk = key[i];
         be = (uint32_t)(lane + 32 * i);
@@ -255,7 +259,7 @@ NVDEV void select_topk(const float* sig, uint32_t* key, int k, float rsf, int la
     // the owner lane marks the winner and broadcasts its sigma
     float s_own = 0.0f;
 #pragma unroll
-    for (int i = 0; i < kMaxE / 32; ++i)
+    for (int i = 0; i < PER; ++i)
       if (lane + 32 * i == win) {
         s_own = sig[i];
         key[i] = 0u;
@@ -271,84 +275,61 @@ NVDEV void select_topk(const float* sig, uint32_t* key, int k, float rsf, int la
   out_w = __fmul_rn(__fdiv_rn(my_sig, sum), rsf);
 }
 
-// Top-k of token t by one warp.  Lane l holds experts l, l+32, ...; each of
-// the k rounds is a warp-wide argmax of sigma + bias (ties to the lower
-// expert).  Lane j < k returns slot j's expert and weight.
-NVDEV void topk_token(const float* __restrict__ src, int splits, const float* __restrict__ offset,
-                      float* __restrict__ logits, const float* __restrict__ bias, int T, int E, int k, float rsf,
-                      int t, int lane, int& out_idx, float& out_w) {
-  float sig[kMaxE / 32];
-  uint32_t key[kMaxE / 32];
-  const int per = (E + 31) >> 5;
-  // every slot's logit first, then the scores.  With up to eight splits
-  // (large batches) all of the lane's partial sums are loaded before any is
-  // added, so their latencies overlap; the sums keep split order.
-  float lg[kMaxE / 32];
-  if (splits > 0 && splits <= 8) {
-    const size_t stride = (size_t)T * E;
-    float v[kMaxE / 32][8];
+// Top-k of one token whose scores sit in shared memory: sigma bits at
+// s_sig[e], selection keys at s_key[e], e < E.
+template <int PER>
+NVDEV void select_topk_smem(const uint32_t* s_sig, const uint32_t* s_key, int E, int k, float rsf, int lane,
+                            int& idx, float& w) {
+  float sig[PER];
+  uint32_t key[PER];
 #pragma unroll
-    for (int i = 0; i < kMaxE / 32; ++i) {
-      const int e = lane + 32 * i;
-      const float* p = src + (size_t)t * E + e;
-#pragma unroll
-      for (int u = 0; u < 8; ++u) v[i][u] = (i < per && e < E && u < splits) ? p[(size_t)u * stride] : 0.0f;
-    }
-#pragma unroll
-    for (int i = 0; i < kMaxE / 32; ++i) {
-      const int e = lane + 32 * i;
-      float l = v[i][0];
-#pragma unroll
-      for (int u = 1; u < 8; ++u)
-        if (u < splits) l = __fadd_rn(l, v[i][u]);
-      if (i < per && e < E) {
-        if (offset) l = __fadd_rn(l, offset[e]);
-        logits[(size_t)t * E + e] = l;
-      }
-      lg[i] = l;
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < kMaxE / 32; ++i) {
-      const int e = lane + 32 * i;
-      lg[i] = (i < per && e < E) ? token_logit(src, splits, offset, logits, T, E, t, e) : 0.0f;   // splits < 0: no write
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < kMaxE / 32; ++i) {
+  for (int i = 0; i < PER; ++i) {
     const int e = lane + 32 * i;
-    sig[i] = 0.0f;
-    key[i] = 0u;
-    if (i < per && e < E) expert_score(lg[i], bias[e], sig[i], key[i]);
+    sig[i] = e < E ? __uint_as_float(s_sig[e]) : 0.0f;
+    key[i] = e < E ? s_key[e] : 0u;
   }
-  select_topk(sig, key, k, rsf, lane, out_idx, out_w);
+  select_topk<PER>(sig, key, k, rsf, lane, idx, w);
 }
 
-__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ src, int splits,
-                                                   const float* __restrict__ offset, float* __restrict__ logits,
-                                                   const float* __restrict__ bias, int T, int E, int k, float rsf,
-                                                   int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
-  griddep_wait();
-  griddep_launch();
-  const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (t >= T) return;
-  int idx;
-  float w;
-  topk_token(src, splits, offset, logits, bias, T, E, k, rsf, t, lane, idx, w);
-  if (lane < k) {
-    topk_idx[(size_t)t * k + lane] = idx;
-    topk_w[(size_t)t * k + lane] = w;
+// The same for any E <= 256, with the fewest slots per lane that cover E.
+NVDEV void select_topk_smem_any(const uint32_t* s_sig, const uint32_t* s_key, int E, int k, float rsf, int lane,
+                                int& idx, float& w) {
+  switch ((E + 31) >> 5) {
+    case 1: select_topk_smem<1>(s_sig, s_key, E, k, rsf, lane, idx, w); break;
+    case 2: select_topk_smem<2>(s_sig, s_key, E, k, rsf, lane, idx, w); break;
+    case 3: select_topk_smem<3>(s_sig, s_key, E, k, rsf, lane, idx, w); break;
+    case 4: select_topk_smem<4>(s_sig, s_key, E, k, rsf, lane, idx, w); break;
+    default: select_topk_smem<kMaxE / 32>(s_sig, s_key, E, k, rsf, lane, idx, w); break;
   }
 }
 
 // ---------------------------------------------------------------------------
-// Permutation.  Tokens are cut into chunks of 256; inside a chunk a bitmap per
-// expert marks the tokens that chose it, so the rank of (token, expert) among
-// the chunk's tokens is a popcount.  A single-block scan turns per-chunk
-// counts into row bases.  Everything is integer and order-independent.
+// Larger batches (more than 256 tokens): two kernels.
+//
+// topk_bitmap_kernel: one block per 32 tokens.  Its threads compute every
+// (token, expert) logit, sigma and selection key of the block's tokens into
+// shared memory, one pair per thread and step; then one warp per token runs
+// the selection rounds from there.  The block's tokens that chose expert e
+// form one 32-bit word (bit = token's place in the block), written to
+// bm[block][e], and its popcount to blk_counts[e][block].  The kernel also
+// fills perm with -1 and row_w with 0 over the padded capacity.
+//
+// perm_scan_scatter_kernel: one block per 256 tokens.  Each block sums
+// blk_counts per expert (one warp per expert) into the totals and the
+// exclusive prefix of its own 32-token blocks, pads the totals to 128 rows
+// and scans them into the experts' first rows, then places each of its
+// (token, slot) pairs: row = expert's first row + rows of the expert's
+// earlier blocks + popcount of the lower bits of the block's word.  That is
+// the token's rank among the expert's tokens, so rows keep token order.
+// Block 0 also writes expert_offsets, the counts and the m-tile map.
+// Everything after the scores is integer and order-independent.
 // ---------------------------------------------------------------------------
-constexpr int kChunk = 256;
+constexpr int kTkTokens = 32;                      // tokens per top-k block: one bitmap word
+constexpr int kTkThreads = 1024;                   // one warp per token for the selection
+constexpr int kTkPairs = kTkTokens * kMaxE / kTkThreads;   // (token, expert) pairs per thread, at most 8
+constexpr int kScWords = 8;                        // bitmap words per scatter block
+constexpr int kScTokens = kScWords * kTkTokens;    // 256 tokens
+constexpr int kScThreads = 1024;
 
 // In-place exclusive scan of sp[0..256) by warp 0 of the block (eight entries
 // per lane, then a shuffle scan of the lane sums); the caller synchronises
@@ -372,93 +353,156 @@ NVDEV void warp0_exclusive_scan256(int32_t* sp) {
   for (int j = 0; j < 8; ++j) sp[lane * 8 + j] = inc - run + ex[j];
 }
 
-NVDEV void build_bitmap(uint32_t (*bm)[kChunk / 32], const int32_t* topk_idx, int T, int E, int k, int t) {
-  for (int i = threadIdx.x; i < E * (kChunk / 32); i += blockDim.x) bm[i / (kChunk / 32)][i % (kChunk / 32)] = 0;
-  __syncthreads();
-  if (t < T)
-    for (int j = 0; j < k; ++j) atomicOr(&bm[topk_idx[(size_t)t * k + j]][threadIdx.x >> 5], 1u << (threadIdx.x & 31));
-  __syncthreads();
-}
+// Dynamic shared memory of topk_bitmap_kernel: sigma bits and keys of the
+// block's 32 tokens (64 KiB at E = 256).
+inline int topk_bitmap_smem_bytes(int E) { return 2 * kTkTokens * E * (int)sizeof(uint32_t); }
 
-// Also fills perm with -1 and row_w with 0 over the padded capacity; the
-// scatter, two launches later, overwrites the real rows.
-__global__ void __launch_bounds__(kChunk) perm_count_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
-                                                            int32_t* __restrict__ chunk_counts, int cap,
-                                                            int32_t* __restrict__ perm, float* __restrict__ row_w) {
-  __shared__ uint32_t bm[kMaxE][kChunk / 32];
+__global__ void __launch_bounds__(kTkThreads, 1) topk_bitmap_kernel(
+    const float* __restrict__ src, int splits, const float* __restrict__ offset, float* __restrict__ logits,
+    const float* __restrict__ bias, int T, int E, int k, float rsf, int cap, int32_t* __restrict__ topk_idx,
+    float* __restrict__ topk_w, uint32_t* __restrict__ bm, int32_t* __restrict__ blk_counts, int nblk,
+    int32_t* __restrict__ perm, float* __restrict__ row_w) {
+  extern __shared__ uint32_t s_score[];           // [32 * E] sigma bits, then [32 * E] keys
+  __shared__ uint32_t s_bm[kMaxE];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int e = tid; e < E; e += blockDim.x) s_bm[e] = 0u;
   griddep_wait();
   griddep_launch();
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < cap; i += gridDim.x * blockDim.x) {
+  for (int i = blockIdx.x * blockDim.x + tid; i < cap; i += gridDim.x * blockDim.x) {
     perm[i] = -1;
     row_w[i] = 0.0f;
   }
-  build_bitmap(bm, topk_idx, T, E, k, blockIdx.x * kChunk + threadIdx.x);
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int n = 0;
+  const int t0 = blockIdx.x * kTkTokens;
+  const int nt = min(kTkTokens, T - t0);
+  const int np = nt * E;                          // the block's pairs are src[t0 * E + i], i < np
+  // the logits of this thread's pairs i = tid + j * 1024: the split-ordered
+  // sum of the partials, two splits' loads of every pair in flight at once
+  float acc[kTkPairs];
+  if (splits > 0) {
+    const size_t stride = (size_t)T * E;
+    const float* base = src + (size_t)t0 * E;
+    for (int u0 = 0; u0 < splits; u0 += 2) {
+      float v[2][kTkPairs];
 #pragma unroll
-    for (int w = 0; w < kChunk / 32; ++w) n += __popc(bm[e][w]);
-    chunk_counts[(size_t)blockIdx.x * E + e] = n;
+      for (int uu = 0; uu < 2; ++uu)
+#pragma unroll
+        for (int j = 0; j < kTkPairs; ++j) {
+          const int i = tid + j * kTkThreads;
+          v[uu][j] = (u0 + uu < splits && i < np) ? base[(size_t)(u0 + uu) * stride + i] : 0.0f;
+        }
+#pragma unroll
+      for (int uu = 0; uu < 2; ++uu)
+#pragma unroll
+        for (int j = 0; j < kTkPairs; ++j)
+          if (u0 + uu < splits) acc[j] = (u0 + uu == 0) ? v[uu][j] : __fadd_rn(acc[j], v[uu][j]);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < kTkPairs; ++j) {
+      const int i = tid + j * kTkThreads;
+      acc[j] = i < np ? src[(size_t)t0 * E + i] : 0.0f;
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < kTkPairs; ++j) {
+    const int i = tid + j * kTkThreads;
+    if (i < np) {
+      const int e = i % E;
+      float l = acc[j];
+      if (splits > 0) {
+        if (offset) l = __fadd_rn(l, offset[e]);
+        logits[(size_t)t0 * E + i] = l;
+      }
+      float sig;
+      uint32_t key;
+      expert_score(l, bias[e], sig, key);
+      s_score[i] = __float_as_uint(sig);
+      s_score[kTkTokens * E + i] = key;
+    }
+  }
+  __syncthreads();
+  if (warp < nt) {
+    int idx;
+    float w;
+    select_topk_smem_any(s_score + warp * E, s_score + kTkTokens * E + warp * E, E, k, rsf, lane, idx, w);
+    if (lane < k) {
+      topk_idx[(size_t)(t0 + warp) * k + lane] = idx;
+      topk_w[(size_t)(t0 + warp) * k + lane] = w;
+      atomicOr(&s_bm[idx], 1u << warp);
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += blockDim.x) {
+    const uint32_t word = s_bm[e];
+    bm[(size_t)blockIdx.x * E + e] = word;
+    blk_counts[(size_t)e * nblk + blockIdx.x] = __popc(word);
   }
 }
 
-// One block of 256 threads (E <= 256): per-expert totals, 128-row padding,
-// exclusive scan into expert_offsets, per-chunk row bases (in place) and the
-// m-tile -> expert map.
-__global__ void __launch_bounds__(256) perm_scan_kernel(int32_t* __restrict__ chunk_counts, int nchunks, int E,
-                                                        int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
-                                                        int32_t* __restrict__ tile_expert,
-                                                        int32_t* __restrict__ num_mtiles) {
+__global__ void __launch_bounds__(kScThreads, 1) perm_scan_scatter_kernel(
+    const int32_t* __restrict__ topk_idx, const float* __restrict__ topk_w, int T, int E, int k,
+    const uint32_t* __restrict__ bm, const int32_t* __restrict__ blk_counts, int nblk,
+    int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ tile_expert,
+    int32_t* __restrict__ num_mtiles, int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm,
+    float* __restrict__ row_w) {
   __shared__ int32_t sp[256];
+  __shared__ int32_t s_total[kMaxE];
+  __shared__ int32_t s_pre[kMaxE][kScWords];       // rows of expert e in the 32-token blocks before b0 + s
   griddep_wait();
   griddep_launch();
-  const int e = threadIdx.x;
-  int total = 0;
-  if (e < E)
-    for (int c = 0; c < nchunks; ++c) total += chunk_counts[(size_t)c * E + e];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int b0 = blockIdx.x * kScWords;
+  // one warp per expert; lane l sums the block counts [l * per, (l + 1) * per)
+  const int per = (nblk + 31) >> 5;
+  const int lo = min(lane * per, nblk), hi = min(lo + per, nblk);
+  for (int e = warp; e < E; e += blockDim.x >> 5) {
+    const int32_t* row = blk_counts + (size_t)e * nblk;
+    int sum = 0;
+#pragma unroll 8
+    for (int b = lo; b < hi; ++b) sum += row[b];
+    int inc = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    if (lane == 31) s_total[e] = inc;
+    if (hi > b0 && lo < b0 + kScWords) {           // this lane's range holds some of the block's words
+      int run = inc - sum;
+      for (int b = lo; b < hi && b < b0 + kScWords; ++b) {
+        if (b >= b0) s_pre[e][b - b0] = run;
+        run += row[b];
+      }
+    }
+  }
+  __syncthreads();
+  const int total = tid < E ? s_total[tid] : 0;
   const int padded = (total + kRowTile - 1) / kRowTile * kRowTile;
-  sp[e] = (e < E) ? padded : 0;
+  if (tid < 256) sp[tid] = tid < E ? padded : 0;
   __syncthreads();
   warp0_exclusive_scan256(sp);
   __syncthreads();
-  const int start = sp[e];
-  if (e < E) {
-    offsets[e] = start;
-    counts[e] = total;
-    int run = start;
-    for (int c = 0; c < nchunks; ++c) {
-      const int n = chunk_counts[(size_t)c * E + e];
-      chunk_counts[(size_t)c * E + e] = run;
-      run += n;
+  if (blockIdx.x == 0 && tid < E) {
+    const int start = sp[tid];
+    offsets[tid] = start;
+    counts[tid] = total;
+    for (int m = start / kRowTile; m < (start + padded) / kRowTile; ++m) tile_expert[m] = tid;
+    if (tid == E - 1) {
+      offsets[E] = start + padded;
+      *num_mtiles = (start + padded) / kRowTile;
     }
-    for (int m = start / kRowTile; m < (start + padded) / kRowTile; ++m) tile_expert[m] = e;
   }
-  if (e == E - 1) {
-    offsets[E] = start + padded;
-    *num_mtiles = (start + padded) / kRowTile;
-  }
-}
-
-__global__ void __launch_bounds__(kChunk) perm_scatter_kernel(const int32_t* __restrict__ topk_idx,
-                                                              const float* __restrict__ topk_w, int T, int E, int k,
-                                                              const int32_t* __restrict__ chunk_base,
-                                                              int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm,
-                                                              float* __restrict__ row_w) {
-  __shared__ uint32_t bm[kMaxE][kChunk / 32];
-  griddep_wait();
-  griddep_launch();
-  const int t = blockIdx.x * kChunk + threadIdx.x;
-  build_bitmap(bm, topk_idx, T, E, k, t);
-  if (t >= T) return;
-  const int wi = threadIdx.x >> 5;
-  const uint32_t below = (1u << (threadIdx.x & 31)) - 1u;
-  for (int j = 0; j < k; ++j) {
-    const int e = topk_idx[(size_t)t * k + j];
-    int rank = __popc(bm[e][wi] & below);
-    for (int w = 0; w < wi; ++w) rank += __popc(bm[e][w]);
-    const int row = chunk_base[(size_t)blockIdx.x * E + e] + rank;
+  // the block's (token, slot) pairs, consecutive pairs to consecutive threads
+  const int p0 = blockIdx.x * kScTokens * k;
+  const int np = min(kScTokens, T - blockIdx.x * kScTokens) * k;
+  for (int q = tid; q < np; q += blockDim.x) {
+    const int t = (p0 + q) / k;
+    const int e = topk_idx[p0 + q];
+    const int b = t >> 5;
+    const int row = sp[e] + s_pre[e][b - b0] + __popc(bm[(size_t)b * E + e] & ((1u << (t & 31)) - 1u));
     perm[row] = t;
-    inv_perm[(size_t)t * k + j] = row;
-    if (row_w) row_w[row] = topk_w[(size_t)t * k + j];
+    inv_perm[p0 + q] = row;
+    row_w[row] = topk_w[p0 + q];
   }
 }
 
@@ -543,7 +587,6 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
   }
   griddep_wait();
   griddep_launch();
-  const int per = (E + 31) >> 5;
   for (int t0 = 0; t0 < T; t0 += chunk_t) {
     const int nt = min(chunk_t, T - t0);
     // every (token, expert) of the chunk, one per thread: the logit (the
@@ -562,18 +605,9 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
     // top-k, one warp per token
     for (int tt = warp; tt < nt; tt += blockDim.x >> 5) {
       const int t = t0 + tt;
-      float sig[kMaxE / 32];
-      uint32_t key[kMaxE / 32];
-#pragma unroll
-      for (int i = 0; i < kMaxE / 32; ++i) {
-        const int e = lane + 32 * i;
-        const bool here = i < per && e < E;
-        sig[i] = here ? __uint_as_float(s_score[tt * E + e]) : 0.0f;
-        key[i] = here ? s_score[chunk_t * E + tt * E + e] : 0u;
-      }
       int idx;
       float w;
-      select_topk(sig, key, k, rsf, lane, idx, w);
+      select_topk_smem_any(s_score + tt * E, s_score + chunk_t * E + tt * E, E, k, rsf, lane, idx, w);
       if (lane < k) {
         topk_idx[(size_t)t * k + lane] = idx;
         topk_w[(size_t)t * k + lane] = w;
@@ -636,30 +670,40 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
   }
 }
 
-// Opts the small-batch kernel into its largest dynamic shared memory, once
-// per device.
-static nvfp4_status allow_route_small_smem() {
+// Opts a routing kernel into `bytes` of dynamic shared memory, once per
+// device (`done` is that kernel's own table).
+template <typename Kernel>
+static nvfp4_status allow_dyn_smem(Kernel kernel, int bytes, bool* done) {
   static std::mutex mu;
-  static bool done[64] = {};
   int dev = 0;
   NV_CHECK(check_cuda(cudaGetDevice(&dev), "cudaGetDevice"));
   if (dev < 0 || dev >= 64) dev = 63;
   std::lock_guard<std::mutex> lock(mu);
   if (!done[dev]) {
-    NV_CHECK(check_cuda(cudaFuncSetAttribute(route_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             kRouteSmallMaxDyn),
+    NV_CHECK(check_cuda(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
                         "cudaFuncSetAttribute"));
     done[dev] = true;
   }
   return NVFP4_OK;
 }
 
+static nvfp4_status allow_route_small_smem() {
+  static bool done[64] = {};
+  return allow_dyn_smem(route_small_kernel, kRouteSmallMaxDyn, done);
+}
+
+static nvfp4_status allow_topk_bitmap_smem() {
+  static bool done[64] = {};
+  return allow_dyn_smem(topk_bitmap_kernel, topk_bitmap_smem_bytes(kMaxE), done);
+}
+
 RouteScratch carve_route_scratch(Carver& c, int T, int E, int k) {
   RouteScratch r;
-  const int nchunks = (T + kChunk - 1) / kChunk;
+  const int nblk = (T + kTkTokens - 1) / kTkTokens;
   const int cap = route_rows_capacity(T, E, k);
   r.status = c.take<uint32_t>(64);
-  r.chunk_counts = c.take<int32_t>((size_t)nchunks * E);
+  r.bm = c.take<uint32_t>((size_t)nblk * E);
+  r.blk_counts = c.take<int32_t>((size_t)nblk * E);
   r.counts = c.take<int32_t>((size_t)E);
   r.tile_expert = c.take<int32_t>((size_t)cap / kRowTile + 1);
   r.num_mtiles = c.take<int32_t>(1);
@@ -677,7 +721,6 @@ int route_rows_capacity(int T, int E, int k) {
 
 nvfp4_status launch_route(const RouteArgs& a, const RouteScratch& r, cudaStream_t s) {
   const int cap = route_rows_capacity(a.T, a.E, a.k);
-  const int nchunks = (a.T + kChunk - 1) / kChunk;
   int splits = 0;
   if (a.x) {
     splits = router_splits(a.T, a.H);
@@ -714,18 +757,19 @@ nvfp4_status launch_route(const RouteArgs& a, const RouteScratch& r, cudaStream_
                             r.tile_expert, r.num_mtiles, a.perm, a.inv_perm, r.row_w, qx ? 1 : 0,
                             static_cast<const uint4*>(a.x), a.H, a.act_gscale, a.a_codes, a.a_scales);
   }
-  // each kernel waits for its predecessor's results (griddepcontrol.wait) as
-  // its first step, so programmatic launch only hides the launch latency
-  NV_CHECK(launch_dependent("topk_kernel", topk_kernel, dim3((a.T + 7) / 8), dim3(256), 0, s,
-                            (const float*)(splits ? r.partial : a.logits), splits, a.logit_offset, a.logits, a.bias,
-                            a.T, a.E, a.k, a.rsf, a.topk_idx, a.topk_w));
-  NV_CHECK(launch_dependent("perm_count_kernel", perm_count_kernel, dim3(nchunks), dim3(kChunk), 0, s,
-                            (const int32_t*)a.topk_idx, a.T, a.E, a.k, r.chunk_counts, cap, a.perm, r.row_w));
-  NV_CHECK(launch_dependent("perm_scan_kernel", perm_scan_kernel, dim3(1), dim3(256), 0, s, r.chunk_counts, nchunks,
-                            a.E, r.counts, a.expert_offsets, r.tile_expert, r.num_mtiles));
-  return launch_dependent("perm_scatter_kernel", perm_scatter_kernel, dim3(nchunks), dim3(kChunk), 0, s,
-                          (const int32_t*)a.topk_idx, (const float*)a.topk_w, a.T, a.E, a.k,
-                          (const int32_t*)r.chunk_counts, a.perm, a.inv_perm, r.row_w);
+  // both kernels wait for their predecessor's results (griddepcontrol.wait)
+  // before reading them, so programmatic launch only hides the launch latency
+  const int nblk = (a.T + kTkTokens - 1) / kTkTokens;
+  NV_CHECK(allow_topk_bitmap_smem());
+  NV_CHECK(launch_dependent("topk_bitmap_kernel", topk_bitmap_kernel, dim3(nblk), dim3(kTkThreads),
+                            topk_bitmap_smem_bytes(a.E), s, (const float*)(splits ? r.partial : a.logits), splits,
+                            a.logit_offset, a.logits, a.bias, a.T, a.E, a.k, a.rsf, cap, a.topk_idx, a.topk_w, r.bm,
+                            r.blk_counts, nblk, a.perm, r.row_w));
+  return launch_dependent("perm_scan_scatter_kernel", perm_scan_scatter_kernel,
+                          dim3((a.T + kScTokens - 1) / kScTokens), dim3(kScThreads), 0, s,
+                          (const int32_t*)a.topk_idx, (const float*)a.topk_w, a.T, a.E, a.k, (const uint32_t*)r.bm,
+                          (const int32_t*)r.blk_counts, nblk, r.counts, a.expert_offsets, r.tile_expert,
+                          r.num_mtiles, a.perm, a.inv_perm, r.row_w);
 }
 
 nvfp4_status check_route_shape(int T, int H, int E, int k) {

@@ -38,7 +38,8 @@ bool route_fuses_x_quantise(int T, int H, int k);
 
 struct RouteScratch {
   uint32_t* status = nullptr;           // device status word (start of the workspace)
-  int32_t* chunk_counts = nullptr;      // [chunks][E], then per-chunk row bases
+  uint32_t* bm = nullptr;               // [ceil(T/32)][E] tokens of each 32-token block that chose e
+  int32_t* blk_counts = nullptr;        // [E][ceil(T/32)] popcounts of bm
   int32_t* counts = nullptr;            // [E] rows routed to each expert
   int32_t* tile_expert = nullptr;       // [capacity / 128] expert of each m-tile
   int32_t* num_mtiles = nullptr;        // [1]

@@ -41,7 +41,7 @@ def test_abi_version_and_sizes():
 
 def test_forward_launch_count_follows_the_shape():
     """The host-only launch count of the forward: router GEMM, routing (one
-    kernel up to 256 tokens, else four), quantise-scatter (inside the routing
+    kernel up to 256 tokens, else two), quantise-scatter (inside the routing
     kernel when at most 64 KiB of permuted rows), gate/up, down, combine, plus
     the shared expert's three kernels (and a reduction after each of its GEMMs
     when few tokens split their K), and the dynamic modes' amax kernels."""
@@ -50,15 +50,15 @@ def test_forward_launch_count_follows_the_shape():
     assert n(32, 8, 256, 128, 2) == 5          # tiny layer: 32 x 2 rows of 144 bytes
     assert n(16, 80, 6144, 2048, 8) == 6       # decode: 442 KB of rows, a separate quantise kernel
     assert n(256, 80, 6144, 2048, 8) == 6
-    assert n(257, 80, 6144, 2048, 8) == 9      # multi-kernel routing above 256 tokens
-    assert n(8192, 80, 6144, 2048, 8) == 9
+    assert n(257, 80, 6144, 2048, 8) == 7      # two routing kernels above 256 tokens
+    assert n(8192, 80, 6144, 2048, 8) == 7
     # the shared expert at 16 tokens: both GEMMs split K, each adding a reduction
     assert n(16, 80, 6144, 2048, 8, I_shared=2048) == 11
-    assert n(8192, 80, 6144, 2048, 8, I_shared=2048) == 12
+    assert n(8192, 80, 6144, 2048, 8, I_shared=2048) == 10
     # the split K of the shared GEMMs starts below half a wave of tiles: 300
     # tokens are 3 x 4 tiles each (both split), 2560 tokens 20 x 4 (neither)
-    assert n(300, 16, 1024, 512, 4, I_shared=512) == 9 + 3 + 2
-    assert n(2560, 16, 1024, 512, 4, I_shared=512) == 9 + 3
+    assert n(300, 16, 1024, 512, 4, I_shared=512) == 7 + 3 + 2
+    assert n(2560, 16, 1024, 512, 4, I_shared=512) == 7 + 3
     assert n(3, 6, 512, 256, 3, I_shared=256) == 5 + 3 + 2
     assert n(32, 8, 256, 128, 2, act_scale_mode="expert") == 6     # per-expert g1: no fused quantisation
     assert n(16, 80, 6144, 2048, 8, act_scale_mode="dynamic") == 7

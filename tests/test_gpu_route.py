@@ -28,10 +28,12 @@ def _check_selection_and_permutation(c, logits, bias, k, rsf):
 
 
 @pytest.mark.parametrize("T,E,k", [(1, 8, 2), (300, 80, 8), (2049, 128, 8), (77, 256, 16), (33, 16, 16),
-                                   (5000, 80, 8), (256, 80, 8), (257, 80, 8), (256, 256, 16)])
+                                   (5000, 80, 8), (256, 80, 8), (257, 80, 8), (256, 256, 16),
+                                   # the large-batch path with one, four and eight experts per lane
+                                   (700, 20, 4), (1000, 100, 6), (600, 256, 16)])
 def test_selection_and_permutation_from_logits(T, E, k):
     """Batches of up to 256 tokens take the single-block path, larger ones the
-    multi-kernel path; both must give the oracle's bytes."""
+    two-kernel path; both must give the oracle's bytes."""
     require_cuda()
     c = capi()
     logits = workloads.random_floats((T, E), 3, f"logits{T}x{E}").numpy()
