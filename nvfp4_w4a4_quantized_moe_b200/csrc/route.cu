@@ -51,8 +51,11 @@ int router_splits(int T, int H) {
   const int mt = std::max(1, (T + kRBM - 1) / kRBM);
   const int kt = H / kRBK;
   int sp = 148 / mt;
-  sp = std::min(sp, std::max(1, kt / 4));
-  return std::max(1, sp);
+  sp = std::max(1, std::min(sp, std::max(1, kt / 4)));
+  // each split takes ceil(kt / sp) stages; recount so that none is left
+  // without any (25 stages over 6 splits of 5 would leave the sixth empty)
+  const int per = (kt + sp - 1) / sp;
+  return (kt + per - 1) / per;
 }
 
 __global__ void __launch_bounds__(kRThreads, 1)
@@ -72,7 +75,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
   const int mt = blockIdx.x;
   const int KT = p.H / kRBK;
   const int kt0 = blockIdx.y * p.kt_per_split;
-  const int kt1 = min(kt0 + p.kt_per_split, KT);
+  const int nkt = min(kt0 + p.kt_per_split, KT) - kt0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.stages; ++s) {
@@ -106,7 +109,8 @@ __global__ void __launch_bounds__(kRThreads, 1)
       int stage = 0;
       uint32_t phase = 0, filled = 0, fill_parity = 0;
       bool ok = true;
-      for (int kt = kt0; kt < kt1; ++kt) {
+      for (int i = 0; i < nkt; ++i) {
+        const int kt = kt0 + i;
         if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) {
           *abort_flag = 1;
           atomicExch(p.status, kDevTimeout);
@@ -136,7 +140,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int kt = kt0; kt < kt1; ++kt) {
+      for (int i = 0; i < nkt; ++i) {
         if (!mbar_wait(&full_bar[stage], phase, abort_flag)) {
           *abort_flag = 1;
           atomicExch(p.status, kDevTimeout);
@@ -148,7 +152,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
         const uint64_t adesc = sdesc_sw128(sA), bdesc = sdesc_sw128(sA + kRAbytes);
 #pragma unroll
         for (int j = 0; j < 4; ++j)      // 16 bf16 = 32 bytes of K per MMA
-          mma_bf16(tmem, adesc + 2 * j, bdesc + 2 * j, idesc, (kt > kt0 || j > 0) ? 1u : 0u);
+          mma_bf16(tmem, adesc + 2 * j, bdesc + 2 * j, idesc, (i > 0 || j > 0) ? 1u : 0u);
         tc_commit(&empty_bar[stage]);
         if (++stage == p.stages) {
           stage = 0;
@@ -163,20 +167,41 @@ __global__ void __launch_bounds__(kRThreads, 1)
     }
   } else {
     const int quad = warp & 3;
-    const int row = mt * kRBM + quad * 32 + lane;
     if (mbar_wait(&acc_bar, 0, abort_flag)) {
       tc_fence_after();
       const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16);
-      float* dst = p.partial + ((size_t)blockIdx.y * p.T + row) * p.E;
+      // The warp's 32 rows go through shared memory (the pipeline's stages,
+      // idle once every MMA has completed) and leave as one contiguous block
+      // of partial[split] with coalesced stores.
+      float* stg = reinterpret_cast<float*>(smem) + (size_t)quad * 32 * p.E;
+      const bool vec = (p.E & 3) == 0;   // rows of 16-byte multiples
       for (int c = 0; c < p.n_mma; c += 32) {
         uint32_t r[32];
         tmem_ld32(tbase + c, r);
         tmem_ld_wait();
-        if (row < p.T) {
+        float* srow = stg + (size_t)lane * p.E + c;
+        if (vec) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            if (c + i < p.E)
+              *reinterpret_cast<float4*>(srow + i) = make_float4(__uint_as_float(r[i]), __uint_as_float(r[i + 1]),
+                                                                  __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
+        } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i)
-            if (c + i < p.E) dst[c + i] = __uint_as_float(r[i]);
+            if (c + i < p.E) srow[i] = __uint_as_float(r[i]);
         }
+      }
+      __syncwarp();
+      const int row0 = mt * kRBM + quad * 32;
+      const size_t n = (size_t)max(0, min(32, p.T - row0)) * p.E;
+      float* dst = p.partial + ((size_t)blockIdx.y * p.T + row0) * p.E;
+      if (vec) {
+        const float4* s4 = reinterpret_cast<const float4*>(stg);
+        float4* d4 = reinterpret_cast<float4*>(dst);
+        for (size_t i = lane; i < n / 4; i += 32) d4[i] = s4[i];
+      } else {
+        for (size_t i = lane; i < n; i += 32) dst[i] = stg[i];
       }
     } else {
       *abort_flag = 1;
@@ -739,6 +764,9 @@ nvfp4_status launch_route(const RouteArgs& a, const RouteScratch& r, cudaStream_
     p.partial = r.partial;
     p.status = r.status;
     const int smem = router_smem_bytes(a.E);
+    // the epilogue stages the 128 x E fp32 tile in the pipeline's buffers
+    NV_REQUIRE(smem - 1024 >= kRBM * a.E * (int)sizeof(float), NVFP4_ERR_UNSUPPORTED_SHAPE,
+               "router: E=%d does not fit the epilogue's staging", a.E);
     NV_CHECK(check_cuda(cudaFuncSetAttribute(router_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
                         "cudaFuncSetAttribute"));
     dim3 grid((a.T + kRBM - 1) / kRBM, splits);

@@ -67,7 +67,11 @@ def test_skewed_loads_and_empty_experts():
                                                      ("prefill", 8192, 6144, 80, 8, 0.5),
                                                      # router split counts 1 and 24 on the large-batch path
                                                      ("one_split", 9600, 512, 80, 8, 0.0),
-                                                     ("many_splits", 600, 6144, 80, 8, 0.0)])
+                                                     ("many_splits", 600, 6144, 80, 8, 0.0),
+                                                     # 25 K stages: six splits of five would leave one empty,
+                                                     # so the router takes five (one token, then the large path)
+                                                     ("odd_stages", 1, 1600, 16, 4, 0.0),
+                                                     ("odd_stages_large", 300, 1600, 80, 8, 0.0)])
 def test_route_from_hidden_states(name, T, H, E, k, offset_std):
     """Logits match fp64 within the fp32 summation bound; top-k sets match
     wherever the oracle's k-th and (k+1)-th biased scores are apart by more
