@@ -6,7 +6,8 @@
  * implementation: the E2M1 and E4M3 conversions used by every quantiser
  * (element formats of the "K-EXAONE-152B-A23B-REAP-80E-NVFP4" model card,
  * "Quantization Setup") and the fixed fp32 sigmoid of the router
- * ("K-EXAONE-152B-A23B-REAP-80E-BF16" model card, "Routing behavior").
+ * ("K-EXAONE-152B-A23B-REAP-80E-BF16" model card, "Routing behavior"), and
+ * the router GEMM's split of K, which fixes the logits' fp32 rounding.
  * Same conventions as nvfp4_moe.h: device pointers, asynchronous on `stream`,
  * nvfp4_status results.  They are not needed to run the layer.
  */
@@ -83,6 +84,15 @@ NVFP4_API nvfp4_status nvfp4_test_block_scale_div(const float* amax, const float
 
 /* out[i] = the router's fp32 sigmoid of l[i]. */
 NVFP4_API nvfp4_status nvfp4_test_sigmoid(const float* l, int n, float* out, void* stream);
+
+/* Host arithmetic only, no CUDA call: the number of K splits the router GEMM
+ * of moe_route and the layer uses for T tokens and hidden size H (one CTA
+ * per 128 tokens and split, at most 148 CTAs, at least four 64-column K
+ * stages per split where H allows, and no split without stages), with the
+ * stages each split takes (the last may take fewer) in *stages_per_split
+ * when it is not NULL.  The logits' fp32 rounding follows this split.
+ * Returns -1 when T < 1 or H is not a positive multiple of 64. */
+NVFP4_API int nvfp4_test_router_splits(int T, int H, int* stages_per_split);
 
 #ifdef __cplusplus
 }

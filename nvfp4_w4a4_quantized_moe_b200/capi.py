@@ -108,6 +108,7 @@ _declare("nvfp4_test_sigmoid", _i, _vp, _i, _vp, _vp)
 _declare("nvfp4_test_mma_peak", _i, _i, _i, _i, _i, _vp, _vp, _vp)
 _declare("nvfp4_test_wait_timeout", _i, _vp, ctypes.c_uint64, _vp, _sz, _vp, _vp, _vp)
 _declare("nvfp4_test_block_scale_div", _i, _vp, _vp, _i, _vp, _vp, _vp, _vp, _vp)
+_declare("nvfp4_test_router_splits", _i, _i, _i, ctypes.POINTER(ctypes.c_int))
 
 # Every symbol the public headers declare (checked by the CPU test suite).
 EXPORTS = ("nvfp4_last_error", "nvfp4_abi_version", "nvfp4_workspace_status",
@@ -121,7 +122,8 @@ EXPORTS = ("nvfp4_last_error", "nvfp4_abi_version", "nvfp4_workspace_status",
            "moe_nvfp4_down", "moe_reap_keep",
            "nvfp4_block_stats_compute",
            "nvfp4_test_e2m1", "nvfp4_test_e2m1_sweep", "nvfp4_test_e4m3", "nvfp4_test_sigmoid",
-           "nvfp4_test_mma_peak", "nvfp4_test_wait_timeout", "nvfp4_test_block_scale_div")
+           "nvfp4_test_mma_peak", "nvfp4_test_wait_timeout", "nvfp4_test_block_scale_div",
+           "nvfp4_test_router_splits")
 
 
 def _check(status: int):
@@ -623,6 +625,15 @@ def nvfp4_test_e4m3(s: torch.Tensor):
     val = torch.empty(s.numel(), dtype=torch.float32, device=s.device)
     _check(lib.nvfp4_test_e4m3(_p(s), s.numel(), _p(codes), _p(val), _stream()))
     return codes, val
+
+
+def nvfp4_test_router_splits(T: int, H: int):
+    """(splits, K stages per split) of the router GEMM for T tokens, hidden H."""
+    per = ctypes.c_int(0)
+    n = lib.nvfp4_test_router_splits(T, H, ctypes.byref(per))
+    if n < 0:
+        raise ValueError(f"no router split for T={T} H={H}")
+    return n, per.value
 
 
 def nvfp4_test_sigmoid(l: torch.Tensor):

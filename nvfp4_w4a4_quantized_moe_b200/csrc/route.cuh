@@ -48,6 +48,9 @@ struct RouteScratch {
 };
 
 int route_rows_capacity(int T, int E, int k);
+// K splits of the router GEMM (64-column K stages, one CTA per 128 tokens
+// and split); a function of the shape only.
+int router_splits(int T, int H);
 RouteScratch carve_route_scratch(Carver& c, int T, int E, int k);
 nvfp4_status check_route_shape(int T, int H, int E, int k);
 nvfp4_status launch_route(const RouteArgs& a, const RouteScratch& r, cudaStream_t s);

@@ -3,6 +3,7 @@
 #include "../../include/nvfp4_moe_testing.h"
 #include "common.cuh"
 #include "host.cuh"
+#include "route.cuh"
 #include "route_math.cuh"
 
 namespace nvfp4moe {
@@ -484,4 +485,11 @@ extern "C" nvfp4_status nvfp4_test_block_scale_div(const float* amax, const floa
   test_block_scale_div_kernel<<<(n + 255) / 256, 256, 0, as_stream(stream)>>>(amax, g, n, q_lib, q_ieee, code_lib,
                                                                               code_ieee);
   return check_launch("test_block_scale_div_kernel");
+}
+
+extern "C" int nvfp4_test_router_splits(int T, int H, int* stages_per_split) {
+  if (T < 1 || H <= 0 || H % 64 != 0) return -1;
+  const int splits = nvfp4moe::router_splits(T, H);
+  if (stages_per_split) *stages_per_split = (H / 64 + splits - 1) / splits;
+  return splits;
 }

@@ -70,6 +70,29 @@ def test_forward_launch_count_follows_the_shape():
     assert c.lib.moe_nvfp4_forward_launches(16, 80, 6144, 2048, 8, 0, 7) == -1
 
 
+def test_router_splits_leave_no_split_empty():
+    """The router GEMM's K split (host arithmetic): every split gets K stages,
+    at least four where it has company, and the CTAs (one per 128 tokens and
+    split) stay within one wave of the 148 SMs."""
+    c = capi()
+    for T in (1, 16, 100, 128, 129, 257, 300, 1000, 2048, 4096, 8192, 9600, 20000):
+        mt = -(-T // 128)
+        for H in range(64, 32768 + 1, 64):
+            sp, per = c.nvfp4_test_router_splits(T, H)
+            kt = H // 64
+            assert sp >= 1 and per >= 1
+            assert (sp - 1) * per < kt <= sp * per, (T, H, sp, per)    # the last split has stages
+            assert sp * mt <= max(148, mt)
+            if sp > 1:
+                assert per >= 4
+    assert c.nvfp4_test_router_splits(16, 6144) == (24, 4)       # decode
+    assert c.nvfp4_test_router_splits(8192, 6144) == (2, 48)     # prefill
+    assert c.nvfp4_test_router_splits(1, 1600) == (5, 5)         # 25 stages: five splits, not six
+    assert c.nvfp4_test_router_splits(129, 19200) == (60, 5)     # 300 stages: 74 splits of 5 would leave 14 empty
+    with pytest.raises(ValueError):
+        c.nvfp4_test_router_splits(1, 100)
+
+
 def test_host_side_argument_checks():
     c = capi()
     lib = c.lib
