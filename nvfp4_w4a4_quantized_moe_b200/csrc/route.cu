@@ -534,10 +534,10 @@ __global__ void __launch_bounds__(kScThreads, 1) perm_scan_scatter_kernel(
 // ---------------------------------------------------------------------------
 // Routing of a small batch (T <= 256) in one block: top-k, per-expert counts,
 // the padded scan, and the scatter, with the padding fill of perm and row_w
-// that the large-batch path does in its count kernel.  The scores (sigma and
+// that the large-batch path does in its top-k kernel.  The scores (sigma and
 // the selection key) are computed one (token, expert) per thread and kept in
 // shared memory, so a token's warp only runs the selection rounds.  The
-// arithmetic is the same as topk_token's (expert_score, select_topk) and so
+// arithmetic is the large-batch path's (expert_score, select_topk) and so
 // is every integer result.  For small layers (route_fuses_x_quantise) the
 // kernel also quantises x and writes it to the permuted rows, the work of the
 // layer's quantise-scatter kernel, with the same bits.
